@@ -1,0 +1,236 @@
+"""CPU oracle for the Switch-FFN layer forward pass.
+
+TEST INFRASTRUCTURE ONLY.  This module is the slow, plainly written
+definition that the CUDA library is checked against.  Only ``tests/``,
+``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` may
+import it; the library never calls it and it never calls the library.  It
+shares no code with the CUDA path: the one thing both sides use is the
+seeded input generator in ``switch_inputs`` (which draws and encodes inputs
+and computes no stage of the layer).
+
+Every stage follows the page "Switch Transformers: scaling to
+trillion-parameter models" (cited below as [P1 §section]):
+
+* router logits ``h(x) = W_r . x`` and the softmax gate
+  [P1 §"Switch Routing: From Top-k to k = 1", gate equation];
+* the routing math in float32 [P1 §"Making Sparse Training Stable",
+  selective precision] -- the oracle computes logits and probabilities in
+  float64 and takes the top-1 decision on the float32-rounded logits;
+* top-1 choice, k = 1 [P1 §"Switch Routing", and the dispatch figure
+  "argmax p_i, k=1" in §"Expert Capacity and the Capacity Factor"];
+* expert capacity = tokens / experts x capacity factor, rounded up
+  [P1 §"Expert Capacity and the Capacity Factor", capacity equation];
+* overflow tokens dropped to the residual, unused slots are padding
+  [same section, the two trade-off bullets and the figure];
+* N independent FFN experts [P1 §"The Core Idea"], ReLU, no biases;
+* the gate-scaled combine ``y = p_i(x) E_i(x)`` over the single selected
+  expert [P1 §"Switch Routing", combine equation with |T| = 1];
+* the load-balancing loss ``alpha . N . sum_i f_i P_i`` with ``f_i`` the
+  fraction of tokens whose argmax is ``i`` and ``P_i`` the mean router
+  probability [P1 §"The Load-Balancing Loss", loss and f/P equations].
+
+Readings taken where the pages leave a step open: capacity rounds up; the
+whole batch is one routing group and tokens take slots in batch order;
+ties go to the lowest expert index; ``f_i`` counts routed tokens including
+dropped ones (the page defines it through the argmax, before capacity);
+the combine adds the residual ``x`` when asked (block output of a dropped
+token is ``x``); no dropout (forward pass).
+
+Arithmetic is float64 throughout (expert matmuls included); floating-point
+inputs are the exact values of the bf16 / fp32 bit patterns the GPU reads.
+Parity pins: every function here is pinned by a ``-m "not gpu"`` test
+(``tests/test_oracle_pins.py``) against closed forms, hand-worked golden
+values, invariants the pages state, and brute force; none is unpinned.
+"""
+from fractions import Fraction
+import math
+
+import numpy as np
+
+from switch_inputs import as_f64
+
+
+# ------------------------------------------------------------------ capacity
+
+def capacity(T: int, n_experts: int, capacity_factor: float) -> int:
+    """Expert capacity C = ceil(T / N x capacity_factor), exactly.
+
+    [P1 §"Expert Capacity and the Capacity Factor", capacity equation]; the
+    page prints no rounding, rounding up is the reading taken.  The float
+    ``capacity_factor`` is taken at its exact binary value.
+    """
+    if T < 0 or n_experts <= 0 or not capacity_factor > 0:
+        raise ValueError("need T >= 0, N > 0, capacity_factor > 0")
+    return math.ceil(Fraction(T) * Fraction(capacity_factor) / n_experts)
+
+
+# -------------------------------------------------------------------- router
+
+def router(x, w_r, b_r=None):
+    """Logits, softmax gate, top-1 expert, gate value and top-1/top-2 margin.
+
+    ``x [T, d]`` (fp32 values or bf16 bits), ``w_r [N, d]`` fp32,
+    ``b_r [N]`` or None.  Returns a dict:
+
+    * ``logits`` float64 ``h = x . W_r^T (+ b)``
+      [P1 §"Switch Routing", router logits];
+    * ``probs`` float64 ``p_i = exp(h_i) / sum_j exp(h_j)`` [gate equation],
+      evaluated with the row maximum subtracted (same value, no overflow);
+    * ``idx`` int64: the expert of largest float32-rounded logit, lowest
+      index on ties [k = 1; routing math in float32, §"Making Sparse
+      Training Stable"];
+    * ``gate`` float64 ``p_idx``;
+    * ``margin`` float64: largest minus second largest probability
+      (``inf`` when N = 1).
+    """
+    h = as_f64(x) @ np.asarray(w_r, dtype=np.float64).T
+    if b_r is not None:
+        h = h + np.asarray(b_r, dtype=np.float64)[None, :]
+    T, N = h.shape
+    if T == 0:
+        z = np.zeros(0)
+        return {"logits": h, "probs": h.copy(), "idx": np.zeros(0, np.int64),
+                "gate": z, "margin": z}
+    shifted = h - h.max(axis=1, keepdims=True)
+    e = np.exp(shifted)
+    p = e / e.sum(axis=1, keepdims=True)
+    idx = np.argmax(h.astype(np.float32), axis=1).astype(np.int64)
+    gate = p[np.arange(T), idx]
+    if N == 1:
+        margin = np.full(T, np.inf)
+    else:
+        top2 = np.sort(p, axis=1)[:, -2:]
+        margin = top2[:, 1] - top2[:, 0]
+    return {"logits": h, "probs": p, "idx": idx, "gate": gate,
+            "margin": margin}
+
+
+# ------------------------------------------------------------------ dispatch
+
+def dispatch(idx, n_experts: int, C: int):
+    """Capacity-bounded dispatch, one pass over the batch in token order.
+
+    Each token takes the next free slot of its expert; once an expert holds
+    C tokens, later tokens routed to it are dropped
+    [P1 §"Expert Capacity and the Capacity Factor": overflow dropped,
+    unused slots are padding].  Returns ``rank [T]`` (slot number within
+    the expert, also for dropped tokens), ``drop [T]`` bool (rank >= C),
+    ``counts [N]`` (tokens routed, before the capacity cut) and
+    ``slot_token [N*C]`` (token in each slot, -1 for padding).
+    """
+    idx = np.asarray(idx)
+    T = idx.shape[0]
+    cnt = [0] * n_experts
+    rank = np.empty(T, dtype=np.int64)
+    drop = np.empty(T, dtype=bool)
+    slot_token = np.full(n_experts * C, -1, dtype=np.int64)
+    for t in range(T):
+        e = int(idx[t])
+        r = cnt[e]
+        cnt[e] = r + 1
+        rank[t] = r
+        drop[t] = r >= C
+        if r < C:
+            slot_token[e * C + r] = t
+    return {"rank": rank, "drop": drop,
+            "counts": np.asarray(cnt, dtype=np.int64),
+            "slot_token": slot_token}
+
+
+# ---------------------------------------------------------------- experts
+
+def expert(x_rows, w1_e, w2_e):
+    """One expert FFN on rows of x: relu(x . W1_e^T) . W2_e^T, float64.
+
+    ``w1_e [F, d]``, ``w2_e [d, F]`` (output-major) [P1 §"The Core Idea":
+    each expert is an independent FFN; ReLU and no biases are the reading].
+    """
+    hid = as_f64(x_rows) @ as_f64(w1_e).T
+    hid = np.maximum(hid, 0.0)
+    return hid @ as_f64(w2_e).T
+
+
+def expert_ffn(x, w1, w2, slot_token, counts, C, experts=None):
+    """Every expert over its capacity buffer: ``Y [N, C, d]`` float64.
+
+    Row r of expert e holds E_e(x[slot_token[e*C + r]]) for the
+    n_e = min(counts[e], C) kept tokens; padding rows stay zero.
+    ``experts`` restricts the work to a subset (others stay zero).
+    """
+    N = len(counts)
+    d = x.shape[1]
+    Y = np.zeros((N, C, d))
+    for e in (range(N) if experts is None else experts):
+        n = min(int(counts[e]), C)
+        if n == 0:
+            continue
+        rows = slot_token[e * C: e * C + n]
+        Y[e, :n] = expert(x[rows], w1[e], w2[e])
+    return Y
+
+
+# ------------------------------------------------------------------ combine
+
+def combine(x, idx, rank, drop, gate, Y, residual=True):
+    """Block output: x + p_idx(x) . E_idx(x) for kept tokens, x for dropped.
+
+    [P1 §"Switch Routing", combine equation with one selected expert;
+    §"Expert Capacity ...", a dropped token passes through the residual.]
+    With ``residual=False`` the residual term is left out (dropped tokens
+    give 0).
+    """
+    T, d = x.shape
+    out = as_f64(x) if residual else np.zeros((T, d))
+    kept = ~np.asarray(drop, dtype=bool)
+    out[kept] += np.asarray(gate)[kept, None] * Y[np.asarray(idx)[kept],
+                                                  np.asarray(rank)[kept]]
+    return out
+
+
+# ----------------------------------------------------------------- aux loss
+
+def aux_loss(counts, probs, alpha: float):
+    """loss = alpha . N . sum_i f_i P_i.
+
+    f_i = counts_i / T (tokens whose argmax is i, dropped ones included),
+    P_i = mean over tokens of p_i(x)
+    [P1 §"The Load-Balancing Loss", loss equation and f/P equations].
+    Returns (loss, f, P) in float64; an empty batch gives loss 0.
+    """
+    counts = np.asarray(counts, dtype=np.float64)
+    N = counts.shape[0]
+    T = probs.shape[0]
+    if T == 0:
+        return 0.0, np.zeros(N), np.zeros(N)
+    f = counts / T
+    P = np.asarray(probs, dtype=np.float64).sum(axis=0) / T
+    return float(alpha * N * np.sum(f * P)), f, P
+
+
+# ------------------------------------------------------------- whole layer
+
+def layer_forward(x, w_r, b_r, w1, w2, capacity_factor, alpha=0.01,
+                  residual=True, experts=None):
+    """All stages in order; returns every intermediate in a dict."""
+    T = x.shape[0]
+    N = w_r.shape[0]
+    C = capacity(T, N, capacity_factor)
+    r = router(x, w_r, b_r)
+    dsp = dispatch(r["idx"], N, C)
+    Y = expert_ffn(x, w1, w2, dsp["slot_token"], dsp["counts"], C, experts)
+    out = combine(x, r["idx"], dsp["rank"], dsp["drop"], r["gate"], Y,
+                  residual)
+    loss, f, P = aux_loss(dsp["counts"], r["probs"], alpha)
+    return {"C": C, **r, **dsp, "Y": Y, "out": out, "loss": loss,
+            "f": f, "P": P}
+
+
+def token_outputs(x, tokens, idx, drop, gate, w1, w2, residual=True):
+    """Block output rows for selected tokens only (for full-size sampling)."""
+    tokens = np.asarray(tokens)
+    rows = as_f64(x[tokens]) if residual else np.zeros((len(tokens), x.shape[1]))
+    for j, t in enumerate(tokens):
+        if not drop[t]:
+            e = int(idx[t])
+            rows[j] += gate[t] * expert(x[t:t + 1], w1[e], w2[e])[0]
+    return rows
