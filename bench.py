@@ -1,0 +1,461 @@
+#!/usr/bin/env python
+"""Switch-FFN layer forward benchmark on B200.
+
+One step = one whole layer forward through the C ABI (router, dispatch,
+expert FFNs, gate-scaled combine with residual, load-balancing loss) on one
+batch of synthetic input already resident in HBM.  The default workload is
+the Switch-Base-like bf16 layer (T = 65536 tokens = batch 128 x seq 512,
+d_model 768, d_ff 3072, 128 experts, capacity factor 1.25).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...     (the CPU oracle, timed)
+
+With N > 1 (torchrun) every rank runs an independent replica on its own
+batch (its own routing group): weak scaling, no collective on the data path.
+Rank 0 prints one JSON line.
+"""
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+from switch_inputs import WORKLOADS, make_x, make_router, make_w1, make_w2, Inputs  # noqa: E402
+
+METRIC = "Switch-layer fwd tokens/s"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="base", choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="budget of the oracle sample timed for cpu_baseline")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_desc(wl):
+    return (f"{wl.name}: Switch-FFN layer, T={wl.T} tokens, d_model={wl.d_model}, "
+            f"d_ff={wl.d_ff}, N={wl.n_experts} experts, capacity_factor={wl.capacity_factor}, "
+            f"{wl.dtype} (fp32 router)")
+
+
+# ------------------------------------------------------------ CPU oracle
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def oracle_sample(inp, budget_s, fixed_experts=None):
+    """Time the oracle on a bounded sample of the workload.
+
+    The router (fp64 logits, softmax, top-1) and the dispatch run on every
+    token; the expert FFNs run for experts 0, 1, ... until the time budget is
+    spent (or for `fixed_experts` of them); the combine and the loss run on
+    every token.  The expert time is scaled by N / (experts run) to estimate
+    the whole layer.  Returns (estimated seconds for the layer, experts run).
+    """
+    import oracle.switch_oracle as orc
+    wl = inp.wl
+    t0 = time.perf_counter()
+    r = orc.router(inp.x, inp.w_r, inp.b_r)
+    C = orc.capacity(wl.T, wl.n_experts, wl.capacity_factor)
+    dsp = orc.dispatch(r["idx"], wl.n_experts, C)
+    t1 = time.perf_counter()
+    Y = np.zeros((wl.n_experts, C, wl.d_model))
+    done = 0
+    t_exp0 = time.perf_counter()
+    limit = fixed_experts if fixed_experts is not None else wl.n_experts
+    while done < limit:
+        part = orc.expert_ffn(inp.x, inp.w1, inp.w2, dsp["slot_token"], dsp["counts"], C,
+                              experts=[done])
+        Y[done] = part[done]
+        done += 1
+        if fixed_experts is None and time.perf_counter() - t0 > budget_s:
+            break
+    t_exp = time.perf_counter() - t_exp0
+    t2 = time.perf_counter()
+    orc.combine(inp.x, r["idx"], dsp["rank"], dsp["drop"], r["gate"], Y)
+    orc.aux_loss(dsp["counts"], r["probs"], wl.alpha)
+    t3 = time.perf_counter()
+    est = (t1 - t0) + (t3 - t2) + t_exp * wl.n_experts / done
+    return est, done
+
+
+def host_inputs(wl, rank=0):
+    w_r, b_r = make_router(wl)
+    x = make_x(wl.with_(seed=wl.seed + 7919 * rank))
+    return Inputs(wl, x, w_r, b_r, make_w1(wl), make_w2(wl))
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = WORKLOADS[args.workload]
+    inp = host_inputs(wl)
+    per_step_budget = max(1.0, min(8.0, 150.0 / max(1, args.steps + args.warmup)))
+    est, n_exp = oracle_sample(inp, per_step_budget)          # sizes the sample
+    for _ in range(max(0, args.warmup - 1)):
+        oracle_sample(inp, per_step_budget, fixed_experts=n_exp)
+    ests = [oracle_sample(inp, per_step_budget, fixed_experts=n_exp)[0]
+            for _ in range(args.steps)]
+    sec = statistics.mean(ests)
+    value = wl.T / sec
+    sample = (f"oracle (numpy float64) on all {wl.T} tokens for router, dispatch, combine "
+              f"and loss; expert FFNs for experts 0..{n_exp - 1} of {wl.n_experts}, "
+              f"time scaled by {wl.n_experts}/{n_exp}")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": workload_desc(wl)},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# -------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.rows = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.gpu_id)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.rows.append((time.time(), [c.strip() for c in ln.split(",")]))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        rows = [r for (t, r) in self.rows if t0 - 0.25 <= t <= t1 + 0.25]
+        if not rows:   # timed region shorter than the sampling period: nearest samples
+            rows = [r for (t, r) in sorted(self.rows, key=lambda tr: abs(tr[0] - (t0 + t1) / 2))[:3]]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows),
+                "power_w_max": max((float(r[3]) for r in rows if r[3].replace(".", "").isdigit()),
+                                   default=None)}
+
+
+# ------------------------------------------------------------- GPU arm
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+    from sparse_mixture_experts_switch_b200 import switch_moe as sm
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+
+    wl = WORKLOADS[args.workload]
+    inp = host_inputs(wl, rank)
+    T, d, F, N = wl.T, wl.d_model, wl.d_ff, wl.n_experts
+    C = sm.switch_capacity(T, N, wl.capacity_factor)
+    bf = wl.dtype == "bf16"
+    tdt = torch.bfloat16 if bf else torch.float32
+
+    def to_dev(a):
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+    x = to_dev(inp.x)
+    w_r = to_dev(inp.w_r)
+    b_r = None if inp.b_r is None else to_dev(inp.b_r)
+    w1 = to_dev(inp.w1)
+    w2 = to_dev(inp.w2)
+    cfg = sm.config(T, d, F, N, wl.capacity_factor, dtype=wl.dtype, alpha=wl.alpha)
+    ws = sm.workspace(cfg, device=dev)
+    out = torch.empty_like(x)
+    idx = torch.empty(T, dtype=torch.int32, device=dev)
+    gate = torch.empty(T, dtype=torch.float32, device=dev)
+    counts = torch.empty(N, dtype=torch.int32, device=dev)
+    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        sm.switch_layer_forward(cfg, x, w_r, b_r, w1, w2, out, idx, gate, counts, loss, ws)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    clocks = ClockSampler(local if not os.environ.get("CUDA_VISIBLE_DEVICES")
+                          else os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local])
+    clocks.start()
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    st, where, info = sm.switch_get_device_error(ws)
+    if st != 0:
+        raise RuntimeError(f"device error {st} at {where} ({info}) during warm-up")
+
+    # ------------------------------------------------ timed region (device)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize(dev)
+    t_wall0 = time.time()
+    for e0, e1 in evs:
+        flush.zero_()                      # L2 flush, outside the events
+        e0.record(stream)
+        step()
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    t_wall1 = time.time()
+    ms = [e0.elapsed_time(e1) for e0, e1 in evs]
+    total_ms = torch.tensor([sum(ms)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(total_ms, op=dist.ReduceOp.MAX)
+    total_ms = float(total_ms.item())
+    st, where, info = sm.switch_get_device_error(ws)
+    if st != 0:
+        raise RuntimeError(f"device error {st} at {where} ({info}) in the timed region")
+    ms_per_step = total_ms / args.steps
+    value = T * args.steps * world / (total_ms / 1e3)
+
+    # ------------------------------------------- end to end (host buffers)
+    x_host = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
+    x_host.copy_(x)
+    out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    loss_host = torch.empty(1, dtype=torch.float32, pin_memory=True)
+
+    def e2e_step():
+        x.copy_(x_host, non_blocking=True)
+        step()
+        out_host.copy_(out, non_blocking=True)
+        loss_host.copy_(loss, non_blocking=True)
+
+    for _ in range(max(3, args.warmup)):
+        e2e_step()
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    e2e_value = T * args.steps * world / (float(e2e_ms.item()) / 1e3)
+    clocks.stop()
+
+    # --------------------------------------- per-kernel roofline (rank 0)
+    line = None
+    if rank == 0:
+        pk, pk_kind = peaks()
+        kern = kernel_rooflines(sm, cfg, wl, C, x, w_r, b_r, w1, w2, ws, flush, stream, dev,
+                                pk, pk_kind)
+        T_kept = kern.pop("_T_kept")
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            est, n_exp = oracle_sample(inp, args.cpu_seconds)
+            cpu = {"value": wl.T / est, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                   "sample": (f"numpy float64 oracle: router, dispatch, combine and loss on "
+                              f"all {wl.T} tokens; expert FFNs of experts 0..{n_exp - 1} of "
+                              f"{wl.n_experts}, their time scaled by {wl.n_experts}/{n_exp}"),
+                   "host_cpus": os.cpu_count()}
+        ffn = kern["expert_ffn"]
+        flops_layer = 2.0 * T * d * N + 4.0 * T_kept * d * F
+        bytes_layer = 3 * T * d * 2 + 2 * N * d * F * 2 + T * d * 2
+        t_layer_min = max(flops_layer / (pk["bf16_tflops"] * 1e12),
+                          bytes_layer / (pk["hbm_gbs"] * 1e9))
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if bf else "f32", "data": "synthetic",
+            "config": {"workload": workload_desc(wl), "T": T, "d_model": d, "d_ff": F,
+                       "n_experts": N, "capacity_factor": wl.capacity_factor, "capacity": C,
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": "flushed (256 MiB write) before every timed step, outside the events"},
+            "roofline": {"kernel": "expert FFN grouped GEMM (GEMM1 + GEMM2, tcgen05)",
+                         "bound": "tensor", "achieved": ffn["tflops"],
+                         "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": ffn["tflops"] / pk["bf16_tflops"],
+                         "peak_kind": f"{pk_kind} bf16 burst", "traffic": ffn.get("traffic"),
+                         "useful_flops": 4.0 * T_kept * d * F},
+            "layer_roofline": {"t_min_us": t_layer_min * 1e6,
+                               "tokens_per_s": T / t_layer_min,
+                               "frac": (T / t_layer_min and value / world / (T / t_layer_min))},
+            "kernels": kern,
+            "routing": {"T_kept": T_kept, "drop_rate": 1.0 - T_kept / T,
+                        "padding": 1.0 - T_kept / (N * C)},
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": x.numel() * x.element_size(),
+                    "d2h_bytes_per_step": out.numel() * out.element_size() + 4},
+            "clocks": clocks.summary(t_wall0, t_wall1),
+            "gpu_launches": launches_per_step(cfg, wl) * args.steps,
+        }
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+def launches_per_step(cfg, wl):
+    """Kernels switch_layer_forward launches with the default flags on this
+    workload: router (weight split + tensor-core router), scan, finalize,
+    GEMM1, GEMM2, dropped-token copy, loss."""
+    tc = wl.dtype == "bf16" and (wl.n_experts + 15) // 16 * 16 <= 256
+    if tc:
+        return 8
+    return 8   # SIMT router + tile ranks replace the two router launches
+
+
+def kernel_rooflines(sm, cfg, wl, C, x, w_r, b_r, w1, w2, ws, flush, stream, dev, pk, pk_kind,
+                     reps=10):
+    """Staged calls timed alone (L2 flushed before each), with their
+    algorithmic bytes / FLOPs."""
+    import torch
+    T, d, F, N = wl.T, wl.d_model, wl.d_ff, wl.n_experts
+    i32 = dict(dtype=torch.int32, device=dev)
+    idx = torch.empty(T, **i32)
+    gate = torch.empty(T, dtype=torch.float32, device=dev)
+    probs = torch.empty(T, N, dtype=torch.float32, device=dev)
+    rank = torch.empty(T, **i32)
+    drop = torch.empty(T, dtype=torch.uint8, device=dev)
+    counts = torch.empty(N, **i32)
+    slot = torch.empty(N * C, **i32)
+    x_disp = torch.empty(N * C, d, dtype=x.dtype, device=dev)
+    y = torch.empty(N * C, d, dtype=x.dtype, device=dev)
+    out = torch.empty_like(x)
+    loss = torch.empty(1, dtype=torch.float32, device=dev)
+
+    def timed(fn):
+        fn()
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            ts.append(e0.elapsed_time(e1) * 1e-3)
+        return statistics.mean(ts)
+
+    es = x.element_size()
+    t_router = timed(lambda: sm.switch_router(cfg, x, w_r, b_r, idx, gate, None, ws))
+    t_router_p = timed(lambda: sm.switch_router(cfg, x, w_r, b_r, idx, gate, probs, ws))
+    t_disp = timed(lambda: sm.switch_dispatch(cfg, idx, None, rank, drop, counts, slot, None,
+                                              None, ws))
+    t_disp_g = timed(lambda: sm.switch_dispatch(cfg, idx, None, rank, drop, counts, slot, x,
+                                                x_disp, ws))
+    cnt = counts.cpu().numpy().astype(np.int64)
+    T_kept = int(np.minimum(cnt, C).sum())
+    t_ffn = timed(lambda: sm.switch_expert_ffn(cfg, x, slot, counts, w1, w2, y, ws))
+    t_comb = timed(lambda: sm.switch_combine(cfg, x, idx, rank, drop, gate, y, out))
+    t_aux = timed(lambda: sm.switch_aux_loss(cfg, counts, probs, loss, None, None, ws))
+    st, where, info = sm.switch_get_device_error(ws)
+    if st != 0:
+        raise RuntimeError(f"device error {st} at {where} ({info}) in kernel timing")
+    hbm = pk["hbm_gbs"]
+
+    def bw(name, t, nbytes):
+        gbs = nbytes / t / 1e9
+        return {"us": t * 1e6, "bytes": nbytes, "gbs": gbs, "frac_hbm": gbs / hbm,
+                "frac_8tbs": gbs / 8000.0}
+
+    flops = 4.0 * T_kept * d * F
+    res = {
+        "router": bw("router", t_router, T * d * es + N * d * 4 + T * 8),
+        "router_with_probs": bw("router", t_router_p, T * d * es + N * d * 4 + T * 8 + T * N * 4),
+        "dispatch_metadata": {"us": t_disp * 1e6,
+                              "bytes": T * 4 + T * 5 + N * 4 + N * C * 4},
+        "dispatch_gather": bw("dispatch", t_disp_g,
+                              T * 9 + N * 4 + N * C * 4 + T_kept * d * es + N * C * d * es),
+        "expert_ffn": {"us": t_ffn * 1e6, "useful_flops": flops, "tflops": flops / t_ffn / 1e12,
+                       "frac_burst": flops / t_ffn / 1e12 / pk["bf16_tflops"],
+                       "frac_sustained": flops / t_ffn / 1e12 / pk["bf16_tflops_sustained"],
+                       "weight_bytes": 2 * N * d * F * es, "traffic": None},
+        "combine": bw("combine", t_comb, 2 * T * d * es + T_kept * d * es + T * 13),
+        "aux_loss_from_probs": bw("aux", t_aux, T * N * 4 + N * 4),
+        "peaks": {"hbm_gbs": hbm, "bf16_tflops": pk["bf16_tflops"], "kind": pk_kind},
+        "_T_kept": T_kept,
+    }
+    return res
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,198 @@
+/*
+ * switch_moe.h -- C ABI of the Switch-FFN layer forward pass on one NVIDIA
+ * B200 (sm_100a).
+ *
+ * The layer is the one of "Switch Transformers: scaling to trillion-parameter
+ * models" (cited below as [P1 section]):
+ *   router logits h(x) = W_r . x and softmax gate p_i(x)
+ *       [P1 "Switch Routing: From Top-k to k = 1", gate equation],
+ *   routing math in float32 [P1 "Making Sparse Training Stable",
+ *       selective precision],
+ *   top-1 expert (k = 1), lowest index on ties,
+ *   expert capacity C = ceil(T / N x capacity_factor)
+ *       [P1 "Expert Capacity and the Capacity Factor", capacity equation],
+ *   tokens take slots in batch order; overflow tokens are dropped and pass
+ *       through on the residual; unused slots are padding [same section],
+ *   N independent ReLU FFN experts E_e(x) = relu(x W1_e^T) W2_e^T
+ *       [P1 "The Core Idea"],
+ *   gate-scaled combine y = p_i(x) E_i(x) [P1 "Switch Routing", combine
+ *       equation, one selected expert], block output x + y,
+ *   load-balancing loss alpha . N . sum_i f_i P_i
+ *       [P1 "The Load-Balancing Loss", loss and f/P equations].
+ *
+ * Conventions for every entry point:
+ *   - Tensor pointers are DEVICE pointers owned by the caller, row-major and
+ *     contiguous, each aligned to at least 16 bytes.  The library never
+ *     allocates or frees device memory.
+ *   - Scratch lives in a caller-owned device workspace of at least
+ *     switch_workspace_size() bytes (256-byte aligned).  Its first 16 bytes
+ *     hold the device error word; zero it once after allocating (a
+ *     zero-filled allocation is fine).  Calls that share a workspace must be
+ *     ordered on one stream.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Calls are asynchronous on it; nothing synchronises the host
+ *     except switch_get_device_error().
+ *   - Host-detectable errors (bad arguments, unsupported shapes, workspace
+ *     too small) return synchronously and launch nothing.  Launch failures
+ *     return SWITCH_ERR_CUDA.  Device-side failures (a bounded wait that ran
+ *     out) are recorded in the error word and read by
+ *     switch_get_device_error().
+ *   - T = 0 is a no-op that returns SWITCH_OK and writes nothing.
+ *   - Inputs must be finite; results for NaN/Inf inputs are unspecified.
+ *   - dtype SWITCH_BF16: x, w1, w2, y, x_disp and out are bf16, the router
+ *     weight/bias/probabilities/gates are fp32, d_model and d_ff must be
+ *     multiples of 64.  dtype SWITCH_F32: every floating tensor is fp32 and
+ *     all arithmetic is fp32 FMA (no TF32).
+ *   - Index tensors are int32, the drop mask is uint8 (0 kept / 1 dropped).
+ *   - Expert weights are stored output-major per expert, like the weight of
+ *     a linear layer: w1 [N, d_ff, d_model], w2 [N, d_model, d_ff], so that
+ *     E_e(x) = relu(x . w1[e]^T) . w2[e]^T.  Router weight w_r [N, d_model].
+ */
+#ifndef SWITCH_MOE_H_
+#define SWITCH_MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SWITCH_OK = 0,
+  SWITCH_ERR_INVALID_ARG = 1,          /* null pointer, bad size, misaligned */
+  SWITCH_ERR_UNSUPPORTED = 2,          /* shape/dtype this build does not run */
+  SWITCH_ERR_WORKSPACE_TOO_SMALL = 3,
+  SWITCH_ERR_CUDA = 4,                 /* a CUDA runtime call or launch failed */
+  SWITCH_ERR_TIMEOUT = 5,              /* device: a bounded wait ran out */
+  SWITCH_ERR_DEVICE_BOUNDS = 6         /* device: an index out of range */
+} switch_status_t;
+
+typedef enum { SWITCH_F32 = 0, SWITCH_BF16 = 1 } switch_dtype_t;
+
+/* Option bits of switch_config_t.flags (0 = the default fast path). */
+enum {
+  SWITCH_FLAG_ROUTER_SIMT = 1,       /* CUDA-core fp32 FMA router */
+  SWITCH_FLAG_ROUTER_2TERM = 2,      /* tensor-core router, W_r split in 2 bf16 terms (default 3) */
+  SWITCH_FLAG_UNFUSED_COMBINE = 4,   /* forward: write Y, then a separate combine kernel */
+  SWITCH_FLAG_GATHER_COPY = 8,       /* forward: copy routed rows to x_disp before GEMM1 */
+  SWITCH_FLAG_NO_RESIDUAL = 16       /* forward: block output is y alone (dropped -> 0) */
+};
+
+typedef struct {
+  int64_t T;                /* tokens in the batch: one routing group, batch order */
+  int32_t d_model;
+  int32_t d_ff;
+  int32_t n_experts;        /* 1 <= N <= 1024 */
+  int32_t dtype;            /* switch_dtype_t */
+  double capacity_factor;   /* > 0; taken at the exact value of the double */
+  float alpha;              /* load-balancing loss coefficient */
+  int32_t flags;            /* SWITCH_FLAG_* */
+  int64_t spin_limit;       /* bounded-wait limit in SM cycles; 0 = default (~2 s) */
+} switch_config_t;
+
+/* Expert capacity C = ceil(T x capacity_factor / N), computed exactly
+ * [P1 "Expert Capacity and the Capacity Factor", capacity equation; the
+ * page prints no rounding, rounding up is the reading taken].
+ * Returns -1 for T < 0, N < 1 or capacity_factor <= 0 (or not finite). */
+int64_t switch_capacity(int64_t T, int32_t n_experts, double capacity_factor);
+
+/* Bytes of device workspace every entry point below accepts for `cfg`
+ * (the maximum over them).  Writes *bytes; validates cfg. */
+switch_status_t switch_workspace_size(const switch_config_t* cfg, size_t* bytes);
+
+/* Router [P1 "Switch Routing", gate equation; top-1; fp32 routing math].
+ *   x      [T, d_model]  bf16 or fp32 (cfg->dtype)
+ *   w_r    [N, d_model]  fp32;  b_r [N] fp32 or NULL (added to the logits)
+ *   idx    [T] int32 out: expert of the largest logit, lowest index on ties
+ *   gate   [T] fp32  out: p_idx(x)
+ *   probs  [T, N] fp32 out, or NULL: softmax probabilities
+ * bf16 x runs on the tensor cores with W_r split into three bf16 terms that
+ * sum to it exactly (two with SWITCH_FLAG_ROUTER_2TERM) and fp32
+ * accumulation; fp32 x (or SWITCH_FLAG_ROUTER_SIMT) uses fp32 FMA. */
+switch_status_t switch_router(const switch_config_t* cfg, const void* x,
+                              const float* w_r, const float* b_r, int32_t* idx,
+                              float* gate, float* probs, void* ws, size_t ws_bytes,
+                              void* stream);
+
+/* Capacity-bounded dispatch [P1 "Expert Capacity and the Capacity
+ * Factor": overflow dropped, padding slots].  Input: idx [T] int32, or, when
+ * idx is NULL, probs [T, N] fp32 whose argmax (lowest index on ties) is the
+ * expert.  Outputs (all required):
+ *   rank       [T] int32: number of earlier tokens routed to the same expert
+ *   drop       [T] uint8: rank >= C
+ *   counts     [N] int32: tokens routed to each expert (before the cut)
+ *   slot_token [N * C] int32: token in slot r of expert e at e*C + r, -1 for
+ *              padding
+ * Optional gather: if x_disp is non-NULL, x [T, d_model] must be given and
+ * x_disp [N, C, d_model] receives x[slot_token] per slot, zeros in padding.
+ * Deterministic: slot order never depends on thread timing.
+ * Expert ids outside [0, N) set SWITCH_ERR_DEVICE_BOUNDS in the error word
+ * (the token is then treated as dropped). */
+switch_status_t switch_dispatch(const switch_config_t* cfg, const int32_t* idx,
+                                const float* probs, int32_t* rank, uint8_t* drop,
+                                int32_t* counts, int32_t* slot_token, const void* x,
+                                void* x_disp, void* ws, size_t ws_bytes, void* stream);
+
+/* Expert FFNs over the capacity buffers [P1 "The Core Idea"]:
+ *   y[e, r, :] = relu(x[slot_token[e*C + r]] . w1[e]^T) . w2[e]^T
+ * for r < n_e = min(counts[e], C).  Rows r >= n_e of y are left untouched.
+ *   x [T, d_model], w1 [N, d_ff, d_model], w2 [N, d_model, d_ff],
+ *   y [N, C, d_model]; slot_token [N*C], counts [N] as from switch_dispatch.
+ * bf16: tcgen05 grouped GEMM, fp32 accumulation, the hidden activation is
+ * rounded once to bf16, y rounded once to bf16.  fp32: CUDA-core FMA. */
+switch_status_t switch_expert_ffn(const switch_config_t* cfg, const void* x,
+                                  const int32_t* slot_token, const int32_t* counts,
+                                  const void* w1, const void* w2, void* y, void* ws,
+                                  size_t ws_bytes, void* stream);
+
+/* Combine [P1 "Switch Routing", combine equation with one expert; dropped
+ * tokens pass through on the residual]:
+ *   out[t] = x_residual[t] + (drop[t] ? 0 : gate[t] * y[idx[t], rank[t], :])
+ * computed in fp32 and rounded once to the output dtype.  x_residual may be
+ * NULL (no residual term).  y [N, C, d_model]. */
+switch_status_t switch_combine(const switch_config_t* cfg, const void* x_residual,
+                               const int32_t* idx, const int32_t* rank,
+                               const uint8_t* drop, const float* gate, const void* y,
+                               void* out, void* stream);
+
+/* Load-balancing loss [P1 "The Load-Balancing Loss"]:
+ *   f_i = counts_i / T, P_i = (1/T) sum_t probs[t, i],
+ *   loss = alpha . N . sum_i f_i P_i.
+ * counts [N] int32 (routed, dropped included), probs [T, N] fp32.
+ * loss: device fp32 scalar; f, P: [N] fp32 or NULL.  Fixed-order
+ * reductions: the result is bit-reproducible run to run. */
+switch_status_t switch_aux_loss(const switch_config_t* cfg, const int32_t* counts,
+                                const float* probs, float* loss, float* f, float* P,
+                                void* ws, size_t ws_bytes, void* stream);
+
+/* The whole layer on one stream with no host synchronisation:
+ * router -> dispatch -> expert FFN (gather fused into GEMM1's operand
+ * load, ReLU in its epilogue) -> gate x expert output + residual (fused
+ * into GEMM2's epilogue) -> load-balancing loss.
+ *   out [T, d_model] (same dtype as x)
+ *   idx [T] int32, gate [T] fp32, counts [N] int32: optional outputs (NULL
+ *   to skip); loss: device fp32 scalar or NULL.
+ * Same results as the staged calls above in sequence. */
+switch_status_t switch_layer_forward(const switch_config_t* cfg, const void* x,
+                                     const float* w_r, const float* b_r,
+                                     const void* w1, const void* w2, void* out,
+                                     int32_t* idx, float* gate, int32_t* counts,
+                                     float* loss, void* ws, size_t ws_bytes,
+                                     void* stream);
+
+/* Synchronises `stream`, reads the workspace's device error word, clears
+ * it, and returns the recorded status (SWITCH_OK if none).  *where_out and
+ * *info_out (either may be NULL) receive the reporting kernel role and a
+ * detail value. */
+switch_status_t switch_get_device_error(void* ws, void* stream, int32_t* where_out,
+                                        int64_t* info_out);
+
+/* Static, human-readable name of a status code. */
+const char* switch_status_string(switch_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SWITCH_MOE_H_ */

@@ -1,0 +1,136 @@
+// Combine and load-balancing loss.
+//
+// Combine: "Switch Transformers: scaling to trillion-parameter models",
+// section "Switch Routing: From Top-k to k = 1", combine equation with one
+// selected expert, y = p_i(x) E_i(x); a dropped token's output is the
+// residual (section "Expert Capacity and the Capacity Factor").
+// Loss: section "The Load-Balancing Loss", alpha . N . sum_i f_i P_i.
+#include "kernels.cuh"
+
+namespace smoe {
+
+// ------------------------------------------------------------------ combine
+
+template <bool kBF16>
+__global__ void __launch_bounds__(256) combine_kernel(
+    int64_t T, int vec_per_row, int64_t C, const uint4* __restrict__ x,
+    const int* __restrict__ idx, const int* __restrict__ rank,
+    const uint8_t* __restrict__ drop, const float* __restrict__ gate,
+    const uint4* __restrict__ y, uint4* __restrict__ out, bool only_dropped) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       t < T; t += warps) {
+    const bool dropped = drop[t] != 0;
+    if (only_dropped && !dropped) continue;
+    const float g = dropped ? 0.f : gate[t];
+    const uint4* yrow =
+        dropped ? nullptr : y + (static_cast<int64_t>(idx[t]) * C + rank[t]) * vec_per_row;
+    const uint4* xrow = x ? x + t * vec_per_row : nullptr;
+    uint4* orow = out + t * vec_per_row;
+    for (int v = lane; v < vec_per_row; v += 32) {
+      const uint4 xv = xrow ? __ldg(xrow + v) : make_uint4(0, 0, 0, 0);
+      const uint4 yv = yrow ? __ldg(yrow + v) : make_uint4(0, 0, 0, 0);
+      uint4 o;
+      if (kBF16) {
+        const uint32_t* xa = &xv.x;
+        const uint32_t* ya = &yv.x;
+        uint32_t* oa = &o.x;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float lo = fmaf(g, bf16_lo(ya[i]), bf16_lo(xa[i]));
+          const float hi = fmaf(g, bf16_hi(ya[i]), bf16_hi(xa[i]));
+          oa[i] = pack_bf16x2(lo, hi);
+        }
+      } else {
+        o.x = __float_as_uint(fmaf(g, __uint_as_float(yv.x), __uint_as_float(xv.x)));
+        o.y = __float_as_uint(fmaf(g, __uint_as_float(yv.y), __uint_as_float(xv.y)));
+        o.z = __float_as_uint(fmaf(g, __uint_as_float(yv.z), __uint_as_float(xv.z)));
+        o.w = __float_as_uint(fmaf(g, __uint_as_float(yv.w), __uint_as_float(xv.w)));
+      }
+      orow[v] = o;
+    }
+  }
+}
+
+cudaError_t launch_combine(int64_t T, int d, int64_t C, bool bf16, const void* x,
+                           const int* idx, const int* rank, const uint8_t* drop,
+                           const float* gate, const void* y, void* out, bool only_dropped,
+                           cudaStream_t st) {
+  const int vec = d * (bf16 ? 2 : 4) / 16;
+  int64_t blocks = (T + 7) / 8;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  if (blocks < 1) blocks = 1;
+  if (bf16)
+    combine_kernel<true><<<static_cast<int>(blocks), 256, 0, st>>>(
+        T, vec, C, static_cast<const uint4*>(x), idx, rank, drop, gate,
+        static_cast<const uint4*>(y), static_cast<uint4*>(out), only_dropped);
+  else
+    combine_kernel<false><<<static_cast<int>(blocks), 256, 0, st>>>(
+        T, vec, C, static_cast<const uint4*>(x), idx, rank, drop, gate,
+        static_cast<const uint4*>(y), static_cast<uint4*>(out), only_dropped);
+  return cudaGetLastError();
+}
+
+// --------------------------------------------------------------- aux loss
+
+// psum[blk][e] = sum over rows blk*128 .. blk*128+127 of probs[row][e],
+// added in row order.
+__global__ void __launch_bounds__(128) prob_colsum_kernel(int64_t T, int N,
+                                                          const float* __restrict__ probs,
+                                                          float* __restrict__ psum) {
+  const int e = blockIdx.y * 128 + threadIdx.x;
+  if (e >= N) return;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kTileTok;
+  const int64_t r1 = r0 + kTileTok < T ? r0 + kTileTok : T;
+  float s = 0.f;
+  for (int64_t r = r0; r < r1; ++r) s += probs[r * N + e];
+  psum[static_cast<int64_t>(blockIdx.x) * N + e] = s;
+}
+
+cudaError_t launch_prob_colsum(int64_t T, int N, const float* probs, float* psum,
+                               cudaStream_t st) {
+  const dim3 grid(static_cast<unsigned>((T + kTileTok - 1) / kTileTok),
+                  static_cast<unsigned>((N + 127) / 128));
+  prob_colsum_kernel<<<grid, 128, 0, st>>>(T, N, probs, psum);
+  return cudaGetLastError();
+}
+
+// One block: P_e = (sum_p psum[p][e]) / T in double, fixed order; then a
+// fixed-shape tree over experts for sum_e f_e P_e.
+__global__ void __launch_bounds__(256) aux_loss_kernel(int64_t T, int N, int nparts,
+                                                       float alpha,
+                                                       const int* __restrict__ counts,
+                                                       const float* __restrict__ psum,
+                                                       float* __restrict__ loss,
+                                                       float* __restrict__ f_out,
+                                                       float* __restrict__ P_out) {
+  __shared__ double red[256];
+  const int tid = threadIdx.x;
+  double acc = 0.0;
+  for (int e = tid; e < N; e += 256) {
+    double s = 0.0;
+    for (int p = 0; p < nparts; ++p) s += static_cast<double>(psum[static_cast<int64_t>(p) * N + e]);
+    const double P = s / static_cast<double>(T);
+    const double f = static_cast<double>(counts[e]) / static_cast<double>(T);
+    if (f_out) f_out[e] = static_cast<float>(f);
+    if (P_out) P_out[e] = static_cast<float>(P);
+    acc += f * P;
+  }
+  red[tid] = acc;
+  __syncthreads();
+  for (int s = 128; s > 0; s >>= 1) {
+    if (tid < s) red[tid] += red[tid + s];
+    __syncthreads();
+  }
+  if (tid == 0 && loss) *loss = static_cast<float>(static_cast<double>(alpha) * N * red[0]);
+}
+
+cudaError_t launch_aux_loss(int64_t T, int N, int nparts, float alpha, const int* counts,
+                            const float* psum, float* loss, float* f, float* P,
+                            cudaStream_t st) {
+  aux_loss_kernel<<<1, 256, 0, st>>>(T, N, nparts, alpha, counts, psum, loss, f, P);
+  return cudaGetLastError();
+}
+
+}  // namespace smoe

@@ -1,0 +1,505 @@
+// Expert FFNs over the capacity buffers: N independent ReLU FFNs
+// ("Switch Transformers: scaling to trillion-parameter models", section
+// "The Core Idea"), each applied to the tokens that hold its slots
+// (section "Expert Capacity and the Capacity Factor"), and optionally the
+// gate-scaled combine with the residual fused into the second GEMM's
+// epilogue (section "Switch Routing: From Top-k to k = 1", combine
+// equation; one writer per output row since k = 1).
+//
+// bf16 path: a persistent tcgen05 grouped GEMM.
+//   * tile = 128 slots (rows) x 256 output columns, K in blocks of 64;
+//   * warp 0 feeds a 4-stage shared-memory ring with TMA (128-byte swizzle);
+//     in GEMM1 the A rows are gathered straight from x through slot_token
+//     with tile::gather4 (four token rows per copy), so the dispatched
+//     tokens are never materialised;
+//   * warp 1 issues tcgen05.mma (M=128, N=256, K=16) into one of two TMEM
+//     accumulators (2 x 256 fp32 columns) so the epilogue of one tile
+//     overlaps the main loop of the next;
+//   * warps 2-5 drain TMEM (one token row per thread): ReLU + bf16 for the
+//     hidden activation, bf16 for Y, or x + gate * acc for the combine;
+//   * the tile list comes from device-side counts (no host sync); experts'
+//     empty capacity tiles are never scheduled; consecutive CTAs take the
+//     M tiles of the same (expert, N tile) so each weight tile is read from
+//     HBM about once and from L2 by the rest.
+// fp32 path: CUDA-core FMA tiles (no TF32), same tile list semantics.
+#include "kernels.cuh"
+
+namespace smoe {
+
+// ----------------------------------------------------------- tensor maps
+
+typedef CUresult (*PFN_encodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                    const cuuint32_t*, CUtensorMapInterleave,
+                                    CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                    CUtensorMapFloatOOBfill);
+
+PFN_encodeTiled get_encode_fn() {
+  static PFN_encodeTiled fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_encodeTiled>(p);
+  }
+  return fn;
+}
+
+// 2-D bf16 tensor [outer, inner] (inner contiguous), 128-byte swizzle,
+// out-of-range elements read as zero.
+bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                       uint32_t box_inner, uint32_t box_outer) {
+  PFN_encodeTiled enc = get_encode_fn();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {inner * 2};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------- tile list
+
+// Tile t belongs to the expert e with mts[e] * ntn <= t < mts[e + 1] * ntn
+// (the last such e, which is never empty).  Inside an expert, M tiles vary
+// fastest so that CTAs running side by side share the weight tile.
+__device__ __forceinline__ void decode_tile(int tile, const int* mts, int N, int ntn, int& e,
+                                            int& m, int& n) {
+  int lo = 0, hi = N;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (mts[mid] * ntn <= tile) lo = mid; else hi = mid;
+  }
+  e = lo;
+  const int mt = mts[e + 1] - mts[e];
+  const int local = tile - mts[e] * ntn;
+  n = local / mt;
+  m = local - n * mt;
+}
+
+// ================================================== tcgen05 grouped GEMM
+
+constexpr int kBM = 128, kBN = 256, kBK = 64;
+constexpr int kStages = 4;
+constexpr uint32_t kABytes = kBM * kBK * 2;             // 16 KB
+constexpr uint32_t kBBytes = kBN * kBK * 2;             // 32 KB
+constexpr uint32_t kStageBytes = kABytes + kBBytes;     // 48 KB
+constexpr int kGemmThreads = 192;
+constexpr uint32_t kTmemCols = 512;                     // 2 accumulators x 256
+
+struct GemmParams {
+  int N, n_out, K, ntiles_n;
+  int64_t C;
+  const int* counts;
+  const int* mtile_start;
+  const int* slot_token;
+  int mode;
+  __nv_bfloat16* out;       // kModeHidden / kModeY: row e*C + r, leading dim ldo
+  int64_t ldo;
+  const __nv_bfloat16* x_res;   // kModeCombine
+  const float* gate;
+  __nv_bfloat16* comb_out;      // [T, n_out]
+  DevErr* err;
+  long long spin;
+};
+
+template <bool kGather>
+__global__ void __launch_bounds__(kGemmThreads, 1) expert_gemm_kernel(
+    const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+    GemmParams p) {
+  const int total = p.mtile_start[p.N] * p.ntiles_n;
+  if (static_cast<int>(blockIdx.x) >= total) return;    // uniform for the block
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint8_t* tail = smem + kStages * kStageBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(tail);
+  uint64_t* empty = full + kStages;
+  uint64_t* tfull = empty + kStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  int* mts = reinterpret_cast<int*>(tail + 128);         // [N + 1]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long lim = p.spin;
+  const int kblocks = p.K / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 128);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  for (int i = threadIdx.x; i <= p.N; i += blockDim.x) mts[i] = p.mtile_start[i];
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // --------------------------------------------------- TMA producer warp
+    if (lane == 0) {
+      tma_prefetch_desc(&tmap_a);
+      tma_prefetch_desc(&tmap_b);
+    }
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t issued_mask = 0, issued_phase = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      if (*abort_flag) break;
+      int e, m, n;
+      decode_tile(tile, mts, p.N, p.ntiles_n, e, m, n);
+      const int64_t slot0 = static_cast<int64_t>(e) * p.C + static_cast<int64_t>(m) * kBM;
+      int tok[4] = {0, 0, 0, 0};
+      if (kGather) {
+        const int64_t cnt = p.counts[e];
+        const int64_t n_e = cnt < p.C ? cnt : p.C;
+        const int first = p.slot_token[slot0];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int64_t r = static_cast<int64_t>(m) * kBM + lane * 4 + i;
+          tok[i] = r < n_e ? p.slot_token[slot0 + lane * 4 + i] : first;
+        }
+      }
+      bool ok = true;
+      for (int kb = 0; kb < kblocks; ++kb) {
+        int w_ok = 1;
+        if (lane == 0) w_ok = mbar_wait(&empty[stage], phase ^ 1u, lim) ? 1 : 0;
+        w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
+        if (!w_ok) {
+          if (lane == 0) {
+            report_error(p.err, SWITCH_ERR_TIMEOUT, kWhereGemmProducer, tile);
+            *abort_flag = 1;
+          }
+          ok = false;
+          break;
+        }
+        uint8_t* sa = smem + stage * kStageBytes;
+        uint8_t* sb = sa + kABytes;
+        if (lane == 0) mbar_arrive_expect_tx(&full[stage], kStageBytes);
+        __syncwarp();
+        if (kGather) {
+          tma_gather4(sa + lane * 512, &tmap_a, &full[stage], kb * kBK, tok[0], tok[1], tok[2],
+                      tok[3]);
+        } else if (lane == 0) {
+          tma_load_2d(sa, &tmap_a, &full[stage], kb * kBK, static_cast<int>(slot0));
+        }
+        if (lane == 0)
+          tma_load_2d(sb, &tmap_b, &full[stage], kb * kBK, e * p.n_out + n * kBN);
+        issued_mask |= 1u << stage;
+        issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+        if (++stage == kStages) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) break;
+    }
+    if (lane == 0) {
+      for (int s = 0; s < kStages; ++s)
+        if (((issued_mask >> s) & 1u) &&
+            !mbar_wait(&full[s], (issued_phase >> s) & 1u, kDefaultSpinCycles))
+          report_error(p.err, SWITCH_ERR_TIMEOUT, kWhereDrain, s);
+    }
+  } else if (warp == 1) {
+    // --------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(kBM, kBN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool any = false;
+      for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, lim)) {
+          report_error(p.err, SWITCH_ERR_TIMEOUT, kWhereGemmMma, tile);
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBN);
+        bool ok = true;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&full[stage], phase, lim)) {
+            report_error(p.err, SWITCH_ERR_TIMEOUT, kWhereGemmMma, tile);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * kStageBytes);
+          const uint32_t sb = sa + kABytes;
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k)
+            umma_bf16(d_tmem, sw128_kmajor_desc(sa + k * 32), sw128_kmajor_desc(sb + k * 32),
+                      idesc, (kb | k) != 0 ? 1u : 0u);
+          any = true;
+          umma_commit(&empty[stage]);
+          if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      if (any && *abort_flag) {
+        umma_commit(drain);
+        if (!mbar_wait(drain, 0, kDefaultSpinCycles))
+          report_error(p.err, SWITCH_ERR_TIMEOUT, kWhereDrain, -1);
+      }
+    }
+  } else {
+    // --------------------------------------------------- epilogue warps
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      if (!mbar_wait(&tfull[acc], acc_phase, lim)) {
+        report_error(p.err, SWITCH_ERR_TIMEOUT, kWhereGemmEpilogue, tile);
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      int e, m, n;
+      decode_tile(tile, mts, p.N, p.ntiles_n, e, m, n);
+      const int64_t cnt = p.counts[e];
+      const int64_t n_e = cnt < p.C ? cnt : p.C;
+      const int64_t r = static_cast<int64_t>(m) * kBM + row;
+      const bool valid = r < n_e;
+      const uint32_t taddr =
+          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * kBN);
+      int tok = 0;
+      float g = 0.f;
+      if (p.mode == kModeCombine && valid) {
+        tok = p.slot_token[static_cast<int64_t>(e) * p.C + r];
+        g = p.gate[tok];
+      }
+#pragma unroll 1
+      for (int c = 0; c < kBN / 32; ++c) {
+        float v[32];
+        tmem_ld32(taddr + c * 32, v);
+        const int col = n * kBN + c * 32;
+        if (!valid || col >= p.n_out) continue;
+        uint32_t pk[16];
+        if (p.mode == kModeHidden) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            pk[j] = pack_bf16x2(fmaxf(v[2 * j], 0.f), fmaxf(v[2 * j + 1], 0.f));
+          uint4* dst = reinterpret_cast<uint4*>(
+              p.out + (static_cast<int64_t>(e) * p.C + r) * p.ldo + col);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+        } else if (p.mode == kModeY) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) pk[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
+          uint4* dst = reinterpret_cast<uint4*>(
+              p.out + (static_cast<int64_t>(e) * p.C + r) * p.ldo + col);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+        } else {
+          const int64_t off = static_cast<int64_t>(tok) * p.n_out + col;
+          uint4 xr[4];
+          if (p.x_res != nullptr) {
+            const uint4* src = reinterpret_cast<const uint4*>(p.x_res + off);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) xr[j] = __ldg(src + j);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) xr[j] = make_uint4(0, 0, 0, 0);
+          }
+          const uint32_t* xw = &xr[0].x;
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            pk[j] = pack_bf16x2(fmaf(g, v[2 * j], bf16_lo(xw[j])),
+                                fmaf(g, v[2 * j + 1], bf16_hi(xw[j])));
+          uint4* dst = reinterpret_cast<uint4*>(p.comb_out + off);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
+}
+
+static size_t gemm_smem_bytes(int N) {
+  return 1024 + kStages * kStageBytes + 128 + sizeof(int) * (N + 1);
+}
+
+template <bool kGather>
+static cudaError_t run_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& gp,
+                            int num_sms, cudaStream_t st) {
+  const size_t smem = gemm_smem_bytes(gp.N);
+  cudaError_t e = cudaFuncSetAttribute(expert_gemm_kernel<kGather>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  expert_gemm_kernel<kGather><<<num_sms, kGemmThreads, smem, st>>>(ta, tb, gp);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_expert_ffn_bf16(const FfnArgs& a, cudaStream_t st) {
+  const uint64_t slots = static_cast<uint64_t>(a.N) * static_cast<uint64_t>(a.C);
+  CUtensorMap ta1, tb1, ta2, tb2;
+  const bool gather = a.x_disp == nullptr;
+  bool ok = gather
+                ? make_tmap_bf16_2d(&ta1, a.x, a.d, a.T, kBK, 1)
+                : make_tmap_bf16_2d(&ta1, a.x_disp, a.d, slots, kBK, kBM);
+  ok = ok && make_tmap_bf16_2d(&tb1, a.w1, a.d, static_cast<uint64_t>(a.N) * a.F, kBK, kBN);
+  ok = ok && make_tmap_bf16_2d(&ta2, a.hbuf, a.F, slots, kBK, kBM);
+  ok = ok && make_tmap_bf16_2d(&tb2, a.w2, a.F, static_cast<uint64_t>(a.N) * a.d, kBK, kBN);
+  if (!ok) return cudaErrorInvalidValue;
+
+  GemmParams g1{};
+  g1.N = a.N;
+  g1.n_out = a.F;
+  g1.K = a.d;
+  g1.ntiles_n = (a.F + kBN - 1) / kBN;
+  g1.C = a.C;
+  g1.counts = a.counts;
+  g1.mtile_start = a.mtile_start;
+  g1.slot_token = a.slot_token;
+  g1.mode = kModeHidden;
+  g1.out = static_cast<__nv_bfloat16*>(a.hbuf);
+  g1.ldo = a.F;
+  g1.err = a.err;
+  g1.spin = a.spin;
+  cudaError_t e = gather ? run_gemm<true>(ta1, tb1, g1, a.num_sms, st)
+                         : run_gemm<false>(ta1, tb1, g1, a.num_sms, st);
+  if (e != cudaSuccess) return e;
+
+  GemmParams g2 = g1;
+  g2.n_out = a.d;
+  g2.K = a.F;
+  g2.ntiles_n = (a.d + kBN - 1) / kBN;
+  g2.mode = a.mode2;
+  g2.out = static_cast<__nv_bfloat16*>(a.y);
+  g2.ldo = a.d;
+  g2.x_res = static_cast<const __nv_bfloat16*>(a.x_res);
+  g2.gate = a.gate;
+  g2.comb_out = static_cast<__nv_bfloat16*>(a.out);
+  return run_gemm<false>(ta2, tb2, g2, a.num_sms, st);
+}
+
+// ===================================================== fp32 CUDA cores
+
+constexpr int kSB = 64, kSK = 16;
+
+// grid (ceil(C / 64), ceil(n_out / 64), N); 256 threads, 4x4 outputs each.
+__global__ void __launch_bounds__(256) ffn_simt_kernel(
+    int mode, int64_t C, int n_out, int K, const int* __restrict__ counts,
+    const int* __restrict__ slot_token, const float* __restrict__ a_src, bool a_gather,
+    const float* __restrict__ w, float* __restrict__ out, const float* __restrict__ x_res,
+    const float* __restrict__ gate) {
+  __shared__ float As[kSK][kSB + 4];
+  __shared__ float Bs[kSK][kSB + 4];
+  const int e = blockIdx.z;
+  const int64_t cnt = counts[e];
+  const int64_t n_e = cnt < C ? cnt : C;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kSB;
+  if (r0 >= n_e) return;
+  const int c0 = blockIdx.y * kSB;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  const float* wE = w + static_cast<int64_t>(e) * n_out * K;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < K; k0 += kSK) {
+    for (int i = threadIdx.x; i < kSB * kSK; i += 256) {
+      const int rr = i / kSK, kk = i % kSK;
+      const int64_t r = r0 + rr;
+      float v = 0.f;
+      if (r < n_e && k0 + kk < K) {
+        const int64_t src_row =
+            a_gather ? static_cast<int64_t>(slot_token[static_cast<int64_t>(e) * C + r])
+                     : static_cast<int64_t>(e) * C + r;
+        v = a_src[src_row * K + k0 + kk];
+      }
+      As[kk][rr] = v;
+      const int cc = c0 + rr;
+      Bs[kk][rr] = (cc < n_out && k0 + kk < K) ? wE[static_cast<int64_t>(cc) * K + k0 + kk] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < kSK; ++kk) {
+      float av[4], bv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) av[i] = As[kk][ty * 4 + i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) bv[j] = Bs[kk][tx * 4 + j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t r = r0 + ty * 4 + i;
+    if (r >= n_e) continue;
+    const int64_t slot = static_cast<int64_t>(e) * C + r;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int col = c0 + tx * 4 + j;
+      if (col >= n_out) continue;
+      if (mode == kModeHidden) {
+        out[slot * n_out + col] = fmaxf(acc[i][j], 0.f);
+      } else if (mode == kModeY) {
+        out[slot * n_out + col] = acc[i][j];
+      } else {
+        const int tok = slot_token[slot];
+        const float xr = x_res ? x_res[static_cast<int64_t>(tok) * n_out + col] : 0.f;
+        out[static_cast<int64_t>(tok) * n_out + col] = fmaf(gate[tok], acc[i][j], xr);
+      }
+    }
+  }
+}
+
+cudaError_t launch_expert_ffn_f32(const FfnArgs& a, cudaStream_t st) {
+  const dim3 g1(static_cast<unsigned>((a.C + kSB - 1) / kSB),
+                static_cast<unsigned>((a.F + kSB - 1) / kSB), static_cast<unsigned>(a.N));
+  ffn_simt_kernel<<<g1, 256, 0, st>>>(kModeHidden, a.C, a.F, a.d, a.counts, a.slot_token,
+                                      static_cast<const float*>(a.x), true,
+                                      static_cast<const float*>(a.w1),
+                                      static_cast<float*>(a.hbuf), nullptr, nullptr);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const dim3 g2(static_cast<unsigned>((a.C + kSB - 1) / kSB),
+                static_cast<unsigned>((a.d + kSB - 1) / kSB), static_cast<unsigned>(a.N));
+  float* out2 = a.mode2 == kModeCombine ? static_cast<float*>(a.out) : static_cast<float*>(a.y);
+  ffn_simt_kernel<<<g2, 256, 0, st>>>(a.mode2, a.C, a.d, a.F, a.counts, a.slot_token,
+                                      static_cast<const float*>(a.hbuf), false,
+                                      static_cast<const float*>(a.w2), out2,
+                                      static_cast<const float*>(a.x_res), a.gate);
+  return cudaGetLastError();
+}
+
+}  // namespace smoe

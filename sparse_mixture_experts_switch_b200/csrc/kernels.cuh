@@ -1,0 +1,99 @@
+// Launch wrappers shared between the kernel files and the C-ABI layer.
+#pragma once
+
+#include "common.cuh"
+
+namespace smoe {
+
+constexpr int kTileTok = 128;   // tokens per dispatch/router tile
+
+// ------------------------------------------------------------- dispatch
+// Per 128-token tile: expert of each token (from idx, or argmax of probs),
+// rank within the tile in token order, and the tile's histogram
+// hist[e * ntiles + tile].
+cudaError_t launch_tile_rank(int64_t T, int N, const int* idx_in, const float* probs,
+                             int* idx_out, int* local_rank, int* hist, int ntiles,
+                             DevErr* err, cudaStream_t st);
+// Exclusive scan of every expert's tile histogram in tile order:
+// base[e * ntiles + tile]; counts[e] = total.
+cudaError_t launch_scan(int N, int ntiles, const int* hist, int* base, int* counts,
+                        cudaStream_t st);
+// rank/drop per token, slot_token (kept tokens and -1 padding), and the
+// per-expert prefix of 128-row M tiles mtile_start[N + 1].
+cudaError_t launch_finalize(int64_t T, int N, int64_t C, int ntiles, const int* idx,
+                            const int* local_rank, const int* base, const int* counts,
+                            int* rank, uint8_t* drop, int* slot_token, int* mtile_start,
+                            cudaStream_t st);
+// Only mtile_start from counts (for a standalone expert-FFN call).
+cudaError_t launch_mtile_table(int N, int64_t C, const int* counts, int* mtile_start,
+                               cudaStream_t st);
+// x_disp[s] = x[slot_token[s]] (zeros for padding), row_bytes % 16 == 0.
+cudaError_t launch_gather_rows(int64_t nslots, int64_t row_bytes, const int* slot_token,
+                               const void* x, void* x_disp, cudaStream_t st);
+
+// ------------------------------------------------------- combine / loss
+// out[t] = x[t] + (drop ? 0 : gate * y[idx*C + rank]); fp32 math, one rounding.
+// only_dropped: touch only dropped tokens (kept ones are written elsewhere).
+cudaError_t launch_combine(int64_t T, int d, int64_t C, bool bf16, const void* x,
+                           const int* idx, const int* rank, const uint8_t* drop,
+                           const float* gate, const void* y, void* out, bool only_dropped,
+                           cudaStream_t st);
+// psum[blk][e] = sum of probs rows [blk*128, blk*128 + 128) (fixed order).
+cudaError_t launch_prob_colsum(int64_t T, int N, const float* probs, float* psum,
+                               cudaStream_t st);
+// loss = alpha * N * sum_e (counts_e / T) * (sum_p psum[p][e] / T).
+cudaError_t launch_aux_loss(int64_t T, int N, int nparts, float alpha, const int* counts,
+                            const float* psum, float* loss, float* f, float* P,
+                            cudaStream_t st);
+
+// ---------------------------------------------------------------- router
+struct RouterOut {
+  int* idx;          // [T]
+  float* gate;       // [T]
+  float* probs;      // [T, N] or null
+  float* psum;       // [nparts, N] or null (per-tile sums of probs)
+  int* hist;         // [N, ntiles] or null (tensor-core router only)
+  int* local_rank;   // [T] or null (tensor-core router only)
+};
+// CUDA-core fp32 router; psum parts are 64-token blocks.  `logits` is a
+// [T, N] fp32 scratch.
+cudaError_t launch_router_simt(int64_t T, int d, int N, bool bf16, const void* x,
+                               const float* w_r, const float* b_r, float* logits,
+                               RouterOut o, int* nparts_out, cudaStream_t st);
+// Tensor-core router (bf16 x).  Writes idx, gate, probs?, psum (128-token
+// parts), hist and local_rank.  wsplit: [terms][N_pad][d] bf16 scratch.
+cudaError_t launch_router_tc(int64_t T, int d, int N, int terms, const void* x,
+                             const float* w_r, const float* b_r, void* wsplit,
+                             RouterOut o, int ntiles, DevErr* err, long long spin,
+                             int num_sms, cudaStream_t st);
+bool router_tc_supported(int N, int d, int terms);
+
+// ------------------------------------------------------------ expert FFN
+enum GemmMode : int { kModeHidden = 0, kModeY = 1, kModeCombine = 2 };
+
+struct FfnArgs {
+  int64_t T;
+  int d, F, N;
+  int64_t C;
+  const void* x;            // [T, d]
+  const void* x_disp;       // [N*C, d] or null (gather inside GEMM1)
+  const int* slot_token;    // [N*C]
+  const int* counts;        // [N]
+  const int* mtile_start;   // [N + 1]
+  const void* w1;           // [N, F, d]
+  const void* w2;           // [N, d, F]
+  void* hbuf;               // [N*C, F]
+  void* y;                  // [N*C, d] (kModeY)
+  // kModeCombine: out[token] = x_res[token] + gate[token] * acc
+  const void* x_res;        // [T, d] or null
+  const float* gate;        // [T]
+  void* out;                // [T, d]
+  int mode2;                // kModeY or kModeCombine for the second GEMM
+  DevErr* err;
+  long long spin;
+  int num_sms;
+};
+cudaError_t launch_expert_ffn_bf16(const FfnArgs& a, cudaStream_t st);
+cudaError_t launch_expert_ffn_f32(const FfnArgs& a, cudaStream_t st);
+
+}  // namespace smoe

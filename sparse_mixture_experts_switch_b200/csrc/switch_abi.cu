@@ -1,0 +1,408 @@
+// C ABI of the Switch-FFN layer (declared in include/switch_moe.h):
+// argument validation, exact capacity, workspace carving and the launch
+// sequence of each entry point.  No device memory is allocated here.
+#include <climits>
+#include <cmath>
+#include <cstring>
+
+#include "kernels.cuh"
+
+using namespace smoe;
+
+namespace {
+
+constexpr size_t kAlign = 1024;
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ceil(T * cf / N) with cf taken at the exact value of the double.
+int64_t capacity_exact(int64_t T, int32_t N, double cf) {
+  if (T < 0 || N < 1 || !(cf > 0.0) || !std::isfinite(cf)) return -1;
+  if (T == 0) return 0;
+  int ex = 0;
+  const double f = std::frexp(cf, &ex);                          // cf = f * 2^ex
+  const uint64_t mant = static_cast<uint64_t>(std::ldexp(f, 53));  // exact, < 2^53
+  int sh = ex - 53;                                               // cf = mant * 2^sh
+  unsigned __int128 num = static_cast<unsigned __int128>(T) * mant;
+  unsigned __int128 den = static_cast<unsigned __int128>(N);
+  if (sh >= 0) {
+    if (sh > 10) return -1;                                       // cf >= 2^63: nonsense
+    num <<= sh;
+  } else {
+    if (-sh > 116) return 1;                                      // 0 < T cf / N < 1
+    den <<= -sh;
+  }
+  const unsigned __int128 q = (num + den - 1) / den;
+  if (q > static_cast<unsigned __int128>(INT64_MAX)) return -1;
+  return static_cast<int64_t>(q);
+}
+
+struct Layout {
+  size_t err, hist, base, psum, local_rank, idx, gate, rank, drop, counts, slot_token,
+      mtile_start, wsplit, logits, xdisp, hbuf, ybuf, total;
+};
+
+int ntiles_of(int64_t T) { return static_cast<int>((T + kTileTok - 1) / kTileTok); }
+
+Layout layout_for(const switch_config_t& c, int64_t C) {
+  const int64_t T = c.T;
+  const int64_t N = c.n_experts;
+  const size_t es = c.dtype == SWITCH_BF16 ? 2 : 4;
+  const int64_t nt = ntiles_of(T);
+  const int64_t nparts = (T + 63) / 64;
+  const int64_t npad = (N + 15) / 16 * 16;
+  const int64_t slots = N * C;
+  Layout L{};
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = align_up(o + (bytes ? bytes : 1), kAlign);
+    return at;
+  };
+  L.err = take(256);
+  L.hist = take(sizeof(int) * N * nt);
+  L.base = take(sizeof(int) * N * nt);
+  L.psum = take(sizeof(float) * N * nparts);
+  L.local_rank = take(sizeof(int) * T);
+  L.idx = take(sizeof(int) * T);
+  L.gate = take(sizeof(float) * T);
+  L.rank = take(sizeof(int) * T);
+  L.drop = take(T);
+  L.counts = take(sizeof(int) * N);
+  L.slot_token = take(sizeof(int) * slots);
+  L.mtile_start = take(sizeof(int) * (N + 1));
+  L.wsplit = take(2 * 3 * npad * static_cast<size_t>(c.d_model));
+  L.logits = take(sizeof(float) * N * T);
+  L.xdisp = take(es * slots * static_cast<size_t>(c.d_model));
+  L.hbuf = take(es * slots * static_cast<size_t>(c.d_ff));
+  L.ybuf = take(es * slots * static_cast<size_t>(c.d_model));
+  L.total = o;
+  return L;
+}
+
+switch_status_t validate(const switch_config_t* c, int64_t* C_out) {
+  if (c == nullptr) return SWITCH_ERR_INVALID_ARG;
+  if (c->T < 0 || c->T > INT_MAX || c->d_model < 1 || c->d_ff < 1 || c->n_experts < 1 ||
+      c->n_experts > 1024 || (c->dtype != SWITCH_F32 && c->dtype != SWITCH_BF16) ||
+      c->spin_limit < 0)
+    return SWITCH_ERR_INVALID_ARG;
+  const int64_t C = capacity_exact(c->T, c->n_experts, c->capacity_factor);
+  if (C < 0) return SWITCH_ERR_INVALID_ARG;
+  if (c->dtype == SWITCH_BF16 && (c->d_model % 64 != 0 || c->d_ff % 64 != 0))
+    return SWITCH_ERR_UNSUPPORTED;
+  if (c->dtype == SWITCH_F32 && (c->d_model % 4 != 0 || c->d_ff % 4 != 0))
+    return SWITCH_ERR_UNSUPPORTED;
+  if (C > INT_MAX / c->n_experts) return SWITCH_ERR_UNSUPPORTED;   // slot ids are int32
+  if (C_out) *C_out = C;
+  return SWITCH_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Ctx {
+  int64_t C;
+  Layout L;
+  uint8_t* ws;
+  DevErr* err;
+  cudaStream_t st;
+  long long spin;
+  int num_sms;
+  template <class P>
+  P* at(size_t off) const { return reinterpret_cast<P*>(ws + off); }
+};
+
+int device_sms() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (cache[dev] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    int major = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cache[dev] = major == 10 ? v : -1;   // the kernels are built for sm_100a only
+  }
+  return cache[dev];
+}
+
+switch_status_t prepare(const switch_config_t* cfg, void* ws, size_t ws_bytes, void* stream,
+                        Ctx* ctx) {
+  int64_t C = 0;
+  switch_status_t s = validate(cfg, &C);
+  if (s != SWITCH_OK) return s;
+  ctx->C = C;
+  ctx->L = layout_for(*cfg, C);
+  if (cfg->T == 0) return SWITCH_OK;
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+    return SWITCH_ERR_INVALID_ARG;
+  if (ws_bytes < ctx->L.total) return SWITCH_ERR_WORKSPACE_TOO_SMALL;
+  ctx->ws = static_cast<uint8_t*>(ws);
+  ctx->err = reinterpret_cast<DevErr*>(ws);
+  ctx->st = static_cast<cudaStream_t>(stream);
+  ctx->spin = cfg->spin_limit > 0 ? cfg->spin_limit : kDefaultSpinCycles;
+  ctx->num_sms = device_sms();
+  if (ctx->num_sms == 0) return SWITCH_ERR_CUDA;
+  if (ctx->num_sms < 0) return SWITCH_ERR_UNSUPPORTED;
+  return SWITCH_OK;
+}
+
+switch_status_t cuda_status(cudaError_t e) {
+  return e == cudaSuccess ? SWITCH_OK : SWITCH_ERR_CUDA;
+}
+
+#define SMOE_TRY(expr)                         \
+  do {                                         \
+    cudaError_t _e = (expr);                   \
+    if (_e != cudaSuccess) return SWITCH_ERR_CUDA; \
+  } while (0)
+
+int router_terms(const switch_config_t* c) {
+  return (c->flags & SWITCH_FLAG_ROUTER_2TERM) ? 2 : 3;
+}
+
+bool use_tc_router(const switch_config_t* c) {
+  return c->dtype == SWITCH_BF16 && !(c->flags & SWITCH_FLAG_ROUTER_SIMT) &&
+         router_tc_supported(c->n_experts, c->d_model, router_terms(c));
+}
+
+}  // namespace
+
+extern "C" {
+
+int64_t switch_capacity(int64_t T, int32_t n_experts, double capacity_factor) {
+  return capacity_exact(T, n_experts, capacity_factor);
+}
+
+switch_status_t switch_workspace_size(const switch_config_t* cfg, size_t* bytes) {
+  int64_t C = 0;
+  switch_status_t s = validate(cfg, &C);
+  if (s != SWITCH_OK) return s;
+  if (bytes == nullptr) return SWITCH_ERR_INVALID_ARG;
+  *bytes = layout_for(*cfg, C).total;
+  return SWITCH_OK;
+}
+
+switch_status_t switch_router(const switch_config_t* cfg, const void* x, const float* w_r,
+                              const float* b_r, int32_t* idx, float* gate, float* probs,
+                              void* ws, size_t ws_bytes, void* stream) {
+  Ctx c{};
+  switch_status_t s = prepare(cfg, ws, ws_bytes, stream, &c);
+  if (s != SWITCH_OK || cfg->T == 0) return s;
+  if (!x || !w_r || !idx || !gate || !aligned16(x) || (probs && !aligned16(probs)))
+    return SWITCH_ERR_INVALID_ARG;
+  RouterOut o{idx, gate, probs, c.at<float>(c.L.psum), nullptr, nullptr};
+  if (use_tc_router(cfg)) {
+    return cuda_status(launch_router_tc(cfg->T, cfg->d_model, cfg->n_experts,
+                                        router_terms(cfg), x, w_r, b_r, c.ws + c.L.wsplit, o,
+                                        ntiles_of(cfg->T), c.err, c.spin, c.num_sms, c.st));
+  }
+  int nparts = 0;
+  return cuda_status(launch_router_simt(cfg->T, cfg->d_model, cfg->n_experts,
+                                        cfg->dtype == SWITCH_BF16, x, w_r, b_r,
+                                        c.at<float>(c.L.logits), o, &nparts, c.st));
+}
+
+switch_status_t switch_dispatch(const switch_config_t* cfg, const int32_t* idx,
+                                const float* probs, int32_t* rank, uint8_t* drop,
+                                int32_t* counts, int32_t* slot_token, const void* x,
+                                void* x_disp, void* ws, size_t ws_bytes, void* stream) {
+  Ctx c{};
+  switch_status_t s = prepare(cfg, ws, ws_bytes, stream, &c);
+  if (s != SWITCH_OK || cfg->T == 0) return s;
+  if ((!idx && !probs) || !rank || !drop || !counts || !slot_token) return SWITCH_ERR_INVALID_ARG;
+  if (x_disp && (!x || !aligned16(x) || !aligned16(x_disp))) return SWITCH_ERR_INVALID_ARG;
+  const int N = cfg->n_experts;
+  const int nt = ntiles_of(cfg->T);
+  int* idx_src = idx ? const_cast<int*>(idx) : c.at<int>(c.L.idx);
+  SMOE_TRY(launch_tile_rank(cfg->T, N, idx, probs, idx ? nullptr : idx_src,
+                            c.at<int>(c.L.local_rank), c.at<int>(c.L.hist), nt, c.err, c.st));
+  SMOE_TRY(launch_scan(N, nt, c.at<int>(c.L.hist), c.at<int>(c.L.base), counts, c.st));
+  SMOE_TRY(launch_finalize(cfg->T, N, c.C, nt, idx_src, c.at<int>(c.L.local_rank),
+                           c.at<int>(c.L.base), counts, rank, drop, slot_token,
+                           c.at<int>(c.L.mtile_start), c.st));
+  if (x_disp) {
+    const int64_t row_bytes =
+        static_cast<int64_t>(cfg->d_model) * (cfg->dtype == SWITCH_BF16 ? 2 : 4);
+    SMOE_TRY(launch_gather_rows(static_cast<int64_t>(N) * c.C, row_bytes, slot_token, x,
+                                x_disp, c.st));
+  }
+  return SWITCH_OK;
+}
+
+switch_status_t switch_expert_ffn(const switch_config_t* cfg, const void* x,
+                                  const int32_t* slot_token, const int32_t* counts,
+                                  const void* w1, const void* w2, void* y, void* ws,
+                                  size_t ws_bytes, void* stream) {
+  Ctx c{};
+  switch_status_t s = prepare(cfg, ws, ws_bytes, stream, &c);
+  if (s != SWITCH_OK || cfg->T == 0) return s;
+  if (!x || !slot_token || !counts || !w1 || !w2 || !y || !aligned16(x) || !aligned16(w1) ||
+      !aligned16(w2) || !aligned16(y))
+    return SWITCH_ERR_INVALID_ARG;
+  FfnArgs a{};
+  a.T = cfg->T;
+  a.d = cfg->d_model;
+  a.F = cfg->d_ff;
+  a.N = cfg->n_experts;
+  a.C = c.C;
+  a.x = x;
+  a.slot_token = slot_token;
+  a.counts = counts;
+  a.mtile_start = c.at<int>(c.L.mtile_start);
+  a.w1 = w1;
+  a.w2 = w2;
+  a.hbuf = c.ws + c.L.hbuf;
+  a.y = y;
+  a.mode2 = kModeY;
+  a.err = c.err;
+  a.spin = c.spin;
+  a.num_sms = c.num_sms;
+  if (cfg->dtype == SWITCH_F32) return cuda_status(launch_expert_ffn_f32(a, c.st));
+  SMOE_TRY(launch_mtile_table(a.N, a.C, counts, c.at<int>(c.L.mtile_start), c.st));
+  if (cfg->flags & SWITCH_FLAG_GATHER_COPY) {
+    SMOE_TRY(launch_gather_rows(static_cast<int64_t>(a.N) * a.C,
+                                static_cast<int64_t>(a.d) * 2, slot_token, x,
+                                c.ws + c.L.xdisp, c.st));
+    a.x_disp = c.ws + c.L.xdisp;
+  }
+  return cuda_status(launch_expert_ffn_bf16(a, c.st));
+}
+
+switch_status_t switch_combine(const switch_config_t* cfg, const void* x_residual,
+                               const int32_t* idx, const int32_t* rank, const uint8_t* drop,
+                               const float* gate, const void* y, void* out, void* stream) {
+  int64_t C = 0;
+  switch_status_t s = validate(cfg, &C);
+  if (s != SWITCH_OK || cfg->T == 0) return s;
+  if (!idx || !rank || !drop || !gate || !y || !out || !aligned16(y) || !aligned16(out) ||
+      (x_residual && !aligned16(x_residual)))
+    return SWITCH_ERR_INVALID_ARG;
+  return cuda_status(launch_combine(cfg->T, cfg->d_model, C, cfg->dtype == SWITCH_BF16,
+                                    x_residual, idx, rank, drop, gate, y, out, false,
+                                    static_cast<cudaStream_t>(stream)));
+}
+
+switch_status_t switch_aux_loss(const switch_config_t* cfg, const int32_t* counts,
+                                const float* probs, float* loss, float* f, float* P, void* ws,
+                                size_t ws_bytes, void* stream) {
+  Ctx c{};
+  switch_status_t s = prepare(cfg, ws, ws_bytes, stream, &c);
+  if (s != SWITCH_OK || cfg->T == 0) return s;
+  if (!counts || !probs || !loss) return SWITCH_ERR_INVALID_ARG;
+  float* psum = c.at<float>(c.L.psum);
+  SMOE_TRY(launch_prob_colsum(cfg->T, cfg->n_experts, probs, psum, c.st));
+  return cuda_status(launch_aux_loss(cfg->T, cfg->n_experts, ntiles_of(cfg->T), cfg->alpha,
+                                     counts, psum, loss, f, P, c.st));
+}
+
+switch_status_t switch_layer_forward(const switch_config_t* cfg, const void* x,
+                                     const float* w_r, const float* b_r, const void* w1,
+                                     const void* w2, void* out, int32_t* idx, float* gate,
+                                     int32_t* counts, float* loss, void* ws, size_t ws_bytes,
+                                     void* stream) {
+  Ctx c{};
+  switch_status_t s = prepare(cfg, ws, ws_bytes, stream, &c);
+  if (s != SWITCH_OK || cfg->T == 0) return s;
+  if (!x || !w_r || !w1 || !w2 || !out || !aligned16(x) || !aligned16(w1) || !aligned16(w2) ||
+      !aligned16(out))
+    return SWITCH_ERR_INVALID_ARG;
+  const int64_t T = cfg->T;
+  const int N = cfg->n_experts;
+  const int nt = ntiles_of(T);
+  const bool bf16 = cfg->dtype == SWITCH_BF16;
+  int* idx_p = idx ? idx : c.at<int>(c.L.idx);
+  float* gate_p = gate ? gate : c.at<float>(c.L.gate);
+  int* counts_p = counts ? counts : c.at<int>(c.L.counts);
+  int* local_rank = c.at<int>(c.L.local_rank);
+  int* hist = c.at<int>(c.L.hist);
+  float* psum = c.at<float>(c.L.psum);
+  int nparts = nt;
+
+  // 1. router (+ per-tile ranks and histograms on the tensor-core path)
+  if (use_tc_router(cfg)) {
+    RouterOut o{idx_p, gate_p, nullptr, psum, hist, local_rank};
+    SMOE_TRY(launch_router_tc(T, cfg->d_model, N, router_terms(cfg), x, w_r, b_r,
+                              c.ws + c.L.wsplit, o, nt, c.err, c.spin, c.num_sms, c.st));
+  } else {
+    RouterOut o{idx_p, gate_p, nullptr, psum, nullptr, nullptr};
+    SMOE_TRY(launch_router_simt(T, cfg->d_model, N, bf16, x, w_r, b_r,
+                                c.at<float>(c.L.logits), o, &nparts, c.st));
+    SMOE_TRY(launch_tile_rank(T, N, idx_p, nullptr, nullptr, local_rank, hist, nt, c.err,
+                              c.st));
+  }
+  // 2-3. dispatch: scan over tiles, then rank / drop / slots / tile table
+  SMOE_TRY(launch_scan(N, nt, hist, c.at<int>(c.L.base), counts_p, c.st));
+  int* slot_token = c.at<int>(c.L.slot_token);
+  int* rank = c.at<int>(c.L.rank);
+  uint8_t* drop = c.at<uint8_t>(c.L.drop);
+  SMOE_TRY(launch_finalize(T, N, c.C, nt, idx_p, local_rank, c.at<int>(c.L.base), counts_p,
+                           rank, drop, slot_token, c.at<int>(c.L.mtile_start), c.st));
+  // 4. experts, with the combine fused into the second GEMM unless asked not to
+  const bool fused = !(cfg->flags & SWITCH_FLAG_UNFUSED_COMBINE);
+  const void* x_res = (cfg->flags & SWITCH_FLAG_NO_RESIDUAL) ? nullptr : x;
+  FfnArgs a{};
+  a.T = T;
+  a.d = cfg->d_model;
+  a.F = cfg->d_ff;
+  a.N = N;
+  a.C = c.C;
+  a.x = x;
+  a.slot_token = slot_token;
+  a.counts = counts_p;
+  a.mtile_start = c.at<int>(c.L.mtile_start);
+  a.w1 = w1;
+  a.w2 = w2;
+  a.hbuf = c.ws + c.L.hbuf;
+  a.y = c.ws + c.L.ybuf;
+  a.x_res = x_res;
+  a.gate = gate_p;
+  a.out = out;
+  a.mode2 = fused ? kModeCombine : kModeY;
+  a.err = c.err;
+  a.spin = c.spin;
+  a.num_sms = c.num_sms;
+  if (bf16 && (cfg->flags & SWITCH_FLAG_GATHER_COPY)) {
+    SMOE_TRY(launch_gather_rows(static_cast<int64_t>(N) * c.C,
+                                static_cast<int64_t>(a.d) * 2, slot_token, x, c.ws + c.L.xdisp,
+                                c.st));
+    a.x_disp = c.ws + c.L.xdisp;
+  }
+  SMOE_TRY(bf16 ? launch_expert_ffn_bf16(a, c.st) : launch_expert_ffn_f32(a, c.st));
+  // 5. dropped tokens (fused) or every token (unfused)
+  SMOE_TRY(launch_combine(T, cfg->d_model, c.C, bf16, x_res, idx_p, rank, drop, gate_p,
+                          c.ws + c.L.ybuf, out, fused, c.st));
+  // 6. load-balancing loss
+  if (loss)
+    SMOE_TRY(launch_aux_loss(T, N, nparts, cfg->alpha, counts_p, psum, loss, nullptr, nullptr,
+                             c.st));
+  return SWITCH_OK;
+}
+
+switch_status_t switch_get_device_error(void* ws, void* stream, int32_t* where_out,
+                                        int64_t* info_out) {
+  if (ws == nullptr) return SWITCH_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return SWITCH_ERR_CUDA;
+  DevErr h{};
+  if (cudaMemcpy(&h, ws, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return SWITCH_ERR_CUDA;
+  if (where_out) *where_out = h.where;
+  if (info_out) *info_out = h.info;
+  if (h.code != 0 && cudaMemset(ws, 0, sizeof(h)) != cudaSuccess) return SWITCH_ERR_CUDA;
+  return static_cast<switch_status_t>(h.code);
+}
+
+const char* switch_status_string(switch_status_t s) {
+  switch (s) {
+    case SWITCH_OK: return "ok";
+    case SWITCH_ERR_INVALID_ARG: return "invalid argument";
+    case SWITCH_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case SWITCH_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case SWITCH_ERR_CUDA: return "CUDA error";
+    case SWITCH_ERR_TIMEOUT: return "device wait timed out";
+    case SWITCH_ERR_DEVICE_BOUNDS: return "device index out of range";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

@@ -29,6 +29,7 @@ Recipe (stated once, used everywhere):
 Every tensor gets its own ``SeedSequence`` (and every expert of ``w1``/``w2``
 its own child), so one expert's weights can be regenerated alone.
 """
+import os
 from dataclasses import dataclass
 from typing import Optional
 
@@ -99,20 +100,31 @@ def make_expert_w2(wl: Workload, e: int) -> np.ndarray:
     return w if wl.dtype == "f32" else f32_to_bf16_bits(w)
 
 
+def _fill_experts(out: np.ndarray, make_one, wl: Workload) -> np.ndarray:
+    """Fill out[e] = make_one(wl, e) for every expert, on a thread pool (each
+    expert has its own generator, so the result does not depend on the
+    number of threads; numpy releases the GIL while drawing)."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    def one(e):
+        out[e] = make_one(wl, e)
+
+    workers = max(1, min(wl.n_experts, os.cpu_count() or 1, 32))
+    with ThreadPoolExecutor(max_workers=workers) as ex:
+        list(ex.map(one, range(wl.n_experts)))
+    return out
+
+
 def make_w1(wl: Workload) -> np.ndarray:
     dt = np.float32 if wl.dtype == "f32" else np.uint16
-    out = np.empty((wl.n_experts, wl.d_ff, wl.d_model), dtype=dt)
-    for e in range(wl.n_experts):
-        out[e] = make_expert_w1(wl, e)
-    return out
+    return _fill_experts(np.empty((wl.n_experts, wl.d_ff, wl.d_model), dtype=dt),
+                         make_expert_w1, wl)
 
 
 def make_w2(wl: Workload) -> np.ndarray:
     dt = np.float32 if wl.dtype == "f32" else np.uint16
-    out = np.empty((wl.n_experts, wl.d_model, wl.d_ff), dtype=dt)
-    for e in range(wl.n_experts):
-        out[e] = make_expert_w2(wl, e)
-    return out
+    return _fill_experts(np.empty((wl.n_experts, wl.d_model, wl.d_ff), dtype=dt),
+                         make_expert_w2, wl)
 
 
 # ------------------------------------------------------------- zipf bias
