@@ -134,6 +134,29 @@ switch_status_t switch_dispatch(const switch_config_t* cfg, const int32_t* idx,
                                 int32_t* counts, int32_t* slot_token, const void* x,
                                 void* x_disp, void* ws, size_t ws_bytes, void* stream);
 
+/* switch_dispatch for callers that cannot allocate device memory (the
+ * pages have no counterpart: this is a deployment convenience).  A plugin
+ * running inside another engine's enqueue step, or a serving loop with a
+ * fixed memory budget that must not call cudaMalloc after start-up (it can
+ * synchronise the device), cannot hand this library a workspace; this entry
+ * point needs none.  Same inputs and outputs as switch_dispatch without the
+ * optional gather (idx or probs in; rank, drop, counts, slot_token out; all
+ * device pointers owned by the caller), bit-identical results.
+ *   - Scratch: a 2 MiB array compiled into the library, held by every GPU
+ *     that loads it until the process exits.  Limits: T <= 131072 and
+ *     N * ceil(T / 128) <= 131072; larger sizes return SWITCH_ERR_UNSUPPORTED
+ *     and launch nothing.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - All calls share the array: calls that overlap on the GPU (different
+ *     streams with no ordering between them) race and give wrong results.
+ *   - No device error word: expert ids outside [0, N) make the token dropped
+ *     (rank -1, drop 1) without a report.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call. */
+switch_status_t switch_dispatch_noalloc(const switch_config_t* cfg, const int32_t* idx,
+                                        const float* probs, int32_t* rank, uint8_t* drop,
+                                        int32_t* counts, int32_t* slot_token, void* stream);
+
 /* Expert FFNs over the capacity buffers [P1 "The Core Idea"]:
  *   y[e, r, :] = relu(x[slot_token[e*C + r]] . w1[e]^T) . w2[e]^T
  * for r < n_e = min(counts[e], C).  Rows r >= n_e of y are left untouched.

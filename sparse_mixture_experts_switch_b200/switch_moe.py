@@ -56,6 +56,8 @@ def _load():
         "switch_dispatch": (c_int32, [cfgp, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                       c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
                                       c_void_p]),
+        "switch_dispatch_noalloc": (c_int32, [cfgp, c_void_p, c_void_p, c_void_p, c_void_p,
+                                              c_void_p, c_void_p, c_void_p]),
         "switch_expert_ffn": (c_int32, [cfgp, c_void_p, c_void_p, c_void_p, c_void_p,
                                         c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
         "switch_combine": (c_int32, [cfgp, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
@@ -136,6 +138,14 @@ def switch_dispatch(cfg, idx, probs, rank, drop, counts, slot_token, x, x_disp, 
     _check(_lib.switch_dispatch(ctypes.byref(cfg), _p(idx), _p(probs), _p(rank), _p(drop),
                                 _p(counts), _p(slot_token), _p(x), _p(x_disp), _p(ws),
                                 ws.numel(), _stream(stream)), "switch_dispatch")
+
+
+def switch_dispatch_noalloc(cfg, idx, probs, rank, drop, counts, slot_token, stream=None):
+    """switch_dispatch without a workspace, for callers that cannot allocate
+    device memory (scratch lives in a fixed array inside the library)."""
+    _check(_lib.switch_dispatch_noalloc(ctypes.byref(cfg), _p(idx), _p(probs), _p(rank),
+                                        _p(drop), _p(counts), _p(slot_token), _stream(stream)),
+           "switch_dispatch_noalloc")
 
 
 def switch_expert_ffn(cfg, x, slot_token, counts, w1, w2, y, ws, stream=None):
