@@ -8,20 +8,26 @@
 //
 // bf16 path: a persistent tcgen05 grouped GEMM.
 //   * tile = 128 slots (rows) x 256 output columns, K in blocks of 64;
-//   * warp 0 feeds a 4-stage shared-memory ring with TMA (128-byte swizzle);
-//     in GEMM1 the A rows are gathered straight from x through slot_token
-//     with tile::gather4 (four token rows per copy), so the dispatched
-//     tokens are never materialised;
+//   * warp 0 feeds a 4-stage shared-memory ring: weights (B) by TMA with
+//     the 128-byte swizzle; in GEMM1 the A rows are gathered straight from x
+//     through slot_token by the warp's 32 lanes with 16-byte cp.async into
+//     the same swizzled layout (the next tile's token ids are fetched while
+//     the current tile streams), so the dispatched tokens are never
+//     materialised; GEMM2 reads the hidden rows by TMA;
 //   * warp 1 issues tcgen05.mma (M=128, N=256, K=16) into one of two TMEM
 //     accumulators (2 x 256 fp32 columns) so the epilogue of one tile
 //     overlaps the main loop of the next;
-//   * warps 2-5 drain TMEM (one token row per thread): ReLU + bf16 for the
-//     hidden activation, bf16 for Y, or x + gate * acc for the combine;
+//   * warps 2-5 drain TMEM (one token row per thread) through a per-warp
+//     shared buffer that turns row-per-thread values into coalesced stores:
+//     ReLU + bf16 for the hidden activation, bf16 for Y, or x + gate * acc
+//     for the combine;
 //   * the tile list comes from device-side counts (no host sync); experts'
 //     empty capacity tiles are never scheduled; consecutive CTAs take the
 //     M tiles of the same (expert, N tile) so each weight tile is read from
 //     HBM about once and from L2 by the rest.
 // fp32 path: CUDA-core FMA tiles (no TF32), same tile list semantics.
+#include <cstring>
+
 #include "kernels.cuh"
 
 namespace smoe {
@@ -89,8 +95,11 @@ constexpr int kStages = 4;
 constexpr uint32_t kABytes = kBM * kBK * 2;             // 16 KB
 constexpr uint32_t kBBytes = kBN * kBK * 2;             // 32 KB
 constexpr uint32_t kStageBytes = kABytes + kBBytes;     // 48 KB
-constexpr int kGemmThreads = 192;
+constexpr int kGemmThreads = 224;   // w0 producer, w1 MMA, w2-5 epilogue, w6 producer
+constexpr int kGatherLanes = 64;    // lanes of warps 0 and 6 that gather A rows
 constexpr uint32_t kTmemCols = 512;                     // 2 accumulators x 256
+constexpr uint32_t kStageOutBytes = 32 * 32 * 4;        // per epilogue warp: 32 rows x 32 fp32
+constexpr uint32_t kTailBytes = 128 + 4 * 32 * 4 + 4 * kStageOutBytes;   // + mts[N + 1]
 
 struct GemmParams {
   int N, n_out, K, ntiles_n;
@@ -98,6 +107,7 @@ struct GemmParams {
   const int* counts;
   const int* mtile_start;
   const int* slot_token;
+  const __nv_bfloat16* a_rows;  // gather mode: x [T, K]
   int mode;
   __nv_bfloat16* out;       // kModeHidden / kModeY: row e*C + r, leading dim ldo
   int64_t ldo;
@@ -107,6 +117,12 @@ struct GemmParams {
   DevErr* err;
   long long spin;
 };
+
+// Rows (m*128 + r) of expert e in this tile that hold a token.
+__device__ __forceinline__ int64_t kept_rows(const GemmParams& p, int e) {
+  const int64_t cnt = p.counts[e];
+  return cnt < p.C ? cnt : p.C;
+}
 
 template <bool kGather>
 __global__ void __launch_bounds__(kGemmThreads, 1) expert_gemm_kernel(
@@ -126,7 +142,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) expert_gemm_kernel(
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-  int* mts = reinterpret_cast<int*>(tail + 128);         // [N + 1]
+  int* tok_s = reinterpret_cast<int*>(tail + 128);                    // [4][32]
+  uint8_t* stage_out = tail + 128 + 4 * 32 * 4;                       // [4][32 x 32 fp32]
+  int* mts = reinterpret_cast<int*>(stage_out + 4 * kStageOutBytes);  // [N + 1]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long lim = p.spin;
@@ -134,7 +152,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) expert_gemm_kernel(
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], 1);
+      // gather mode: one cp.async arrival per gathering lane + the B copy
+      mbar_init(&full[s], kGather ? kGatherLanes + 1 : 1);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -156,68 +175,105 @@ __global__ void __launch_bounds__(kGemmThreads, 1) expert_gemm_kernel(
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
-  if (warp == 0) {
-    // --------------------------------------------------- TMA producer warp
-    if (lane == 0) {
-      tma_prefetch_desc(&tmap_a);
-      tma_prefetch_desc(&tmap_b);
-    }
-    int stage = 0;
-    uint32_t phase = 0;
-    uint32_t issued_mask = 0, issued_phase = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-      if (*abort_flag) break;
-      int e, m, n;
-      decode_tile(tile, mts, p.N, p.ntiles_n, e, m, n);
-      const int64_t slot0 = static_cast<int64_t>(e) * p.C + static_cast<int64_t>(m) * kBM;
-      int tok[4] = {0, 0, 0, 0};
-      if (kGather) {
-        const int64_t cnt = p.counts[e];
-        const int64_t n_e = cnt < p.C ? cnt : p.C;
-        const int first = p.slot_token[slot0];
+  if (warp == 0 || warp == 6) {
+    // --------------------------------------------------- producer warps
+    // B (weights) by TMA from warp 0; A by TMA (tiled), or in gather mode by
+    // the 64 lanes of warps 0 and 6 with 16-byte cp.async: warp 0 fills rows
+    // 0-63, warp 6 rows 64-127; lane = (row lane / 8 within a group of 4
+    // rows, 16-byte chunk lane % 8), so one instruction reads four whole
+    // 128-byte row segments, and each chunk lands where the 128-byte swizzle
+    // puts it (chunk ^ row % 8).
+    const bool lead = warp == 0;
+    if (!kGather && !lead) goto producer_done;
+    {
+      if (lead && lane == 0 && !kGather) tma_prefetch_desc(&tmap_a);
+      if (lead && lane == 0) tma_prefetch_desc(&tmap_b);
+      const int ch = lane & 7;
+      const int row0 = (lead ? 0 : 64) + (lane >> 3);        // rows row0 + 4 j, j < 16
+      const uint32_t vec_per_row = static_cast<uint32_t>(p.K / 8);   // 16-byte units
+      // per-lane shared-memory offsets of the 16 rows (two swizzle phases)
+      const uint32_t sw_even = static_cast<uint32_t>((ch ^ (row0 & 7)) << 4);
+      const uint32_t sw_odd = static_cast<uint32_t>((ch ^ ((row0 + 4) & 7)) << 4);
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0, issued_phase = 0;
+      // 16-byte-unit offset of each row's token in x (~0u: padding row)
+      uint32_t roff[16];
+      auto load_rows = [&](int t_tile, uint32_t* dst) {
+        int e, m, n;
+        decode_tile(t_tile, mts, p.N, p.ntiles_n, e, m, n);
+        const int64_t n_e = kept_rows(p, e);
+        const int64_t slot0 = static_cast<int64_t>(e) * p.C + static_cast<int64_t>(m) * kBM;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int64_t r = static_cast<int64_t>(m) * kBM + lane * 4 + i;
-          tok[i] = r < n_e ? p.slot_token[slot0 + lane * 4 + i] : first;
+        for (int j = 0; j < 16; ++j) {
+          const int r = row0 + 4 * j;
+          dst[j] = (static_cast<int64_t>(m) * kBM + r < n_e)
+                       ? static_cast<uint32_t>(p.slot_token[slot0 + r]) * vec_per_row
+                       : ~0u;
         }
-      }
-      bool ok = true;
-      for (int kb = 0; kb < kblocks; ++kb) {
-        int w_ok = 1;
-        if (lane == 0) w_ok = mbar_wait(&empty[stage], phase ^ 1u, lim) ? 1 : 0;
-        w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
-        if (!w_ok) {
-          if (lane == 0) {
-            report_error(p.err, SWITCH_ERR_TIMEOUT, kWhereGemmProducer, tile);
-            *abort_flag = 1;
+      };
+      if (kGather) load_rows(blockIdx.x, roff);
+      for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+        if (__shfl_sync(0xffffffffu, *abort_flag, 0)) break;   // warp-uniform
+        int e, m, n;
+        decode_tile(tile, mts, p.N, p.ntiles_n, e, m, n);
+        const int64_t slot0 = static_cast<int64_t>(e) * p.C + static_cast<int64_t>(m) * kBM;
+        uint32_t roff_next[16];
+        const int next = tile + gridDim.x;
+        if (kGather && next < total) load_rows(next, roff_next);   // in flight meanwhile
+        bool ok = true;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          int w_ok = 1;
+          if (lane == 0) w_ok = mbar_wait(&empty[stage], phase ^ 1u, lim) ? 1 : 0;
+          w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
+          if (!w_ok) {
+            if (lane == 0) {
+              report_error(p.err, SWITCH_ERR_TIMEOUT, kWhereGemmProducer, tile);
+              *abort_flag = 1;
+            }
+            ok = false;
+            break;
           }
-          ok = false;
-          break;
+          uint8_t* sa = smem + stage * kStageBytes;
+          uint8_t* sb = sa + kABytes;
+          if (kGather) {
+            const uint4* src0 = reinterpret_cast<const uint4*>(p.a_rows) + kb * 8 + ch;
+            const uint32_t dst0 = smem_u32(sa) + static_cast<uint32_t>(row0 * 128);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              if (roff[j] != ~0u)
+                cp_async16_s(dst0 + j * 512 + ((j & 1) ? sw_odd : sw_even), src0 + roff[j]);
+            }
+            cp_async_mbar_arrive_noinc(&full[stage]);
+            if (lead && lane == 0) {
+              mbar_arrive_expect_tx(&full[stage], kBBytes);
+              tma_load_2d(sb, &tmap_b, &full[stage], kb * kBK, e * p.n_out + n * kBN);
+            }
+          } else if (lane == 0) {
+            mbar_arrive_expect_tx(&full[stage], kStageBytes);
+            tma_load_2d(sa, &tmap_a, &full[stage], kb * kBK, static_cast<int>(slot0));
+            tma_load_2d(sb, &tmap_b, &full[stage], kb * kBK, e * p.n_out + n * kBN);
+          }
+          issued_mask |= 1u << stage;
+          issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+          if (++stage == kStages) { stage = 0; phase ^= 1u; }
         }
-        uint8_t* sa = smem + stage * kStageBytes;
-        uint8_t* sb = sa + kABytes;
-        if (lane == 0) mbar_arrive_expect_tx(&full[stage], kStageBytes);
-        __syncwarp();
+        if (!ok) break;
         if (kGather) {
-          tma_gather4(sa + lane * 512, &tmap_a, &full[stage], kb * kBK, tok[0], tok[1], tok[2],
-                      tok[3]);
-        } else if (lane == 0) {
-          tma_load_2d(sa, &tmap_a, &full[stage], kb * kBK, static_cast<int>(slot0));
+#pragma unroll
+          for (int j = 0; j < 16; ++j) roff[j] = roff_next[j];
         }
-        if (lane == 0)
-          tma_load_2d(sb, &tmap_b, &full[stage], kb * kBK, e * p.n_out + n * kBN);
-        issued_mask |= 1u << stage;
-        issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
-        if (++stage == kStages) { stage = 0; phase ^= 1u; }
       }
-      if (!ok) break;
+      // Never leave with copies in flight into this CTA's shared memory.
+      if (kGather) cp_async_wait_all();
+      if (lead && lane == 0) {
+        for (int s = 0; s < kStages; ++s)
+          if (((issued_mask >> s) & 1u) &&
+              !mbar_wait(&full[s], (issued_phase >> s) & 1u, kDefaultSpinCycles))
+            report_error(p.err, SWITCH_ERR_TIMEOUT, kWhereDrain, s);
+      }
     }
-    if (lane == 0) {
-      for (int s = 0; s < kStages; ++s)
-        if (((issued_mask >> s) & 1u) &&
-            !mbar_wait(&full[s], (issued_phase >> s) & 1u, kDefaultSpinCycles))
-          report_error(p.err, SWITCH_ERR_TIMEOUT, kWhereDrain, s);
-    }
+  producer_done:;
   } else if (warp == 1) {
     // --------------------------------------------------- MMA issuer
     if (lane == 0) {
@@ -243,6 +299,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) expert_gemm_kernel(
             ok = false;
             break;
           }
+          if (kGather) fence_proxy_async_smem();   // cp.async data -> tensor-core reads
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + stage * kStageBytes);
           const uint32_t sb = sa + kABytes;
@@ -267,76 +324,86 @@ __global__ void __launch_bounds__(kGemmThreads, 1) expert_gemm_kernel(
     }
   } else {
     // --------------------------------------------------- epilogue warps
+    // Each thread owns one accumulator row (TMEM lane).  Per 32-column chunk
+    // the row's values (ReLU'd, or scaled by its gate) go through a per-warp
+    // shared buffer so that global stores are written 8 rows x 64 bytes per
+    // instruction instead of 32 scattered 16-byte pieces.
     const int q = warp & 3;
     const int row = q * 32 + lane;
+    const uint32_t stg = smem_u32(stage_out + q * kStageOutBytes);
+    int* tokw = tok_s + q * 32;
+    const int qq = lane & 3;          // 8-column group in the transposed pass
+    const int rr0 = lane >> 2;        // row within an 8-row pass
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-      if (!mbar_wait(&tfull[acc], acc_phase, lim)) {
-        report_error(p.err, SWITCH_ERR_TIMEOUT, kWhereGemmEpilogue, tile);
-        *abort_flag = 1;
+      // warp-uniform outcome: the TMEM loads below are warp-collective
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull[acc], acc_phase, lim));
+      if (!ok) {
+        if (lane == 0) {
+          report_error(p.err, SWITCH_ERR_TIMEOUT, kWhereGemmEpilogue, tile);
+          *abort_flag = 1;
+        }
         break;
       }
       tc_fence_after();
       int e, m, n;
       decode_tile(tile, mts, p.N, p.ntiles_n, e, m, n);
-      const int64_t cnt = p.counts[e];
-      const int64_t n_e = cnt < p.C ? cnt : p.C;
-      const int64_t r = static_cast<int64_t>(m) * kBM + row;
-      const bool valid = r < n_e;
+      const int64_t n_e = kept_rows(p, e);
+      const int64_t rbase = static_cast<int64_t>(m) * kBM + q * 32;   // first row of this warp
+      const bool valid = rbase + lane < n_e;
       const uint32_t taddr =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * kBN);
-      int tok = 0;
-      float g = 0.f;
-      if (p.mode == kModeCombine && valid) {
-        tok = p.slot_token[static_cast<int64_t>(e) * p.C + r];
-        g = p.gate[tok];
+      float g = 1.f;
+      if (p.mode == kModeCombine) {
+        const int tk = valid ? p.slot_token[static_cast<int64_t>(e) * p.C + rbase + lane] : 0;
+        g = valid ? p.gate[tk] : 0.f;
+        tokw[lane] = tk;
       }
+      __syncwarp();
 #pragma unroll 1
       for (int c = 0; c < kBN / 32; ++c) {
         float v[32];
         tmem_ld32(taddr + c * 32, v);
-        const int col = n * kBN + c * 32;
-        if (!valid || col >= p.n_out) continue;
-        uint32_t pk[16];
-        if (p.mode == kModeHidden) {
+        const int col0 = n * kBN + c * 32;
+        if (col0 >= p.n_out) continue;     // uniform across the warp
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            pk[j] = pack_bf16x2(fmaxf(v[2 * j], 0.f), fmaxf(v[2 * j + 1], 0.f));
-          uint4* dst = reinterpret_cast<uint4*>(
-              p.out + (static_cast<int64_t>(e) * p.C + r) * p.ldo + col);
+        for (int j = 0; j < 32; ++j)
+          v[j] = p.mode == kModeHidden ? fmaxf(v[j], 0.f) : (p.mode == kModeCombine ? g * v[j] : v[j]);
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-        } else if (p.mode == kModeY) {
+        for (int k = 0; k < 8; ++k)
+          st_shared_v4(stg + lane * 128 + ((k ^ (lane & 7)) << 4), v[4 * k], v[4 * k + 1],
+                       v[4 * k + 2], v[4 * k + 3]);
+        __syncwarp();
 #pragma unroll
-          for (int j = 0; j < 16; ++j) pk[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
-          uint4* dst = reinterpret_cast<uint4*>(
-              p.out + (static_cast<int64_t>(e) * p.C + r) * p.ldo + col);
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-        } else {
-          const int64_t off = static_cast<int64_t>(tok) * p.n_out + col;
-          uint4 xr[4];
-          if (p.x_res != nullptr) {
-            const uint4* src = reinterpret_cast<const uint4*>(p.x_res + off);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) xr[j] = __ldg(src + j);
-          } else {
-#pragma unroll
-            for (int j = 0; j < 4; ++j) xr[j] = make_uint4(0, 0, 0, 0);
+        for (int pass = 0; pass < 4; ++pass) {
+          const int rr = pass * 8 + rr0;
+          const int64_t r = rbase + rr;
+          if (r < n_e) {
+            const float4 a = ld_shared_v4(stg + rr * 128 + (((2 * qq) ^ (rr & 7)) << 4));
+            const float4 b = ld_shared_v4(stg + rr * 128 + (((2 * qq + 1) ^ (rr & 7)) << 4));
+            uint4 o;
+            if (p.mode == kModeCombine) {
+              const int tk = tokw[rr];
+              const int64_t off = static_cast<int64_t>(tk) * p.n_out + col0 + qq * 8;
+              uint4 xr = make_uint4(0, 0, 0, 0);
+              if (p.x_res != nullptr) xr = __ldg(reinterpret_cast<const uint4*>(p.x_res + off));
+              o.x = pack_bf16x2(a.x + bf16_lo(xr.x), a.y + bf16_hi(xr.x));
+              o.y = pack_bf16x2(a.z + bf16_lo(xr.y), a.w + bf16_hi(xr.y));
+              o.z = pack_bf16x2(b.x + bf16_lo(xr.z), b.y + bf16_hi(xr.z));
+              o.w = pack_bf16x2(b.z + bf16_lo(xr.w), b.w + bf16_hi(xr.w));
+              *reinterpret_cast<uint4*>(p.comb_out + off) = o;
+            } else {
+              o.x = pack_bf16x2(a.x, a.y);
+              o.y = pack_bf16x2(a.z, a.w);
+              o.z = pack_bf16x2(b.x, b.y);
+              o.w = pack_bf16x2(b.z, b.w);
+              *reinterpret_cast<uint4*>(p.out + (static_cast<int64_t>(e) * p.C + r) * p.ldo +
+                                        col0 + qq * 8) = o;
+            }
           }
-          const uint32_t* xw = &xr[0].x;
-#pragma unroll
-          for (int j = 0; j < 16; ++j)
-            pk[j] = pack_bf16x2(fmaf(g, v[2 * j], bf16_lo(xw[j])),
-                                fmaf(g, v[2 * j + 1], bf16_hi(xw[j])));
-          uint4* dst = reinterpret_cast<uint4*>(p.comb_out + off);
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
         }
+        __syncwarp();
       }
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
@@ -352,7 +419,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) expert_gemm_kernel(
 }
 
 static size_t gemm_smem_bytes(int N) {
-  return 1024 + kStages * kStageBytes + 128 + sizeof(int) * (N + 1);
+  return 1024 + kStages * kStageBytes + kTailBytes + sizeof(int) * (N + 1);
 }
 
 template <bool kGather>
@@ -371,9 +438,11 @@ cudaError_t launch_expert_ffn_bf16(const FfnArgs& a, cudaStream_t st) {
   const uint64_t slots = static_cast<uint64_t>(a.N) * static_cast<uint64_t>(a.C);
   CUtensorMap ta1, tb1, ta2, tb2;
   const bool gather = a.x_disp == nullptr;
-  bool ok = gather
-                ? make_tmap_bf16_2d(&ta1, a.x, a.d, a.T, kBK, 1)
-                : make_tmap_bf16_2d(&ta1, a.x_disp, a.d, slots, kBK, kBM);
+  bool ok = true;
+  if (gather)
+    memset(&ta1, 0, sizeof(ta1));          // unused: rows are gathered with cp.async
+  else
+    ok = make_tmap_bf16_2d(&ta1, a.x_disp, a.d, slots, kBK, kBM);
   ok = ok && make_tmap_bf16_2d(&tb1, a.w1, a.d, static_cast<uint64_t>(a.N) * a.F, kBK, kBN);
   ok = ok && make_tmap_bf16_2d(&ta2, a.hbuf, a.F, slots, kBK, kBM);
   ok = ok && make_tmap_bf16_2d(&tb2, a.w2, a.F, static_cast<uint64_t>(a.N) * a.d, kBK, kBN);
@@ -388,6 +457,7 @@ cudaError_t launch_expert_ffn_bf16(const FfnArgs& a, cudaStream_t st) {
   g1.counts = a.counts;
   g1.mtile_start = a.mtile_start;
   g1.slot_token = a.slot_token;
+  g1.a_rows = static_cast<const __nv_bfloat16*>(a.x);
   g1.mode = kModeHidden;
   g1.out = static_cast<__nv_bfloat16*>(a.hbuf);
   g1.ldo = a.F;
@@ -401,6 +471,7 @@ cudaError_t launch_expert_ffn_bf16(const FfnArgs& a, cudaStream_t st) {
   g2.n_out = a.d;
   g2.K = a.F;
   g2.ntiles_n = (a.d + kBN - 1) / kBN;
+  g2.a_rows = nullptr;
   g2.mode = a.mode2;
   g2.out = static_cast<__nv_bfloat16*>(a.y);
   g2.ldo = a.d;
