@@ -73,7 +73,7 @@ typedef enum { SWITCH_F32 = 0, SWITCH_BF16 = 1 } switch_dtype_t;
 /* Option bits of switch_config_t.flags (0 = the default fast path). */
 enum {
   SWITCH_FLAG_ROUTER_SIMT = 1,       /* CUDA-core fp32 FMA router */
-  SWITCH_FLAG_ROUTER_2TERM = 2,      /* tensor-core router, W_r split in 2 bf16 terms (default 3) */
+  SWITCH_FLAG_ROUTER_3TERM = 2,      /* tensor-core router, W_r split in 3 bf16 terms (default 2) */
   SWITCH_FLAG_UNFUSED_COMBINE = 4,   /* forward: write Y, then a separate combine kernel */
   SWITCH_FLAG_GATHER_COPY = 8,       /* forward: copy routed rows to x_disp before GEMM1 */
   SWITCH_FLAG_NO_RESIDUAL = 16       /* forward: block output is y alone (dropped -> 0) */
@@ -107,9 +107,13 @@ switch_status_t switch_workspace_size(const switch_config_t* cfg, size_t* bytes)
  *   idx    [T] int32 out: expert of the largest logit, lowest index on ties
  *   gate   [T] fp32  out: p_idx(x)
  *   probs  [T, N] fp32 out, or NULL: softmax probabilities
- * bf16 x runs on the tensor cores with W_r split into three bf16 terms that
- * sum to it exactly (two with SWITCH_FLAG_ROUTER_2TERM) and fp32
- * accumulation; fp32 x (or SWITCH_FLAG_ROUTER_SIMT) uses fp32 FMA. */
+ * bf16 x runs on the tensor cores: bf16 x is exact, W_r is split into bf16
+ * terms hi + lo (W_r to about 2^-17 relative; SWITCH_FLAG_ROUTER_3TERM adds
+ * a third term, whose sum is W_r exactly), each term accumulated in its
+ * own fp32 TMEM columns and the logits summed in fp32.  Measured max
+ * relative error of the probabilities against a float64 reference: about
+ * 4e-6 (two terms), 2e-6 (three).  Probabilities below 2^-126 are returned
+ * as 0.  fp32 x (or SWITCH_FLAG_ROUTER_SIMT) uses fp32 FMA. */
 switch_status_t switch_router(const switch_config_t* cfg, const void* x,
                               const float* w_r, const float* b_r, int32_t* idx,
                               float* gate, float* probs, void* ws, size_t ws_bytes,

@@ -338,7 +338,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) expert_gemm_kernel(
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
       // warp-uniform outcome: the TMEM loads below are warp-collective
-      const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull[acc], acc_phase, lim));
+      const bool ok = __all_sync(0xffffffffu, mbar_wait_sleepy(&tfull[acc], acc_phase, lim));
       if (!ok) {
         if (lane == 0) {
           report_error(p.err, SWITCH_ERR_TIMEOUT, kWhereGemmEpilogue, tile);

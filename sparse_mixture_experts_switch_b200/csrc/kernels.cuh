@@ -67,6 +67,8 @@ cudaError_t launch_router_tc(int64_t T, int d, int N, int terms, const void* x,
                              RouterOut o, int ntiles, DevErr* err, long long spin,
                              int num_sms, cudaStream_t st);
 bool router_tc_supported(int N, int d, int terms);
+// Bytes of the bf16 split-weight scratch launch_router_tc needs (3 terms).
+size_t router_wsplit_bytes(int N, int d);
 
 // ------------------------------------------------------------ expert FFN
 enum GemmMode : int { kModeHidden = 0, kModeY = 1, kModeCombine = 2 };

@@ -21,6 +21,15 @@ namespace smoe {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
+// 2^x on the special-function unit (one instruction).  Results below the
+// smallest normal float (2^-126) flush to zero: a probability that small is
+// reported as 0.
+__device__ __forceinline__ float exp2_fast(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // ================================================================ SIMT
 
 constexpr int kSimtTok = 64;      // tokens per block (8 warps x 8)
@@ -172,18 +181,22 @@ __global__ void wsplit_kernel(int N, int N_pad, int d, int terms,
 
 struct RouterTcParams {
   int64_t T;
-  int d, N, N_pad, acc_stride, terms, stages, ntiles;
-  uint32_t stage_bytes, tmem_cols;
+  int d, N, N_pad, acc_stride, terms, ntiles, subs;
+  int xstages, wstages;
+  uint32_t wstage_bytes, tmem_cols;
   const float* b_r;
   RouterOut o;
   DevErr* err;
   long long spin;
 };
 
-constexpr int kRouterThreads = 192;   // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+// warp 0 TMA, warp 1 MMA, warps 2-9 epilogue (two groups of four)
+constexpr int kRouterThreads = 64 + 256;
+constexpr int kRouterMaxXStages = 12;
+constexpr int kRouterMaxWStages = 4;
 
-__device__ __forceinline__ void transpose_reduce32(float (&v)[32], int lane) {
-  // After this, lane j holds the sum over the warp's lanes of v[j].
+__device__ __forceinline__ void transpose_reduce32(float* v, int lane) {
+  // After this, lane j holds in v[0] the sum over the warp's lanes of v[j].
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) {
     const bool upper = (lane & off) != 0;
@@ -196,49 +209,73 @@ __device__ __forceinline__ void transpose_reduce32(float (&v)[32], int lane) {
   }
 }
 
+// Logits of experts 32c .. 32c + 31 of this thread's token: the sum of the
+// weight terms' accumulator columns (term p at column p * NCH * 32).
+template <int NCH, int TERMS>
+__device__ __forceinline__ void load_logits(uint32_t taddr, int c, float* v) {
+  tmem_ld32(taddr + c * 32, v);
+#pragma unroll
+  for (int p = 1; p < TERMS; ++p) {
+    float w[32];
+    tmem_ld32(taddr + p * NCH * 32 + c * 32, w);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] += w[j];
+  }
+}
+
+// Each CTA owns `subs` consecutive 128-token tiles, all accumulated at once
+// (subs x N_pad fp32 TMEM columns).  The K loop is outermost: every k-block
+// of the split router weight is loaded into shared memory once per CTA and
+// used for all its tiles, so the weight is read from L2 once per CTA rather
+// than once per tile; x streams through a deeper ring of its own.
+template <int NCH, int TERMS>
 __global__ void __launch_bounds__(kRouterThreads, 1) router_tc_kernel(
     const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
     RouterTcParams prm) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-  const int S = prm.stages;
-  uint8_t* tail = smem + static_cast<size_t>(S) * prm.stage_bytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(tail);
-  uint64_t* empty = full + 8;
-  uint64_t* tfull = empty + 8;
-  uint64_t* tempty = tfull + 2;
-  uint64_t* drain = tempty + 2;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  const int XS = prm.xstages, WS = prm.wstages, SUBS = prm.subs;
+  const int N = prm.N, N_pad = prm.N_pad, NS = prm.acc_stride;
+  constexpr uint32_t kXBytes = 128 * 128;                // one 128-token x block
+  uint8_t* xring = smem;
+  uint8_t* wring = smem + static_cast<size_t>(XS) * kXBytes;
+  uint8_t* tail = wring + static_cast<size_t>(WS) * prm.wstage_bytes;
+  uint64_t* xfull = reinterpret_cast<uint64_t*>(tail);
+  uint64_t* xempty = xfull + kRouterMaxXStages;
+  uint64_t* wfull = xempty + kRouterMaxXStages;
+  uint64_t* wempty = wfull + kRouterMaxWStages;
+  uint64_t* tfull = wempty + kRouterMaxWStages;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tfull + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-  volatile int* epi_abort = abort_flag + 1;
-  const int NS = prm.acc_stride;                       // N_pad rounded up to 32
-  float* bias_s = reinterpret_cast<float*>(tail + 256);  // [NS]
-  float* red = bias_s + NS;                              // [4][NS]
-  int* cnt = reinterpret_cast<int*>(red + 4 * NS);       // [4][N_pad]
+  volatile int* epi_abort = abort_flag + 1;              // [2] one per epilogue group
+  float* bias_s = reinterpret_cast<float*>(tail + 512);  // [N_pad]
+  float* red = bias_s + N_pad;                           // [2][4][N_pad]
+  int* cnt = reinterpret_cast<int*>(red + 2 * 4 * N_pad);   // [2][4][N_pad]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int N = prm.N, N_pad = prm.N_pad;
   const int kblocks = prm.d / 64;
   const long long lim = prm.spin;
-  const uint32_t a_bytes = 128 * 128;
+  const int tile0 = blockIdx.x * SUBS;
+  const int ntile_here = min(SUBS, prm.ntiles - tile0);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+    for (int s = 0; s < XS; ++s) {
+      mbar_init(&xfull[s], 1);
+      mbar_init(&xempty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 128);
+    for (int s = 0; s < WS; ++s) {
+      mbar_init(&wfull[s], 1);
+      mbar_init(&wempty[s], 1);
     }
-    mbar_init(drain, 1);
+    mbar_init(tfull, 1);
     *abort_flag = 0;
-    *epi_abort = 0;
+    epi_abort[0] = 0;
+    epi_abort[1] = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
   }
-  for (int i = threadIdx.x; i < NS; i += blockDim.x)
+  for (int i = threadIdx.x; i < N_pad; i += blockDim.x)
     bias_s[i] = (prm.b_r != nullptr && i < N) ? prm.b_r[i] : 0.f;
   if (warp == 1) {
     tmem_alloc(tmem_holder, prm.tmem_cols);
@@ -254,182 +291,210 @@ __global__ void __launch_bounds__(kRouterThreads, 1) router_tc_kernel(
     if (lane == 0) {
       tma_prefetch_desc(&tmap_x);
       tma_prefetch_desc(&tmap_w);
-      int stage = 0;
-      uint32_t phase = 0;
-      uint32_t issued_mask = 0, issued_phase = 0;
-      for (int tile = blockIdx.x; tile < prm.ntiles && !*abort_flag; tile += gridDim.x) {
-        for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, lim)) {
-            report_error(prm.err, SWITCH_ERR_TIMEOUT, kWhereRouterProducer, tile);
-            *abort_flag = 1;
-            break;
-          }
-          uint8_t* sa = smem + static_cast<size_t>(stage) * prm.stage_bytes;
-          uint8_t* sb = sa + a_bytes;
-          mbar_arrive_expect_tx(&full[stage], prm.stage_bytes);
-          tma_load_2d(sa, &tmap_x, &full[stage], kb * 64, tile * 128);
-          for (int p = 0; p < prm.terms; ++p)
-            tma_load_2d(sb + static_cast<size_t>(p) * N_pad * 128, &tmap_w, &full[stage],
-                        kb * 64, p * N_pad);
-          issued_mask |= 1u << stage;
-          issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
-          if (++stage == S) { stage = 0; phase ^= 1u; }
+      int xs = 0, ws = 0;
+      uint32_t xph = 0, wph = 0;
+      uint32_t xmask = 0, xphs = 0, wmask = 0, wphs = 0;
+      bool ok = true;
+      for (int kb = 0; kb < kblocks && ok; ++kb) {
+        if (!mbar_wait(&wempty[ws], wph ^ 1u, lim)) { ok = false; break; }
+        mbar_arrive_expect_tx(&wfull[ws], prm.wstage_bytes);
+        uint8_t* wb = wring + static_cast<size_t>(ws) * prm.wstage_bytes;
+        for (int p = 0; p < prm.terms; ++p)
+          tma_load_2d(wb + static_cast<size_t>(p) * N_pad * 128, &tmap_w, &wfull[ws], kb * 64,
+                      p * N_pad);
+        wmask |= 1u << ws;
+        wphs = (wphs & ~(1u << ws)) | (wph << ws);
+        if (++ws == WS) { ws = 0; wph ^= 1u; }
+        for (int s = 0; s < ntile_here; ++s) {
+          if (!mbar_wait(&xempty[xs], xph ^ 1u, lim)) { ok = false; break; }
+          mbar_arrive_expect_tx(&xfull[xs], kXBytes);
+          tma_load_2d(xring + static_cast<size_t>(xs) * kXBytes, &tmap_x, &xfull[xs], kb * 64,
+                      (tile0 + s) * 128);
+          xmask |= 1u << xs;
+          xphs = (xphs & ~(1u << xs)) | (xph << xs);
+          if (++xs == XS) { xs = 0; xph ^= 1u; }
         }
       }
+      if (!ok) {
+        report_error(prm.err, SWITCH_ERR_TIMEOUT, kWhereRouterProducer, blockIdx.x);
+        *abort_flag = 1;
+      }
       // Never leave with copies in flight into this CTA's shared memory.
-      for (int s = 0; s < S; ++s)
-        if (((issued_mask >> s) & 1u) &&
-            !mbar_wait(&full[s], (issued_phase >> s) & 1u, kDefaultSpinCycles))
+      for (int s = 0; s < XS; ++s)
+        if (((xmask >> s) & 1u) && !mbar_wait(&xfull[s], (xphs >> s) & 1u, kDefaultSpinCycles))
+          report_error(prm.err, SWITCH_ERR_TIMEOUT, kWhereDrain, s);
+      for (int s = 0; s < WS; ++s)
+        if (((wmask >> s) & 1u) && !mbar_wait(&wfull[s], (wphs >> s) & 1u, kDefaultSpinCycles))
           report_error(prm.err, SWITCH_ERR_TIMEOUT, kWhereDrain, s);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(128, N_pad);
-      int stage = 0;
-      uint32_t phase = 0;
-      int acc = 0;
-      uint32_t acc_phase = 0;
-      bool any = false;
-      for (int tile = blockIdx.x; tile < prm.ntiles && !*abort_flag; tile += gridDim.x) {
-        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, lim)) {
-          report_error(prm.err, SWITCH_ERR_TIMEOUT, kWhereRouterMma, tile);
-          *abort_flag = 1;
-          break;
-        }
+      // Terms are stacked along the MMA's N dimension (each term has its own
+      // N_PAD accumulator columns), GSIZE terms per instruction.
+      constexpr int N_PAD = NCH * 32;
+      constexpr int GSIZE = (256 / N_PAD) < TERMS ? (256 / N_PAD) : TERMS;
+      constexpr int NGROUPS = (TERMS + GSIZE - 1) / GSIZE;
+      constexpr int LAST = TERMS - (NGROUPS - 1) * GSIZE;
+      constexpr uint32_t idesc_full = idesc_bf16_f32(128, GSIZE * N_PAD);
+      constexpr uint32_t idesc_last = idesc_bf16_f32(128, LAST * N_PAD);
+      int xs = 0, ws = 0;
+      uint32_t xph = 0, wph = 0;
+      bool ok = true, any = false;
+      // Descriptors are built once per ring slot and advanced by constants
+      // (the start-address field counts 16-byte units): the MMA issue loop
+      // must stay well under the 64 tensor-core cycles of one MMA.
+      const uint64_t xdesc0 = sw128_kmajor_desc(smem_u32(xring));
+      const uint64_t wdesc0 = sw128_kmajor_desc(smem_u32(wring));
+      const uint64_t term_step = static_cast<uint64_t>(N_pad * 128 / 16);
+      for (int kb = 0; kb < kblocks && ok && !*abort_flag; ++kb) {
+        if (!mbar_wait(&wfull[ws], wph, lim)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * prm.acc_stride);
-        bool ok = true;
-        for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait(&full[stage], phase, lim)) {
-            report_error(prm.err, SWITCH_ERR_TIMEOUT, kWhereRouterMma, tile);
-            *abort_flag = 1;
-            ok = false;
-            break;
-          }
+        const uint64_t wd = wdesc0 + static_cast<uint64_t>(ws) * (prm.wstage_bytes / 16);
+        for (int s = 0; s < ntile_here; ++s) {
+          if (!mbar_wait(&xfull[xs], xph, lim)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t sa = smem_u32(smem + static_cast<size_t>(stage) * prm.stage_bytes);
-          const uint32_t sb = sa + a_bytes;
+          const uint64_t xd = xdesc0 + static_cast<uint64_t>(xs) * (kXBytes / 16);
+          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(s * NS);
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            const uint64_t ad = sw128_kmajor_desc(sa + k * 32);
-            for (int p = 0; p < prm.terms; ++p) {
-              const uint64_t bd =
-                  sw128_kmajor_desc(sb + static_cast<uint32_t>(p * N_pad * 128) + k * 32);
-              umma_bf16(d_tmem, ad, bd, idesc, (kb | k | p) != 0 ? 1u : 0u);
-            }
+#pragma unroll
+            for (int g = 0; g < NGROUPS; ++g)
+              umma_bf16(d_tmem + static_cast<uint32_t>(g * GSIZE * N_PAD), xd + 2 * k,
+                        wd + g * GSIZE * term_step + 2 * k,
+                        g == NGROUPS - 1 ? idesc_last : idesc_full, (kb | k) != 0 ? 1u : 0u);
           }
           any = true;
-          umma_commit(&empty[stage]);
-          if (++stage == S) { stage = 0; phase ^= 1u; }
+          umma_commit(&xempty[xs]);
+          if (++xs == XS) { xs = 0; xph ^= 1u; }
         }
         if (!ok) break;
-        umma_commit(&tfull[acc]);
-        acc ^= 1;
-        if (acc == 0) acc_phase ^= 1u;
+        umma_commit(&wempty[ws]);
+        if (++ws == WS) { ws = 0; wph ^= 1u; }
       }
-      if (any && *abort_flag) {
-        // Let every issued MMA finish before TMEM is released.
-        umma_commit(drain);
-        if (!mbar_wait(drain, 0, kDefaultSpinCycles))
-          report_error(prm.err, SWITCH_ERR_TIMEOUT, kWhereDrain, -1);
+      if (!ok) {
+        report_error(prm.err, SWITCH_ERR_TIMEOUT, kWhereRouterMma, blockIdx.x);
+        *abort_flag = 1;
       }
+      // Accumulators complete (or, after an error, every issued MMA done):
+      // the epilogue may read TMEM, and TMEM may be released.
+      if (any || ok) umma_commit(tfull);
+      else mbar_arrive(tfull);
+      // After an error nobody else may wait for the MMAs: do it here, so
+      // TMEM is never released under an MMA still in flight.
+      if ((!ok || *abort_flag) && !mbar_wait(tfull, 0, kDefaultSpinCycles))
+        report_error(prm.err, SWITCH_ERR_TIMEOUT, kWhereDrain, -1);
     }
   } else {
     // ------------------------------------------------------- epilogue
-    const int q = warp & 3;                 // TMEM lane quarter of this warp
+    // group g (warps 2-5: g = 0, warps 6-9: g = 1) takes tiles g, g + 2, ...
+    // of the CTA; each warp owns the 32 TMEM lanes (tokens) of its quarter.
+    const int g = (warp - 2) >> 2;
+    const int q = warp & 3;
     const int row = q * 32 + lane;
-    const int et = threadIdx.x - 64;        // 0..127
-    int acc = 0;
-    uint32_t acc_phase = 0;
-    for (int tile = blockIdx.x; tile < prm.ntiles; tile += gridDim.x) {
-      const bool ok = mbar_wait(&tfull[acc], acc_phase, lim);
-      if (!ok) *epi_abort = 1;
-      for (int i = et; i < 4 * N_pad; i += 128) cnt[i] = 0;
-      named_bar_sync(1, 128);
-      if (*epi_abort || *abort_flag) {
-        if (et == 0) {
-          report_error(prm.err, SWITCH_ERR_TIMEOUT, kWhereRouterEpilogue, tile);
-          *abort_flag = 1;
-        }
-        break;
-      }
+    const int et = (threadIdx.x - 64) & 127;
+    float* redg = red + g * 4 * N_pad;
+    int* cntg = cnt + g * 4 * N_pad;
+    volatile int* my_abort = epi_abort + g;
+    const bool ok = mbar_wait_sleepy(tfull, 0, lim);
+    if (!ok || *abort_flag) *my_abort = 1;
+    named_bar_sync(1 + g, 128);
+    if (*my_abort) {
+      if (et == 0) report_error(prm.err, SWITCH_ERR_TIMEOUT, kWhereRouterEpilogue, blockIdx.x);
+    } else {
       tc_fence_after();
-      const int64_t t = static_cast<int64_t>(tile) * 128 + row;
-      const bool valid = t < prm.T;
-      const uint32_t taddr =
-          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * prm.acc_stride);
-      float v[32];
-      // pass 1: max and argmax (lowest index on ties)
-      float m = -INFINITY;
-      int best = 0;
-      for (int c = 0; c < N_pad; c += 32) {
-        tmem_ld32(taddr + c, v);
+      for (int s = g; s < ntile_here; s += 2) {
+        const int tile = tile0 + s;
+        for (int i = et; i < 4 * N_pad; i += 128) cntg[i] = 0;
+        named_bar_sync(1 + g, 128);
+        const int64_t t = static_cast<int64_t>(tile) * 128 + row;
+        const bool valid = t < prm.T;
+        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                               static_cast<uint32_t>(s * NS);
+        // Three streaming passes over the row's logits in TMEM (max; sum of
+        // exponentials and the first index of the max; scaled probabilities
+        // and their column sums), 32 values live at a time.
+        const bool has_bias = prm.b_r != nullptr;
+        float v[32];
+        float m = -INFINITY;
+#pragma unroll 1
+        for (int c = 0; c < NCH; ++c) {
+          load_logits<NCH, TERMS>(taddr, c, v);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int e = c + j;
-          const float h = v[j] + bias_s[e];
-          if (e < N && h > m) { m = h; best = e; }
-        }
-      }
-      // pass 2: sum of exponentials
-      float s = 0.f;
-      for (int c = 0; c < N_pad; c += 32) {
-        tmem_ld32(taddr + c, v);
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (c + j < N) s += exp2f((v[j] + bias_s[c + j] - m) * kLog2e);
-      }
-      const float inv = 1.f / s;
-      // pass 3: probabilities, their column sums over the tile
-      for (int c = 0; c < N_pad; c += 32) {
-        tmem_ld32(taddr + c, v);
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          v[j] = (valid && c + j < N) ? exp2f((v[j] + bias_s[c + j] - m) * kLog2e) * inv : 0.f;
-        if (valid && prm.o.probs != nullptr) {
-          float4* dst = reinterpret_cast<float4*>(prm.o.probs + t * N + c);
-          if (c + 32 <= N && (N % 4) == 0) {
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-              dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-          } else {
-            for (int j = 0; j < 32 && c + j < N; ++j) prm.o.probs[t * N + c + j] = v[j];
+          for (int j = 0; j < 32; ++j) {
+            const float hv = has_bias ? v[j] + bias_s[c * 32 + j] : v[j];
+            if (c * 32 + j < N) m = fmaxf(m, hv);
           }
         }
-        transpose_reduce32(v, lane);
-        red[q * NS + c + lane] = v[0];
+        const float mL = m * kLog2e;
+        float s4[4] = {0.f, 0.f, 0.f, 0.f};
+        int best = 0x7fffffff;
+#pragma unroll 1
+        for (int c = 0; c < NCH; ++c) {
+          load_logits<NCH, TERMS>(taddr, c, v);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int e = c * 32 + j;
+            const float hv = has_bias ? v[j] + bias_s[e] : v[j];
+            if (e < N) {
+              s4[j & 3] += exp2_fast(fmaf(hv, kLog2e, -mL));
+              if (hv == m && e < best) best = e;
+            }
+          }
+        }
+        const float inv = 1.f / ((s4[0] + s4[1]) + (s4[2] + s4[3]));
+        const float scale = valid ? inv : 0.f;
+#pragma unroll 1
+        for (int c = 0; c < NCH; ++c) {
+          load_logits<NCH, TERMS>(taddr, c, v);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int e = c * 32 + j;
+            const float hv = has_bias ? v[j] + bias_s[e] : v[j];
+            v[j] = e < N ? exp2_fast(fmaf(hv, kLog2e, -mL)) * scale : 0.f;
+          }
+          if (valid && prm.o.probs != nullptr) {
+            float* dst = prm.o.probs + t * N + c * 32;
+            if ((N % 4) == 0 && c * 32 + 32 <= N) {
+#pragma unroll
+              for (int j = 0; j < 32; j += 4)
+                *reinterpret_cast<float4*>(dst + j) =
+                    make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (c * 32 + j < N) dst[j] = v[j];
+            }
+          }
+          transpose_reduce32(v, lane);
+          redg[q * N_pad + c * 32 + lane] = v[0];
+        }
+        if (valid) {
+          prm.o.idx[t] = best;
+          prm.o.gate[t] = inv;
+        }
+        // rank within the 128-token tile, token order (quarter q holds
+        // rows 32q .. 32q + 31)
+        const int e_key = valid ? best : -1;
+        const unsigned peers = __match_any_sync(0xffffffffu, e_key);
+        const int rank_w = __popc(peers & ((1u << lane) - 1u));
+        if (valid && rank_w == 0) cntg[q * N_pad + best] = __popc(peers);
+        named_bar_sync(1 + g, 128);
+        if (valid && prm.o.local_rank != nullptr) {
+          int r = rank_w;
+          for (int qq = 0; qq < q; ++qq) r += cntg[qq * N_pad + best];
+          prm.o.local_rank[t] = r;
+        }
+        for (int e = et; e < N; e += 128) {
+          if (prm.o.psum != nullptr)
+            prm.o.psum[static_cast<int64_t>(tile) * N + e] =
+                ((redg[e] + redg[N_pad + e]) + redg[2 * N_pad + e]) + redg[3 * N_pad + e];
+          if (prm.o.hist != nullptr)
+            prm.o.hist[static_cast<int64_t>(e) * prm.ntiles + tile] =
+                cntg[e] + cntg[N_pad + e] + cntg[2 * N_pad + e] + cntg[3 * N_pad + e];
+        }
+        named_bar_sync(1 + g, 128);
       }
-      // accumulator consumed: hand it back to the MMA warp
-      tc_fence_before();
-      mbar_arrive(&tempty[acc]);
-      acc ^= 1;
-      if (acc == 0) acc_phase ^= 1u;
-
-      if (valid) {
-        prm.o.idx[t] = best;
-        prm.o.gate[t] = inv;
-      }
-      // rank within the tile, token order (quarter q holds rows 32q..32q+31)
-      const int e_key = valid ? best : -1;
-      const unsigned peers = __match_any_sync(0xffffffffu, e_key);
-      const int rank_w = __popc(peers & ((1u << lane) - 1u));
-      if (valid && rank_w == 0) cnt[q * N_pad + best] = __popc(peers);
-      named_bar_sync(1, 128);
-      if (valid && prm.o.local_rank != nullptr) {
-        int r = rank_w;
-        for (int qq = 0; qq < q; ++qq) r += cnt[qq * N_pad + best];
-        prm.o.local_rank[t] = r;
-      }
-      for (int e = et; e < N; e += 128) {
-        if (prm.o.psum != nullptr)
-          prm.o.psum[static_cast<int64_t>(tile) * N + e] =
-              ((red[e] + red[NS + e]) + red[2 * NS + e]) + red[3 * NS + e];
-        if (prm.o.hist != nullptr)
-          prm.o.hist[static_cast<int64_t>(e) * prm.ntiles + tile] =
-              cnt[e] + cnt[N_pad + e] + cnt[2 * N_pad + e] + cnt[3 * N_pad + e];
-      }
-      named_bar_sync(1, 128);
     }
   }
 
@@ -452,11 +517,36 @@ PFN_encodeTiled get_encode_fn();   // defined in expert_ffn.cu
 bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
                        uint32_t box_inner, uint32_t box_outer);   // expert_ffn.cu
 
-static int router_n_pad(int N) { return (N + 15) / 16 * 16; }
+static int router_n_pad(int N) { return (N + 31) / 32 * 32; }
 
+size_t router_wsplit_bytes(int N, int d) {
+  return sizeof(__nv_bfloat16) * 3 * static_cast<size_t>(router_n_pad(N)) * d;
+}
+
+// Every weight term keeps its own accumulator columns: terms x N_pad <= 512.
 bool router_tc_supported(int N, int d, int terms) {
   const int n_pad = router_n_pad(N);
-  return (terms == 2 || terms == 3) && n_pad <= 256 && d % 64 == 0 && d > 0;
+  return (terms == 2 || terms == 3) && terms * n_pad <= 512 && d % 64 == 0 && d > 0;
+}
+
+template <int NCH, int TERMS>
+static cudaError_t run_router_tc_t(const CUtensorMap& tx, const CUtensorMap& tw,
+                                   const RouterTcParams& p, size_t smem, int grid,
+                                   cudaStream_t st) {
+  cudaError_t e = cudaFuncSetAttribute(router_tc_kernel<NCH, TERMS>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  router_tc_kernel<NCH, TERMS><<<grid, kRouterThreads, smem, st>>>(tx, tw, p);
+  return cudaGetLastError();
+}
+
+template <int NCH>
+static cudaError_t run_router_tc(const CUtensorMap& tx, const CUtensorMap& tw,
+                                 const RouterTcParams& p, size_t smem, int grid,
+                                 cudaStream_t st) {
+  return p.terms == 2 ? run_router_tc_t<NCH, 2>(tx, tw, p, smem, grid, st)
+                      : run_router_tc_t<NCH, 3>(tx, tw, p, smem, grid, st);
 }
 
 cudaError_t launch_router_tc(int64_t T, int d, int N, int terms, const void* x,
@@ -487,32 +577,45 @@ cudaError_t launch_router_tc(int64_t T, int d, int N, int terms, const void* x,
   p.N_pad = N_pad;
   p.terms = terms;
   p.ntiles = ntiles;
-  p.stage_bytes = 128u * 128u + static_cast<uint32_t>(terms) * N_pad * 128u;
-  const int ns = (N_pad + 31) / 32 * 32;
-  const size_t tail_bytes = 256 + sizeof(float) * ns * 5 + sizeof(int) * N_pad * 4;
-  const size_t budget = 227 * 1024 - 1024 - tail_bytes;
-  int stages = static_cast<int>(budget / p.stage_bytes);
-  if (stages > 8) stages = 8;
-  if (stages < 2) return cudaErrorInvalidConfiguration;
-  p.stages = stages;
-  // Accumulators start 32-column aligned so that the epilogue's 32-column
-  // TMEM loads stay inside the allocation.
+  // One tile's accumulator: the terms side by side, N_pad (a multiple of 32)
+  // columns each.
+  const int ns = terms * N_pad;
   p.acc_stride = ns;
+  // Tiles per CTA: enough to cover the tokens in about one wave, at most
+  // what TMEM holds (512 fp32 columns).
+  int subs = (ntiles + num_sms - 1) / num_sms;
+  if (subs > 512 / ns) subs = 512 / ns;
+  if (subs < 1) subs = 1;
+  p.subs = subs;
+  p.wstage_bytes = static_cast<uint32_t>(terms) * N_pad * 128u;
+  const size_t tail_bytes = 512 + sizeof(float) * N_pad * 9 + sizeof(int) * N_pad * 8;
+  const size_t budget = 227 * 1024 - 1024 - tail_bytes;
+  int wst = 2;
+  int xst = static_cast<int>((budget - wst * p.wstage_bytes) / (128 * 128));
+  if (xst > kRouterMaxXStages) xst = kRouterMaxXStages;
+  if (xst < 2) return cudaErrorInvalidConfiguration;
+  p.xstages = xst;
+  p.wstages = wst;
   uint32_t cols = 32;
-  while (cols < static_cast<uint32_t>(2 * p.acc_stride)) cols <<= 1;
+  while (cols < static_cast<uint32_t>(subs * ns)) cols <<= 1;
   p.tmem_cols = cols;
   p.b_r = b_r;
   p.o = o;
   p.err = err;
   p.spin = spin;
-  const size_t smem = 1024 + static_cast<size_t>(stages) * p.stage_bytes + tail_bytes;
-  cudaError_t e = cudaFuncSetAttribute(router_tc_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  int grid = ntiles < num_sms ? ntiles : num_sms;
-  router_tc_kernel<<<grid, kRouterThreads, smem, st>>>(tx, tw, p);
-  return cudaGetLastError();
+  const size_t smem = 1024 + static_cast<size_t>(xst) * 128 * 128 +
+                      static_cast<size_t>(wst) * p.wstage_bytes + tail_bytes;
+  const int grid = (ntiles + subs - 1) / subs;
+  switch (N_pad / 32) {
+    case 1: return run_router_tc<1>(tx, tw, p, smem, grid, st);
+    case 2: return run_router_tc<2>(tx, tw, p, smem, grid, st);
+    case 3: return run_router_tc<3>(tx, tw, p, smem, grid, st);
+    case 4: return run_router_tc<4>(tx, tw, p, smem, grid, st);
+    case 5: return run_router_tc<5>(tx, tw, p, smem, grid, st);
+    case 6: return run_router_tc<6>(tx, tw, p, smem, grid, st);
+    case 7: return run_router_tc<7>(tx, tw, p, smem, grid, st);
+    default: return run_router_tc<8>(tx, tw, p, smem, grid, st);
+  }
 }
 
 }  // namespace smoe

@@ -50,7 +50,6 @@ Layout layout_for(const switch_config_t& c, int64_t C) {
   const size_t es = c.dtype == SWITCH_BF16 ? 2 : 4;
   const int64_t nt = ntiles_of(T);
   const int64_t nparts = (T + 63) / 64;
-  const int64_t npad = (N + 15) / 16 * 16;
   const int64_t slots = N * C;
   Layout L{};
   size_t o = 0;
@@ -71,7 +70,7 @@ Layout layout_for(const switch_config_t& c, int64_t C) {
   L.counts = take(sizeof(int) * N);
   L.slot_token = take(sizeof(int) * slots);
   L.mtile_start = take(sizeof(int) * (N + 1));
-  L.wsplit = take(2 * 3 * npad * static_cast<size_t>(c.d_model));
+  L.wsplit = take(router_wsplit_bytes(c.n_experts, c.d_model));
   L.logits = take(sizeof(float) * N * T);
   L.xdisp = take(es * slots * static_cast<size_t>(c.d_model));
   L.hbuf = take(es * slots * static_cast<size_t>(c.d_ff));
@@ -157,7 +156,7 @@ switch_status_t cuda_status(cudaError_t e) {
   } while (0)
 
 int router_terms(const switch_config_t* c) {
-  return (c->flags & SWITCH_FLAG_ROUTER_2TERM) ? 2 : 3;
+  return (c->flags & SWITCH_FLAG_ROUTER_3TERM) ? 3 : 2;
 }
 
 bool use_tc_router(const switch_config_t* c) {

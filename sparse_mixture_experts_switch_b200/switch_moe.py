@@ -21,7 +21,7 @@ STATUS_NAMES = {0: "SWITCH_OK", 1: "SWITCH_ERR_INVALID_ARG", 2: "SWITCH_ERR_UNSU
                 5: "SWITCH_ERR_TIMEOUT", 6: "SWITCH_ERR_DEVICE_BOUNDS"}
 SWITCH_F32, SWITCH_BF16 = 0, 1
 FLAG_ROUTER_SIMT = 1
-FLAG_ROUTER_2TERM = 2
+FLAG_ROUTER_3TERM = 2
 FLAG_UNFUSED_COMBINE = 4
 FLAG_GATHER_COPY = 8
 FLAG_NO_RESIDUAL = 16

@@ -72,7 +72,7 @@ E2E = Workload("e2e", T=3000, d_model=320, d_ff=576, n_experts=8, capacity_facto
 
 
 @pytest.mark.parametrize("flags", [0, 1, 2, 4, 8, 1 | 4 | 8],
-                         ids=["fused", "simt_router", "two_term", "unfused", "gather_copy",
+                         ids=["fused", "simt_router", "three_term", "unfused", "gather_copy",
                               "simt_unfused_copy"])
 def test_layer_bf16(sm, flags):
     flips, drop_rate = check_layer(sm, E2E, flags)
@@ -122,3 +122,28 @@ def test_layer_single_token_and_capacity_one(sm):
         wl = Workload("t", T=T, d_model=64, d_ff=128, n_experts=4, capacity_factor=cf,
                       dtype="bf16", seed=75 + T)
         check_layer(sm, wl)
+
+
+@pytest.mark.parametrize("T,N,d,F,flags", [(1, 4, 64, 128, 0), (37, 4, 64, 128, 0),
+                                           (300, 37, 128, 192, 0), (300, 300, 64, 64, 0),
+                                           (513, 16, 64, 128, 8), (129, 64, 128, 64, 4)])
+def test_workspace_bounds_respected(sm, T, N, d, F, flags):
+    """Canary bytes right after the workspace stay untouched, for small and
+    odd shapes where padded per-expert scratch is easiest to mis-size."""
+    wl = Workload("ws", T=T, d_model=d, d_ff=F, n_experts=N, capacity_factor=1.0,
+                  dtype="bf16", seed=81)
+    inp = make_inputs(wl)
+    cfg = sm.config(T, d, F, N, 1.0, flags=flags)
+    n = sm.switch_workspace_size(cfg)
+    canary = 1 << 16
+    buf = torch.full((n + canary,), 0xA5, dtype=torch.uint8, device="cuda")
+    buf[:n].zero_()
+    ws = buf[:n]
+    x = dev_float(inp.x)
+    out = torch.empty_like(x)
+    loss = torch.empty(1, dtype=torch.float32, device="cuda")
+    sm.switch_layer_forward(cfg, x, dev_float(inp.w_r), None, dev_float(inp.w1),
+                            dev_float(inp.w2), out, None, None, None, loss, ws)
+    st, where, info = sm.switch_get_device_error(ws)
+    assert st == 0
+    assert (buf[n:] == 0xA5).all(), "a kernel wrote past the end of the workspace"

@@ -74,14 +74,14 @@ def test_router(sm, wl, flags):
     assert rel_err(gate.cpu().numpy(), want_gate).max() <= PROB_RTOL
 
 
-def test_router_two_term_split(sm):
-    """Two bf16 terms (W_r rounded to ~16 significant bits): reported, and
-    held to the same probability tolerance."""
+def test_router_three_term_split(sm):
+    """Three bf16 terms (their sum is W_r exactly): reported, and held to
+    the same probability tolerance."""
     wl = ROUTER_CASES[1]
     x = make_x(wl)
     w_r, b_r = make_router(wl)
     r = orc.router(x, w_r, b_r)
-    cfg = _cfg(sm, wl, sm.FLAG_ROUTER_2TERM)
+    cfg = _cfg(sm, wl, sm.FLAG_ROUTER_3TERM)
     ws = sm.workspace(cfg)
     idx = torch.empty(wl.T, **I32)
     gate = torch.empty(wl.T, **F32)
@@ -89,7 +89,7 @@ def test_router_two_term_split(sm):
     sm.switch_router(cfg, dev_float(x), dev_float(w_r), None, idx, gate, probs, ws)
     _ok(sm, ws)
     err = rel_err(probs.cpu().numpy(), r["probs"]).max()
-    print(f"two-term router: max prob rel err {err:.3e}")
+    print(f"three-term router: max prob rel err {err:.3e}")
     assert err <= PROB_RTOL
     check_routing(idx.cpu().numpy(), r)
 
