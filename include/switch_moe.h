@@ -76,7 +76,10 @@ enum {
   SWITCH_FLAG_ROUTER_3TERM = 2,      /* tensor-core router, W_r split in 3 bf16 terms (default 2) */
   SWITCH_FLAG_UNFUSED_COMBINE = 4,   /* forward: write Y, then a separate combine kernel */
   SWITCH_FLAG_GATHER_COPY = 8,       /* forward: copy routed rows to x_disp before GEMM1 */
-  SWITCH_FLAG_NO_RESIDUAL = 16       /* forward: block output is y alone (dropped -> 0) */
+  SWITCH_FLAG_NO_RESIDUAL = 16,      /* forward: block output is y alone (dropped -> 0) */
+  SWITCH_FLAG_GEMM_1SM = 32,         /* both expert GEMMs on single CTAs */
+  SWITCH_FLAG_GEMM_PAIRS = 64        /* GEMM1 on CTA pairs too (default: GEMM1 single CTAs,
+                                        GEMM2 CTA pairs) */
 };
 
 typedef struct {

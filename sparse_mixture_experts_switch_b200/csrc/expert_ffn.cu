@@ -28,7 +28,7 @@
 // fp32 path: CUDA-core FMA tiles (no TF32), same tile list semantics.
 #include <cstring>
 
-#include "kernels.cuh"
+#include "gemm_common.cuh"
 
 namespace smoe {
 
@@ -69,60 +69,10 @@ bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint6
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// ------------------------------------------------------------- tile list
-
-// Tile t belongs to the expert e with mts[e] * ntn <= t < mts[e + 1] * ntn
-// (the last such e, which is never empty).  Inside an expert, M tiles vary
-// fastest so that CTAs running side by side share the weight tile.
-__device__ __forceinline__ void decode_tile(int tile, const int* mts, int N, int ntn, int& e,
-                                            int& m, int& n) {
-  int lo = 0, hi = N;
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (mts[mid] * ntn <= tile) lo = mid; else hi = mid;
-  }
-  e = lo;
-  const int mt = mts[e + 1] - mts[e];
-  const int local = tile - mts[e] * ntn;
-  n = local / mt;
-  m = local - n * mt;
-}
-
 // ================================================== tcgen05 grouped GEMM
 
-constexpr int kBM = 128, kBN = 256, kBK = 64;
 constexpr int kStages = 4;
-constexpr uint32_t kABytes = kBM * kBK * 2;             // 16 KB
-constexpr uint32_t kBBytes = kBN * kBK * 2;             // 32 KB
 constexpr uint32_t kStageBytes = kABytes + kBBytes;     // 48 KB
-constexpr int kGemmThreads = 224;   // w0 producer, w1 MMA, w2-5 epilogue, w6 producer
-constexpr int kGatherLanes = 64;    // lanes of warps 0 and 6 that gather A rows
-constexpr uint32_t kTmemCols = 512;                     // 2 accumulators x 256
-constexpr uint32_t kStageOutBytes = 32 * 32 * 4;        // per epilogue warp: 32 rows x 32 fp32
-constexpr uint32_t kTailBytes = 128 + 4 * 32 * 4 + 4 * kStageOutBytes;   // + mts[N + 1]
-
-struct GemmParams {
-  int N, n_out, K, ntiles_n;
-  int64_t C;
-  const int* counts;
-  const int* mtile_start;
-  const int* slot_token;
-  const __nv_bfloat16* a_rows;  // gather mode: x [T, K]
-  int mode;
-  __nv_bfloat16* out;       // kModeHidden / kModeY: row e*C + r, leading dim ldo
-  int64_t ldo;
-  const __nv_bfloat16* x_res;   // kModeCombine
-  const float* gate;
-  __nv_bfloat16* comb_out;      // [T, n_out]
-  DevErr* err;
-  long long spin;
-};
-
-// Rows (m*128 + r) of expert e in this tile that hold a token.
-__device__ __forceinline__ int64_t kept_rows(const GemmParams& p, int e) {
-  const int64_t cnt = p.counts[e];
-  return cnt < p.C ? cnt : p.C;
-}
 
 template <bool kGather>
 __global__ void __launch_bounds__(kGemmThreads, 1) expert_gemm_kernel(
@@ -175,21 +125,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1) expert_gemm_kernel(
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
-  if (warp == 0 || warp == 6) {
+  if (warp == 0 || warp >= 6) {
     // --------------------------------------------------- producer warps
     // B (weights) by TMA from warp 0; A by TMA (tiled), or in gather mode by
-    // the 64 lanes of warps 0 and 6 with 16-byte cp.async: warp 0 fills rows
-    // 0-63, warp 6 rows 64-127; lane = (row lane / 8 within a group of 4
-    // rows, 16-byte chunk lane % 8), so one instruction reads four whole
-    // 128-byte row segments, and each chunk lands where the 128-byte swizzle
-    // puts it (chunk ^ row % 8).
+    // the lanes of warps 0, 6, 7, 8 with 16-byte cp.async, 32 rows per warp;
+    // lane = (row lane / 8 within a group of 4 rows, 16-byte chunk lane % 8),
+    // so one instruction reads four whole 128-byte row segments, and each
+    // chunk lands where the 128-byte swizzle puts it (chunk ^ row % 8).
     const bool lead = warp == 0;
     if (!kGather && !lead) goto producer_done;
     {
       if (lead && lane == 0 && !kGather) tma_prefetch_desc(&tmap_a);
       if (lead && lane == 0) tma_prefetch_desc(&tmap_b);
       const int ch = lane & 7;
-      const int row0 = (lead ? 0 : 64) + (lane >> 3);        // rows row0 + 4 j, j < 16
+      const int gw = lead ? 0 : warp - 5;                      // 0..3
+      const int row0 = 32 * gw + (lane >> 3);                  // rows row0 + 4 j, j < 8
       const uint32_t vec_per_row = static_cast<uint32_t>(p.K / 8);   // 16-byte units
       // per-lane shared-memory offsets of the 16 rows (two swizzle phases)
       const uint32_t sw_even = static_cast<uint32_t>((ch ^ (row0 & 7)) << 4);
@@ -198,14 +148,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) expert_gemm_kernel(
       uint32_t phase = 0;
       uint32_t issued_mask = 0, issued_phase = 0;
       // 16-byte-unit offset of each row's token in x (~0u: padding row)
-      uint32_t roff[16];
+      uint32_t roff[8];
       auto load_rows = [&](int t_tile, uint32_t* dst) {
         int e, m, n;
         decode_tile(t_tile, mts, p.N, p.ntiles_n, e, m, n);
         const int64_t n_e = kept_rows(p, e);
         const int64_t slot0 = static_cast<int64_t>(e) * p.C + static_cast<int64_t>(m) * kBM;
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
+        for (int j = 0; j < 8; ++j) {
           const int r = row0 + 4 * j;
           dst[j] = (static_cast<int64_t>(m) * kBM + r < n_e)
                        ? static_cast<uint32_t>(p.slot_token[slot0 + r]) * vec_per_row
@@ -218,7 +168,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) expert_gemm_kernel(
         int e, m, n;
         decode_tile(tile, mts, p.N, p.ntiles_n, e, m, n);
         const int64_t slot0 = static_cast<int64_t>(e) * p.C + static_cast<int64_t>(m) * kBM;
-        uint32_t roff_next[16];
+        uint32_t roff_next[8];
         const int next = tile + gridDim.x;
         if (kGather && next < total) load_rows(next, roff_next);   // in flight meanwhile
         bool ok = true;
@@ -240,7 +190,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) expert_gemm_kernel(
             const uint4* src0 = reinterpret_cast<const uint4*>(p.a_rows) + kb * 8 + ch;
             const uint32_t dst0 = smem_u32(sa) + static_cast<uint32_t>(row0 * 128);
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
+            for (int j = 0; j < 8; ++j) {
               if (roff[j] != ~0u)
                 cp_async16_s(dst0 + j * 512 + ((j & 1) ? sw_odd : sw_even), src0 + roff[j]);
             }
@@ -261,7 +211,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) expert_gemm_kernel(
         if (!ok) break;
         if (kGather) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) roff[j] = roff_next[j];
+          for (int j = 0; j < 8; ++j) roff[j] = roff_next[j];
         }
       }
       // Never leave with copies in flight into this CTA's shared memory.
@@ -329,11 +279,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) expert_gemm_kernel(
     // shared buffer so that global stores are written 8 rows x 64 bytes per
     // instruction instead of 32 scattered 16-byte pieces.
     const int q = warp & 3;
-    const int row = q * 32 + lane;
     const uint32_t stg = smem_u32(stage_out + q * kStageOutBytes);
     int* tokw = tok_s + q * 32;
-    const int qq = lane & 3;          // 8-column group in the transposed pass
-    const int rr0 = lane >> 2;        // row within an 8-row pass
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
@@ -349,62 +296,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) expert_gemm_kernel(
       tc_fence_after();
       int e, m, n;
       decode_tile(tile, mts, p.N, p.ntiles_n, e, m, n);
-      const int64_t n_e = kept_rows(p, e);
-      const int64_t rbase = static_cast<int64_t>(m) * kBM + q * 32;   // first row of this warp
-      const bool valid = rbase + lane < n_e;
-      const uint32_t taddr =
-          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * kBN);
-      float g = 1.f;
-      if (p.mode == kModeCombine) {
-        const int tk = valid ? p.slot_token[static_cast<int64_t>(e) * p.C + rbase + lane] : 0;
-        g = valid ? p.gate[tk] : 0.f;
-        tokw[lane] = tk;
-      }
-      __syncwarp();
-#pragma unroll 1
-      for (int c = 0; c < kBN / 32; ++c) {
-        float v[32];
-        tmem_ld32(taddr + c * 32, v);
-        const int col0 = n * kBN + c * 32;
-        if (col0 >= p.n_out) continue;     // uniform across the warp
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          v[j] = p.mode == kModeHidden ? fmaxf(v[j], 0.f) : (p.mode == kModeCombine ? g * v[j] : v[j]);
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-          st_shared_v4(stg + lane * 128 + ((k ^ (lane & 7)) << 4), v[4 * k], v[4 * k + 1],
-                       v[4 * k + 2], v[4 * k + 3]);
-        __syncwarp();
-#pragma unroll
-        for (int pass = 0; pass < 4; ++pass) {
-          const int rr = pass * 8 + rr0;
-          const int64_t r = rbase + rr;
-          if (r < n_e) {
-            const float4 a = ld_shared_v4(stg + rr * 128 + (((2 * qq) ^ (rr & 7)) << 4));
-            const float4 b = ld_shared_v4(stg + rr * 128 + (((2 * qq + 1) ^ (rr & 7)) << 4));
-            uint4 o;
-            if (p.mode == kModeCombine) {
-              const int tk = tokw[rr];
-              const int64_t off = static_cast<int64_t>(tk) * p.n_out + col0 + qq * 8;
-              uint4 xr = make_uint4(0, 0, 0, 0);
-              if (p.x_res != nullptr) xr = __ldg(reinterpret_cast<const uint4*>(p.x_res + off));
-              o.x = pack_bf16x2(a.x + bf16_lo(xr.x), a.y + bf16_hi(xr.x));
-              o.y = pack_bf16x2(a.z + bf16_lo(xr.y), a.w + bf16_hi(xr.y));
-              o.z = pack_bf16x2(b.x + bf16_lo(xr.z), b.y + bf16_hi(xr.z));
-              o.w = pack_bf16x2(b.z + bf16_lo(xr.w), b.w + bf16_hi(xr.w));
-              *reinterpret_cast<uint4*>(p.comb_out + off) = o;
-            } else {
-              o.x = pack_bf16x2(a.x, a.y);
-              o.y = pack_bf16x2(a.z, a.w);
-              o.z = pack_bf16x2(b.x, b.y);
-              o.w = pack_bf16x2(b.z, b.w);
-              *reinterpret_cast<uint4*>(p.out + (static_cast<int64_t>(e) * p.C + r) * p.ldo +
-                                        col0 + qq * 8) = o;
-            }
-          }
-        }
-        __syncwarp();
-      }
+      epilogue_tile(p, e, m, n,
+                    tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                        static_cast<uint32_t>(acc * kBN),
+                    stg, tokw, q, lane);
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
       acc ^= 1;
@@ -438,14 +333,17 @@ cudaError_t launch_expert_ffn_bf16(const FfnArgs& a, cudaStream_t st) {
   const uint64_t slots = static_cast<uint64_t>(a.N) * static_cast<uint64_t>(a.C);
   CUtensorMap ta1, tb1, ta2, tb2;
   const bool gather = a.x_disp == nullptr;
+  // CTA pairs load half a weight tile each (128 rows); single CTAs all 256.
+  const uint32_t b_rows1 = a.pair1 ? 128u : static_cast<uint32_t>(kBN);
+  const uint32_t b_rows2 = a.pair2 ? 128u : static_cast<uint32_t>(kBN);
   bool ok = true;
   if (gather)
     memset(&ta1, 0, sizeof(ta1));          // unused: rows are gathered with cp.async
   else
     ok = make_tmap_bf16_2d(&ta1, a.x_disp, a.d, slots, kBK, kBM);
-  ok = ok && make_tmap_bf16_2d(&tb1, a.w1, a.d, static_cast<uint64_t>(a.N) * a.F, kBK, kBN);
+  ok = ok && make_tmap_bf16_2d(&tb1, a.w1, a.d, static_cast<uint64_t>(a.N) * a.F, kBK, b_rows1);
   ok = ok && make_tmap_bf16_2d(&ta2, a.hbuf, a.F, slots, kBK, kBM);
-  ok = ok && make_tmap_bf16_2d(&tb2, a.w2, a.F, static_cast<uint64_t>(a.N) * a.d, kBK, kBN);
+  ok = ok && make_tmap_bf16_2d(&tb2, a.w2, a.F, static_cast<uint64_t>(a.N) * a.d, kBK, b_rows2);
   if (!ok) return cudaErrorInvalidValue;
 
   GemmParams g1{};
@@ -463,8 +361,13 @@ cudaError_t launch_expert_ffn_bf16(const FfnArgs& a, cudaStream_t st) {
   g1.ldo = a.F;
   g1.err = a.err;
   g1.spin = a.spin;
-  cudaError_t e = gather ? run_gemm<true>(ta1, tb1, g1, a.num_sms, st)
-                         : run_gemm<false>(ta1, tb1, g1, a.num_sms, st);
+  cudaError_t e;
+  if (a.pair1)
+    e = gather ? run_gemm_pair<true>(ta1, tb1, g1, a.num_sms, st)
+               : run_gemm_pair<false>(ta1, tb1, g1, a.num_sms, st);
+  else
+    e = gather ? run_gemm<true>(ta1, tb1, g1, a.num_sms, st)
+               : run_gemm<false>(ta1, tb1, g1, a.num_sms, st);
   if (e != cudaSuccess) return e;
 
   GemmParams g2 = g1;
@@ -478,7 +381,8 @@ cudaError_t launch_expert_ffn_bf16(const FfnArgs& a, cudaStream_t st) {
   g2.x_res = static_cast<const __nv_bfloat16*>(a.x_res);
   g2.gate = a.gate;
   g2.comb_out = static_cast<__nv_bfloat16*>(a.out);
-  return run_gemm<false>(ta2, tb2, g2, a.num_sms, st);
+  return a.pair2 ? run_gemm_pair<false>(ta2, tb2, g2, a.num_sms, st)
+                : run_gemm<false>(ta2, tb2, g2, a.num_sms, st);
 }
 
 // ===================================================== fp32 CUDA cores

@@ -1,0 +1,350 @@
+// Expert FFN GEMMs on CTA pairs (2-SM tcgen05): same math and epilogues as
+// expert_gemm_kernel, with each output tile 256 rows x 256 columns computed
+// by a cluster of two CTAs on two SMs.
+//
+//   * CTA r of the pair holds rows 128 r .. 128 r + 127 of the A tile and
+//     rows 128 r .. 128 r + 127 of the weight (B) tile in its own shared
+//     memory; the pair's leader (r = 0) issues tcgen05.mma.cta_group::2
+//     (M = 256, N = 256, K = 16) over both CTAs' operands, and each CTA's
+//     TMEM receives its 128 rows x 256 columns.  Every SM thus streams 32 KB
+//     per 64-deep K step instead of 48 KB, and the ring is six stages deep.
+//   * Weight (and tiled A) copies are TMA loads whose byte counts land on the
+//     leader's mbarrier; in GEMM1 each CTA gathers its own token rows with
+//     cp.async, and the follower's completion is relayed to the leader.
+//   * Commits are multicast to both CTAs (stage release, accumulator ready);
+//     both CTAs' epilogue warps hand an accumulator back to the leader.
+//   * Pair tiles come from device-side counts: an expert's 128-row M tiles
+//     are taken two at a time; an odd last tile leaves the follower's half
+//     empty (computed, not stored).
+// No copy here is multicast: each CTA loads only its own operands.
+#include <cstring>
+
+#include "gemm_common.cuh"
+
+namespace smoe {
+
+constexpr int kPairStages = 6;
+constexpr uint32_t kPairBHalf = 128 * kBK * 2;                 // 16 KB
+constexpr uint32_t kPairStageBytes = kABytes + kPairBHalf;     // 32 KB
+constexpr uint32_t kPairTail = 768 + 4 * kStageOutBytes;       // + mts, pts
+
+// Prefix over experts of ceil(M tiles / 2), one warp.
+__device__ void pair_prefix_warp(int N, const int* mts, int* pts) {
+  const int lane = threadIdx.x & 31;
+  const int per = (N + 31) / 32;
+  int s = 0;
+  for (int i = 0; i < per; ++i) {
+    const int e = lane * per + i;
+    if (e < N) s += (mts[e + 1] - mts[e] + 1) >> 1;
+  }
+  int inc = s;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, inc, off);
+    if (lane >= off) inc += v;
+  }
+  int run = inc - s;
+  for (int i = 0; i < per; ++i) {
+    const int e = lane * per + i;
+    if (e < N) {
+      pts[e] = run;
+      run += (mts[e + 1] - mts[e] + 1) >> 1;
+    }
+  }
+  if (lane == 31) pts[N] = inc;
+}
+
+template <bool kGather>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    expert_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
+                            const __grid_constant__ CUtensorMap tmap_b, GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint8_t* tail = smem + kPairStages * kPairStageBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(tail);   // leader: TMA bytes of both CTAs
+  uint64_t* afull = full + kPairStages;                  // local: gathered A rows
+  uint64_t* empty = afull + kPairStages;                 // local: stage free (MMA done)
+  uint64_t* tfull = empty + kPairStages;                 // local: accumulator ready
+  uint64_t* tempty = tfull + 2;                          // leader: accumulator drained
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tail + 192);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tail + 196);
+  int* tok_s = reinterpret_cast<int*>(tail + 256);                      // [4][32]
+  uint8_t* stage_out = tail + 768;                                      // [4][32 x 32 fp32]
+  int* mts = reinterpret_cast<int*>(stage_out + 4 * kStageOutBytes);    // [N + 1]
+  int* pts = mts + (p.N + 1);                                           // [N + 1]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int cid = static_cast<int>(cluster_id_x());
+  const int ncl = static_cast<int>(cluster_count_x());
+  const long long lim = p.spin;
+  const int kblocks = p.K / kBK;
+
+  for (int i = threadIdx.x; i <= p.N; i += blockDim.x) mts[i] = p.mtile_start[i];
+  __syncthreads();
+  if (warp == 0) pair_prefix_warp(p.N, mts, pts);
+  __syncthreads();
+  const int total = pts[p.N] * p.ntiles_n;
+  if (cid >= total) return;                 // same decision in both CTAs of the pair
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kPairStages; ++s) {
+      mbar_init(&full[s], kGather ? 2 : 1);   // leader's expect_tx (+ follower's relay)
+      mbar_init(&afull[s], kGatherLanes);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 8);               // 4 epilogue warps x 2 CTAs
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_holder, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();                          // the peer's barriers exist before any remote use
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const uint32_t full_lead = map_to_rank(smem_u32(full), 0);
+  const uint32_t tempty_lead = map_to_rank(smem_u32(tempty), 0);
+
+  if (warp == 0 || warp >= 6) {
+    // ------------------------------------------------------- producer warps
+    // (warp 0: weights, A rows 0-31; warps 6-8: A rows 32-127 when gathered)
+    const bool lead_warp = warp == 0;
+    if (!kGather && !lead_warp) goto producer_done;
+    {
+      if (lead_warp && lane == 0 && !kGather) tma_prefetch_desc(&tmap_a);
+      if (lead_warp && lane == 0) tma_prefetch_desc(&tmap_b);
+      const int ch = lane & 7;
+      const int gw = lead_warp ? 0 : warp - 5;                // 0..3
+      const int row0 = 32 * gw + (lane >> 3);                  // rows row0 + 4 j, j < 8
+      const uint32_t vec_per_row = static_cast<uint32_t>(p.K / 8);
+      const uint32_t sw_even = static_cast<uint32_t>((ch ^ (row0 & 7)) << 4);
+      const uint32_t sw_odd = static_cast<uint32_t>((ch ^ ((row0 + 4) & 7)) << 4);
+      const uint32_t tx_bytes = kGather ? 2 * kPairBHalf : 2 * kPairStageBytes;
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0, issued_phase = 0;
+      uint32_t roff[8];
+      auto load_rows = [&](int t_tile, uint32_t* dst) {
+        int e, mp, n;
+        decode_tile(t_tile, pts, p.N, p.ntiles_n, e, mp, n);
+        const int m = 2 * mp + static_cast<int>(rank);
+        const int64_t n_e = kept_rows(p, e);
+        const int64_t slot0 = static_cast<int64_t>(e) * p.C + static_cast<int64_t>(m) * kBM;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int r = row0 + 4 * j;
+          dst[j] = (static_cast<int64_t>(m) * kBM + r < n_e)
+                       ? static_cast<uint32_t>(p.slot_token[slot0 + r]) * vec_per_row
+                       : ~0u;
+        }
+      };
+      if (kGather) load_rows(cid, roff);
+      for (int tile = cid; tile < total; tile += ncl) {
+        if (__shfl_sync(0xffffffffu, *abort_flag, 0)) break;   // warp-uniform
+        int e, mp, n;
+        decode_tile(tile, pts, p.N, p.ntiles_n, e, mp, n);
+        const int m = 2 * mp + static_cast<int>(rank);
+        const int64_t slot0 = static_cast<int64_t>(e) * p.C + static_cast<int64_t>(m) * kBM;
+        uint32_t roff_next[8];
+        const int next = tile + ncl;
+        if (kGather && next < total) load_rows(next, roff_next);
+        bool ok = true;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          int w_ok = 1;
+          if (lane == 0) w_ok = mbar_wait(&empty[stage], phase ^ 1u, lim) ? 1 : 0;
+          w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
+          if (!w_ok) {
+            if (lane == 0) {
+              report_error(p.err, SWITCH_ERR_TIMEOUT, kWhereGemmProducer, tile);
+              *abort_flag = 1;
+            }
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + stage * kPairStageBytes;
+          uint8_t* sb = sa + kABytes;
+          if (kGather) {
+            const uint4* src0 = reinterpret_cast<const uint4*>(p.a_rows) + kb * 8 + ch;
+            const uint32_t dst0 = smem_u32(sa) + static_cast<uint32_t>(row0 * 128);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              if (roff[j] != ~0u)
+                cp_async16_s(dst0 + j * 512 + ((j & 1) ? sw_odd : sw_even), src0 + roff[j]);
+            }
+            cp_async_mbar_arrive_noinc(&afull[stage]);
+          }
+          if (lead_warp && lane == 0) {
+            const uint32_t bar = full_lead + 8u * stage;
+            if (leader) mbar_arrive_expect_tx(&full[stage], tx_bytes);
+            if (!kGather) tma_load_2d_pair(sa, &tmap_a, bar, kb * kBK, static_cast<int>(slot0));
+            tma_load_2d_pair(sb, &tmap_b, bar, kb * kBK,
+                             e * p.n_out + n * kBN + static_cast<int>(rank) * 128);
+          }
+          issued_mask |= 1u << stage;
+          issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+          if (++stage == kPairStages) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        if (kGather) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) roff[j] = roff_next[j];
+        }
+      }
+      // Never leave with copies in flight into shared memory: own cp.async
+      // here; both CTAs' TMA bytes complete on the leader's barriers, which
+      // the leader drains before the final cluster barrier.
+      if (kGather) cp_async_wait_all();
+      if (lead_warp && lane == 0 && leader) {
+        for (int s = 0; s < kPairStages; ++s)
+          if (((issued_mask >> s) & 1u) &&
+              !mbar_wait_cluster(&full[s], (issued_phase >> s) & 1u, kDefaultSpinCycles))
+            report_error(p.err, SWITCH_ERR_TIMEOUT, kWhereDrain, s);
+      }
+    }
+  producer_done:;
+  } else if (warp == 1) {
+    if (leader && lane == 0) {
+      // ----------------------------------------------------- MMA issuer
+      constexpr uint32_t idesc = idesc_bf16_f32(2 * kBM, kBN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool any = false;
+      for (int tile = cid; tile < total && !*abort_flag; tile += ncl) {
+        if (!mbar_wait_cluster(&tempty[acc], acc_phase ^ 1u, lim)) {
+          report_error(p.err, SWITCH_ERR_TIMEOUT, kWhereGemmMma, tile);
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBN);
+        bool ok = true;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait_cluster(&full[stage], phase, lim) ||
+              (kGather && !mbar_wait(&afull[stage], phase, lim))) {
+            report_error(p.err, SWITCH_ERR_TIMEOUT, kWhereGemmMma, tile);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          if (kGather) fence_proxy_async_smem();   // cp.async data -> tensor-core reads
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * kPairStageBytes);
+          const uint32_t sb = sa + kABytes;
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k)
+            umma_bf16_pair(d_tmem, sw128_kmajor_desc(sa + k * 32),
+                           sw128_kmajor_desc(sb + k * 32), idesc, (kb | k) != 0 ? 1u : 0u);
+          any = true;
+          umma_commit_pair(&empty[stage], 0x3);
+          if (++stage == kPairStages) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit_pair(&tfull[acc], 0x3);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      if (any && *abort_flag) {
+        umma_commit_pair(drain, 0x1);
+        if (!mbar_wait(drain, 0, kDefaultSpinCycles))
+          report_error(p.err, SWITCH_ERR_TIMEOUT, kWhereDrain, -1);
+      }
+    } else if (!leader && lane == 0 && kGather) {
+      // ------------------------------------------- follower: relay A rows
+      // Tell the leader when this CTA's gathered rows of each stage landed.
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int tile = cid; tile < total && !*abort_flag; tile += ncl) {
+        bool ok = true;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&afull[stage], phase, lim)) {
+            report_error(p.err, SWITCH_ERR_TIMEOUT, kWhereGemmProducer, tile);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          fence_proxy_async_smem();
+          mbar_arrive_remote(full_lead + 8u * stage);
+          if (++stage == kPairStages) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+      }
+    }
+  } else {
+    // ------------------------------------------------------- epilogue warps
+    const int q = warp & 3;
+    const uint32_t stg = smem_u32(stage_out + q * kStageOutBytes);
+    int* tokw = tok_s + q * 32;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = cid; tile < total; tile += ncl) {
+      // warp-uniform outcome: the TMEM loads below are warp-collective
+      const bool ok = __all_sync(0xffffffffu, mbar_wait_sleepy(&tfull[acc], acc_phase, lim));
+      if (!ok) {
+        if (lane == 0) {
+          report_error(p.err, SWITCH_ERR_TIMEOUT, kWhereGemmEpilogue, tile);
+          *abort_flag = 1;
+        }
+        break;
+      }
+      tc_fence_after();
+      int e, mp, n;
+      decode_tile(tile, pts, p.N, p.ntiles_n, e, mp, n);
+      epilogue_tile(p, e, 2 * mp + static_cast<int>(rank), n,
+                    tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                        static_cast<uint32_t>(acc * kBN),
+                    stg, tokw, q, lane);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (leader) mbar_arrive(&tempty[acc]);
+        else mbar_arrive_remote(tempty_lead + 8u * acc);
+      }
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();                          // no CTA leaves while its peer may still signal it
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_pair(tmem_base, kTmemCols);
+}
+
+size_t gemm_pair_smem_bytes(int N) {
+  return 1024 + kPairStages * kPairStageBytes + kPairTail + 2 * sizeof(int) * (N + 1);
+}
+
+template <bool kGather>
+cudaError_t run_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& gp,
+                          int num_sms, cudaStream_t st) {
+  const size_t smem = gemm_pair_smem_bytes(gp.N);
+  cudaError_t e = cudaFuncSetAttribute(expert_gemm_pair_kernel<kGather>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const int grid = (num_sms / 2) * 2;
+  expert_gemm_pair_kernel<kGather><<<grid, kGemmThreads, smem, st>>>(ta, tb, gp);
+  return cudaGetLastError();
+}
+
+template cudaError_t run_gemm_pair<true>(const CUtensorMap&, const CUtensorMap&,
+                                         const GemmParams&, int, cudaStream_t);
+template cudaError_t run_gemm_pair<false>(const CUtensorMap&, const CUtensorMap&,
+                                          const GemmParams&, int, cudaStream_t);
+
+}  // namespace smoe

@@ -1,0 +1,139 @@
+// Shared pieces of the tcgen05 grouped expert GEMMs (one-SM and CTA-pair
+// kernels): tile geometry, parameters, the device-side tile list, and the
+// epilogue that drains one 128-row x 256-column accumulator to memory.
+#pragma once
+
+#include "kernels.cuh"
+
+namespace smoe {
+
+bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                       uint32_t box_inner, uint32_t box_outer);
+
+// ------------------------------------------------------------- tile list
+
+// Tile t belongs to the expert e with mts[e] * ntn <= t < mts[e + 1] * ntn
+// (the last such e, which is never empty).  Inside an expert, M tiles vary
+// fastest so that CTAs running side by side share the weight tile.
+__device__ __forceinline__ void decode_tile(int tile, const int* mts, int N, int ntn, int& e,
+                                            int& m, int& n) {
+  int lo = 0, hi = N;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (mts[mid] * ntn <= tile) lo = mid; else hi = mid;
+  }
+  e = lo;
+  const int mt = mts[e + 1] - mts[e];
+  const int local = tile - mts[e] * ntn;
+  n = local / mt;
+  m = local - n * mt;
+}
+
+constexpr int kBM = 128, kBN = 256, kBK = 64;
+constexpr uint32_t kABytes = kBM * kBK * 2;             // 16 KB
+constexpr uint32_t kBBytes = kBN * kBK * 2;             // 32 KB
+// w0 producer (weights + A rows 0-31), w1 MMA, w2-5 epilogue, w6-8 producers
+// (A rows 32-127 when rows are gathered)
+constexpr int kGemmThreads = 288;
+constexpr int kGatherWarps = 4;
+constexpr int kGatherLanes = 32 * kGatherWarps;
+constexpr uint32_t kTmemCols = 512;                     // 2 accumulators x 256
+constexpr uint32_t kStageOutBytes = 32 * 32 * 4;        // per epilogue warp: 32 rows x 32 fp32
+constexpr uint32_t kTailBytes = 128 + 4 * 32 * 4 + 4 * kStageOutBytes;   // + mts[N + 1]
+
+struct GemmParams {
+  int N, n_out, K, ntiles_n;
+  int64_t C;
+  const int* counts;
+  const int* mtile_start;
+  const int* slot_token;
+  const __nv_bfloat16* a_rows;  // gather mode: x [T, K]
+  int mode;
+  __nv_bfloat16* out;       // kModeHidden / kModeY: row e*C + r, leading dim ldo
+  int64_t ldo;
+  const __nv_bfloat16* x_res;   // kModeCombine
+  const float* gate;
+  __nv_bfloat16* comb_out;      // [T, n_out]
+  DevErr* err;
+  long long spin;
+};
+
+// Rows (m*128 + r) of expert e in this tile that hold a token.
+__device__ __forceinline__ int64_t kept_rows(const GemmParams& p, int e) {
+  const int64_t cnt = p.counts[e];
+  return cnt < p.C ? cnt : p.C;
+}
+
+
+// Epilogue of one tile for the calling warp (quarter q of the accumulator's
+// 128 TMEM lanes: rows m * 128 + q * 32 + lane of expert e).  Each thread
+// owns one accumulator row; per 32-column chunk the row's values (ReLU'd,
+// or scaled by its gate) go through the warp's shared buffer `stg` so that
+// global stores are written 8 rows x 64 bytes per instruction.
+__device__ __forceinline__ void epilogue_tile(const GemmParams& p, int e, int m, int n,
+                                              uint32_t taddr, uint32_t stg, int* tokw, int q,
+                                              int lane) {
+  const int qq = lane & 3;          // 8-column group in the transposed pass
+  const int rr0 = lane >> 2;        // row within an 8-row pass
+  const int64_t n_e = kept_rows(p, e);
+  const int64_t rbase = static_cast<int64_t>(m) * kBM + q * 32;   // first row of this warp
+  const bool valid = rbase + lane < n_e;
+  float g = 1.f;
+  if (p.mode == kModeCombine) {
+    const int tk = valid ? p.slot_token[static_cast<int64_t>(e) * p.C + rbase + lane] : 0;
+    g = valid ? p.gate[tk] : 0.f;
+    tokw[lane] = tk;
+  }
+  __syncwarp();
+#pragma unroll 1
+  for (int c = 0; c < kBN / 32; ++c) {
+    float v[32];
+    tmem_ld32(taddr + c * 32, v);
+    const int col0 = n * kBN + c * 32;
+    if (col0 >= p.n_out) continue;     // uniform across the warp
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      v[j] = p.mode == kModeHidden ? fmaxf(v[j], 0.f) : (p.mode == kModeCombine ? g * v[j] : v[j]);
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      st_shared_v4(stg + lane * 128 + ((k ^ (lane & 7)) << 4), v[4 * k], v[4 * k + 1],
+                   v[4 * k + 2], v[4 * k + 3]);
+    __syncwarp();
+#pragma unroll
+    for (int pass = 0; pass < 4; ++pass) {
+      const int rr = pass * 8 + rr0;
+      const int64_t r = rbase + rr;
+      if (r < n_e) {
+        const float4 a = ld_shared_v4(stg + rr * 128 + (((2 * qq) ^ (rr & 7)) << 4));
+        const float4 b = ld_shared_v4(stg + rr * 128 + (((2 * qq + 1) ^ (rr & 7)) << 4));
+        uint4 o;
+        if (p.mode == kModeCombine) {
+          const int tk = tokw[rr];
+          const int64_t off = static_cast<int64_t>(tk) * p.n_out + col0 + qq * 8;
+          uint4 xr = make_uint4(0, 0, 0, 0);
+          if (p.x_res != nullptr) xr = __ldg(reinterpret_cast<const uint4*>(p.x_res + off));
+          o.x = pack_bf16x2(a.x + bf16_lo(xr.x), a.y + bf16_hi(xr.x));
+          o.y = pack_bf16x2(a.z + bf16_lo(xr.y), a.w + bf16_hi(xr.y));
+          o.z = pack_bf16x2(b.x + bf16_lo(xr.z), b.y + bf16_hi(xr.z));
+          o.w = pack_bf16x2(b.z + bf16_lo(xr.w), b.w + bf16_hi(xr.w));
+          *reinterpret_cast<uint4*>(p.comb_out + off) = o;
+        } else {
+          o.x = pack_bf16x2(a.x, a.y);
+          o.y = pack_bf16x2(a.z, a.w);
+          o.z = pack_bf16x2(b.x, b.y);
+          o.w = pack_bf16x2(b.z, b.w);
+          *reinterpret_cast<uint4*>(p.out + (static_cast<int64_t>(e) * p.C + r) * p.ldo +
+                                    col0 + qq * 8) = o;
+        }
+      }
+    }
+    __syncwarp();
+  }
+}
+
+// CTA-pair kernel launcher (expert_ffn_pair.cu).
+template <bool kGather>
+cudaError_t run_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& gp,
+                          int num_sms, cudaStream_t st);
+
+}  // namespace smoe

@@ -91,6 +91,8 @@ struct FfnArgs {
   const float* gate;        // [T]
   void* out;                // [T, d]
   int mode2;                // kModeY or kModeCombine for the second GEMM
+  bool pair1;               // GEMM1 on CTA pairs (2-SM), else one CTA per tile
+  bool pair2;               // GEMM2 on CTA pairs
   DevErr* err;
   long long spin;
   int num_sms;

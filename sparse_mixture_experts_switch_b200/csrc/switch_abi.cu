@@ -256,6 +256,8 @@ switch_status_t switch_expert_ffn(const switch_config_t* cfg, const void* x,
   a.err = c.err;
   a.spin = c.spin;
   a.num_sms = c.num_sms;
+  a.pair1 = (cfg->flags & SWITCH_FLAG_GEMM_PAIRS) != 0;
+  a.pair2 = !(cfg->flags & SWITCH_FLAG_GEMM_1SM);
   if (cfg->dtype == SWITCH_F32) return cuda_status(launch_expert_ffn_f32(a, c.st));
   SMOE_TRY(launch_mtile_table(a.N, a.C, counts, c.at<int>(c.L.mtile_start), c.st));
   if (cfg->flags & SWITCH_FLAG_GATHER_COPY) {
@@ -360,6 +362,8 @@ switch_status_t switch_layer_forward(const switch_config_t* cfg, const void* x,
   a.err = c.err;
   a.spin = c.spin;
   a.num_sms = c.num_sms;
+  a.pair1 = (cfg->flags & SWITCH_FLAG_GEMM_PAIRS) != 0;
+  a.pair2 = !(cfg->flags & SWITCH_FLAG_GEMM_1SM);
   if (bf16 && (cfg->flags & SWITCH_FLAG_GATHER_COPY)) {
     SMOE_TRY(launch_gather_rows(static_cast<int64_t>(N) * c.C,
                                 static_cast<int64_t>(a.d) * 2, slot_token, x, c.ws + c.L.xdisp,

@@ -25,6 +25,8 @@ FLAG_ROUTER_3TERM = 2
 FLAG_UNFUSED_COMBINE = 4
 FLAG_GATHER_COPY = 8
 FLAG_NO_RESIDUAL = 16
+FLAG_GEMM_1SM = 32
+FLAG_GEMM_PAIRS = 64
 
 
 class SwitchConfig(ctypes.Structure):

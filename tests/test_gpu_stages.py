@@ -207,7 +207,9 @@ FFN_CASES = [
 ]
 
 
-@pytest.mark.parametrize("flags", [0, 8], ids=["gather_in_gemm", "gather_copy"])
+@pytest.mark.parametrize("flags", [0, 8, 32, 40, 64, 72],
+                         ids=["gather_in_gemm", "gather_copy", "one_sm", "one_sm_copy", "pairs",
+                              "pairs_copy"])
 @pytest.mark.parametrize("wl", FFN_CASES, ids=lambda w: w.name)
 def test_expert_ffn(sm, wl, flags):
     inp = make_inputs(wl)
