@@ -278,15 +278,12 @@ def main():
     barrier()
     t_wall1 = time.time()
     ms = [e0.elapsed_time(e1) for e0, e1 in evs]
-    total_ms = torch.tensor([sum(ms)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(total_ms, op=dist.ReduceOp.MAX)
-    total_ms = float(total_ms.item())
+    total_ms = max_over_ranks(sum(ms), dev, world)
     st, where, info = sm.switch_get_device_error(ws)
     if st != 0:
         raise RuntimeError(f"device error {st} at {where} ({info}) in the timed region")
     ms_per_step = total_ms / args.steps
-    value = T * args.steps * world / (total_ms / 1e3)
+    value = job_throughput(T, args.steps, world, total_ms)
 
     # ------------------------------------------- end to end (host buffers)
     x_host = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
@@ -312,10 +309,8 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
-    e2e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-    e2e_value = T * args.steps * world / (float(e2e_ms.item()) / 1e3)
+    e2e_value = job_throughput(T, args.steps, world,
+                               max_over_ranks(e0.elapsed_time(e1), dev, world))
     clocks.stop()
 
     # --------------------------------------- per-kernel roofline (rank 0)
@@ -370,6 +365,22 @@ def main():
         dist.destroy_process_group()
     if line is not None:
         print(json.dumps(line), flush=True)
+
+
+def max_over_ranks(value, device, world):
+    """The largest per-rank value (rank timings are aggregated by their max)."""
+    if world == 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank, steps, world, max_total_ms):
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's time."""
+    return tokens_per_rank * steps * world / (max_total_ms / 1e3)
 
 
 def launches_per_step(cfg, wl):
