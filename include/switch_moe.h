@@ -25,10 +25,10 @@
  *     contiguous, each aligned to at least 16 bytes.  The library never
  *     allocates or frees device memory.
  *   - Scratch lives in a caller-owned device workspace of at least
- *     switch_workspace_size() bytes (256-byte aligned).  Its first 16 bytes
- *     hold the device error word; zero it once after allocating (a
- *     zero-filled allocation is fine).  Calls that share a workspace must be
- *     ordered on one stream.
+ *     switch_workspace_size() bytes (256-byte aligned).  Its first 256 bytes
+ *     hold the device error word and a counter that the calls leave at zero;
+ *     zero them once after allocating (a zero-filled allocation is fine).
+ *     Calls that share a workspace must be ordered on one stream.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream).  Calls are asynchronous on it; nothing synchronises the host
  *     except switch_get_device_error().

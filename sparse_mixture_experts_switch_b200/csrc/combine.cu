@@ -96,40 +96,65 @@ cudaError_t launch_prob_colsum(int64_t T, int N, const float* probs, float* psum
   return cudaGetLastError();
 }
 
-// One block: P_e = (sum_p psum[p][e]) / T in double, fixed order; then a
-// fixed-shape tree over experts for sum_e f_e P_e.
+// Two fixed-order stages in one launch.  Block b owns experts
+// [32 b, 32 b + 32): its 8 warps split the parts, each lane one expert,
+// partial sums in double; the warps' sums are added in warp order.  The
+// last block to finish (a ticket counter decides only *which* block, not
+// any order of additions) forms sum_e f_e P_e in expert order and the loss.
 __global__ void __launch_bounds__(256) aux_loss_kernel(int64_t T, int N, int nparts,
                                                        float alpha,
                                                        const int* __restrict__ counts,
                                                        const float* __restrict__ psum,
                                                        float* __restrict__ loss,
                                                        float* __restrict__ f_out,
-                                                       float* __restrict__ P_out) {
-  __shared__ double red[256];
-  const int tid = threadIdx.x;
-  double acc = 0.0;
-  for (int e = tid; e < N; e += 256) {
-    double s = 0.0;
-    for (int p = 0; p < nparts; ++p) s += static_cast<double>(psum[static_cast<int64_t>(p) * N + e]);
-    const double P = s / static_cast<double>(T);
+                                                       float* __restrict__ P_out,
+                                                       double* __restrict__ fp_scratch,
+                                                       unsigned* __restrict__ ticket) {
+  __shared__ double part[8][32];
+  __shared__ bool last;
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int e = blockIdx.x * 32 + lane;
+  double s = 0.0;
+  if (e < N)
+    for (int pp = w; pp < nparts; pp += 8) s += static_cast<double>(psum[static_cast<int64_t>(pp) * N + e]);
+  part[w][lane] = s;
+  __syncthreads();
+  if (w == 0 && e < N) {
+    double tot = 0.0;
+    for (int q = 0; q < 8; ++q) tot += part[q][lane];
+    const double P = tot / static_cast<double>(T);
     const double f = static_cast<double>(counts[e]) / static_cast<double>(T);
     if (f_out) f_out[e] = static_cast<float>(f);
     if (P_out) P_out[e] = static_cast<float>(P);
-    acc += f * P;
+    fp_scratch[e] = f * P;
   }
-  red[tid] = acc;
+  __threadfence();
   __syncthreads();
-  for (int s = 128; s > 0; s >>= 1) {
-    if (tid < s) red[tid] += red[tid + s];
+  if (threadIdx.x == 0) last = atomicAdd(ticket, 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  // last block: sum over experts in a fixed shape
+  __shared__ double red[256];
+  double acc = 0.0;
+  for (int i = threadIdx.x; i < N; i += 256) acc += const_cast<volatile double*>(fp_scratch)[i];
+  red[threadIdx.x] = acc;
+  __syncthreads();
+  for (int st = 128; st > 0; st >>= 1) {
+    if (threadIdx.x < st) red[threadIdx.x] += red[threadIdx.x + st];
     __syncthreads();
   }
-  if (tid == 0 && loss) *loss = static_cast<float>(static_cast<double>(alpha) * N * red[0]);
+  if (threadIdx.x == 0) {
+    if (loss) *loss = static_cast<float>(static_cast<double>(alpha) * N * red[0]);
+    *ticket = 0;                 // ready for the next call on this workspace
+  }
 }
 
 cudaError_t launch_aux_loss(int64_t T, int N, int nparts, float alpha, const int* counts,
                             const float* psum, float* loss, float* f, float* P,
-                            cudaStream_t st) {
-  aux_loss_kernel<<<1, 256, 0, st>>>(T, N, nparts, alpha, counts, psum, loss, f, P);
+                            double* fp_scratch, unsigned* ticket, cudaStream_t st) {
+  aux_loss_kernel<<<(N + 31) / 32, 256, 0, st>>>(T, N, nparts, alpha, counts, psum, loss, f,
+                                                 P, fp_scratch, ticket);
   return cudaGetLastError();
 }
 

@@ -416,6 +416,26 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
          | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
 }
 
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
+// --------------------------------------------------------------- host side
+
+// Raise a kernel's dynamic shared-memory limit to `bytes`, once per kernel
+// and device (steady-state calls then launch with no extra driver call).
+// `cache` is a per-kernel array of 64 entries, one per device.
+inline cudaError_t ensure_smem_limit(const void* func, size_t bytes, size_t* cache) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < 64 && cache[dev] >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(bytes));
+  if (e == cudaSuccess && dev >= 0 && dev < 64) cache[dev] = bytes;
+  return e;
+}
+
 // ------------------------------------------------------------- numerics
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -296,12 +296,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1) expert_gemm_kernel(
       tc_fence_after();
       int e, m, n;
       decode_tile(tile, mts, p.N, p.ntiles_n, e, m, n);
+      // combine: fetch the next tile's token now, prefetch its residual row
+      // after this tile (the next tile's main loop then hides the latency)
+      int ntok = -1, nn = 0;
+      if (p.mode == kModeCombine) {
+        if (tile == static_cast<int>(blockIdx.x)) prefetch_residual(p, combine_row_token(p, e, m, q, lane), n);
+        const int nt = tile + gridDim.x;
+        if (nt < total) {
+          int e2, m2;
+          decode_tile(nt, mts, p.N, p.ntiles_n, e2, m2, nn);
+          ntok = combine_row_token(p, e2, m2, q, lane);
+        }
+      }
       epilogue_tile(p, e, m, n,
                     tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                         static_cast<uint32_t>(acc * kBN),
                     stg, tokw, q, lane);
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
+      prefetch_residual(p, ntok, nn);
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
@@ -321,9 +334,8 @@ template <bool kGather>
 static cudaError_t run_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& gp,
                             int num_sms, cudaStream_t st) {
   const size_t smem = gemm_smem_bytes(gp.N);
-  cudaError_t e = cudaFuncSetAttribute(expert_gemm_kernel<kGather>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  static size_t smem_set[64] = {};
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(&expert_gemm_kernel<kGather>), smem, smem_set);
   if (e != cudaSuccess) return e;
   expert_gemm_kernel<kGather><<<num_sms, kGemmThreads, smem, st>>>(ta, tb, gp);
   return cudaGetLastError();

@@ -303,7 +303,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       int e, mp, n;
       decode_tile(tile, pts, p.N, p.ntiles_n, e, mp, n);
-      epilogue_tile(p, e, 2 * mp + static_cast<int>(rank), n,
+      const int m = 2 * mp + static_cast<int>(rank);
+      // combine: fetch the next tile's token now, prefetch its residual row
+      // after this tile (the next tile's main loop then hides the latency)
+      int ntok = -1, nn = 0;
+      if (p.mode == kModeCombine) {
+        if (tile == cid) prefetch_residual(p, combine_row_token(p, e, m, q, lane), n);
+        const int nt = tile + ncl;
+        if (nt < total) {
+          int e2, mp2;
+          decode_tile(nt, pts, p.N, p.ntiles_n, e2, mp2, nn);
+          ntok = combine_row_token(p, e2, 2 * mp2 + static_cast<int>(rank), q, lane);
+        }
+      }
+      epilogue_tile(p, e, m, n,
                     tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                         static_cast<uint32_t>(acc * kBN),
                     stg, tokw, q, lane);
@@ -313,6 +326,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         if (leader) mbar_arrive(&tempty[acc]);
         else mbar_arrive_remote(tempty_lead + 8u * acc);
       }
+      prefetch_residual(p, ntok, nn);
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
@@ -333,9 +347,8 @@ template <bool kGather>
 cudaError_t run_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& gp,
                           int num_sms, cudaStream_t st) {
   const size_t smem = gemm_pair_smem_bytes(gp.N);
-  cudaError_t e = cudaFuncSetAttribute(expert_gemm_pair_kernel<kGather>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  static size_t smem_set[64] = {};
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(&expert_gemm_pair_kernel<kGather>), smem, smem_set);
   if (e != cudaSuccess) return e;
   const int grid = (num_sms / 2) * 2;
   expert_gemm_pair_kernel<kGather><<<grid, kGemmThreads, smem, st>>>(ta, tb, gp);

@@ -65,6 +65,24 @@ __device__ __forceinline__ int64_t kept_rows(const GemmParams& p, int e) {
 }
 
 
+// Combine epilogue: the token whose row this thread drains in a given tile
+// (row m * 128 + q * 32 + lane of expert e), or -1.
+__device__ __forceinline__ int combine_row_token(const GemmParams& p, int e, int m, int q,
+                                                 int lane) {
+  const int64_t r = static_cast<int64_t>(m) * kBM + q * 32 + lane;
+  return r < kept_rows(p, e) ? p.slot_token[static_cast<int64_t>(e) * p.C + r] : -1;
+}
+
+// Pull a token's residual row segment (256 columns of x) into L2 ahead of
+// the tile that adds it, so the epilogue's reads do not wait on DRAM.
+__device__ __forceinline__ void prefetch_residual(const GemmParams& p, int tok, int n) {
+  if (tok < 0 || p.x_res == nullptr) return;
+  const char* base = reinterpret_cast<const char*>(p.x_res + static_cast<int64_t>(tok) * p.n_out +
+                                                   n * kBN);
+  const int bytes = (p.n_out - n * kBN < kBN ? p.n_out - n * kBN : kBN) * 2;
+  for (int off = 0; off < bytes; off += 128) prefetch_l2(base + off);
+}
+
 // Epilogue of one tile for the calling warp (quarter q of the accumulator's
 // 128 TMEM lanes: rows m * 128 + q * 32 + lane of expert e).  Each thread
 // owns one accumulator row; per 32-column chunk the row's values (ReLU'd,

@@ -42,9 +42,10 @@ cudaError_t launch_combine(int64_t T, int d, int64_t C, bool bf16, const void* x
 cudaError_t launch_prob_colsum(int64_t T, int N, const float* probs, float* psum,
                                cudaStream_t st);
 // loss = alpha * N * sum_e (counts_e / T) * (sum_p psum[p][e] / T).
+// fp_scratch: [N] doubles; ticket: one zero-initialised counter (left zero).
 cudaError_t launch_aux_loss(int64_t T, int N, int nparts, float alpha, const int* counts,
                             const float* psum, float* loss, float* f, float* P,
-                            cudaStream_t st);
+                            double* fp_scratch, unsigned* ticket, cudaStream_t st);
 
 // ---------------------------------------------------------------- router
 struct RouterOut {

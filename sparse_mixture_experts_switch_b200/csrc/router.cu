@@ -533,9 +533,8 @@ template <int NCH, int TERMS>
 static cudaError_t run_router_tc_t(const CUtensorMap& tx, const CUtensorMap& tw,
                                    const RouterTcParams& p, size_t smem, int grid,
                                    cudaStream_t st) {
-  cudaError_t e = cudaFuncSetAttribute(router_tc_kernel<NCH, TERMS>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  static size_t smem_set[64] = {};
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(&router_tc_kernel<NCH, TERMS>), smem, smem_set);
   if (e != cudaSuccess) return e;
   router_tc_kernel<NCH, TERMS><<<grid, kRouterThreads, smem, st>>>(tx, tw, p);
   return cudaGetLastError();

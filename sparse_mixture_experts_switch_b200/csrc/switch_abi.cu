@@ -38,9 +38,13 @@ int64_t capacity_exact(int64_t T, int32_t N, double cf) {
 }
 
 struct Layout {
-  size_t err, hist, base, psum, local_rank, idx, gate, rank, drop, counts, slot_token,
+  size_t err, hist, base, psum, fpsc, local_rank, idx, gate, rank, drop, counts, slot_token,
       mtile_start, wsplit, logits, xdisp, hbuf, ybuf, total;
 };
+
+// Bytes 16..19 of the workspace: the loss kernel's completion ticket (kept
+// at zero between calls, like the error word in bytes 0..15).
+constexpr size_t kTicketOffset = 16;
 
 int ntiles_of(int64_t T) { return static_cast<int>((T + kTileTok - 1) / kTileTok); }
 
@@ -62,6 +66,7 @@ Layout layout_for(const switch_config_t& c, int64_t C) {
   L.hist = take(sizeof(int) * N * nt);
   L.base = take(sizeof(int) * N * nt);
   L.psum = take(sizeof(float) * N * nparts);
+  L.fpsc = take(sizeof(double) * N);
   L.local_rank = take(sizeof(int) * T);
   L.idx = take(sizeof(int) * T);
   L.gate = take(sizeof(float) * T);
@@ -293,7 +298,8 @@ switch_status_t switch_aux_loss(const switch_config_t* cfg, const int32_t* count
   float* psum = c.at<float>(c.L.psum);
   SMOE_TRY(launch_prob_colsum(cfg->T, cfg->n_experts, probs, psum, c.st));
   return cuda_status(launch_aux_loss(cfg->T, cfg->n_experts, ntiles_of(cfg->T), cfg->alpha,
-                                     counts, psum, loss, f, P, c.st));
+                                     counts, psum, loss, f, P, c.at<double>(c.L.fpsc),
+                                     c.at<unsigned>(kTicketOffset), c.st));
 }
 
 switch_status_t switch_layer_forward(const switch_config_t* cfg, const void* x,
@@ -377,7 +383,7 @@ switch_status_t switch_layer_forward(const switch_config_t* cfg, const void* x,
   // 6. load-balancing loss
   if (loss)
     SMOE_TRY(launch_aux_loss(T, N, nparts, cfg->alpha, counts_p, psum, loss, nullptr, nullptr,
-                             c.st));
+                             c.at<double>(c.L.fpsc), c.at<unsigned>(kTicketOffset), c.st));
   return SWITCH_OK;
 }
 
