@@ -409,12 +409,10 @@ def job_throughput(tokens_per_rank, steps, world, max_total_ms):
 
 def launches_per_step(cfg, wl):
     """Kernels switch_layer_forward launches with the default flags on this
-    workload: router (weight split + tensor-core router), scan, finalize,
-    GEMM1, GEMM2, dropped-token copy, loss."""
-    tc = wl.dtype == "bf16" and (wl.n_experts + 15) // 16 * 16 <= 256
-    if tc:
-        return 8
-    return 8   # SIMT router + tile ranks replace the two router launches
+    workload: router (weight split + tensor-core router, or SIMT router +
+    tile ranks), scan, finalize, the row copy (bf16), GEMM1, GEMM2, the
+    dropped-token copy and the loss."""
+    return 2 + 2 + (1 if wl.dtype == "bf16" else 0) + 2 + 1 + 1
 
 
 def kernel_rooflines(sm, cfg, wl, C, x, w_r, b_r, w1, w2, ws, flush, stream, dev, pk, pk_kind,
@@ -460,7 +458,10 @@ def kernel_rooflines(sm, cfg, wl, C, x, w_r, b_r, w1, w2, ws, flush, stream, dev
                                                 x_disp, ws))
     cnt = counts.cpu().numpy().astype(np.int64)
     T_kept = int(np.minimum(cnt, C).sum())
-    t_ffn = timed(lambda: sm.switch_expert_ffn(cfg, x, slot, counts, w1, w2, y, ws))
+    # GEMM1 + GEMM2 alone: the rows dispatch_gather laid out, fed straight in
+    cfg_rows = sm.config(T, d, F, N, wl.capacity_factor, dtype=wl.dtype, alpha=wl.alpha,
+                         flags=sm.FLAG_ROWS_DISPATCHED)
+    t_ffn = timed(lambda: sm.switch_expert_ffn(cfg_rows, x_disp, None, counts, w1, w2, y, ws))
     t_comb = timed(lambda: sm.switch_combine(cfg, x, idx, rank, drop, gate, y, out))
     t_aux = timed(lambda: sm.switch_aux_loss(cfg, counts, probs, loss, None, None, ws))
     st, where, info = sm.switch_get_device_error(ws)

@@ -75,11 +75,15 @@ enum {
   SWITCH_FLAG_ROUTER_SIMT = 1,       /* CUDA-core fp32 FMA router */
   SWITCH_FLAG_ROUTER_3TERM = 2,      /* tensor-core router, W_r split in 3 bf16 terms (default 2) */
   SWITCH_FLAG_UNFUSED_COMBINE = 4,   /* forward: write Y, then a separate combine kernel */
-  SWITCH_FLAG_GATHER_COPY = 8,       /* forward: copy routed rows to x_disp before GEMM1 */
+  SWITCH_FLAG_GATHER_IN_GEMM = 8,    /* bf16 expert FFN: GEMM1 gathers the routed rows of x
+                                        itself (default: one copy kernel first lays them out
+                                        expert by expert, then GEMM1 reads tiles by TMA) */
   SWITCH_FLAG_NO_RESIDUAL = 16,      /* forward: block output is y alone (dropped -> 0) */
   SWITCH_FLAG_GEMM_1SM = 32,         /* both expert GEMMs on single CTAs */
-  SWITCH_FLAG_GEMM_PAIRS = 64        /* GEMM1 on CTA pairs too (default: GEMM1 single CTAs,
+  SWITCH_FLAG_GEMM_PAIRS = 64,       /* GEMM1 on CTA pairs too (default: GEMM1 single CTAs,
                                         GEMM2 CTA pairs) */
+  SWITCH_FLAG_ROWS_DISPATCHED = 128  /* switch_expert_ffn: x is the dispatched row buffer
+                                        x_disp [N*C, d_model] from switch_dispatch */
 };
 
 typedef struct {
@@ -169,6 +173,9 @@ switch_status_t switch_dispatch_noalloc(const switch_config_t* cfg, const int32_
  * for r < n_e = min(counts[e], C).  Rows r >= n_e of y are left untouched.
  *   x [T, d_model], w1 [N, d_ff, d_model], w2 [N, d_model, d_ff],
  *   y [N, C, d_model]; slot_token [N*C], counts [N] as from switch_dispatch.
+ * With SWITCH_FLAG_ROWS_DISPATCHED, x is instead the dispatched buffer
+ * x_disp [N*C, d_model] (row e*C + r = x[slot_token[e*C + r]]) that
+ * switch_dispatch writes; slot_token is then not read (may be NULL).
  * bf16: tcgen05 grouped GEMM, fp32 accumulation, the hidden activation is
  * rounded once to bf16, y rounded once to bf16.  fp32: CUDA-core FMA. */
 switch_status_t switch_expert_ffn(const switch_config_t* cfg, const void* x,

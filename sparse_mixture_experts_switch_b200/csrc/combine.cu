@@ -96,11 +96,13 @@ cudaError_t launch_prob_colsum(int64_t T, int N, const float* probs, float* psum
   return cudaGetLastError();
 }
 
-// Two fixed-order stages in one launch.  Block b owns experts
-// [32 b, 32 b + 32): its 8 warps split the parts, each lane one expert,
-// partial sums in double; the warps' sums are added in warp order.  The
-// last block to finish (a ticket counter decides only *which* block, not
-// any order of additions) forms sum_e f_e P_e in expert order and the loss.
+// Two fixed-order stages in one launch.  Block (bx, by) owns experts
+// [32 bx, 32 bx + 32) and the by-th of kAuxChunks equal runs of parts: its 8
+// warps split the run, each lane one expert, partial sums in double, the
+// warps' sums added in warp order into part_sum[by][e].  The last block to
+// finish (a ticket counter decides only *which* block, not any order of
+// additions) adds the runs in order, forms f_e P_e and sums over experts in
+// a fixed tree.
 __global__ void __launch_bounds__(256) aux_loss_kernel(int64_t T, int N, int nparts,
                                                        float alpha,
                                                        const int* __restrict__ counts,
@@ -108,36 +110,44 @@ __global__ void __launch_bounds__(256) aux_loss_kernel(int64_t T, int N, int npa
                                                        float* __restrict__ loss,
                                                        float* __restrict__ f_out,
                                                        float* __restrict__ P_out,
-                                                       double* __restrict__ fp_scratch,
+                                                       double* __restrict__ part_sum,
                                                        unsigned* __restrict__ ticket) {
   __shared__ double part[8][32];
+  __shared__ double red[256];
   __shared__ bool last;
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int e = blockIdx.x * 32 + lane;
+  const int per = (nparts + gridDim.y - 1) / gridDim.y;
+  const int p0 = blockIdx.y * per;
+  const int p1 = p0 + per < nparts ? p0 + per : nparts;
   double s = 0.0;
   if (e < N)
-    for (int pp = w; pp < nparts; pp += 8) s += static_cast<double>(psum[static_cast<int64_t>(pp) * N + e]);
+    for (int pp = p0 + w; pp < p1; pp += 8)
+      s += static_cast<double>(psum[static_cast<int64_t>(pp) * N + e]);
   part[w][lane] = s;
   __syncthreads();
   if (w == 0 && e < N) {
     double tot = 0.0;
     for (int q = 0; q < 8; ++q) tot += part[q][lane];
-    const double P = tot / static_cast<double>(T);
-    const double f = static_cast<double>(counts[e]) / static_cast<double>(T);
-    if (f_out) f_out[e] = static_cast<float>(f);
-    if (P_out) P_out[e] = static_cast<float>(P);
-    fp_scratch[e] = f * P;
+    part_sum[static_cast<int64_t>(blockIdx.y) * N + e] = tot;
   }
   __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) last = atomicAdd(ticket, 1u) == gridDim.x - 1;
+  if (threadIdx.x == 0) last = atomicAdd(ticket, 1u) == gridDim.x * gridDim.y - 1;
   __syncthreads();
   if (!last) return;
   __threadfence();
-  // last block: sum over experts in a fixed shape
-  __shared__ double red[256];
   double acc = 0.0;
-  for (int i = threadIdx.x; i < N; i += 256) acc += const_cast<volatile double*>(fp_scratch)[i];
+  for (int i = threadIdx.x; i < N; i += 256) {
+    double tot = 0.0;
+    for (unsigned c = 0; c < gridDim.y; ++c)
+      tot += const_cast<volatile double*>(part_sum)[static_cast<int64_t>(c) * N + i];
+    const double P = tot / static_cast<double>(T);
+    const double f = static_cast<double>(counts[i]) / static_cast<double>(T);
+    if (f_out) f_out[i] = static_cast<float>(f);
+    if (P_out) P_out[i] = static_cast<float>(P);
+    acc += f * P;
+  }
   red[threadIdx.x] = acc;
   __syncthreads();
   for (int st = 128; st > 0; st >>= 1) {
@@ -152,9 +162,11 @@ __global__ void __launch_bounds__(256) aux_loss_kernel(int64_t T, int N, int npa
 
 cudaError_t launch_aux_loss(int64_t T, int N, int nparts, float alpha, const int* counts,
                             const float* psum, float* loss, float* f, float* P,
-                            double* fp_scratch, unsigned* ticket, cudaStream_t st) {
-  aux_loss_kernel<<<(N + 31) / 32, 256, 0, st>>>(T, N, nparts, alpha, counts, psum, loss, f,
-                                                 P, fp_scratch, ticket);
+                            double* part_sum, unsigned* ticket, cudaStream_t st) {
+  const int chunks = nparts < kAuxChunks ? (nparts > 0 ? nparts : 1) : kAuxChunks;
+  const dim3 grid(static_cast<unsigned>((N + 31) / 32), static_cast<unsigned>(chunks));
+  aux_loss_kernel<<<grid, 256, 0, st>>>(T, N, nparts, alpha, counts, psum, loss, f, P,
+                                        part_sum, ticket);
   return cudaGetLastError();
 }
 

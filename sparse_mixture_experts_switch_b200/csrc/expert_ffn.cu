@@ -53,10 +53,10 @@ PFN_encodeTiled get_encode_fn() {
   return fn;
 }
 
-// 2-D bf16 tensor [outer, inner] (inner contiguous), 128-byte swizzle,
-// out-of-range elements read as zero.
+// 2-D bf16 tensor [outer, inner] (inner contiguous), 128-byte swizzle by
+// default; out-of-range elements read as zero and are never written.
 bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
-                       uint32_t box_inner, uint32_t box_outer) {
+                       uint32_t box_inner, uint32_t box_outer, bool swizzle64) {
   PFN_encodeTiled enc = get_encode_fn();
   if (enc == nullptr) return false;
   const cuuint64_t dims[2] = {inner, outer};
@@ -64,7 +64,8 @@ bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint6
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t estr[2] = {1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
-             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             swizzle64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -77,14 +78,15 @@ constexpr uint32_t kStageBytes = kABytes + kBBytes;     // 48 KB
 template <bool kGather>
 __global__ void __launch_bounds__(kGemmThreads, 1) expert_gemm_kernel(
     const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-    GemmParams p) {
+    const __grid_constant__ CUtensorMap tmap_out, GemmParams p) {
   const int total = p.mtile_start[p.N] * p.ntiles_n;
   if (static_cast<int>(blockIdx.x) >= total) return;    // uniform for the block
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-  uint8_t* tail = smem + kStages * kStageBytes;
+  uint8_t* stage_out = smem + kStages * kStageBytes;                 // [4][4 KB], 1024-aligned
+  uint8_t* tail = stage_out + 4 * kStageOutBytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(tail);
   uint64_t* empty = full + kStages;
   uint64_t* tfull = empty + kStages;
@@ -93,8 +95,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) expert_gemm_kernel(
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   int* tok_s = reinterpret_cast<int*>(tail + 128);                    // [4][32]
-  uint8_t* stage_out = tail + 128 + 4 * 32 * 4;                       // [4][32 x 32 fp32]
-  int* mts = reinterpret_cast<int*>(stage_out + 4 * kStageOutBytes);  // [N + 1]
+  int* mts = reinterpret_cast<int*>(tail + 128 + 4 * 32 * 4);         // [N + 1]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long lim = p.spin;
@@ -283,6 +284,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) expert_gemm_kernel(
     int* tokw = tok_s + q * 32;
     int acc = 0;
     uint32_t acc_phase = 0;
+    if (lane == 0 && p.mode != kModeCombine) tma_prefetch_desc(&tmap_out);
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
       // warp-uniform outcome: the TMEM loads below are warp-collective
       const bool ok = __all_sync(0xffffffffu, mbar_wait_sleepy(&tfull[acc], acc_phase, lim));
@@ -308,7 +310,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) expert_gemm_kernel(
           ntok = combine_row_token(p, e2, m2, q, lane);
         }
       }
-      epilogue_tile(p, e, m, n,
+      epilogue_tile(p, &tmap_out, e, m, n,
                     tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                         static_cast<uint32_t>(acc * kBN),
                     stg, tokw, q, lane);
@@ -318,6 +320,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) expert_gemm_kernel(
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
+    if (lane == 0) bulk_wait_all();        // boxes stored from shared memory are written
   }
 
   tc_fence_before();
@@ -331,19 +334,19 @@ static size_t gemm_smem_bytes(int N) {
 }
 
 template <bool kGather>
-static cudaError_t run_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& gp,
-                            int num_sms, cudaStream_t st) {
+static cudaError_t run_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to,
+                            const GemmParams& gp, int num_sms, cudaStream_t st) {
   const size_t smem = gemm_smem_bytes(gp.N);
   static size_t smem_set[64] = {};
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(&expert_gemm_kernel<kGather>), smem, smem_set);
   if (e != cudaSuccess) return e;
-  expert_gemm_kernel<kGather><<<num_sms, kGemmThreads, smem, st>>>(ta, tb, gp);
+  expert_gemm_kernel<kGather><<<num_sms, kGemmThreads, smem, st>>>(ta, tb, to, gp);
   return cudaGetLastError();
 }
 
 cudaError_t launch_expert_ffn_bf16(const FfnArgs& a, cudaStream_t st) {
   const uint64_t slots = static_cast<uint64_t>(a.N) * static_cast<uint64_t>(a.C);
-  CUtensorMap ta1, tb1, ta2, tb2;
+  CUtensorMap ta1, tb1, ta2, tb2, to1, to2;
   const bool gather = a.x_disp == nullptr;
   // CTA pairs load half a weight tile each (128 rows); single CTAs all 256.
   const uint32_t b_rows1 = a.pair1 ? 128u : static_cast<uint32_t>(kBN);
@@ -356,6 +359,12 @@ cudaError_t launch_expert_ffn_bf16(const FfnArgs& a, cudaStream_t st) {
   ok = ok && make_tmap_bf16_2d(&tb1, a.w1, a.d, static_cast<uint64_t>(a.N) * a.F, kBK, b_rows1);
   ok = ok && make_tmap_bf16_2d(&ta2, a.hbuf, a.F, slots, kBK, kBM);
   ok = ok && make_tmap_bf16_2d(&tb2, a.w2, a.F, static_cast<uint64_t>(a.N) * a.d, kBK, b_rows2);
+  // epilogue boxes: 32 rows x 32 columns of H (GEMM1) or Y (GEMM2, unfused)
+  ok = ok && make_tmap_bf16_2d(&to1, a.hbuf, a.F, slots, 32, 32, true);
+  if (a.mode2 == kModeY)
+    ok = ok && make_tmap_bf16_2d(&to2, a.y, a.d, slots, 32, 32, true);
+  else
+    memset(&to2, 0, sizeof(to2));          // unused: the combine scatters rows by token
   if (!ok) return cudaErrorInvalidValue;
 
   GemmParams g1{};
@@ -375,11 +384,11 @@ cudaError_t launch_expert_ffn_bf16(const FfnArgs& a, cudaStream_t st) {
   g1.spin = a.spin;
   cudaError_t e;
   if (a.pair1)
-    e = gather ? run_gemm_pair<true>(ta1, tb1, g1, a.num_sms, st)
-               : run_gemm_pair<false>(ta1, tb1, g1, a.num_sms, st);
+    e = gather ? run_gemm_pair<true>(ta1, tb1, to1, g1, a.num_sms, st)
+               : run_gemm_pair<false>(ta1, tb1, to1, g1, a.num_sms, st);
   else
-    e = gather ? run_gemm<true>(ta1, tb1, g1, a.num_sms, st)
-               : run_gemm<false>(ta1, tb1, g1, a.num_sms, st);
+    e = gather ? run_gemm<true>(ta1, tb1, to1, g1, a.num_sms, st)
+               : run_gemm<false>(ta1, tb1, to1, g1, a.num_sms, st);
   if (e != cudaSuccess) return e;
 
   GemmParams g2 = g1;
@@ -393,8 +402,8 @@ cudaError_t launch_expert_ffn_bf16(const FfnArgs& a, cudaStream_t st) {
   g2.x_res = static_cast<const __nv_bfloat16*>(a.x_res);
   g2.gate = a.gate;
   g2.comb_out = static_cast<__nv_bfloat16*>(a.out);
-  return a.pair2 ? run_gemm_pair<false>(ta2, tb2, g2, a.num_sms, st)
-                : run_gemm<false>(ta2, tb2, g2, a.num_sms, st);
+  return a.pair2 ? run_gemm_pair<false>(ta2, tb2, to2, g2, a.num_sms, st)
+                : run_gemm<false>(ta2, tb2, to2, g2, a.num_sms, st);
 }
 
 // ===================================================== fp32 CUDA cores
@@ -473,8 +482,10 @@ __global__ void __launch_bounds__(256) ffn_simt_kernel(
 cudaError_t launch_expert_ffn_f32(const FfnArgs& a, cudaStream_t st) {
   const dim3 g1(static_cast<unsigned>((a.C + kSB - 1) / kSB),
                 static_cast<unsigned>((a.F + kSB - 1) / kSB), static_cast<unsigned>(a.N));
+  // token rows gathered through slot_token, or already dispatched
+  const bool gather = a.x_disp == nullptr;
   ffn_simt_kernel<<<g1, 256, 0, st>>>(kModeHidden, a.C, a.F, a.d, a.counts, a.slot_token,
-                                      static_cast<const float*>(a.x), true,
+                                      static_cast<const float*>(gather ? a.x : a.x_disp), gather,
                                       static_cast<const float*>(a.w1),
                                       static_cast<float*>(a.hbuf), nullptr, nullptr);
   cudaError_t e = cudaGetLastError();

@@ -7,9 +7,6 @@
 
 namespace smoe {
 
-bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
-                       uint32_t box_inner, uint32_t box_outer);
-
 // ------------------------------------------------------------- tile list
 
 // Tile t belongs to the expert e with mts[e] * ntn <= t < mts[e + 1] * ntn
@@ -39,7 +36,7 @@ constexpr int kGatherWarps = 4;
 constexpr int kGatherLanes = 32 * kGatherWarps;
 constexpr uint32_t kTmemCols = 512;                     // 2 accumulators x 256
 constexpr uint32_t kStageOutBytes = 32 * 32 * 4;        // per epilogue warp: 32 rows x 32 fp32
-constexpr uint32_t kTailBytes = 128 + 4 * 32 * 4 + 4 * kStageOutBytes;   // + mts[N + 1]
+constexpr uint32_t kTailBytes = 4 * kStageOutBytes + 128 + 4 * 32 * 4;   // + mts[N + 1]
 
 struct GemmParams {
   int N, n_out, K, ntiles_n;
@@ -85,33 +82,71 @@ __device__ __forceinline__ void prefetch_residual(const GemmParams& p, int tok, 
 
 // Epilogue of one tile for the calling warp (quarter q of the accumulator's
 // 128 TMEM lanes: rows m * 128 + q * 32 + lane of expert e).  Each thread
-// owns one accumulator row; per 32-column chunk the row's values (ReLU'd,
-// or scaled by its gate) go through the warp's shared buffer `stg` so that
-// global stores are written 8 rows x 64 bytes per instruction.
-__device__ __forceinline__ void epilogue_tile(const GemmParams& p, int e, int m, int n,
-                                              uint32_t taddr, uint32_t stg, int* tokw, int q,
-                                              int lane) {
+// owns one accumulator row.  The 32-column chunks are read from TMEM one
+// ahead of their use, so a chunk's load is in flight while the previous one
+// is stored.  Two store paths, both through the warp's 4 KB shared buffer
+// `stg` (1024-byte aligned):
+//   * hidden / Y rows, when all 32 rows of the quarter hold tokens: ReLU (or
+//     nothing) + bf16 into a 32 x 32 box in the 64-byte-swizzled layout,
+//     written out by one TMA store per chunk (two boxes alternate);
+//   * otherwise (combine, or a quarter with padding rows): fp32 values are
+//     transposed through the buffer so that each global store instruction
+//     writes 8 rows x 64 bytes, rows past the expert's count skipped; the
+//     combine adds the residual row and scales by the token's gate.
+__device__ __forceinline__ void epilogue_tile(const GemmParams& p, const CUtensorMap* tmap_out,
+                                              int e, int m, int n, uint32_t taddr, uint32_t stg,
+                                              int* tokw, int q, int lane) {
   const int qq = lane & 3;          // 8-column group in the transposed pass
   const int rr0 = lane >> 2;        // row within an 8-row pass
   const int64_t n_e = kept_rows(p, e);
   const int64_t rbase = static_cast<int64_t>(m) * kBM + q * 32;   // first row of this warp
   const bool valid = rbase + lane < n_e;
+  const bool bulk = p.mode != kModeCombine && rbase + 32 <= n_e;
+  const int nch = (p.n_out - n * kBN < kBN ? p.n_out - n * kBN : kBN) / 32;   // even: n_out % 64 == 0
   float g = 1.f;
   if (p.mode == kModeCombine) {
     const int tk = valid ? p.slot_token[static_cast<int64_t>(e) * p.C + rbase + lane] : 0;
     g = valid ? p.gate[tk] : 0.f;
     tokw[lane] = tk;
   }
+  if (!bulk && p.mode != kModeCombine) {
+    if (lane == 0) bulk_wait_read<0>();      // earlier boxes have left the buffer
+  }
   __syncwarp();
-#pragma unroll 1
-  for (int c = 0; c < kBN / 32; ++c) {
-    float v[32];
-    tmem_ld32(taddr + c * 32, v);
-    const int col0 = n * kBN + c * 32;
-    if (col0 >= p.n_out) continue;     // uniform across the warp
+  const int box_row = static_cast<int>(static_cast<int64_t>(e) * p.C + rbase);
+  const uint32_t swz = static_cast<uint32_t>((lane >> 1) & 3);
+
+  auto chunk_bulk = [&](int c, const uint32_t* v) {
+    uint32_t pk[16];
 #pragma unroll
-    for (int j = 0; j < 32; ++j)
-      v[j] = p.mode == kModeHidden ? fmaxf(v[j], 0.f) : (p.mode == kModeCombine ? g * v[j] : v[j]);
+    for (int j = 0; j < 16; ++j) {
+      float a = __uint_as_float(v[2 * j]), b = __uint_as_float(v[2 * j + 1]);
+      if (p.mode == kModeHidden) { a = fmaxf(a, 0.f); b = fmaxf(b, 0.f); }
+      pk[j] = pack_bf16x2(a, b);
+    }
+    const uint32_t buf = stg + static_cast<uint32_t>(c & 1) * 2048u;
+    if (lane == 0) bulk_wait_read<1>();      // the box stored from `buf` two chunks ago is out
+    __syncwarp();
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      st_shared_v4u(buf + lane * 64 + ((static_cast<uint32_t>(k) ^ swz) << 4), pk[4 * k],
+                    pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(tmap_out, buf, n * kBN + c * 32, box_row);
+      bulk_commit();
+    }
+  };
+
+  auto chunk_lsu = [&](int c, const uint32_t* u) {
+    const int col0 = n * kBN + c * 32;
+    float v[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const float a = __uint_as_float(u[j]);
+      v[j] = p.mode == kModeHidden ? fmaxf(a, 0.f) : (p.mode == kModeCombine ? g * a : a);
+    }
 #pragma unroll
     for (int k = 0; k < 8; ++k)
       st_shared_v4(stg + lane * 128 + ((k ^ (lane & 7)) << 4), v[4 * k], v[4 * k + 1],
@@ -146,12 +181,25 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, int e, int m,
       }
     }
     __syncwarp();
+  };
+
+  // Chunk c + 1 is loaded while chunk c is stored (nch is even).
+  uint32_t ra[32], rb[32];
+  tmem_ld32_issue(taddr, ra);
+#pragma unroll 1
+  for (int c = 0; c < nch; c += 2) {
+    tmem_ld_wait(ra);
+    tmem_ld32_issue(taddr + static_cast<uint32_t>((c + 1) * 32), rb);
+    if (bulk) chunk_bulk(c, ra); else chunk_lsu(c, ra);
+    tmem_ld_wait(rb);
+    if (c + 2 < nch) tmem_ld32_issue(taddr + static_cast<uint32_t>((c + 2) * 32), ra);
+    if (bulk) chunk_bulk(c + 1, rb); else chunk_lsu(c + 1, rb);
   }
 }
 
 // CTA-pair kernel launcher (expert_ffn_pair.cu).
 template <bool kGather>
-cudaError_t run_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& gp,
-                          int num_sms, cudaStream_t st);
+cudaError_t run_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to,
+                          const GemmParams& gp, int num_sms, cudaStream_t st);
 
 }  // namespace smoe

@@ -42,10 +42,12 @@ cudaError_t launch_combine(int64_t T, int d, int64_t C, bool bf16, const void* x
 cudaError_t launch_prob_colsum(int64_t T, int N, const float* probs, float* psum,
                                cudaStream_t st);
 // loss = alpha * N * sum_e (counts_e / T) * (sum_p psum[p][e] / T).
-// fp_scratch: [N] doubles; ticket: one zero-initialised counter (left zero).
+// part_sum: [kAuxChunks][N] doubles; ticket: one zero-initialised counter
+// (left zero).
+constexpr int kAuxChunks = 16;
 cudaError_t launch_aux_loss(int64_t T, int N, int nparts, float alpha, const int* counts,
                             const float* psum, float* loss, float* f, float* P,
-                            double* fp_scratch, unsigned* ticket, cudaStream_t st);
+                            double* part_sum, unsigned* ticket, cudaStream_t st);
 
 // ---------------------------------------------------------------- router
 struct RouterOut {
@@ -70,6 +72,11 @@ cudaError_t launch_router_tc(int64_t T, int d, int N, int terms, const void* x,
 bool router_tc_supported(int N, int d, int terms);
 // Bytes of the bf16 split-weight scratch launch_router_tc needs (3 terms).
 size_t router_wsplit_bytes(int N, int d);
+
+// 2-D bf16 TMA descriptor (expert_ffn.cu): [outer, inner], box
+// box_outer x box_inner, 128-byte swizzle (64-byte when swizzle64).
+bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                       uint32_t box_inner, uint32_t box_outer, bool swizzle64 = false);
 
 // ------------------------------------------------------------ expert FFN
 enum GemmMode : int { kModeHidden = 0, kModeY = 1, kModeCombine = 2 };

@@ -514,8 +514,6 @@ typedef CUresult (*PFN_encodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_
 
 PFN_encodeTiled get_encode_fn();   // defined in expert_ffn.cu
 
-bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
-                       uint32_t box_inner, uint32_t box_outer);   // expert_ffn.cu
 
 static int router_n_pad(int N) { return (N + 31) / 32 * 32; }
 

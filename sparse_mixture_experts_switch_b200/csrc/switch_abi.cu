@@ -66,7 +66,7 @@ Layout layout_for(const switch_config_t& c, int64_t C) {
   L.hist = take(sizeof(int) * N * nt);
   L.base = take(sizeof(int) * N * nt);
   L.psum = take(sizeof(float) * N * nparts);
-  L.fpsc = take(sizeof(double) * N);
+  L.fpsc = take(sizeof(double) * N * kAuxChunks);
   L.local_rank = take(sizeof(int) * T);
   L.idx = take(sizeof(int) * T);
   L.gate = take(sizeof(float) * T);
@@ -240,8 +240,9 @@ switch_status_t switch_expert_ffn(const switch_config_t* cfg, const void* x,
   Ctx c{};
   switch_status_t s = prepare(cfg, ws, ws_bytes, stream, &c);
   if (s != SWITCH_OK || cfg->T == 0) return s;
-  if (!x || !slot_token || !counts || !w1 || !w2 || !y || !aligned16(x) || !aligned16(w1) ||
-      !aligned16(w2) || !aligned16(y))
+  const bool dispatched = (cfg->flags & SWITCH_FLAG_ROWS_DISPATCHED) != 0;
+  if (!x || (!slot_token && !dispatched) || !counts || !w1 || !w2 || !y || !aligned16(x) ||
+      !aligned16(w1) || !aligned16(w2) || !aligned16(y))
     return SWITCH_ERR_INVALID_ARG;
   FfnArgs a{};
   a.T = cfg->T;
@@ -263,9 +264,13 @@ switch_status_t switch_expert_ffn(const switch_config_t* cfg, const void* x,
   a.num_sms = c.num_sms;
   a.pair1 = (cfg->flags & SWITCH_FLAG_GEMM_PAIRS) != 0;
   a.pair2 = !(cfg->flags & SWITCH_FLAG_GEMM_1SM);
+  if (dispatched) {
+    a.x = nullptr;
+    a.x_disp = x;
+  }
   if (cfg->dtype == SWITCH_F32) return cuda_status(launch_expert_ffn_f32(a, c.st));
   SMOE_TRY(launch_mtile_table(a.N, a.C, counts, c.at<int>(c.L.mtile_start), c.st));
-  if (cfg->flags & SWITCH_FLAG_GATHER_COPY) {
+  if (!dispatched && !(cfg->flags & SWITCH_FLAG_GATHER_IN_GEMM)) {
     SMOE_TRY(launch_gather_rows(static_cast<int64_t>(a.N) * a.C,
                                 static_cast<int64_t>(a.d) * 2, slot_token, x,
                                 c.ws + c.L.xdisp, c.st));
@@ -370,7 +375,7 @@ switch_status_t switch_layer_forward(const switch_config_t* cfg, const void* x,
   a.num_sms = c.num_sms;
   a.pair1 = (cfg->flags & SWITCH_FLAG_GEMM_PAIRS) != 0;
   a.pair2 = !(cfg->flags & SWITCH_FLAG_GEMM_1SM);
-  if (bf16 && (cfg->flags & SWITCH_FLAG_GATHER_COPY)) {
+  if (bf16 && !(cfg->flags & SWITCH_FLAG_GATHER_IN_GEMM)) {
     SMOE_TRY(launch_gather_rows(static_cast<int64_t>(N) * c.C,
                                 static_cast<int64_t>(a.d) * 2, slot_token, x, c.ws + c.L.xdisp,
                                 c.st));

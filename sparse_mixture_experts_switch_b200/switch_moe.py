@@ -23,10 +23,11 @@ SWITCH_F32, SWITCH_BF16 = 0, 1
 FLAG_ROUTER_SIMT = 1
 FLAG_ROUTER_3TERM = 2
 FLAG_UNFUSED_COMBINE = 4
-FLAG_GATHER_COPY = 8
+FLAG_GATHER_IN_GEMM = 8
 FLAG_NO_RESIDUAL = 16
 FLAG_GEMM_1SM = 32
 FLAG_GEMM_PAIRS = 64
+FLAG_ROWS_DISPATCHED = 128
 
 
 class SwitchConfig(ctypes.Structure):

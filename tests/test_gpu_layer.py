@@ -72,9 +72,9 @@ E2E = Workload("e2e", T=3000, d_model=320, d_ff=576, n_experts=8, capacity_facto
 
 
 @pytest.mark.parametrize("flags", [0, 1, 2, 4, 8, 1 | 4 | 8, 32, 32 | 8, 64, 64 | 8],
-                         ids=["fused", "simt_router", "three_term", "unfused", "gather_copy",
-                              "simt_unfused_copy", "gemm_1sm", "gemm_1sm_copy", "gemm_pairs",
-                              "gemm_pairs_copy"])
+                         ids=["fused", "simt_router", "three_term", "unfused", "gather_in_gemm",
+                              "simt_unfused_gather", "gemm_1sm", "gemm_1sm_gather", "gemm_pairs",
+                              "gemm_pairs_gather"])
 def test_layer_bf16(sm, flags):
     flips, drop_rate = check_layer(sm, E2E, flags)
     assert drop_rate > 0     # cf = 1.0 with random routing overflows some experts

@@ -208,8 +208,8 @@ FFN_CASES = [
 
 
 @pytest.mark.parametrize("flags", [0, 8, 32, 40, 64, 72],
-                         ids=["gather_in_gemm", "gather_copy", "one_sm", "one_sm_copy", "pairs",
-                              "pairs_copy"])
+                         ids=["default", "gather_in_gemm", "one_sm", "one_sm_gather", "pairs",
+                              "pairs_gather"])
 @pytest.mark.parametrize("wl", FFN_CASES, ids=lambda w: w.name)
 def test_expert_ffn(sm, wl, flags):
     inp = make_inputs(wl)
@@ -233,6 +233,44 @@ def test_expert_ffn(sm, wl, flags):
     tol = BF16_RMS_TOL if wl.dtype == "bf16" else F32_RMS_TOL
     assert rms_ratio(yg[kept], Y[kept]) <= tol
     assert np.isnan(yg[~kept]).all()     # padding rows untouched
+
+
+@pytest.mark.parametrize("flags", [128, 128 | 32, 128 | 64], ids=["default", "one_sm", "pairs"])
+@pytest.mark.parametrize("wl", FFN_CASES, ids=lambda w: w.name)
+def test_expert_ffn_rows_dispatched(sm, wl, flags):
+    """x_disp from switch_dispatch fed to switch_expert_ffn (ROWS_DISPATCHED):
+    same rows as the oracle's FFN, and bit-identical to the call that
+    dispatches the rows itself."""
+    inp = make_inputs(wl)
+    r = orc.router(inp.x, inp.w_r, inp.b_r)
+    C = orc.capacity(wl.T, wl.n_experts, wl.capacity_factor)
+    dsp = orc.dispatch(r["idx"], wl.n_experts, C)
+    Y = orc.expert_ffn(inp.x, inp.w1, inp.w2, dsp["slot_token"], dsp["counts"], C)
+    x = dev_float(inp.x)
+    _, st, _, _, counts, slot, xd = _dispatch_gpu(sm, wl, idx=r["idx"], x=x, want_xdisp=True)
+    assert st[0] == 0
+    np.testing.assert_array_equal(counts, dsp["counts"])
+    dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    counts_d = torch.from_numpy(counts.astype(np.int32)).cuda()
+    w1, w2 = dev_float(inp.w1), dev_float(inp.w2)
+    cfg = _cfg(sm, wl, flags)
+    ws = sm.workspace(cfg)
+    y = torch.full((wl.n_experts * C, wl.d_model), float("nan"), dtype=dt, device="cuda")
+    sm.switch_expert_ffn(cfg, xd, None, counts_d, w1, w2, y, ws)
+    _ok(sm, ws)
+    y_ref = torch.full_like(y, float("nan"))
+    cfg0 = _cfg(sm, wl, flags & ~128)
+    sm.switch_expert_ffn(cfg0, x, torch.from_numpy(slot.astype(np.int32)).cuda(), counts_d,
+                         w1, w2, y_ref, ws)
+    _ok(sm, ws)
+    kept = np.zeros((wl.n_experts, C), bool)
+    for e in range(wl.n_experts):
+        kept[e, : min(int(counts[e]), C)] = True
+    yg = host_f64(y).reshape(wl.n_experts, C, wl.d_model)
+    tol = BF16_RMS_TOL if wl.dtype == "bf16" else F32_RMS_TOL
+    assert rms_ratio(yg[kept], Y[kept]) <= tol
+    assert np.isnan(yg[~kept]).all()
+    np.testing.assert_array_equal(yg[kept], host_f64(y_ref).reshape(wl.n_experts, C, -1)[kept])
 
 
 def test_expert_ffn_dense_reduction(sm):
