@@ -36,6 +36,31 @@ UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
 
+# DRAM bytes (read + written) of one GEMM1 + GEMM2 launch pair on the Base
+# workload, from ncu captures of those kernels (profiles/
+# expert_gemm_base_full.md), valid only for the kernel sources they were
+# taken on: the bench reports them as `traffic` while the sources hash the
+# same, and null once a kernel has changed.
+GEMM_SOURCES = ("common.cuh", "gemm_common.cuh", "expert_ffn.cu", "expert_ffn_pair.cu")
+GEMM_TRAFFIC = {"workload": "base", "sources_sha256": None, "bytes": None}
+
+
+def gemm_sources_sha256():
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "sparse_mixture_experts_switch_b200", "csrc")
+    for name in GEMM_SOURCES:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def gemm_traffic(workload):
+    if workload != GEMM_TRAFFIC["workload"] or GEMM_TRAFFIC["bytes"] is None:
+        return None
+    return GEMM_TRAFFIC["bytes"] if gemm_sources_sha256() == GEMM_TRAFFIC["sources_sha256"] \
+        else None
+
 
 def parse_args():
     ap = argparse.ArgumentParser()
@@ -353,7 +378,8 @@ def main():
                          "bound": "tensor", "achieved": ffn["tflops"],
                          "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                          "frac": ffn["tflops"] / pk["bf16_tflops"],
-                         "peak_kind": f"{pk_kind} bf16 burst", "traffic": ffn.get("traffic"),
+                         "peak_kind": f"{pk_kind} bf16 burst",
+                         "traffic": gemm_traffic(args.workload),
                          "useful_flops": 4.0 * T_kept * d * F},
             "layer_roofline": {"t_min_us": t_layer_min * 1e6,
                                "tokens_per_s": T / t_layer_min,

@@ -162,20 +162,29 @@ cudaError_t launch_router_simt(int64_t T, int d, int N, bool bf16, const void* x
 
 // ======================================================== tensor cores
 
-__global__ void wsplit_kernel(int N, int N_pad, int d, int terms,
+// W_r [N, d] fp32 -> bf16 terms [rows, d].  Row of (term p, expert e):
+// stacked, p * N_pad + e (each term's experts together); interleaved,
+// (e / 32 * terms + p) * 32 + e % 32 (the terms of 32 experts side by side,
+// so one accumulator chunk of 32 x terms columns holds all of them).
+__global__ void wsplit_kernel(int N, int N_pad, int d, int terms, bool interleave,
                               const float* __restrict__ w_r, __nv_bfloat16* __restrict__ out) {
   const int64_t n = static_cast<int64_t>(N_pad) * d;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int e = static_cast<int>(i / d);
+    const int64_t k = i - static_cast<int64_t>(e) * d;
     const float w = e < N ? w_r[i] : 0.f;
     const __nv_bfloat16 hi = __float2bfloat16_rn(w);
     const float r1 = w - __bfloat162float(hi);           // exact
     const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
     const float r2 = r1 - __bfloat162float(mid);          // exact
-    out[i] = hi;
-    out[n + i] = mid;
-    if (terms == 3) out[2 * n + i] = __float2bfloat16_rn(r2);   // exact: r2 has <= 8 bits
+    auto row = [&](int p) -> int64_t {
+      return interleave ? static_cast<int64_t>((e >> 5) * terms + p) * 32 + (e & 31)
+                        : static_cast<int64_t>(p) * N_pad + e;
+    };
+    out[row(0) * d + k] = hi;
+    out[row(1) * d + k] = mid;
+    if (terms == 3) out[row(2) * d + k] = __float2bfloat16_rn(r2);   // exact: <= 8 bits
   }
 }
 
@@ -209,6 +218,15 @@ __device__ __forceinline__ void transpose_reduce32(float* v, int lane) {
   }
 }
 
+// What the epilogue of a 128-token tile needs.
+struct RouterEpi {
+  int64_t T;
+  int N, N_pad, ntiles;
+  bool has_bias;
+  const float* bias_s;     // [N_pad] in shared memory
+  RouterOut o;
+};
+
 // Logits of experts 32c .. 32c + 31 of this thread's token: the sum of the
 // weight terms' accumulator columns (term p at column p * NCH * 32).
 template <int NCH, int TERMS>
@@ -221,6 +239,111 @@ __device__ __forceinline__ void load_logits(uint32_t taddr, int c, float* v) {
 #pragma unroll
     for (int j = 0; j < 32; ++j) v[j] += w[j];
   }
+}
+
+// Softmax of one token (this thread's TMEM lane) of a 128-token tile, in
+// three streaming passes over its logits in TMEM, 32 values live at a time:
+// the max; the sum of exponentials and the first index of the max; the
+// scaled probabilities (stored when asked) and the warp's column sums of
+// them into redq[e] (a butterfly transpose-reduce over the warp's 32
+// tokens).  All TMEM reads of the tile are done when this returns.
+template <int NCH, int TERMS>
+__device__ __forceinline__ void router_softmax(const RouterEpi& ep, uint32_t taddr, int64_t t,
+                                               float* redq, int lane, int& best_out,
+                                               float& inv_out) {
+  const bool valid = t < ep.T;
+  const int N = ep.N;
+  float v[32];
+  float m = -INFINITY;
+#pragma unroll 1
+  for (int c = 0; c < NCH; ++c) {
+    load_logits<NCH, TERMS>(taddr, c, v);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const float hv = ep.has_bias ? v[j] + ep.bias_s[c * 32 + j] : v[j];
+      if (c * 32 + j < N) m = fmaxf(m, hv);
+    }
+  }
+  const float mL = m * kLog2e;
+  float s4[4] = {0.f, 0.f, 0.f, 0.f};
+  int best = 0x7fffffff;
+#pragma unroll 1
+  for (int c = 0; c < NCH; ++c) {
+    load_logits<NCH, TERMS>(taddr, c, v);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const int e = c * 32 + j;
+      const float hv = ep.has_bias ? v[j] + ep.bias_s[e] : v[j];
+      if (e < N) {
+        s4[j & 3] += exp2_fast(fmaf(hv, kLog2e, -mL));
+        if (hv == m && e < best) best = e;
+      }
+    }
+  }
+  const float inv = 1.f / ((s4[0] + s4[1]) + (s4[2] + s4[3]));
+  const float scale = valid ? inv : 0.f;
+#pragma unroll 1
+  for (int c = 0; c < NCH; ++c) {
+    load_logits<NCH, TERMS>(taddr, c, v);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const int e = c * 32 + j;
+      const float hv = ep.has_bias ? v[j] + ep.bias_s[e] : v[j];
+      v[j] = e < N ? exp2_fast(fmaf(hv, kLog2e, -mL)) * scale : 0.f;
+    }
+    if (valid && ep.o.probs != nullptr) {
+      float* dst = ep.o.probs + t * N + c * 32;
+      if ((N % 4) == 0 && c * 32 + 32 <= N) {
+#pragma unroll
+        for (int j = 0; j < 32; j += 4)
+          *reinterpret_cast<float4*>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (c * 32 + j < N) dst[j] = v[j];
+      }
+    }
+    transpose_reduce32(v, lane);
+    redq[c * 32 + lane] = v[0];
+  }
+  best_out = best;
+  inv_out = inv;
+}
+
+// The rest of a tile's epilogue, by its four warps (128 threads, named
+// barrier `bar`; warp quarter q holds tokens 32q .. 32q + 31): idx and gate,
+// each token's rank among the tile's tokens with the same expert (token
+// order), the tile's histogram and its column sums of the probabilities.
+__device__ __forceinline__ void router_finish(const RouterEpi& ep, int tile, int64_t t, int best,
+                                              float inv, int q, int lane, int et, int bar,
+                                              const float* redg, int* cntg) {
+  const bool valid = t < ep.T;
+  const int N = ep.N, N_pad = ep.N_pad;
+  for (int i = et; i < 4 * N_pad; i += 128) cntg[i] = 0;
+  named_bar_sync(bar, 128);
+  if (valid) {
+    ep.o.idx[t] = best;
+    ep.o.gate[t] = inv;
+  }
+  const int e_key = valid ? best : -1;
+  const unsigned peers = __match_any_sync(0xffffffffu, e_key);
+  const int rank_w = __popc(peers & ((1u << lane) - 1u));
+  if (valid && rank_w == 0) cntg[q * N_pad + best] = __popc(peers);
+  named_bar_sync(bar, 128);
+  if (valid && ep.o.local_rank != nullptr) {
+    int r = rank_w;
+    for (int qq = 0; qq < q; ++qq) r += cntg[qq * N_pad + best];
+    ep.o.local_rank[t] = r;
+  }
+  for (int e = et; e < N; e += 128) {
+    if (ep.o.psum != nullptr)
+      ep.o.psum[static_cast<int64_t>(tile) * N + e] =
+          ((redg[e] + redg[N_pad + e]) + redg[2 * N_pad + e]) + redg[3 * N_pad + e];
+    if (ep.o.hist != nullptr)
+      ep.o.hist[static_cast<int64_t>(e) * ep.ntiles + tile] =
+          cntg[e] + cntg[N_pad + e] + cntg[2 * N_pad + e] + cntg[3 * N_pad + e];
+  }
+  named_bar_sync(bar, 128);
 }
 
 // Each CTA owns `subs` consecutive 128-token tiles, all accumulated at once
@@ -403,97 +526,16 @@ __global__ void __launch_bounds__(kRouterThreads, 1) router_tc_kernel(
       if (et == 0) report_error(prm.err, SWITCH_ERR_TIMEOUT, kWhereRouterEpilogue, blockIdx.x);
     } else {
       tc_fence_after();
+      const RouterEpi ep{prm.T, N, N_pad, prm.ntiles, prm.b_r != nullptr, bias_s, prm.o};
       for (int s = g; s < ntile_here; s += 2) {
         const int tile = tile0 + s;
-        for (int i = et; i < 4 * N_pad; i += 128) cntg[i] = 0;
-        named_bar_sync(1 + g, 128);
         const int64_t t = static_cast<int64_t>(tile) * 128 + row;
-        const bool valid = t < prm.T;
         const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                static_cast<uint32_t>(s * NS);
-        // Three streaming passes over the row's logits in TMEM (max; sum of
-        // exponentials and the first index of the max; scaled probabilities
-        // and their column sums), 32 values live at a time.
-        const bool has_bias = prm.b_r != nullptr;
-        float v[32];
-        float m = -INFINITY;
-#pragma unroll 1
-        for (int c = 0; c < NCH; ++c) {
-          load_logits<NCH, TERMS>(taddr, c, v);
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float hv = has_bias ? v[j] + bias_s[c * 32 + j] : v[j];
-            if (c * 32 + j < N) m = fmaxf(m, hv);
-          }
-        }
-        const float mL = m * kLog2e;
-        float s4[4] = {0.f, 0.f, 0.f, 0.f};
-        int best = 0x7fffffff;
-#pragma unroll 1
-        for (int c = 0; c < NCH; ++c) {
-          load_logits<NCH, TERMS>(taddr, c, v);
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int e = c * 32 + j;
-            const float hv = has_bias ? v[j] + bias_s[e] : v[j];
-            if (e < N) {
-              s4[j & 3] += exp2_fast(fmaf(hv, kLog2e, -mL));
-              if (hv == m && e < best) best = e;
-            }
-          }
-        }
-        const float inv = 1.f / ((s4[0] + s4[1]) + (s4[2] + s4[3]));
-        const float scale = valid ? inv : 0.f;
-#pragma unroll 1
-        for (int c = 0; c < NCH; ++c) {
-          load_logits<NCH, TERMS>(taddr, c, v);
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int e = c * 32 + j;
-            const float hv = has_bias ? v[j] + bias_s[e] : v[j];
-            v[j] = e < N ? exp2_fast(fmaf(hv, kLog2e, -mL)) * scale : 0.f;
-          }
-          if (valid && prm.o.probs != nullptr) {
-            float* dst = prm.o.probs + t * N + c * 32;
-            if ((N % 4) == 0 && c * 32 + 32 <= N) {
-#pragma unroll
-              for (int j = 0; j < 32; j += 4)
-                *reinterpret_cast<float4*>(dst + j) =
-                    make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
-            } else {
-#pragma unroll
-              for (int j = 0; j < 32; ++j)
-                if (c * 32 + j < N) dst[j] = v[j];
-            }
-          }
-          transpose_reduce32(v, lane);
-          redg[q * N_pad + c * 32 + lane] = v[0];
-        }
-        if (valid) {
-          prm.o.idx[t] = best;
-          prm.o.gate[t] = inv;
-        }
-        // rank within the 128-token tile, token order (quarter q holds
-        // rows 32q .. 32q + 31)
-        const int e_key = valid ? best : -1;
-        const unsigned peers = __match_any_sync(0xffffffffu, e_key);
-        const int rank_w = __popc(peers & ((1u << lane) - 1u));
-        if (valid && rank_w == 0) cntg[q * N_pad + best] = __popc(peers);
-        named_bar_sync(1 + g, 128);
-        if (valid && prm.o.local_rank != nullptr) {
-          int r = rank_w;
-          for (int qq = 0; qq < q; ++qq) r += cntg[qq * N_pad + best];
-          prm.o.local_rank[t] = r;
-        }
-        for (int e = et; e < N; e += 128) {
-          if (prm.o.psum != nullptr)
-            prm.o.psum[static_cast<int64_t>(tile) * N + e] =
-                ((redg[e] + redg[N_pad + e]) + redg[2 * N_pad + e]) + redg[3 * N_pad + e];
-          if (prm.o.hist != nullptr)
-            prm.o.hist[static_cast<int64_t>(e) * prm.ntiles + tile] =
-                cntg[e] + cntg[N_pad + e] + cntg[2 * N_pad + e] + cntg[3 * N_pad + e];
-        }
-        named_bar_sync(1 + g, 128);
+        int best;
+        float inv;
+        router_softmax<NCH, TERMS>(ep, taddr, t, redg + q * N_pad, lane, best, inv);
+        router_finish(ep, tile, t, best, inv, q, lane, et, 1 + g, redg, cntg);
       }
     }
   }
@@ -502,6 +544,339 @@ __global__ void __launch_bounds__(kRouterThreads, 1) router_tc_kernel(
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem_base, prm.tmem_cols);
+}
+
+// ---------------------------------------------------------- CTA pairs
+//
+// Persistent router on CTA pairs with double-buffered accumulators, for
+// terms x N_pad <= 256 (one MMA covers every expert and every weight term).
+// A pair tile is 256 tokens: CTA r holds tokens 128 r .. 128 r + 127 (the A
+// operand) and half of the stacked weight split (rows r * Nt/2 .. of the
+// B operand, Nt = terms x N_pad; with two terms, one term per CTA).  The
+// leader issues tcgen05.mma.cta_group::2 (M = 256, N = Nt, K = 16); each
+// CTA's TMEM receives its 128 tokens x all Nt columns.  Every SM streams 16 KB
+// of x and Nt/2 x 128 B of weights per 64-deep K step through a six-stage
+// ring.  Two TMEM accumulators alternate between tiles, each drained by its
+// own group of four epilogue warps, so the softmax of one tile overlaps the
+// main loop of the next.
+struct RouterPairParams {
+  int64_t T;
+  int d, N, N_pad, ntiles, npairs, stages;
+  uint32_t x_bytes, w_bytes;       // per stage and CTA
+  int w_half_rows;
+  const float* b_r;
+  RouterOut o;
+  DevErr* err;
+  long long spin;
+};
+
+constexpr int kRouterPairMaxStages = 8;
+
+template <int NCH, int TERMS>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kRouterThreads, 1)
+    router_pair_kernel(const __grid_constant__ CUtensorMap tmap_x,
+                       const __grid_constant__ CUtensorMap tmap_w, RouterPairParams prm) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  const int STAGES = prm.stages;
+  const uint32_t stage_bytes = prm.x_bytes + prm.w_bytes;
+  const int N = prm.N, N_pad = prm.N_pad;
+  constexpr int NT = NCH * 32 * TERMS;                   // accumulator columns per tile
+  uint8_t* tail = smem + static_cast<size_t>(STAGES) * stage_bytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(tail);    // leader: bytes of both CTAs
+  uint64_t* empty = full + kRouterPairMaxStages;         // local: stage consumed
+  uint64_t* tfull = empty + kRouterPairMaxStages;        // local: accumulator g ready
+  uint64_t* tempty = tfull + 2;                          // leader: accumulator g drained
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  volatile int* epi_fail = abort_flag + 1;   // [2] by tile parity: an epilogue wait gave up
+  float* bias_s = reinterpret_cast<float*>(tail + 512);  // [N_pad]
+  float* red = bias_s + N_pad;                           // [2 parity][4 quarter][N_pad]
+  int* cnt = reinterpret_cast<int*>(red + 2 * 4 * N_pad);   // [2 parity][4 quarter][N_pad]
+  float* xm = reinterpret_cast<float*>(cnt + 2 * 4 * N_pad);  // [2 parity][2 half][128]
+  float* xs = xm + 2 * 2 * 128;
+  int* xb = reinterpret_cast<int*>(xs + 2 * 2 * 128);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int cid = static_cast<int>(cluster_id_x());
+  const int ncl = static_cast<int>(cluster_count_x());
+  const int kblocks = prm.d / 64;
+  const long long lim = prm.spin;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 16);            // 8 epilogue warps x 2 CTAs
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    epi_fail[0] = 0;
+    epi_fail[1] = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  for (int i = threadIdx.x; i < N_pad; i += blockDim.x)
+    bias_s[i] = (prm.b_r != nullptr && i < N) ? prm.b_r[i] : 0.f;
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_holder, 2 * 256);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();                          // the peer's barriers exist before any remote use
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const uint32_t full_lead = map_to_rank(smem_u32(full), 0);
+  const uint32_t tempty_lead = map_to_rank(smem_u32(tempty), 0);
+
+  if (warp == 0) {
+    // ------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmap_x);
+      tma_prefetch_desc(&tmap_w);
+      int stage = 0;
+      uint32_t phase = 0, issued_mask = 0, issued_phase = 0;
+      bool ok = true;
+      for (int pt = cid; pt < prm.npairs && ok && !*abort_flag; pt += ncl) {
+        const int xrow = pt * 256 + static_cast<int>(rank) * 128;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, lim)) { ok = false; break; }
+          uint8_t* sx = smem + static_cast<size_t>(stage) * stage_bytes;
+          const uint32_t bar = full_lead + 8u * stage;
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * stage_bytes);
+          tma_load_2d_pair(sx, &tmap_x, bar, kb * 64, xrow);
+          tma_load_2d_pair(sx + prm.x_bytes, &tmap_w, bar, kb * 64,
+                           static_cast<int>(rank) * prm.w_half_rows);
+          issued_mask |= 1u << stage;
+          issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {
+        report_error(prm.err, SWITCH_ERR_TIMEOUT, kWhereRouterProducer, blockIdx.x);
+        *abort_flag = 1;
+      }
+      // Both CTAs' bytes land on the leader's barriers: the leader waits for
+      // every issued stage before the final cluster barrier.
+      if (leader)
+        for (int s = 0; s < STAGES; ++s)
+          if (((issued_mask >> s) & 1u) &&
+              !mbar_wait_cluster(&full[s], (issued_phase >> s) & 1u, kDefaultSpinCycles))
+            report_error(prm.err, SWITCH_ERR_TIMEOUT, kWhereDrain, s);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------- MMA issuer
+    if (leader && lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(256, NT);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true, any = false;
+      int li = 0;                                        // local tile count
+      for (int pt = cid; pt < prm.npairs && ok && !*abort_flag; pt += ncl, ++li) {
+        const int acc = li & 1;
+        const uint32_t use = static_cast<uint32_t>(li >> 1);   // earlier uses of `acc`
+        if (!mbar_wait_cluster(&tempty[acc], (use & 1u) ^ 1u, lim)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * 256);
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait_cluster(&full[stage], phase, lim)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sx = smem_u32(smem + static_cast<size_t>(stage) * stage_bytes);
+          const uint64_t xd = sw128_kmajor_desc(sx);
+          const uint64_t wd = sw128_kmajor_desc(sx + prm.x_bytes);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            umma_bf16_pair(d_tmem, xd + 2 * k, wd + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+          any = true;
+          umma_commit_pair(&empty[stage], 0x3);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit_pair(&tfull[acc], 0x3);
+      }
+      if (!ok) {
+        report_error(prm.err, SWITCH_ERR_TIMEOUT, kWhereRouterMma, blockIdx.x);
+        *abort_flag = 1;
+      }
+      if (any && *abort_flag) {
+        umma_commit_pair(drain, 0x1);
+        if (!mbar_wait(drain, 0, kDefaultSpinCycles))
+          report_error(prm.err, SWITCH_ERR_TIMEOUT, kWhereDrain, -1);
+      }
+    }
+  } else {
+    // ------------------------------------------------------- epilogue
+    // All eight warps drain every tile: warp quarter q = warp % 4 owns TMEM
+    // lanes (tokens) 32q .. 32q + 31, half h = (warp - 2) / 4 owns expert
+    // chunks h * NH .. of them.  One TMEM pass per thread (its token's logits
+    // of its half, all weight terms), after which the accumulator is handed
+    // back; the halves then exchange (max, sum of exponentials, first index
+    // of the max) through shared memory.  Per-tile shared arrays alternate
+    // with the tile's parity.
+    constexpr int NH = (NCH + 1) / 2;                  // chunks per half
+    const int q = warp & 3;
+    const int h = (warp - 2) >> 2;
+    const int row = q * 32 + lane;
+    const int et = threadIdx.x - 64;                   // 0 .. 255
+    const int N_h = N - h * NH * 32;                   // experts of this half (may be <= 0)
+    int li = 0;
+    for (int pt = cid; pt < prm.npairs; pt += ncl, ++li) {
+      const int acc = li & 1;
+      // One outcome for all eight warps (they meet at named barriers below):
+      // a warp whose wait gave up raises this tile's flag before the
+      // barrier, every warp reads it after.  No warp gets a whole tile ahead
+      // of another (each tile passes this barrier), so alternating two
+      // flags keeps a later tile's failure out of this tile's decision.
+      const bool ok = __all_sync(0xffffffffu,
+                                 mbar_wait_sleepy(&tfull[acc], static_cast<uint32_t>(li >> 1) & 1u, lim));
+      if (!ok && lane == 0) epi_fail[li & 1] = 1;
+      named_bar_sync(1, 256);
+      if (epi_fail[li & 1]) {
+        if (et == 0) {
+          report_error(prm.err, SWITCH_ERR_TIMEOUT, kWhereRouterEpilogue, blockIdx.x);
+          *abort_flag = 1;
+        }
+        break;
+      }
+      tc_fence_after();
+      const int tile = pt * 2 + static_cast<int>(rank);   // this CTA's 128-token tile
+      const bool here = tile < prm.ntiles;                // uniform for the CTA
+      const int64_t t = static_cast<int64_t>(tile) * 128 + row;
+      const bool valid = t < prm.T;
+      // this half's logits (sum of the weight terms, + bias), one chunk of
+      // TMEM loads in flight at a time
+      float v[NH * 32];
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                             static_cast<uint32_t>(acc * 256);
+      if (here) {
+#pragma unroll
+        for (int cc = 0; cc < NH; ++cc) {
+          const int c = h * NH + cc;
+#pragma unroll
+          for (int p = 0; p < TERMS; ++p) {
+            uint32_t r[32];
+            if (c < NCH) {                                // warp-uniform
+              tmem_ld32_issue(taddr + static_cast<uint32_t>((c * TERMS + p) * 32), r);
+              tmem_ld_wait(r);
+            }
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              v[cc * 32 + j] = p == 0 ? __uint_as_float(r[j]) : v[cc * 32 + j] + __uint_as_float(r[j]);
+          }
+          if (prm.b_r != nullptr)
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (c * 32 + j < N) v[cc * 32 + j] += bias_s[c * 32 + j];
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {                                    // TMEM of this tile no longer read
+        if (leader) mbar_arrive(&tempty[acc]);
+        else mbar_arrive_remote(tempty_lead + 8u * acc);
+      }
+      if (!here) continue;
+      const int par = li & 1;
+      float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int i = 0; i < NH * 32; ++i)
+        if (i < N_h) mq[i & 3] = fmaxf(mq[i & 3], v[i]);
+      const float m_h = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
+      int bq[4] = {0x7fffffff, 0x7fffffff, 0x7fffffff, 0x7fffffff};
+#pragma unroll
+      for (int i = 0; i < NH * 32; ++i)
+        if (i < N_h && v[i] == m_h) bq[i & 3] = min(bq[i & 3], i);
+      const int b_h = min(min(bq[0], bq[1]), min(bq[2], bq[3]));
+      const float mL_h = m_h * kLog2e;
+      float sq[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int i = 0; i < NH * 32; ++i) {
+        v[i] = i < N_h ? exp2_fast(fmaf(v[i], kLog2e, -mL_h)) : 0.f;
+        sq[i & 3] += v[i];
+      }
+      float* xm_p = xm + par * 256;
+      float* xs_p = xs + par * 256;
+      int* xb_p = xb + par * 256;
+      xm_p[h * 128 + row] = m_h;
+      xs_p[h * 128 + row] = (sq[0] + sq[1]) + (sq[2] + sq[3]);
+      xb_p[h * 128 + row] = b_h == 0x7fffffff ? b_h : h * NH * 32 + b_h;
+      int* cnt_p = cnt + par * 4 * N_pad;
+      for (int i = et; i < 4 * N_pad; i += 256) cnt_p[i] = 0;
+      named_bar_sync(1, 256);
+      // the token's max, sum and expert, the same in both halves
+      const float m0 = xm_p[row], m1 = xm_p[128 + row];
+      const float m = fmaxf(m0, m1);
+      const float s = xs_p[row] * exp2_fast((m0 - m) * kLog2e) +
+                      xs_p[128 + row] * exp2_fast((m1 - m) * kLog2e);
+      const int best = m0 >= m1 ? xb_p[row] : xb_p[128 + row];
+      const float inv = 1.f / s;
+      const float scale = valid ? exp2_fast((m_h - m) * kLog2e) * inv : 0.f;
+      float* red_p = red + par * 4 * N_pad;
+#pragma unroll
+      for (int cc = 0; cc < NH; ++cc) {
+        const int c = h * NH + cc;
+        if (c >= NCH) break;                              // warp-uniform
+        float pv[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) pv[j] = v[cc * 32 + j] * scale;
+        if (valid && prm.o.probs != nullptr) {
+          float* dst = prm.o.probs + t * N + c * 32;
+          if ((N % 4) == 0 && c * 32 + 32 <= N) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 4)
+              *reinterpret_cast<float4*>(dst + j) =
+                  make_float4(pv[j], pv[j + 1], pv[j + 2], pv[j + 3]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (c * 32 + j < N) dst[j] = pv[j];
+          }
+        }
+        transpose_reduce32(pv, lane);
+        red_p[q * N_pad + c * 32 + lane] = pv[0];
+      }
+      // dispatch ranks within the tile (token order), by half 0
+      int rank_w = 0;
+      if (h == 0) {
+        const int e_key = valid ? best : -1;
+        const unsigned peers = __match_any_sync(0xffffffffu, e_key);
+        rank_w = __popc(peers & ((1u << lane) - 1u));
+        if (valid && rank_w == 0) cnt_p[q * N_pad + best] = __popc(peers);
+      }
+      named_bar_sync(1, 256);
+      if (h == 0 && valid) {
+        prm.o.idx[t] = best;
+        prm.o.gate[t] = inv;
+        if (prm.o.local_rank != nullptr) {
+          int rr = rank_w;
+          for (int qq = 0; qq < q; ++qq) rr += cnt_p[qq * N_pad + best];
+          prm.o.local_rank[t] = rr;
+        }
+      }
+      for (int e = et; e < N; e += 256) {
+        if (prm.o.psum != nullptr)
+          prm.o.psum[static_cast<int64_t>(tile) * N + e] =
+              ((red_p[e] + red_p[N_pad + e]) + red_p[2 * N_pad + e]) + red_p[3 * N_pad + e];
+        if (prm.o.hist != nullptr)
+          prm.o.hist[static_cast<int64_t>(e) * prm.ntiles + tile] =
+              cnt_p[e] + cnt_p[N_pad + e] + cnt_p[2 * N_pad + e] + cnt_p[3 * N_pad + e];
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();                          // no CTA leaves while its peer may still signal it
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_pair(tmem_base, 2 * 256);
 }
 
 // ------------------------------------------------------------------ host
@@ -546,20 +921,90 @@ static cudaError_t run_router_tc(const CUtensorMap& tx, const CUtensorMap& tw,
                       : run_router_tc_t<NCH, 3>(tx, tw, p, smem, grid, st);
 }
 
+template <int NCH, int TERMS>
+static cudaError_t run_router_pair_t(const CUtensorMap& tx, const CUtensorMap& tw,
+                                     const RouterPairParams& p, size_t smem, int grid,
+                                     cudaStream_t st) {
+  static size_t smem_set[64] = {};
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(&router_pair_kernel<NCH, TERMS>),
+                                    smem, smem_set);
+  if (e != cudaSuccess) return e;
+  router_pair_kernel<NCH, TERMS><<<grid, kRouterThreads, smem, st>>>(tx, tw, p);
+  return cudaGetLastError();
+}
+
+// CTA-pair router: terms x N_pad <= 256.
+static cudaError_t launch_router_pair(int64_t T, int d, int N, int N_pad, int terms,
+                                      const void* x, const float* b_r, const void* wsplit,
+                                      RouterOut o, int ntiles, DevErr* err, long long spin,
+                                      int num_sms, cudaStream_t st) {
+  const int nt = terms * N_pad;
+  RouterPairParams p;
+  p.T = T;
+  p.d = d;
+  p.N = N;
+  p.N_pad = N_pad;
+  p.ntiles = ntiles;
+  p.npairs = (ntiles + 1) / 2;
+  p.w_half_rows = nt / 2;
+  p.x_bytes = 128u * 128u;
+  p.w_bytes = static_cast<uint32_t>(nt / 2) * 128u;
+  p.b_r = b_r;
+  p.o = o;
+  p.err = err;
+  p.spin = spin;
+  const size_t tail_bytes =
+      512 + sizeof(float) * N_pad * 9 + sizeof(int) * N_pad * 8 + 3 * sizeof(float) * 512;
+  const size_t budget = 227 * 1024 - 1024 - tail_bytes;
+  int stages = static_cast<int>(budget / (p.x_bytes + p.w_bytes));
+  if (stages > kRouterPairMaxStages) stages = kRouterPairMaxStages;
+  if (stages < 2) return cudaErrorInvalidConfiguration;
+  p.stages = stages;
+  CUtensorMap tx, tw;
+  if (!make_tmap_bf16_2d(&tx, x, static_cast<uint64_t>(d), static_cast<uint64_t>(T), 64, 128))
+    return cudaErrorInvalidValue;
+  if (!make_tmap_bf16_2d(&tw, wsplit, static_cast<uint64_t>(d), static_cast<uint64_t>(nt), 64,
+                         static_cast<uint32_t>(nt / 2)))
+    return cudaErrorInvalidValue;
+  const size_t smem =
+      1024 + static_cast<size_t>(stages) * (p.x_bytes + p.w_bytes) + tail_bytes;
+  int clusters = num_sms / 2;
+  if (clusters > p.npairs) clusters = p.npairs;
+  if (clusters < 1) clusters = 1;
+  const int grid = 2 * clusters;
+  const int nch = N_pad / 32;
+  if (terms == 2) {
+    switch (nch) {
+      case 1: return run_router_pair_t<1, 2>(tx, tw, p, smem, grid, st);
+      case 2: return run_router_pair_t<2, 2>(tx, tw, p, smem, grid, st);
+      case 3: return run_router_pair_t<3, 2>(tx, tw, p, smem, grid, st);
+      default: return run_router_pair_t<4, 2>(tx, tw, p, smem, grid, st);
+    }
+  }
+  switch (nch) {
+    case 1: return run_router_pair_t<1, 3>(tx, tw, p, smem, grid, st);
+    default: return run_router_pair_t<2, 3>(tx, tw, p, smem, grid, st);
+  }
+}
+
 cudaError_t launch_router_tc(int64_t T, int d, int N, int terms, const void* x,
                              const float* w_r, const float* b_r, void* wsplit, RouterOut o,
                              int ntiles, DevErr* err, long long spin, int num_sms,
                              cudaStream_t st) {
   const int N_pad = router_n_pad(N);
+  const bool pair = terms * N_pad <= 256 && num_sms >= 2;
   {
     const int64_t n = static_cast<int64_t>(N_pad) * d;
     int blocks = static_cast<int>((n + 255) / 256);
     if (blocks > 1024) blocks = 1024;
-    wsplit_kernel<<<blocks, 256, 0, st>>>(N, N_pad, d, terms, w_r,
+    wsplit_kernel<<<blocks, 256, 0, st>>>(N, N_pad, d, terms, pair, w_r,
                                           static_cast<__nv_bfloat16*>(wsplit));
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
+  if (pair)
+    return launch_router_pair(T, d, N, N_pad, terms, x, b_r, wsplit, o, ntiles, err, spin,
+                              num_sms, st);
   CUtensorMap tx, tw;
   if (!make_tmap_bf16_2d(&tx, x, static_cast<uint64_t>(d), static_cast<uint64_t>(T), 64, 128))
     return cudaErrorInvalidValue;
