@@ -41,9 +41,10 @@ L2_FLUSH_BYTES = 256 << 20
 # expert_gemm_base_full.md), valid only for the kernel sources they were
 # taken on: the bench reports them as `traffic` while the sources hash the
 # same, and null once a kernel has changed.
-GEMM_SOURCES = ("common.cuh", "gemm_common.cuh", "expert_ffn.cu", "expert_ffn_pair.cu")
+GEMM_SOURCES = ("common.cuh", "gemm_common.cuh", "gemm_pair.cuh", "expert_ffn.cu",
+                "expert_ffn_pair.cu")
 GEMM_TRAFFIC = {"workload": "base",
-                "sources_sha256": "155f30364d5fcc40c067d9658700a6f050897d9d4064480d76f7866e0827bcca",
+                "sources_sha256": "0ab85744d10d1b7781851740503a59e5be0ac68493ab955484fd233810972f4a",
                 # GEMM1 715.7 MB read + 373.0 MB written; GEMM2 1239.5 + 93.7 MB
                 "bytes": 715.732480e6 + 372.987392e6 + 1239.501e6 + 93.651456e6}
 
