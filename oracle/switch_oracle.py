@@ -27,14 +27,21 @@ trillion-parameter models" (cited below as [P1 §section]):
   expert [P1 §"Switch Routing", combine equation with |T| = 1];
 * the load-balancing loss ``alpha . N . sum_i f_i P_i`` with ``f_i`` the
   fraction of tokens whose argmax is ``i`` and ``P_i`` the mean router
-  probability [P1 §"The Load-Balancing Loss", loss and f/P equations].
+  probability [P1 §"The Load-Balancing Loss", loss and f/P equations];
+* the top-k variant with k = 2 that the pages contrast with k = 1
+  [P1 §"Switch Routing: From Top-k to k = 1"]: the two largest gates, the
+  output summed over both, each expert's capacity doubled.
 
 Readings taken where the pages leave a step open: capacity rounds up; the
 whole batch is one routing group and tokens take slots in batch order;
 ties go to the lowest expert index; ``f_i`` counts routed tokens including
 dropped ones (the page defines it through the argmax, before capacity);
 the combine adds the residual ``x`` when asked (block output of a dropped
-token is ``x``); no dropout (forward pass).
+token is ``x``); no dropout (forward pass).  Top-2: the second choice is
+the largest of the other logits (lowest index on ties); the gates are the
+softmax over all experts, not renormalised; the 2T assignments take slots
+first choices first, each route in batch order; ``f_i`` still counts first
+choices.
 
 Arithmetic is float64 throughout (expert matmuls included); floating-point
 inputs are the exact values of the bf16 / fp32 bit patterns the GPU reads.
@@ -223,6 +230,97 @@ def layer_forward(x, w_r, b_r, w1, w2, capacity_factor, alpha=0.01,
     loss, f, P = aux_loss(dsp["counts"], r["probs"], alpha)
     return {"C": C, **r, **dsp, "Y": Y, "out": out, "loss": loss,
             "f": f, "P": P}
+
+
+# ------------------------------------------------------- top-2 routing
+
+def router_top2(x, w_r, b_r=None):
+    """Top-k routing with k = 2 [P1 §"Switch Routing: From Top-k to k = 1":
+    the top-k set T, output sum_{i in T} p_i(x) E_i(x), p the softmax over all
+    N experts (not renormalised over T)].
+
+    Returns the single-route dict of ``router`` plus:
+
+    * ``idx2`` int64 ``[2, T]``: row 0 the top-1 expert (as ``idx``), row 1
+      the expert of largest float32-rounded logit among the others, lowest
+      index on ties;
+    * ``gate2`` float64 ``[2, T]``: ``p`` at those experts;
+    * ``margin2`` float64 ``[2, T]``: row 0 ``p(1st) - p(2nd)``, row 1
+      ``p(2nd) - p(3rd)`` (``inf`` when there is no next expert).
+    """
+    r = router(x, w_r, b_r)
+    h32 = r["logits"].astype(np.float32)
+    p = r["probs"]
+    T, N = p.shape
+    if N < 2:
+        raise ValueError("top-2 routing needs at least two experts")
+    first = r["idx"]
+    rest = h32.copy()
+    rest[np.arange(T), first] = -np.inf
+    second = np.argmax(rest, axis=1).astype(np.int64)
+    idx2 = np.stack([first, second])
+    gate2 = np.stack([p[np.arange(T), first], p[np.arange(T), second]])
+    ps = -np.sort(-p, axis=1)
+    third = ps[:, 2] if N > 2 else np.full(T, -np.inf)
+    margin2 = np.stack([ps[:, 0] - ps[:, 1], ps[:, 1] - third])
+    return {**r, "idx2": idx2, "gate2": gate2, "margin2": margin2}
+
+
+def dispatch_top2(idx2, n_experts: int, C: int):
+    """Capacity-bounded dispatch of both routes, first choices first.
+
+    The 2T (token, expert) assignments take slots in route-major order:
+    every token's first choice in batch order, then every token's second
+    choice in batch order, sharing each expert's C slots (the reading for
+    k = 2: the pages give the capacity per expert, not the priority between
+    routes; first choices first keeps k = 1's behaviour for route 1).
+    Assignment a = r * T + t.  Returns ``rank [2, T]``, ``drop [2, T]``,
+    ``counts [N]`` (assignments routed to each expert, both routes, before
+    the capacity cut) and ``slot_token [N*C]`` (the token of each slot, -1
+    for padding).
+    """
+    idx2 = np.asarray(idx2)
+    T = idx2.shape[1]
+    d = dispatch(idx2.reshape(-1), n_experts, C)
+    st = d["slot_token"]
+    st = np.where(st >= 0, st % max(T, 1), -1)
+    return {"rank": d["rank"].reshape(2, T), "drop": d["drop"].reshape(2, T),
+            "counts": d["counts"], "slot_token": st}
+
+
+def combine_top2(x, idx2, rank2, drop2, gate2, Y, residual=True):
+    """x + sum over the two routes of p_i(x) . E_i(x), dropped routes give 0
+    [P1 §"Switch Routing", combine equation with |T| = 2; a dropped
+    assignment passes nothing, as in §"Expert Capacity ..."]."""
+    T, d = x.shape
+    out = as_f64(x) if residual else np.zeros((T, d))
+    for r in range(2):
+        kept = ~np.asarray(drop2[r], dtype=bool)
+        out[kept] += np.asarray(gate2[r])[kept, None] * \
+            Y[np.asarray(idx2[r])[kept], np.asarray(rank2[r])[kept]]
+    return out
+
+
+def layer_forward_top2(x, w_r, b_r, w1, w2, capacity_factor, alpha=0.01,
+                       residual=True, experts=None):
+    """Top-2 layer: capacity ceil(2T / N x capacity_factor) (each expert
+    receives tokens from two routes [P1 §"Switch Routing", the k = 1 win
+    "half the expert capacity"]); the load-balancing loss keeps its
+    definition through the argmax, i.e. the first choices
+    [P1 §"The Load-Balancing Loss", f_i]."""
+    T = x.shape[0]
+    N = w_r.shape[0]
+    C = capacity(2 * T, N, capacity_factor)
+    r = router_top2(x, w_r, b_r)
+    dsp = dispatch_top2(r["idx2"], N, C)
+    Y = expert_ffn(x, w1, w2, dsp["slot_token"], dsp["counts"], C, experts)
+    out = combine_top2(x, r["idx2"], dsp["rank"], dsp["drop"], r["gate2"], Y,
+                       residual)
+    counts1 = np.bincount(r["idx2"][0], minlength=N)
+    loss, f, P = aux_loss(counts1, r["probs"], alpha)
+    return {"C": C, **r, "rank2": dsp["rank"], "drop2": dsp["drop"],
+            "counts": dsp["counts"], "slot_token": dsp["slot_token"],
+            "counts1": counts1, "Y": Y, "out": out, "loss": loss, "f": f, "P": P}
 
 
 def token_outputs(x, tokens, idx, drop, gate, w1, w2, residual=True):

@@ -49,3 +49,24 @@ def dispatch_case():
         k, *v = ln.split()
         kv[k] = [int(x) for x in v]
     return kv
+
+
+def top2_router_cases():
+    out = []
+    for ln in _lines("top2_hand.txt"):
+        if not ln.startswith("router"):
+            continue
+        a, g, top = (s.strip() for s in ln[len("router"):].split("|"))
+        out.append(([int(v) for v in a.split(",")], [Fraction(v) for v in g.split()],
+                    [int(v) for v in top.split()]))
+    return out
+
+
+def top2_dispatch_case():
+    kv = {}
+    for ln in _lines("top2_hand.txt"):
+        if ln.startswith("router"):
+            continue
+        k, *v = ln.split()
+        kv[k] = [int(x) for x in v]
+    return kv

@@ -4,7 +4,8 @@ invariants the pages state, closed forms, and brute force on tiny inputs.
 
 Pages cited: "Switch Transformers: scaling to trillion-parameter models"
 (sections "Switch Routing: From Top-k to k = 1", "Expert Capacity and the
-Capacity Factor", "The Load-Balancing Loss", "The Core Idea").
+Capacity Factor", "The Load-Balancing Loss", "The Core Idea"); the top-2
+pins follow the top-k set and combine of "Switch Routing".
 
 The last test plants plausible mistakes in the oracle (on the CPU) and checks
 that at least one pin catches each of them.
@@ -270,10 +271,120 @@ def pin_relu_active(O):
     np.testing.assert_array_equal(O.expert(x, w1, w2), [[2.0, 7.0]])
 
 
+# ---------------------------------------------------------- top-2 pins
+
+def pin_top2_router_hand(O):
+    """Hand-worked top-2 sets and gates (tests/golden/top2_hand.txt)."""
+    for a, gates, top in golden_io.top2_router_cases():
+        x, w_r = _logit_router_inputs([a])
+        r = O.router_top2(x, w_r)
+        assert r["idx2"][:, 0].tolist() == top, (a, r["idx2"][:, 0])
+        np.testing.assert_allclose(r["gate2"][:, 0], [float(g) for g in gates],
+                                   rtol=1e-6, atol=0)
+
+
+def pin_top2_router_invariants(O):
+    """W_r = 0: all logits tie, every token takes experts (0, 1) with gates
+    1/N each; on random inputs the two choices differ, the first gate is the
+    k = 1 gate and the second is no larger than the first."""
+    rng = np.random.default_rng(21)
+    x = rng.standard_normal((50, 8)).astype(np.float32)
+    for N in (2, 4, 8):
+        r = O.router_top2(x, np.zeros((N, 8), np.float32))
+        assert (r["idx2"][0] == 0).all() and (r["idx2"][1] == 1).all()
+        np.testing.assert_allclose(r["gate2"], 1.0 / N, rtol=1e-12)
+        w_r = rng.standard_normal((N, 8)).astype(np.float32)
+        r = O.router_top2(x, w_r)
+        r1 = O.router(x, w_r)
+        assert (r["idx2"][0] != r["idx2"][1]).all()
+        assert (r["idx2"][0] == r1["idx"]).all()
+        assert (r["gate2"][1] <= r["gate2"][0]).all()
+        # the second choice is the argmax of p with the first removed
+        p = r1["probs"].copy()
+        p[np.arange(50), r1["idx"]] = -1.0
+        assert (np.argmax(p, axis=1) == r["idx2"][1]).all()
+
+
+def pin_top2_dispatch_hand(O):
+    g = golden_io.top2_dispatch_case()
+    d = O.dispatch_top2(np.array([g["idx1"], g["idx2"]]), g["N"][0], g["C"][0])
+    assert d["rank"].tolist() == [g["rank1"], g["rank2"]]
+    assert d["drop"].astype(int).tolist() == [g["drop1"], g["drop2"]]
+    assert d["counts"].tolist() == g["counts"]
+    assert d["slot_token"].tolist() == g["slot_token"]
+
+
+def pin_top2_dispatch_bruteforce(O):
+    """Every (first, second) assignment of 3 tokens over 3 experts, C = 1..4:
+    rank of assignment (r, t) = #{earlier assignments, first choices before
+    second choices, each in batch order, with the same expert}."""
+    N = 3
+    pairs = [(a, b) for a in range(N) for b in range(N) if a != b]
+    for choice in itertools.product(pairs, repeat=3):
+        idx2 = np.array([[c[0] for c in choice], [c[1] for c in choice]])
+        order = [(r, t) for r in range(2) for t in range(3)]
+        for C in (1, 2, 3, 4):
+            d = O.dispatch_top2(idx2, N, C)
+            for i, (r, t) in enumerate(order):
+                e = idx2[r, t]
+                want = sum(1 for (r2, t2) in order[:i] if idx2[r2, t2] == e)
+                assert d["rank"][r, t] == want and d["drop"][r, t] == (want >= C)
+            assert d["counts"].tolist() == np.bincount(idx2.reshape(-1), minlength=N).tolist()
+
+
+def pin_top2_dense_reduction(O):
+    """N = 2 with two identical experts and capacity factor >= 1: both routes
+    of every token are kept (C = T), the gates sum to 1, so the layer is the
+    dense residual FFN out = x + relu(x W1^T) W2^T (explicit loops)."""
+    rng = np.random.default_rng(31)
+    T, dm, F = 5, 4, 3
+    x = rng.standard_normal((T, dm)).astype(np.float32)
+    w_r = rng.standard_normal((2, dm)).astype(np.float32)
+    w1 = np.repeat(rng.standard_normal((1, F, dm)).astype(np.float32), 2, axis=0)
+    w2 = np.repeat(rng.standard_normal((1, dm, F)).astype(np.float32), 2, axis=0)
+    res = O.layer_forward_top2(x, w_r, None, w1, w2, 1.0, ALPHA)
+    assert res["C"] == T and not res["drop2"].any()
+    np.testing.assert_allclose(res["gate2"].sum(axis=0), 1.0, rtol=1e-12)
+    np.testing.assert_allclose(res["out"], _brute_dense(x, w1[0], w2[0]), rtol=1e-10,
+                               atol=1e-10)
+
+
+def pin_top2_signature(O):
+    """Each expert writes its own signature 100 (e + 1) unit(e): out - x holds
+    exactly the two chosen experts' signatures scaled by their gates, and a
+    dropped second route contributes nothing."""
+    rng = np.random.default_rng(41)
+    N, dm, T = 3, 4, 24
+    x = rng.standard_normal((T, dm)).astype(np.float32)
+    x[:, 3] = 1.0
+    w_r = rng.standard_normal((N, dm)).astype(np.float32)
+    w1 = np.zeros((N, N, dm), np.float32)
+    w2 = np.zeros((N, dm, N), np.float32)
+    for e in range(N):
+        w1[e, e, 3] = 1.0
+        w2[e, e, e] = 100.0 * (e + 1)
+    for cf in (4.0, 0.5):
+        res = O.layer_forward_top2(x, w_r, None, w1, w2, cf, ALPHA)
+        delta = res["out"] - x.astype(np.float64)
+        for t in range(T):
+            want = np.zeros(dm)
+            for r in range(2):
+                if not res["drop2"][r, t]:
+                    e = res["idx2"][r, t]
+                    want[e] += res["gate2"][r, t] * 100.0 * (e + 1)
+            np.testing.assert_allclose(delta[t], want, rtol=1e-12, atol=1e-12)
+        if cf == 0.5:
+            assert res["drop2"].any()
+    assert res["loss"] == pytest.approx(
+        ALPHA * N * np.sum(np.bincount(res["idx2"][0], minlength=N) / T * res["probs"].mean(0)))
+
+
 PINS = [pin_capacity, pin_softmax_hand, pin_router_invariants, pin_dispatch_hand,
         pin_dispatch_bruteforce, pin_dispatch_via_router, pin_aux_hand,
         pin_aux_uniform, pin_dense_reduction, pin_single_expert_signature,
-        pin_dropped_residual, pin_relu_active]
+        pin_dropped_residual, pin_relu_active, pin_top2_router_hand,
+        pin_top2_router_invariants, pin_top2_dispatch_hand, pin_top2_dispatch_bruteforce,
+        pin_top2_dense_reduction, pin_top2_signature]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda p: p.__name__)
@@ -363,7 +474,42 @@ def _mut_aux_no_N(real):
     return f
 
 
+def _mut_top2_second_highest_index(real):
+    def f(x, w_r, b_r=None):
+        r = real(x, w_r, b_r)
+        h32 = r["logits"].astype(np.float32)
+        T, N = h32.shape
+        rest = h32.copy()
+        rest[np.arange(T), r["idx2"][0]] = -np.inf
+        r["idx2"][1] = (N - 1 - np.argmax(rest[:, ::-1], axis=1)).astype(np.int64)
+        r["gate2"][1] = r["probs"][np.arange(T), r["idx2"][1]]
+        return r
+    return f
+
+
+def _mut_top2_renormalised(real):
+    def f(x, w_r, b_r=None):
+        r = real(x, w_r, b_r)
+        r["gate2"] = r["gate2"] / r["gate2"].sum(axis=0, keepdims=True)
+        return r
+    return f
+
+
+def _mut_top2_token_major(real):
+    def f(idx2, N, C):
+        idx2 = np.asarray(idx2)
+        T = idx2.shape[1]
+        d = orc.dispatch(idx2.T.reshape(-1), N, C)      # (t, r) order instead
+        rank = d["rank"].reshape(T, 2).T
+        st = np.where(d["slot_token"] >= 0, d["slot_token"] // 2, -1)
+        return {"rank": rank, "drop": rank >= C, "counts": d["counts"], "slot_token": st}
+    return f
+
+
 MUTANTS = {
+    "top2_second_on_last_tie": ("router_top2", _mut_top2_second_highest_index),
+    "top2_gates_renormalised": ("router_top2", _mut_top2_renormalised),
+    "top2_token_major_slots": ("dispatch_top2", _mut_top2_token_major),
     "capacity_floor": ("capacity", lambda real: _mut_capacity_floor),
     "argmax_last_on_tie": ("router", _mut_router_last_tie),
     "router_ignores_bias": ("router", _mut_router_no_bias),
