@@ -493,6 +493,20 @@ def kernel_rooflines(sm, cfg, wl, C, x, w_r, b_r, w1, w2, ws, flush, stream, dev
                          flags=sm.FLAG_ROWS_DISPATCHED)
     t_ffn = timed(lambda: sm.switch_expert_ffn(cfg_rows, x_disp, None, counts, w1, w2, y, ws))
     t_comb = timed(lambda: sm.switch_combine(cfg, x, idx, rank, drop, gate, y, out))
+    # the top-2 routing variant of the whole layer (capacity over 2T)
+    t_top2 = None
+    if N >= 2:
+        cfg2 = sm.config(T, d, F, N, wl.capacity_factor, dtype=wl.dtype, alpha=wl.alpha,
+                         flags=sm.FLAG_TOP2)
+        ws2 = sm.workspace(cfg2, device=dev)
+        idx2 = torch.empty(2 * T, **i32)
+        gate2 = torch.empty(2 * T, dtype=torch.float32, device=dev)
+        t_top2 = timed(lambda: sm.switch_layer_forward(cfg2, x, w_r, b_r, w1, w2, out, idx2,
+                                                       gate2, counts, loss, ws2))
+        st2, where2, info2 = sm.switch_get_device_error(ws2)
+        if st2 != 0:
+            raise RuntimeError(f"device error {st2} at {where2} ({info2}) in the top-2 layer")
+        del ws2
     t_aux = timed(lambda: sm.switch_aux_loss(cfg, counts, probs, loss, None, None, ws))
     st, where, info = sm.switch_get_device_error(ws)
     if st != 0:
@@ -518,6 +532,9 @@ def kernel_rooflines(sm, cfg, wl, C, x, w_r, b_r, w1, w2, ws, flush, stream, dev
                        "weight_bytes": 2 * N * d * F * es, "traffic": None},
         "combine": bw("combine", t_comb, 2 * T * d * es + T_kept * d * es + T * 13),
         "aux_loss_from_probs": bw("aux", t_aux, T * N * 4 + N * 4),
+        "layer_top2": None if t_top2 is None else {
+            "us": t_top2 * 1e6, "tokens_per_s": T / t_top2,
+            "capacity": sm.switch_capacity(2 * T, N, wl.capacity_factor)},
         "peaks": {"hbm_gbs": hbm, "bf16_tflops": pk["bf16_tflops"], "kind": pk_kind},
         "_T_kept": T_kept,
     }

@@ -82,8 +82,9 @@ enum {
   SWITCH_FLAG_GEMM_1SM = 32,         /* both expert GEMMs on single CTAs */
   SWITCH_FLAG_GEMM_PAIRS = 64,       /* GEMM1 on CTA pairs too (default: GEMM1 single CTAs,
                                         GEMM2 CTA pairs) */
-  SWITCH_FLAG_ROWS_DISPATCHED = 128  /* switch_expert_ffn: x is the dispatched row buffer
+  SWITCH_FLAG_ROWS_DISPATCHED = 128, /* switch_expert_ffn: x is the dispatched row buffer
                                         x_disp [N*C, d_model] from switch_dispatch */
+  SWITCH_FLAG_TOP2 = 512             /* top-k routing with k = 2 (see "Top-2 routing" below) */
 };
 
 typedef struct {
@@ -97,6 +98,25 @@ typedef struct {
   int32_t flags;            /* SWITCH_FLAG_* */
   int64_t spin_limit;       /* bounded-wait limit in SM cycles; 0 = default (~2 s) */
 } switch_config_t;
+
+/* Top-2 routing [P1 "Switch Routing: From Top-k to k = 1": the top-k set
+ * T of largest gates, output sum_{i in T} p_i(x) E_i(x), p the softmax over
+ * all N experts, not renormalised].  With SWITCH_FLAG_TOP2 (needs N >= 2):
+ *   - every per-token routing array has 2T entries, route-major: entry t is
+ *     the token's first choice, entry T + t its second (the largest other
+ *     logit, lowest index on ties);
+ *   - expert capacity is taken over the 2T assignments:
+ *     C = switch_capacity(2 T, N, capacity_factor) (each expert receives
+ *     tokens from two routes);
+ *   - dispatch ranks the assignments in that order, so every first choice
+ *     takes a slot before any second choice; slot_token holds tokens;
+ *   - combine adds both kept routes: x + sum_r gate_r * y[idx_r, rank_r];
+ *   - the load-balancing loss keeps f_i over the first choices;
+ *   - the tensor-core router supports it for terms x round_up(N, 32) <= 256
+ *     (else the fp32 FMA router runs); switch_dispatch needs idx (not
+ *     probs); switch_dispatch_noalloc returns SWITCH_ERR_UNSUPPORTED.
+ * Readings of the pages (first choices first, f over first choices) are the
+ * library's; the pages fix only the top-k set, the gates and the sum. */
 
 /* Expert capacity C = ceil(T x capacity_factor / N), computed exactly
  * [P1 "Expert Capacity and the Capacity Factor", capacity equation; the
@@ -113,6 +133,7 @@ switch_status_t switch_workspace_size(const switch_config_t* cfg, size_t* bytes)
  *   w_r    [N, d_model]  fp32;  b_r [N] fp32 or NULL (added to the logits)
  *   idx    [T] int32 out: expert of the largest logit, lowest index on ties
  *   gate   [T] fp32  out: p_idx(x)
+ *   (top-2: idx and gate [2T], see "Top-2 routing")
  *   probs  [T, N] fp32 out, or NULL: softmax probabilities
  * bf16 x runs on the tensor cores: bf16 x is exact, W_r is split into bf16
  * terms hi + lo (W_r to about 2^-17 relative; SWITCH_FLAG_ROUTER_3TERM adds
@@ -139,7 +160,8 @@ switch_status_t switch_router(const switch_config_t* cfg, const void* x,
  * x_disp [N, C, d_model] receives x[slot_token] per slot, zeros in padding.
  * Deterministic: slot order never depends on thread timing.
  * Expert ids outside [0, N) set SWITCH_ERR_DEVICE_BOUNDS in the error word
- * (the token is then treated as dropped). */
+ * (the token is then treated as dropped).  Top-2: idx, rank and drop have
+ * 2T entries (see "Top-2 routing"), counts counts both routes. */
 switch_status_t switch_dispatch(const switch_config_t* cfg, const int32_t* idx,
                                 const float* probs, int32_t* rank, uint8_t* drop,
                                 int32_t* counts, int32_t* slot_token, const void* x,
@@ -187,7 +209,8 @@ switch_status_t switch_expert_ffn(const switch_config_t* cfg, const void* x,
  * tokens pass through on the residual]:
  *   out[t] = x_residual[t] + (drop[t] ? 0 : gate[t] * y[idx[t], rank[t], :])
  * computed in fp32 and rounded once to the output dtype.  x_residual may be
- * NULL (no residual term).  y [N, C, d_model]. */
+ * NULL (no residual term).  y [N, C, d_model].  Top-2: both kept routes are
+ * added (first route first), idx/rank/drop/gate [2T]. */
 switch_status_t switch_combine(const switch_config_t* cfg, const void* x_residual,
                                const int32_t* idx, const int32_t* rank,
                                const uint8_t* drop, const float* gate, const void* y,
@@ -204,12 +227,14 @@ switch_status_t switch_aux_loss(const switch_config_t* cfg, const int32_t* count
                                 void* ws, size_t ws_bytes, void* stream);
 
 /* The whole layer on one stream with no host synchronisation:
- * router -> dispatch -> expert FFN (gather fused into GEMM1's operand
- * load, ReLU in its epilogue) -> gate x expert output + residual (fused
- * into GEMM2's epilogue) -> load-balancing loss.
+ * router -> dispatch (and, bf16, one copy of the routed rows) -> expert FFN
+ * (ReLU in GEMM1's epilogue) -> gate x expert output + residual (fused into
+ * GEMM2's epilogue; a separate combine with SWITCH_FLAG_UNFUSED_COMBINE or
+ * top-2) -> load-balancing loss.
  *   out [T, d_model] (same dtype as x)
  *   idx [T] int32, gate [T] fp32, counts [N] int32: optional outputs (NULL
- *   to skip); loss: device fp32 scalar or NULL.
+ *   to skip); loss: device fp32 scalar or NULL.  Top-2: idx and gate [2T],
+ *   counts over both routes.
  * Same results as the staged calls above in sequence. */
 switch_status_t switch_layer_forward(const switch_config_t* cfg, const void* x,
                                      const float* w_r, const float* b_r,

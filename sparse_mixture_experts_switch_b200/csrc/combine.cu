@@ -1,9 +1,11 @@
 // Combine and load-balancing loss.
 //
 // Combine: "Switch Transformers: scaling to trillion-parameter models",
-// section "Switch Routing: From Top-k to k = 1", combine equation with one
-// selected expert, y = p_i(x) E_i(x); a dropped token's output is the
-// residual (section "Expert Capacity and the Capacity Factor").
+// section "Switch Routing: From Top-k to k = 1", combine equation
+// y = sum over the selected set of p_i(x) E_i(x) (one expert, or two with
+// top-2 routing); a dropped assignment contributes nothing and a token with
+// none left is its residual (section "Expert Capacity and the Capacity
+// Factor").
 // Loss: section "The Load-Balancing Loss", alpha . N . sum_i f_i P_i.
 #include "kernels.cuh"
 
@@ -16,37 +18,53 @@ __global__ void __launch_bounds__(256) combine_kernel(
     int64_t T, int vec_per_row, int64_t C, const uint4* __restrict__ x,
     const int* __restrict__ idx, const int* __restrict__ rank,
     const uint8_t* __restrict__ drop, const float* __restrict__ gate,
-    const uint4* __restrict__ y, uint4* __restrict__ out, bool only_dropped) {
+    const uint4* __restrict__ y, uint4* __restrict__ out, bool only_dropped, int routes) {
   const int lane = threadIdx.x & 31;
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   for (int64_t t = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
        t < T; t += warps) {
+    // route r of token t is entry r * T + t (routes <= 2)
     const bool dropped = drop[t] != 0;
     if (only_dropped && !dropped) continue;
-    const float g = dropped ? 0.f : gate[t];
-    const uint4* yrow =
-        dropped ? nullptr : y + (static_cast<int64_t>(idx[t]) * C + rank[t]) * vec_per_row;
+    float g[2];
+    const uint4* yrow[2];
+    for (int r = 0; r < 2; ++r) {
+      const int64_t a = r * T + t;
+      const bool here = r < routes && drop[a] == 0;
+      g[r] = here ? gate[a] : 0.f;
+      yrow[r] = here ? y + (static_cast<int64_t>(idx[a]) * C + rank[a]) * vec_per_row : nullptr;
+    }
     const uint4* xrow = x ? x + t * vec_per_row : nullptr;
     uint4* orow = out + t * vec_per_row;
+    if (yrow[0] == nullptr && yrow[1] == nullptr) {
+      // nothing kept: the residual row as it is (bit for bit, -0 included)
+      for (int v = lane; v < vec_per_row; v += 32)
+        orow[v] = xrow ? __ldg(xrow + v) : make_uint4(0, 0, 0, 0);
+      continue;
+    }
     for (int v = lane; v < vec_per_row; v += 32) {
       const uint4 xv = xrow ? __ldg(xrow + v) : make_uint4(0, 0, 0, 0);
-      const uint4 yv = yrow ? __ldg(yrow + v) : make_uint4(0, 0, 0, 0);
+      const uint4 y0 = yrow[0] ? __ldg(yrow[0] + v) : make_uint4(0, 0, 0, 0);
+      const uint4 y1 = yrow[1] ? __ldg(yrow[1] + v) : make_uint4(0, 0, 0, 0);
       uint4 o;
       if (kBF16) {
         const uint32_t* xa = &xv.x;
-        const uint32_t* ya = &yv.x;
+        const uint32_t* ya = &y0.x;
+        const uint32_t* yb = &y1.x;
         uint32_t* oa = &o.x;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const float lo = fmaf(g, bf16_lo(ya[i]), bf16_lo(xa[i]));
-          const float hi = fmaf(g, bf16_hi(ya[i]), bf16_hi(xa[i]));
+          const float lo = fmaf(g[1], bf16_lo(yb[i]), fmaf(g[0], bf16_lo(ya[i]), bf16_lo(xa[i])));
+          const float hi = fmaf(g[1], bf16_hi(yb[i]), fmaf(g[0], bf16_hi(ya[i]), bf16_hi(xa[i])));
           oa[i] = pack_bf16x2(lo, hi);
         }
       } else {
-        o.x = __float_as_uint(fmaf(g, __uint_as_float(yv.x), __uint_as_float(xv.x)));
-        o.y = __float_as_uint(fmaf(g, __uint_as_float(yv.y), __uint_as_float(xv.y)));
-        o.z = __float_as_uint(fmaf(g, __uint_as_float(yv.z), __uint_as_float(xv.z)));
-        o.w = __float_as_uint(fmaf(g, __uint_as_float(yv.w), __uint_as_float(xv.w)));
+        const float* xa = reinterpret_cast<const float*>(&xv);
+        const float* ya = reinterpret_cast<const float*>(&y0);
+        const float* yb = reinterpret_cast<const float*>(&y1);
+        float* oa = reinterpret_cast<float*>(&o);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) oa[i] = fmaf(g[1], yb[i], fmaf(g[0], ya[i], xa[i]));
       }
       orow[v] = o;
     }
@@ -56,7 +74,7 @@ __global__ void __launch_bounds__(256) combine_kernel(
 cudaError_t launch_combine(int64_t T, int d, int64_t C, bool bf16, const void* x,
                            const int* idx, const int* rank, const uint8_t* drop,
                            const float* gate, const void* y, void* out, bool only_dropped,
-                           cudaStream_t st) {
+                           int routes, cudaStream_t st) {
   const int vec = d * (bf16 ? 2 : 4) / 16;
   int64_t blocks = (T + 7) / 8;
   if (blocks > 148 * 16) blocks = 148 * 16;
@@ -64,11 +82,11 @@ cudaError_t launch_combine(int64_t T, int d, int64_t C, bool bf16, const void* x
   if (bf16)
     combine_kernel<true><<<static_cast<int>(blocks), 256, 0, st>>>(
         T, vec, C, static_cast<const uint4*>(x), idx, rank, drop, gate,
-        static_cast<const uint4*>(y), static_cast<uint4*>(out), only_dropped);
+        static_cast<const uint4*>(y), static_cast<uint4*>(out), only_dropped, routes);
   else
     combine_kernel<false><<<static_cast<int>(blocks), 256, 0, st>>>(
         T, vec, C, static_cast<const uint4*>(x), idx, rank, drop, gate,
-        static_cast<const uint4*>(y), static_cast<uint4*>(out), only_dropped);
+        static_cast<const uint4*>(y), static_cast<uint4*>(out), only_dropped, routes);
   return cudaGetLastError();
 }
 

@@ -159,7 +159,7 @@ __global__ void __launch_bounds__(256) finalize_kernel(
     int64_t T, int N, int64_t C, int ntiles, const int* __restrict__ idx,
     const int* __restrict__ local_rank, const int* __restrict__ base,
     const int* __restrict__ counts, int* __restrict__ rank, uint8_t* __restrict__ drop,
-    int* __restrict__ slot_token, int* __restrict__ mtile_start) {
+    int* __restrict__ slot_token, int* __restrict__ mtile_start, int64_t tok_mod) {
   if (blockIdx.x == 0 && threadIdx.x < 32 && mtile_start != nullptr)
     mtile_prefix_warp(N, C, counts, mtile_start);
   const int64_t nslots = static_cast<int64_t>(N) * C;
@@ -174,7 +174,9 @@ __global__ void __launch_bounds__(256) finalize_kernel(
       if (e >= 0 && e < N && lr >= 0) {
         r = base[static_cast<int64_t>(e) * ntiles + (i / kTileTok)] + lr;
         dropped = r >= C;
-        if (!dropped) slot_token[static_cast<int64_t>(e) * C + r] = static_cast<int>(i);
+        if (!dropped)
+          slot_token[static_cast<int64_t>(e) * C + r] =
+              static_cast<int>(tok_mod > 0 && i >= tok_mod ? i - tok_mod : i);
       }
       rank[i] = r;
       drop[i] = dropped ? 1 : 0;
@@ -191,13 +193,14 @@ __global__ void __launch_bounds__(256) finalize_kernel(
 cudaError_t launch_finalize(int64_t T, int N, int64_t C, int ntiles, const int* idx,
                             const int* local_rank, const int* base, const int* counts,
                             int* rank, uint8_t* drop, int* slot_token, int* mtile_start,
-                            cudaStream_t st) {
+                            int64_t tok_mod, cudaStream_t st) {
   const int64_t work = T > static_cast<int64_t>(N) * C ? T : static_cast<int64_t>(N) * C;
   int64_t blocks = (work + 255) / 256;
   if (blocks > 148 * 16) blocks = 148 * 16;
   if (blocks < 1) blocks = 1;
   finalize_kernel<<<static_cast<int>(blocks), 256, 0, st>>>(
-      T, N, C, ntiles, idx, local_rank, base, counts, rank, drop, slot_token, mtile_start);
+      T, N, C, ntiles, idx, local_rank, base, counts, rank, drop, slot_token, mtile_start,
+      tok_mod);
   return cudaGetLastError();
 }
 

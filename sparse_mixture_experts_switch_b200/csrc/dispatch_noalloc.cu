@@ -64,6 +64,7 @@ extern "C" switch_status_t switch_dispatch_noalloc(const switch_config_t* cfg,
   const int64_t T = cfg->T;
   const int N = cfg->n_experts;
   if (T < 0 || N < 1 || N > 1024) return SWITCH_ERR_INVALID_ARG;
+  if (cfg->flags & SWITCH_FLAG_TOP2) return SWITCH_ERR_UNSUPPORTED;   // one route only
   const int64_t C = switch_capacity(T, N, cfg->capacity_factor);
   if (C < 0) return SWITCH_ERR_INVALID_ARG;
   if (C > INT_MAX / N) return SWITCH_ERR_UNSUPPORTED;
@@ -92,7 +93,7 @@ extern "C" switch_status_t switch_dispatch_noalloc(const switch_config_t* cfg,
     return SWITCH_ERR_CUDA;
   if (smoe::launch_scan(N, nt, hist, scan, counts, st) != cudaSuccess) return SWITCH_ERR_CUDA;
   if (smoe::launch_finalize(T, N, C, nt, idx_src, local_rank, scan, counts, rank, drop,
-                            slot_token, nullptr, st) != cudaSuccess)
+                            slot_token, nullptr, 0, st) != cudaSuccess)
     return SWITCH_ERR_CUDA;
   return SWITCH_OK;
 }

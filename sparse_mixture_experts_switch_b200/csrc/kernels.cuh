@@ -20,10 +20,12 @@ cudaError_t launch_scan(int N, int ntiles, const int* hist, int* base, int* coun
                         cudaStream_t st);
 // rank/drop per token, slot_token (kept tokens and -1 padding), and the
 // per-expert prefix of 128-row M tiles mtile_start[N + 1].
+// tok_mod > 0: entries are route-major assignments of tok_mod tokens, and
+// slot_token holds the token (assignment mod tok_mod).
 cudaError_t launch_finalize(int64_t T, int N, int64_t C, int ntiles, const int* idx,
                             const int* local_rank, const int* base, const int* counts,
                             int* rank, uint8_t* drop, int* slot_token, int* mtile_start,
-                            cudaStream_t st);
+                            int64_t tok_mod, cudaStream_t st);
 // Only mtile_start from counts (for a standalone expert-FFN call).
 cudaError_t launch_mtile_table(int N, int64_t C, const int* counts, int* mtile_start,
                                cudaStream_t st);
@@ -32,12 +34,13 @@ cudaError_t launch_gather_rows(int64_t nslots, int64_t row_bytes, const int* slo
                                const void* x, void* x_disp, cudaStream_t st);
 
 // ------------------------------------------------------- combine / loss
-// out[t] = x[t] + (drop ? 0 : gate * y[idx*C + rank]); fp32 math, one rounding.
-// only_dropped: touch only dropped tokens (kept ones are written elsewhere).
+// out[t] = x[t] + sum over routes r of (drop ? 0 : gate * y[idx*C + rank]) at
+// entry r*T + t; fp32 math, one rounding.  only_dropped (one route): touch
+// only dropped tokens (kept ones are written elsewhere).
 cudaError_t launch_combine(int64_t T, int d, int64_t C, bool bf16, const void* x,
                            const int* idx, const int* rank, const uint8_t* drop,
                            const float* gate, const void* y, void* out, bool only_dropped,
-                           cudaStream_t st);
+                           int routes, cudaStream_t st);
 // psum[blk][e] = sum of probs rows [blk*128, blk*128 + 128) (fixed order).
 cudaError_t launch_prob_colsum(int64_t T, int N, const float* probs, float* psum,
                                cudaStream_t st);
@@ -57,6 +60,8 @@ struct RouterOut {
   float* psum;       // [nparts, N] or null (per-tile sums of probs)
   int* hist;         // [N, ntiles] or null (tensor-core router only)
   int* local_rank;   // [T] or null (tensor-core router only)
+  int* idx2;         // top-2: [T] second choices, else null
+  float* gate2;      // top-2: [T] their gates
 };
 // CUDA-core fp32 router; psum parts are 64-token blocks.  `logits` is a
 // [T, N] fp32 scratch.
@@ -70,6 +75,8 @@ cudaError_t launch_router_tc(int64_t T, int d, int N, int terms, const void* x,
                              RouterOut o, int ntiles, DevErr* err, long long spin,
                              int num_sms, cudaStream_t st);
 bool router_tc_supported(int N, int d, int terms);
+// The CTA-pair router (the one with top-2 support) applies: terms x N_pad <= 256.
+bool router_pair_supported(int N, int terms);
 // Bytes of the bf16 split-weight scratch launch_router_tc needs (3 terms).
 size_t router_wsplit_bytes(int N, int d);
 

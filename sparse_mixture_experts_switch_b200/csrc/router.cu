@@ -39,7 +39,8 @@ template <bool kBF16>
 __global__ void __launch_bounds__(256) router_simt_kernel(
     int64_t T, int d, int N, const void* __restrict__ xv, const float* __restrict__ w_r,
     const float* __restrict__ b_r, float* __restrict__ logits, int* __restrict__ idx,
-    float* __restrict__ gate, float* __restrict__ probs, float* __restrict__ psum) {
+    float* __restrict__ gate, float* __restrict__ probs, float* __restrict__ psum,
+    int* __restrict__ idx2, float* __restrict__ gate2) {
   extern __shared__ float sh[];
   float* Xs = sh;                              // [64][33]
   float* Ws = sh + kSimtTok * (kSimtKC + 1);   // [32][128]
@@ -107,17 +108,33 @@ __global__ void __launch_bounds__(256) router_simt_kernel(
     const int64_t t = tok0 + w * 8 + i;
     if (t >= T) break;
     const float* row = logits + t * N;
-    float best = -INFINITY;
-    int best_e = 0x7fffffff;
+    // the two largest logits (value, index), lowest index first on ties:
+    // per lane over its experts in increasing order, then merged across lanes
+    float best = -INFINITY, sec = -INFINITY;
+    int best_e = 0x7fffffff, sec_e = 0x7fffffff;
     for (int e = lane; e < N; e += 32) {
       const float h = row[e];
-      if (h > best) { best = h; best_e = e; }
+      if (h > best) { sec = best; sec_e = best_e; best = h; best_e = e; }
+      else if (h > sec) { sec = h; sec_e = e; }
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {
       const float ob = __shfl_xor_sync(0xffffffffu, best, off);
       const int oe = __shfl_xor_sync(0xffffffffu, best_e, off);
-      if (ob > best || (ob == best && oe < best_e)) { best = ob; best_e = oe; }
+      const float os = __shfl_xor_sync(0xffffffffu, sec, off);
+      const int ose = __shfl_xor_sync(0xffffffffu, sec_e, off);
+      if (ob > best || (ob == best && oe < best_e)) {
+        // theirs first; second = better of ours-first and theirs-second
+        const bool mine = best > os || (best == os && best_e < ose);
+        sec = mine ? best : os;
+        sec_e = mine ? best_e : ose;
+        best = ob;
+        best_e = oe;
+      } else {
+        const bool mine = sec > ob || (sec == ob && sec_e < oe);
+        sec = mine ? sec : ob;
+        sec_e = mine ? sec_e : oe;
+      }
     }
     float s = 0.f;
     for (int e = lane; e < N; e += 32) s += exp2f((row[e] - best) * kLog2e);
@@ -132,6 +149,10 @@ __global__ void __launch_bounds__(256) router_simt_kernel(
     if (lane == 0) {
       idx[t] = best_e;
       gate[t] = inv;
+      if (idx2 != nullptr) {
+        idx2[t] = sec_e;
+        gate2[t] = exp2f((sec - best) * kLog2e) * inv;
+      }
     }
   }
   __syncthreads();
@@ -153,10 +174,11 @@ cudaError_t launch_router_simt(int64_t T, int d, int N, bool bf16, const void* x
   if (sizeof(float) * 8 * N > sm) sm = sizeof(float) * 8 * N;
   if (bf16)
     router_simt_kernel<true><<<blocks, 256, sm, st>>>(T, d, N, x, w_r, b_r, logits, o.idx,
-                                                     o.gate, o.probs, o.psum);
+                                                     o.gate, o.probs, o.psum, o.idx2, o.gate2);
   else
     router_simt_kernel<false><<<blocks, 256, sm, st>>>(T, d, N, x, w_r, b_r, logits, o.idx,
-                                                      o.gate, o.probs, o.psum);
+                                                      o.gate, o.probs, o.psum, o.idx2,
+                                                      o.gate2);
   return cudaGetLastError();
 }
 
@@ -598,6 +620,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kRouterThreads, 1)
   float* xm = reinterpret_cast<float*>(cnt + 2 * 4 * N_pad);  // [2 parity][2 half][128]
   float* xs = xm + 2 * 2 * 128;
   int* xb = reinterpret_cast<int*>(xs + 2 * 2 * 128);
+  float* xm2 = reinterpret_cast<float*>(xb + 2 * 2 * 128);      // top-2: the half's second
+  int* xb2 = reinterpret_cast<int*>(xm2 + 2 * 2 * 128);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -795,6 +819,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kRouterThreads, 1)
       for (int i = 0; i < NH * 32; ++i)
         if (i < N_h && v[i] == m_h) bq[i & 3] = min(bq[i & 3], i);
       const int b_h = min(min(bq[0], bq[1]), min(bq[2], bq[3]));
+      // top-2: the half's largest logit other than b_h, first index of it
+      float m2_h = -INFINITY;
+      int b2_h = 0x7fffffff;
+      if (prm.o.idx2 != nullptr) {
+        float mq2[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int i = 0; i < NH * 32; ++i)
+          if (i < N_h && i != b_h) mq2[i & 3] = fmaxf(mq2[i & 3], v[i]);
+        m2_h = fmaxf(fmaxf(mq2[0], mq2[1]), fmaxf(mq2[2], mq2[3]));
+        int bq2[4] = {0x7fffffff, 0x7fffffff, 0x7fffffff, 0x7fffffff};
+#pragma unroll
+        for (int i = 0; i < NH * 32; ++i)
+          if (i < N_h && i != b_h && v[i] == m2_h) bq2[i & 3] = min(bq2[i & 3], i);
+        b2_h = min(min(bq2[0], bq2[1]), min(bq2[2], bq2[3]));
+      }
       const float mL_h = m_h * kLog2e;
       float sq[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -808,6 +847,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kRouterThreads, 1)
       xm_p[h * 128 + row] = m_h;
       xs_p[h * 128 + row] = (sq[0] + sq[1]) + (sq[2] + sq[3]);
       xb_p[h * 128 + row] = b_h == 0x7fffffff ? b_h : h * NH * 32 + b_h;
+      if (prm.o.idx2 != nullptr) {
+        xm2[par * 256 + h * 128 + row] = m2_h;
+        xb2[par * 256 + h * 128 + row] = b2_h == 0x7fffffff ? b2_h : h * NH * 32 + b2_h;
+      }
       int* cnt_p = cnt + par * 4 * N_pad;
       for (int i = et; i < 4 * N_pad; i += 256) cnt_p[i] = 0;
       named_bar_sync(1, 256);
@@ -818,6 +861,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kRouterThreads, 1)
                       xs_p[128 + row] * exp2_fast((m1 - m) * kLog2e);
       const int best = m0 >= m1 ? xb_p[row] : xb_p[128 + row];
       const float inv = 1.f / s;
+      // top-2: the better of the other half's first and this half's second
+      // (half 0 holds the lower indices, so it wins ties)
+      int second = 0;
+      float gate_2 = 0.f;
+      if (prm.o.idx2 != nullptr) {
+        float v2;
+        if (m0 >= m1) {
+          const float a2 = xm2[par * 256 + row];
+          v2 = a2 >= m1 ? a2 : m1;
+          second = a2 >= m1 ? xb2[par * 256 + row] : xb_p[128 + row];
+        } else {
+          const float b2 = xm2[par * 256 + 128 + row];
+          v2 = m0 >= b2 ? m0 : b2;
+          second = m0 >= b2 ? xb_p[row] : xb2[par * 256 + 128 + row];
+        }
+        gate_2 = exp2_fast((v2 - m) * kLog2e) * inv;
+      }
       const float scale = valid ? exp2_fast((m_h - m) * kLog2e) * inv : 0.f;
       float* red_p = red + par * 4 * N_pad;
 #pragma unroll
@@ -855,6 +915,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kRouterThreads, 1)
       if (h == 0 && valid) {
         prm.o.idx[t] = best;
         prm.o.gate[t] = inv;
+        if (prm.o.idx2 != nullptr) {
+          prm.o.idx2[t] = second;
+          prm.o.gate2[t] = gate_2;
+        }
         if (prm.o.local_rank != nullptr) {
           int rr = rank_w;
           for (int qq = 0; qq < q; ++qq) rr += cnt_p[qq * N_pad + best];
@@ -895,6 +959,8 @@ static int router_n_pad(int N) { return (N + 31) / 32 * 32; }
 size_t router_wsplit_bytes(int N, int d) {
   return sizeof(__nv_bfloat16) * 3 * static_cast<size_t>(router_n_pad(N)) * d;
 }
+
+bool router_pair_supported(int N, int terms) { return terms * router_n_pad(N) <= 256; }
 
 // Every weight term keeps its own accumulator columns: terms x N_pad <= 512.
 bool router_tc_supported(int N, int d, int terms) {
@@ -954,7 +1020,7 @@ static cudaError_t launch_router_pair(int64_t T, int d, int N, int N_pad, int te
   p.err = err;
   p.spin = spin;
   const size_t tail_bytes =
-      512 + sizeof(float) * N_pad * 9 + sizeof(int) * N_pad * 8 + 3 * sizeof(float) * 512;
+      512 + sizeof(float) * N_pad * 9 + sizeof(int) * N_pad * 8 + 5 * sizeof(float) * 512;
   const size_t budget = 227 * 1024 - 1024 - tail_bytes;
   int stages = static_cast<int>(budget / (p.x_bytes + p.w_bytes));
   if (stages > kRouterPairMaxStages) stages = kRouterPairMaxStages;

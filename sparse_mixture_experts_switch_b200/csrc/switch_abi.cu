@@ -38,8 +38,8 @@ int64_t capacity_exact(int64_t T, int32_t N, double cf) {
 }
 
 struct Layout {
-  size_t err, hist, base, psum, fpsc, local_rank, idx, gate, rank, drop, counts, slot_token,
-      mtile_start, wsplit, logits, xdisp, hbuf, ybuf, total;
+  size_t err, hist, base, psum, fpsc, local_rank, idx, gate, rank, drop, counts, counts1,
+      slot_token, mtile_start, wsplit, logits, xdisp, hbuf, ybuf, total;
 };
 
 // Bytes 16..19 of the workspace: the loss kernel's completion ticket (kept
@@ -48,11 +48,16 @@ constexpr size_t kTicketOffset = 16;
 
 int ntiles_of(int64_t T) { return static_cast<int>((T + kTileTok - 1) / kTileTok); }
 
+// Routes per token: 2 with SWITCH_FLAG_TOP2, else 1.  Dispatch works on the
+// routes x T (token, expert) assignments, route-major.
+int routes_of(const switch_config_t& c) { return (c.flags & SWITCH_FLAG_TOP2) ? 2 : 1; }
+
 Layout layout_for(const switch_config_t& c, int64_t C) {
   const int64_t T = c.T;
+  const int64_t A = routes_of(c) * T;        // assignments
   const int64_t N = c.n_experts;
   const size_t es = c.dtype == SWITCH_BF16 ? 2 : 4;
-  const int64_t nt = ntiles_of(T);
+  const int64_t nt = ntiles_of(A);
   const int64_t nparts = (T + 63) / 64;
   const int64_t slots = N * C;
   Layout L{};
@@ -67,12 +72,13 @@ Layout layout_for(const switch_config_t& c, int64_t C) {
   L.base = take(sizeof(int) * N * nt);
   L.psum = take(sizeof(float) * N * nparts);
   L.fpsc = take(sizeof(double) * N * kAuxChunks);
-  L.local_rank = take(sizeof(int) * T);
-  L.idx = take(sizeof(int) * T);
-  L.gate = take(sizeof(float) * T);
-  L.rank = take(sizeof(int) * T);
-  L.drop = take(T);
+  L.local_rank = take(sizeof(int) * A);
+  L.idx = take(sizeof(int) * A);
+  L.gate = take(sizeof(float) * A);
+  L.rank = take(sizeof(int) * A);
+  L.drop = take(A);
   L.counts = take(sizeof(int) * N);
+  L.counts1 = take(sizeof(int) * N);
   L.slot_token = take(sizeof(int) * slots);
   L.mtile_start = take(sizeof(int) * (N + 1));
   L.wsplit = take(router_wsplit_bytes(c.n_experts, c.d_model));
@@ -90,7 +96,11 @@ switch_status_t validate(const switch_config_t* c, int64_t* C_out) {
       c->n_experts > 1024 || (c->dtype != SWITCH_F32 && c->dtype != SWITCH_BF16) ||
       c->spin_limit < 0)
     return SWITCH_ERR_INVALID_ARG;
-  const int64_t C = capacity_exact(c->T, c->n_experts, c->capacity_factor);
+  if ((c->flags & SWITCH_FLAG_TOP2) && (c->n_experts < 2 || c->T > INT_MAX / 2))
+    return SWITCH_ERR_INVALID_ARG;
+  // capacity over the routes x T assignments: each expert takes tokens from
+  // every route
+  const int64_t C = capacity_exact(routes_of(*c) * c->T, c->n_experts, c->capacity_factor);
   if (C < 0) return SWITCH_ERR_INVALID_ARG;
   if (c->dtype == SWITCH_BF16 && (c->d_model % 64 != 0 || c->d_ff % 64 != 0))
     return SWITCH_ERR_UNSUPPORTED;
@@ -164,9 +174,11 @@ int router_terms(const switch_config_t* c) {
   return (c->flags & SWITCH_FLAG_ROUTER_3TERM) ? 3 : 2;
 }
 
+// Tensor-core router; top-2 only on the CTA-pair kernel (terms x N_pad <= 256).
 bool use_tc_router(const switch_config_t* c) {
   return c->dtype == SWITCH_BF16 && !(c->flags & SWITCH_FLAG_ROUTER_SIMT) &&
-         router_tc_supported(c->n_experts, c->d_model, router_terms(c));
+         router_tc_supported(c->n_experts, c->d_model, router_terms(c)) &&
+         (!(c->flags & SWITCH_FLAG_TOP2) || router_pair_supported(c->n_experts, router_terms(c)));
 }
 
 }  // namespace
@@ -194,7 +206,9 @@ switch_status_t switch_router(const switch_config_t* cfg, const void* x, const f
   if (s != SWITCH_OK || cfg->T == 0) return s;
   if (!x || !w_r || !idx || !gate || !aligned16(x) || (probs && !aligned16(probs)))
     return SWITCH_ERR_INVALID_ARG;
-  RouterOut o{idx, gate, probs, c.at<float>(c.L.psum), nullptr, nullptr};
+  const bool top2 = routes_of(*cfg) == 2;
+  RouterOut o{idx, gate, probs, c.at<float>(c.L.psum), nullptr, nullptr,
+              top2 ? idx + cfg->T : nullptr, top2 ? gate + cfg->T : nullptr};
   if (use_tc_router(cfg)) {
     return cuda_status(launch_router_tc(cfg->T, cfg->d_model, cfg->n_experts,
                                         router_terms(cfg), x, w_r, b_r, c.ws + c.L.wsplit, o,
@@ -215,15 +229,18 @@ switch_status_t switch_dispatch(const switch_config_t* cfg, const int32_t* idx,
   if (s != SWITCH_OK || cfg->T == 0) return s;
   if ((!idx && !probs) || !rank || !drop || !counts || !slot_token) return SWITCH_ERR_INVALID_ARG;
   if (x_disp && (!x || !aligned16(x) || !aligned16(x_disp))) return SWITCH_ERR_INVALID_ARG;
+  const bool top2 = routes_of(*cfg) == 2;
+  if (top2 && !idx) return SWITCH_ERR_INVALID_ARG;      // top-2 dispatch takes the choices
   const int N = cfg->n_experts;
-  const int nt = ntiles_of(cfg->T);
+  const int64_t A = routes_of(*cfg) * cfg->T;           // assignments, route-major
+  const int nt = ntiles_of(A);
   int* idx_src = idx ? const_cast<int*>(idx) : c.at<int>(c.L.idx);
-  SMOE_TRY(launch_tile_rank(cfg->T, N, idx, probs, idx ? nullptr : idx_src,
+  SMOE_TRY(launch_tile_rank(A, N, idx, probs, idx ? nullptr : idx_src,
                             c.at<int>(c.L.local_rank), c.at<int>(c.L.hist), nt, c.err, c.st));
   SMOE_TRY(launch_scan(N, nt, c.at<int>(c.L.hist), c.at<int>(c.L.base), counts, c.st));
-  SMOE_TRY(launch_finalize(cfg->T, N, c.C, nt, idx_src, c.at<int>(c.L.local_rank),
+  SMOE_TRY(launch_finalize(A, N, c.C, nt, idx_src, c.at<int>(c.L.local_rank),
                            c.at<int>(c.L.base), counts, rank, drop, slot_token,
-                           c.at<int>(c.L.mtile_start), c.st));
+                           c.at<int>(c.L.mtile_start), top2 ? cfg->T : 0, c.st));
   if (x_disp) {
     const int64_t row_bytes =
         static_cast<int64_t>(cfg->d_model) * (cfg->dtype == SWITCH_BF16 ? 2 : 4);
@@ -290,7 +307,7 @@ switch_status_t switch_combine(const switch_config_t* cfg, const void* x_residua
     return SWITCH_ERR_INVALID_ARG;
   return cuda_status(launch_combine(cfg->T, cfg->d_model, C, cfg->dtype == SWITCH_BF16,
                                     x_residual, idx, rank, drop, gate, y, out, false,
-                                    static_cast<cudaStream_t>(stream)));
+                                    routes_of(*cfg), static_cast<cudaStream_t>(stream)));
 }
 
 switch_status_t switch_aux_loss(const switch_config_t* cfg, const int32_t* counts,
@@ -322,6 +339,9 @@ switch_status_t switch_layer_forward(const switch_config_t* cfg, const void* x,
   const int N = cfg->n_experts;
   const int nt = ntiles_of(T);
   const bool bf16 = cfg->dtype == SWITCH_BF16;
+  const bool top2 = routes_of(*cfg) == 2;
+  const int64_t A = routes_of(*cfg) * T;                // assignments, route-major
+  const int nta = ntiles_of(A);
   int* idx_p = idx ? idx : c.at<int>(c.L.idx);
   float* gate_p = gate ? gate : c.at<float>(c.L.gate);
   int* counts_p = counts ? counts : c.at<int>(c.L.counts);
@@ -330,27 +350,41 @@ switch_status_t switch_layer_forward(const switch_config_t* cfg, const void* x,
   float* psum = c.at<float>(c.L.psum);
   int nparts = nt;
 
-  // 1. router (+ per-tile ranks and histograms on the tensor-core path)
+  // 1. router (+ per-tile ranks and histograms of the first choices on the
+  // tensor-core path)
+  RouterOut o{idx_p, gate_p, nullptr, psum, nullptr, nullptr,
+              top2 ? idx_p + T : nullptr, top2 ? gate_p + T : nullptr};
   if (use_tc_router(cfg)) {
-    RouterOut o{idx_p, gate_p, nullptr, psum, hist, local_rank};
+    o.hist = hist;
+    o.local_rank = local_rank;
     SMOE_TRY(launch_router_tc(T, cfg->d_model, N, router_terms(cfg), x, w_r, b_r,
                               c.ws + c.L.wsplit, o, nt, c.err, c.spin, c.num_sms, c.st));
   } else {
-    RouterOut o{idx_p, gate_p, nullptr, psum, nullptr, nullptr};
     SMOE_TRY(launch_router_simt(T, cfg->d_model, N, bf16, x, w_r, b_r,
                                 c.at<float>(c.L.logits), o, &nparts, c.st));
     SMOE_TRY(launch_tile_rank(T, N, idx_p, nullptr, nullptr, local_rank, hist, nt, c.err,
                               c.st));
   }
-  // 2-3. dispatch: scan over tiles, then rank / drop / slots / tile table
-  SMOE_TRY(launch_scan(N, nt, hist, c.at<int>(c.L.base), counts_p, c.st));
+  // 2-3. dispatch: scan over tiles, then rank / drop / slots / tile table.
+  // Top-2: the first choices' totals are the loss's counts; then the 2T
+  // assignments are ranked as one sequence, first choices first.
+  int* counts_loss = counts_p;
+  if (top2) {
+    counts_loss = c.at<int>(c.L.counts1);
+    SMOE_TRY(launch_scan(N, nt, hist, c.at<int>(c.L.base), counts_loss, c.st));
+    SMOE_TRY(launch_tile_rank(A, N, idx_p, nullptr, nullptr, local_rank, hist, nta, c.err,
+                              c.st));
+  }
+  SMOE_TRY(launch_scan(N, nta, hist, c.at<int>(c.L.base), counts_p, c.st));
   int* slot_token = c.at<int>(c.L.slot_token);
   int* rank = c.at<int>(c.L.rank);
   uint8_t* drop = c.at<uint8_t>(c.L.drop);
-  SMOE_TRY(launch_finalize(T, N, c.C, nt, idx_p, local_rank, c.at<int>(c.L.base), counts_p,
-                           rank, drop, slot_token, c.at<int>(c.L.mtile_start), c.st));
-  // 4. experts, with the combine fused into the second GEMM unless asked not to
-  const bool fused = !(cfg->flags & SWITCH_FLAG_UNFUSED_COMBINE);
+  SMOE_TRY(launch_finalize(A, N, c.C, nta, idx_p, local_rank, c.at<int>(c.L.base), counts_p,
+                           rank, drop, slot_token, c.at<int>(c.L.mtile_start),
+                           top2 ? T : 0, c.st));
+  // 4. experts, with the combine fused into the second GEMM unless asked not
+  // to (or top-2: two experts write each token, so Y, then one combine)
+  const bool fused = !(cfg->flags & SWITCH_FLAG_UNFUSED_COMBINE) && !top2;
   const void* x_res = (cfg->flags & SWITCH_FLAG_NO_RESIDUAL) ? nullptr : x;
   FfnArgs a{};
   a.T = T;
@@ -384,11 +418,12 @@ switch_status_t switch_layer_forward(const switch_config_t* cfg, const void* x,
   SMOE_TRY(bf16 ? launch_expert_ffn_bf16(a, c.st) : launch_expert_ffn_f32(a, c.st));
   // 5. dropped tokens (fused) or every token (unfused)
   SMOE_TRY(launch_combine(T, cfg->d_model, c.C, bf16, x_res, idx_p, rank, drop, gate_p,
-                          c.ws + c.L.ybuf, out, fused, c.st));
-  // 6. load-balancing loss
+                          c.ws + c.L.ybuf, out, fused, routes_of(*cfg), c.st));
+  // 6. load-balancing loss (f_i over the first choices)
   if (loss)
-    SMOE_TRY(launch_aux_loss(T, N, nparts, cfg->alpha, counts_p, psum, loss, nullptr, nullptr,
-                             c.at<double>(c.L.fpsc), c.at<unsigned>(kTicketOffset), c.st));
+    SMOE_TRY(launch_aux_loss(T, N, nparts, cfg->alpha, counts_loss, psum, loss, nullptr,
+                             nullptr, c.at<double>(c.L.fpsc), c.at<unsigned>(kTicketOffset),
+                             c.st));
   return SWITCH_OK;
 }
 

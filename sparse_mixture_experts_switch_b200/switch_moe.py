@@ -28,6 +28,7 @@ FLAG_NO_RESIDUAL = 16
 FLAG_GEMM_1SM = 32
 FLAG_GEMM_PAIRS = 64
 FLAG_ROWS_DISPATCHED = 128
+FLAG_TOP2 = 512
 
 
 class SwitchConfig(ctypes.Structure):

@@ -1,0 +1,267 @@
+"""GPU parity of top-2 routing (SWITCH_FLAG_TOP2) against the oracle's top-2
+functions: router choices and gates, dispatch of the 2T assignments, the
+two-route combine and the whole layer, end to end and at full size.
+
+Routing rule: the GPU's first choice may differ from the oracle's only where
+the oracle's first/second probability margin is below 1e-6; its second
+choice only there or where the second/third margin is below 1e-6 (flips
+counted).  The oracle is then re-based on the GPU's choices, as in the
+top-1 tests, so every other output is compared element by element.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle.switch_oracle as orc
+from switch_inputs import Workload, WORKLOADS, make_inputs, make_x, make_router, as_f64
+from gpu_util import (dev_float, host_f64, rms_ratio, rel_err, PROB_RTOL, MARGIN_FLIP,
+                      BF16_RMS_TOL, F32_RMS_TOL, LOSS_RTOL)
+
+pytestmark = pytest.mark.gpu
+
+I32 = dict(dtype=torch.int32, device="cuda")
+
+
+@pytest.fixture(scope="module")
+def sm():
+    from sparse_mixture_experts_switch_b200 import switch_moe
+    return switch_moe
+
+
+def _cfg(sm, wl, flags=0):
+    return sm.config(wl.T, wl.d_model, wl.d_ff, wl.n_experts, wl.capacity_factor,
+                     dtype=wl.dtype, alpha=wl.alpha, flags=sm.FLAG_TOP2 | flags)
+
+
+def _ok(sm, ws):
+    st, where, info = sm.switch_get_device_error(ws)
+    assert st == 0, f"device error {st} at {where} ({info})"
+
+
+def check_top2_routing(idx2_gpu, r):
+    """Both choices equal the oracle's except where a margin is below 1e-6."""
+    idx2_gpu = np.asarray(idx2_gpu).reshape(2, -1)
+    m = r["margin2"]
+    d1 = idx2_gpu[0] != r["idx2"][0]
+    assert not (d1 & (m[0] >= MARGIN_FLIP)).any(), "first choice differs on a clear margin"
+    d2 = idx2_gpu[1] != r["idx2"][1]
+    ok2 = d1 | (m[0] < MARGIN_FLIP) | (m[1] < MARGIN_FLIP)
+    assert not (d2 & ~ok2).any(), "second choice differs on a clear margin"
+    assert (idx2_gpu[0] != idx2_gpu[1]).all()
+    return int(d1.sum() + d2.sum())
+
+
+ROUTER_CASES = [
+    Workload("t2_base", T=1000, d_model=768, d_ff=64, n_experts=128, capacity_factor=1.25,
+             dtype="bf16", seed=61),
+    Workload("t2_small", T=3000, d_model=320, d_ff=64, n_experts=8, capacity_factor=1.25,
+             dtype="bf16", seed=62),
+    Workload("t2_odd", T=333, d_model=128, d_ff=64, n_experts=37, capacity_factor=1.0,
+             dtype="bf16", seed=63),
+    Workload("t2_two", T=257, d_model=64, d_ff=64, n_experts=2, capacity_factor=1.0,
+             dtype="bf16", seed=64),
+    Workload("t2_wide", T=300, d_model=64, d_ff=64, n_experts=300, capacity_factor=1.0,
+             dtype="bf16", seed=65),
+    Workload("t2_f32", T=515, d_model=64, d_ff=64, n_experts=4, capacity_factor=1.25,
+             dtype="f32", seed=66),
+]
+
+
+@pytest.mark.parametrize("flags", [0, 1], ids=["default", "simt"])
+@pytest.mark.parametrize("wl", ROUTER_CASES, ids=lambda w: w.name)
+def test_router_top2(sm, wl, flags):
+    x = make_x(wl)
+    w_r, b_r = make_router(wl)
+    r = orc.router_top2(x, w_r, b_r)
+    cfg = _cfg(sm, wl, flags)
+    ws = sm.workspace(cfg)
+    idx = torch.empty(2 * wl.T, **I32)
+    gate = torch.empty(2 * wl.T, dtype=torch.float32, device="cuda")
+    sm.switch_router(cfg, dev_float(x), dev_float(w_r), None if b_r is None else dev_float(b_r),
+                     idx, gate, None, ws)
+    _ok(sm, ws)
+    ig = idx.cpu().numpy().astype(np.int64).reshape(2, -1)
+    check_top2_routing(ig, r)
+    g = gate.cpu().numpy().reshape(2, -1)
+    want = np.stack([r["probs"][np.arange(wl.T), ig[k]] for k in range(2)])
+    assert rel_err(g, want).max() <= PROB_RTOL
+
+
+def test_router_top2_ties(sm):
+    """W_r = 0: all logits tie, so every token takes experts (0, 1), gates 1/N."""
+    wl = Workload("t2_tie", T=300, d_model=128, d_ff=64, n_experts=16, capacity_factor=1.0,
+                  dtype="bf16", seed=67)
+    x = make_x(wl)
+    for flags in (0, 1):
+        cfg = _cfg(sm, wl, flags)
+        ws = sm.workspace(cfg)
+        idx = torch.empty(2 * wl.T, **I32)
+        gate = torch.empty(2 * wl.T, dtype=torch.float32, device="cuda")
+        sm.switch_router(cfg, dev_float(x), torch.zeros(16, 128, device="cuda"), None, idx,
+                         gate, None, ws)
+        _ok(sm, ws)
+        ig = idx.cpu().numpy().reshape(2, -1)
+        assert (ig[0] == 0).all() and (ig[1] == 1).all()
+        np.testing.assert_allclose(gate.cpu().numpy(), 1.0 / 16, rtol=PROB_RTOL)
+
+
+@pytest.mark.parametrize("T,N,cf", [(3000, 8, 1.25), (1000, 128, 1.0), (777, 64, 0.3),
+                                    (129, 3, 4.0), (1, 2, 1.0), (5000, 1000, 1.0)])
+def test_dispatch_top2_bitexact(sm, T, N, cf):
+    rng = np.random.default_rng(T * 7 + N)
+    first = rng.integers(0, N, size=T)
+    second = (first + rng.integers(1, N, size=T)) % N
+    idx2 = np.stack([first, second]).astype(np.int64)
+    C = orc.capacity(2 * T, N, cf)
+    want = orc.dispatch_top2(idx2, N, C)
+    wl = Workload("d", T=T, d_model=64, d_ff=64, n_experts=N, capacity_factor=cf,
+                  dtype="bf16", seed=1)
+    cfg = _cfg(sm, wl)
+    assert sm.switch_capacity(2 * T, N, cf) == C
+    ws = sm.workspace(cfg)
+    rank = torch.empty(2 * T, **I32)
+    drop = torch.empty(2 * T, dtype=torch.uint8, device="cuda")
+    counts = torch.empty(N, **I32)
+    slot = torch.empty(N * C, **I32)
+    sm.switch_dispatch(cfg, torch.from_numpy(idx2.reshape(-1).astype(np.int32)).cuda(), None,
+                       rank, drop, counts, slot, None, None, ws)
+    _ok(sm, ws)
+    np.testing.assert_array_equal(rank.cpu().numpy().reshape(2, -1), want["rank"])
+    np.testing.assert_array_equal(drop.cpu().numpy().reshape(2, -1).astype(bool), want["drop"])
+    np.testing.assert_array_equal(counts.cpu().numpy(), want["counts"])
+    np.testing.assert_array_equal(slot.cpu().numpy(), want["slot_token"])
+
+
+def run_layer_top2(sm, wl, inp, flags=0):
+    cfg = _cfg(sm, wl, flags)
+    ws = sm.workspace(cfg)
+    x = dev_float(inp.x)
+    out = torch.full_like(x, float("nan"))
+    idx = torch.empty(2 * wl.T, **I32)
+    gate = torch.empty(2 * wl.T, dtype=torch.float32, device="cuda")
+    counts = torch.empty(wl.n_experts, **I32)
+    loss = torch.empty(1, dtype=torch.float32, device="cuda")
+    sm.switch_layer_forward(cfg, x, dev_float(inp.w_r),
+                            None if inp.b_r is None else dev_float(inp.b_r),
+                            dev_float(inp.w1), dev_float(inp.w2), out, idx, gate, counts, loss,
+                            ws)
+    _ok(sm, ws)
+    return (host_f64(out), idx.cpu().numpy().astype(np.int64).reshape(2, -1),
+            gate.cpu().numpy().reshape(2, -1), counts.cpu().numpy(), float(loss.item()))
+
+
+def rebased_top2(inp, wl, ig):
+    """The oracle's top-2 layer re-based on the GPU's choices `ig` [2, T]."""
+    r = orc.router_top2(inp.x, inp.w_r, inp.b_r)
+    C = orc.capacity(2 * wl.T, wl.n_experts, wl.capacity_factor)
+    dsp = orc.dispatch_top2(ig, wl.n_experts, C)
+    g64 = np.stack([r["probs"][np.arange(wl.T), ig[k]] for k in range(2)])
+    return r, C, dsp, g64
+
+
+LAYER_CASES = [
+    Workload("t2_e2e", T=3000, d_model=320, d_ff=576, n_experts=8, capacity_factor=1.0,
+             dtype="bf16", seed=71),
+    Workload("t2_tight", T=2000, d_model=256, d_ff=512, n_experts=16, capacity_factor=0.5,
+             dtype="bf16", seed=72),
+    Workload("t2_f32", T=600, d_model=64, d_ff=128, n_experts=4, capacity_factor=1.25,
+             dtype="f32", seed=73),
+]
+
+
+@pytest.mark.parametrize("flags", [0, 1, 32, 64, 8], ids=["default", "simt_router", "gemm_1sm",
+                                                       "gemm_pairs", "gather_in_gemm"])
+@pytest.mark.parametrize("wl", LAYER_CASES, ids=lambda w: w.name)
+def test_layer_top2(sm, wl, flags):
+    inp = make_inputs(wl)
+    out, ig, gate, counts, loss = run_layer_top2(sm, wl, inp, flags)
+    r, C, dsp, g64 = rebased_top2(inp, wl, ig)
+    check_top2_routing(ig, r)
+    np.testing.assert_array_equal(counts, dsp["counts"])
+    assert rel_err(gate, g64).max() <= PROB_RTOL
+    Y = orc.expert_ffn(inp.x, inp.w1, inp.w2, dsp["slot_token"], dsp["counts"], C)
+    want = orc.combine_top2(inp.x, ig, dsp["rank"], dsp["drop"], g64, Y)
+    tol = BF16_RMS_TOL if wl.dtype == "bf16" else F32_RMS_TOL
+    assert rms_ratio(out, want) <= tol
+    both = dsp["drop"].all(axis=0)
+    assert (out[both] == as_f64(inp.x)[both]).all()
+    if wl.capacity_factor < 1.0:
+        assert both.any() and (dsp["drop"].any(axis=0) & ~both).any()
+    loss_w, _, _ = orc.aux_loss(np.bincount(ig[0], minlength=wl.n_experts), r["probs"], wl.alpha)
+    assert abs(loss - loss_w) <= LOSS_RTOL * loss_w
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_combine_top2(sm, dtype):
+    wl = Workload("t2_comb", T=1000, d_model=256 if dtype == "bf16" else 64, d_ff=64,
+                  n_experts=8, capacity_factor=0.4, dtype=dtype, seed=74)
+    inp = make_inputs(wl)
+    r = orc.router_top2(inp.x, inp.w_r, inp.b_r)
+    C = orc.capacity(2 * wl.T, wl.n_experts, wl.capacity_factor)
+    dsp = orc.dispatch_top2(r["idx2"], wl.n_experts, C)
+    rng = np.random.default_rng(3)
+    Y = rng.standard_normal((wl.n_experts, C, wl.d_model))
+    dt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    y_dev = torch.from_numpy(Y.reshape(-1, wl.d_model).astype(np.float32)).to(dt).cuda()
+    Yq = host_f64(y_dev).reshape(wl.n_experts, C, wl.d_model)
+    gate = r["gate2"].astype(np.float32)
+    want = orc.combine_top2(inp.x, r["idx2"], dsp["rank"], dsp["drop"],
+                            gate.astype(np.float64), Yq)
+    cfg = _cfg(sm, wl)
+    x = dev_float(inp.x)
+    out = torch.empty_like(x)
+    sm.switch_combine(cfg, x, torch.from_numpy(r["idx2"].reshape(-1).astype(np.int32)).cuda(),
+                      torch.from_numpy(dsp["rank"].reshape(-1).astype(np.int32)).cuda(),
+                      torch.from_numpy(dsp["drop"].reshape(-1).astype(np.uint8)).cuda(),
+                      torch.from_numpy(gate.reshape(-1)).cuda(), y_dev, out)
+    torch.cuda.synchronize()
+    got = host_f64(out)
+    tol = BF16_RMS_TOL if dtype == "bf16" else F32_RMS_TOL
+    assert rms_ratio(got, want) <= tol
+    both = dsp["drop"].all(axis=0)
+    assert both.any() and (got[both] == as_f64(inp.x)[both]).all()
+
+
+def test_top2_needs_two_experts(sm):
+    with pytest.raises(sm.SwitchError):
+        sm.workspace(sm.config(100, 64, 64, 1, 1.0, flags=sm.FLAG_TOP2))
+
+
+def test_fullsize_base_top2(sm):
+    """Base workload with top-2 routing: all routing outputs in full, sampled
+    block-output rows computed one by one by the oracle."""
+    wl = WORKLOADS["base"]
+    inp = make_inputs(wl)
+    out_d = None
+    cfg = _cfg(sm, wl)
+    ws = sm.workspace(cfg)
+    x = dev_float(inp.x)
+    w1, w2 = dev_float(inp.w1), dev_float(inp.w2)
+    out_d = torch.empty_like(x)
+    idx = torch.empty(2 * wl.T, **I32)
+    gate = torch.empty(2 * wl.T, dtype=torch.float32, device="cuda")
+    counts = torch.empty(wl.n_experts, **I32)
+    loss = torch.empty(1, dtype=torch.float32, device="cuda")
+    sm.switch_layer_forward(cfg, x, dev_float(inp.w_r), None, w1, w2, out_d, idx, gate, counts,
+                            loss, ws)
+    _ok(sm, ws)
+    del w1, w2
+    ig = idx.cpu().numpy().astype(np.int64).reshape(2, -1)
+    r, C, dsp, g64 = rebased_top2(inp, wl, ig)
+    flips = check_top2_routing(ig, r)
+    np.testing.assert_array_equal(counts.cpu().numpy(), dsp["counts"])
+    assert rel_err(gate.cpu().numpy().reshape(2, -1), g64).max() <= PROB_RTOL
+    loss_w, _, _ = orc.aux_loss(np.bincount(ig[0], minlength=wl.n_experts), r["probs"],
+                                wl.alpha)
+    assert abs(loss.item() - loss_w) <= LOSS_RTOL * loss_w
+    rng = np.random.default_rng(99)
+    toks = np.unique(np.concatenate([[0, wl.T - 1], rng.choice(wl.T, 40, replace=False)]))
+    want = as_f64(inp.x[toks]).copy()
+    for j, t in enumerate(toks):
+        for k in range(2):
+            if not dsp["drop"][k, t]:
+                e = ig[k, t]
+                want[j] += g64[k, t] * orc.expert(inp.x[t:t + 1], inp.w1[e], inp.w2[e])[0]
+    got = host_f64(out_d[torch.from_numpy(toks).cuda()])
+    assert rms_ratio(got, want) <= BF16_RMS_TOL
+    print(f"base top-2: flips {flips}, C {C}, dropped assignments {dsp['drop'].mean():.4f}")
