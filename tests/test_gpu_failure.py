@@ -19,7 +19,7 @@ def sm():
     return switch_moe
 
 
-@pytest.mark.parametrize("flags", [0, 32, 64])
+@pytest.mark.parametrize("flags", [0, 32, 64, 512])
 def test_forced_timeouts_report_and_recover(sm, flags):
     wl = Workload("f", T=4096, d_model=256, d_ff=512, n_experts=16, capacity_factor=1.0,
                   dtype="bf16", seed=91)

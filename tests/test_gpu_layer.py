@@ -127,7 +127,9 @@ def test_layer_single_token_and_capacity_one(sm):
 
 @pytest.mark.parametrize("T,N,d,F,flags", [(1, 4, 64, 128, 0), (37, 4, 64, 128, 0),
                                            (300, 37, 128, 192, 0), (300, 300, 64, 64, 0),
-                                           (513, 16, 64, 128, 8), (129, 64, 128, 64, 4)])
+                                           (513, 16, 64, 128, 8), (129, 64, 128, 64, 4),
+                                           (1, 2, 64, 128, 512), (300, 37, 128, 192, 512),
+                                           (300, 300, 64, 64, 512), (513, 16, 64, 128, 512 | 8)])
 def test_workspace_bounds_respected(sm, T, N, d, F, flags):
     """Canary bytes right after the workspace stay untouched, for small and
     odd shapes where padded per-expert scratch is easiest to mis-size."""

@@ -265,3 +265,49 @@ def test_fullsize_base_top2(sm):
     got = host_f64(out_d[torch.from_numpy(toks).cuda()])
     assert rms_ratio(got, want) <= BF16_RMS_TOL
     print(f"base top-2: flips {flips}, C {C}, dropped assignments {dsp['drop'].mean():.4f}")
+
+
+def test_top2_expert_ffn_rows_dispatched(sm):
+    """Top-2 staged path: dispatch with the row copy, then the expert FFN on
+    the copied rows (ROWS_DISPATCHED) and the two-route combine, equal to the
+    fused top-2 layer's output."""
+    wl = LAYER_CASES[0]
+    inp = make_inputs(wl)
+    out_l, ig, gate, counts, _ = run_layer_top2(sm, wl, inp, sm.FLAG_UNFUSED_COMBINE)
+    C = orc.capacity(2 * wl.T, wl.n_experts, wl.capacity_factor)
+    cfg = _cfg(sm, wl)
+    ws = sm.workspace(cfg)
+    x = dev_float(inp.x)
+    idx_d = torch.from_numpy(ig.reshape(-1).astype(np.int32)).cuda()
+    rank = torch.empty(2 * wl.T, **I32)
+    drop = torch.empty(2 * wl.T, dtype=torch.uint8, device="cuda")
+    cnt = torch.empty(wl.n_experts, **I32)
+    slot = torch.empty(wl.n_experts * C, **I32)
+    xd = torch.empty(wl.n_experts * C, wl.d_model, dtype=torch.bfloat16, device="cuda")
+    sm.switch_dispatch(cfg, idx_d, None, rank, drop, cnt, slot, x, xd, ws)
+    y = torch.empty(wl.n_experts * C, wl.d_model, dtype=torch.bfloat16, device="cuda")
+    cfg_rows = _cfg(sm, wl, sm.FLAG_ROWS_DISPATCHED)
+    sm.switch_expert_ffn(cfg_rows, xd, None, cnt, dev_float(inp.w1), dev_float(inp.w2), y, ws)
+    out = torch.empty_like(x)
+    sm.switch_combine(cfg, x, idx_d, rank, drop,
+                      torch.from_numpy(gate.reshape(-1).astype(np.float32)).cuda(), y, out)
+    _ok(sm, ws)
+    np.testing.assert_array_equal(cnt.cpu().numpy(), counts)
+    np.testing.assert_array_equal(host_f64(out), out_l)
+
+
+def test_top2_rejected_where_unsupported(sm):
+    """Top-2 dispatch needs the choices (not probs); the no-alloc dispatch is
+    single-route only."""
+    wl = Workload("u", T=64, d_model=64, d_ff=64, n_experts=4, capacity_factor=1.0,
+                  dtype="bf16", seed=2)
+    cfg = _cfg(sm, wl)
+    ws = sm.workspace(cfg)
+    C = sm.switch_capacity(128, 4, 1.0)
+    out = (torch.empty(128, **I32), torch.empty(128, dtype=torch.uint8, device="cuda"),
+           torch.empty(4, **I32), torch.empty(4 * C, **I32))
+    probs = torch.full((64, 4), 0.25, device="cuda")
+    with pytest.raises(sm.SwitchError):
+        sm.switch_dispatch(cfg, None, probs, *out, None, None, ws)
+    with pytest.raises(sm.SwitchError):
+        sm.switch_dispatch_noalloc(cfg, torch.zeros(128, **I32), None, *out)
