@@ -150,3 +150,30 @@ def test_workspace_bounds_respected(sm, T, N, d, F, flags):
     st, where, info = sm.switch_get_device_error(ws)
     assert st == 0
     assert (buf[n:] == 0xA5).all(), "a kernel wrote past the end of the workspace"
+
+
+@pytest.mark.parametrize("flags", [0, 512, 4, 64])
+def test_layer_ignores_stale_workspace(sm, flags):
+    """Scratch contents do not matter: a workspace full of 0xFF bytes (NaN in
+    bf16 and fp32) past its zeroed error word gives the same output, bit for
+    bit, as a zero-filled one (padding rows of the internal buffers are never
+    stored from)."""
+    wl = Workload("stale", T=2000, d_model=256, d_ff=512, n_experts=16, capacity_factor=1.0,
+                  dtype="bf16", seed=83)
+    inp = make_inputs(wl)
+    cfg = sm.config(wl.T, wl.d_model, wl.d_ff, wl.n_experts, 1.0, flags=flags)
+    n = sm.switch_workspace_size(cfg)
+    x = dev_float(inp.x)
+    w_r, w1, w2 = dev_float(inp.w_r), dev_float(inp.w1), dev_float(inp.w2)
+    outs = []
+    for fill in (0x00, 0xFF):
+        ws = torch.full((n,), fill, dtype=torch.uint8, device="cuda")
+        ws[:256].zero_()
+        out = torch.empty_like(x)
+        loss = torch.empty(1, dtype=torch.float32, device="cuda")
+        sm.switch_layer_forward(cfg, x, w_r, None, w1, w2, out, None, None, None, loss, ws)
+        st, where, info = sm.switch_get_device_error(ws)
+        assert st == 0, f"device error {st} at {where} ({info})"
+        outs.append((out.clone(), loss.item()))
+    assert torch.equal(outs[0][0], outs[1][0]) and outs[0][1] == outs[1][1]
+    assert torch.isfinite(outs[1][0].float()).all()
