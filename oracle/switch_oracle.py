@@ -1,4 +1,4 @@
-"""CPU oracle for the Switch-FFN layer forward pass.
+"""CPU oracle for the Switch-FFN layer: forward pass and its gradient.
 
 TEST INFRASTRUCTURE ONLY.  This module is the slow, plainly written
 definition that the CUDA library is checked against.  Only ``tests/``,
@@ -42,6 +42,10 @@ the largest of the other logits (lowest index on ties); the gates are the
 softmax over all experts, not renormalised; the 2T assignments take slots
 first choices first, each route in batch order; ``f_i`` still counts first
 choices.
+
+The backward pass (``layer_backward``) is the chain rule through those
+stages for J = sum(dout * out) + dloss * loss, routing decisions held fixed
+(they are piecewise constant).
 
 Arithmetic is float64 throughout (expert matmuls included); floating-point
 inputs are the exact values of the bf16 / fp32 bit patterns the GPU reads.
@@ -332,3 +336,103 @@ def token_outputs(x, tokens, idx, drop, gate, w1, w2, residual=True):
             e = int(idx[t])
             rows[j] += gate[t] * expert(x[t:t + 1], w1[e], w2[e])[0]
     return rows
+
+
+# ------------------------------------------------------------ backward pass
+#
+# The gradient of  J = sum(dout * out) + dloss * loss  with respect to x, W_r,
+# b_r, W1 and W2, at the forward pass above.  Routing decisions (the argmax,
+# the capacity cut) and f_i are piecewise constant in the inputs, so no
+# gradient flows through them; the gradient reaches the router through the
+# gate value p_idx(x) that scales the expert output [P1 §"Switch Routing:
+# From Top-k to k = 1": the gate value makes the router differentiable] and
+# through P_i of the load-balancing loss [P1 §"The Load-Balancing Loss":
+# P_i is the differentiable factor, f_i is not].  Each step below is the
+# chain rule through one forward stage, in float64.
+
+
+def expert_backward(x_rows, w1_e, w2_e, g_rows, dout_rows):
+    """Backward of out_t = x_t + g_t . E_e(x_t) over one expert's kept rows.
+
+    E_e(x) = relu(x W1_e^T) W2_e^T [P1 §"The Core Idea"].  Returns
+    ``(dgate [n], dx [n, d], dW1_e [F, d], dW2_e [d, F])``: dgate_t is
+    dout_t . E_e(x_t); the expert's input gradient excludes the residual.
+    """
+    X = as_f64(x_rows)
+    W1 = as_f64(w1_e)
+    W2 = as_f64(w2_e)
+    G = as_f64(dout_rows)
+    g = np.asarray(g_rows, dtype=np.float64)
+    A = X @ W1.T                       # pre-activation
+    H = np.maximum(A, 0.0)
+    Y = H @ W2.T                       # expert output
+    dgate = np.sum(G * Y, axis=1)
+    dY = g[:, None] * G                # gradient at the expert output
+    dW2 = dY.T @ H
+    dA = (dY @ W2) * (A > 0.0)         # through the ReLU
+    dW1 = dA.T @ X
+    dX = dA @ W1
+    return dgate, dX, dW1, dW2
+
+
+def router_backward(x, w_r, probs, idx, drop, dgate, counts, alpha, dloss):
+    """Backward of the router for top-1 routing.
+
+    dJ/dp_{t,i} = dgate_t [i = idx_t, token kept]
+                  + dloss . alpha . N . f_i / T     (loss = alpha N sum f_i P_i,
+                                                     P_i = mean_t p_{t,i});
+    the softmax Jacobian gives dh_{t,i} = p_{t,i} (dp_{t,i} - sum_j p_{t,j} dp_{t,j});
+    h = x W_r^T + b gives dx = dh W_r, dW_r = dh^T x, db = sum_t dh.
+    Returns ``(dx_router [T, d], dW_r [N, d], db [N], dh [T, N])``.
+    """
+    X = as_f64(x)
+    Wr = np.asarray(w_r, dtype=np.float64)
+    p = np.asarray(probs, dtype=np.float64)
+    T, N = p.shape
+    f = np.asarray(counts, dtype=np.float64) / T
+    dp = np.tile(dloss * alpha * N * f / T, (T, 1))
+    kept = ~np.asarray(drop, dtype=bool)
+    rows = np.nonzero(kept)[0]
+    dp[rows, np.asarray(idx)[rows]] += np.asarray(dgate, dtype=np.float64)[rows]
+    dh = p * (dp - np.sum(p * dp, axis=1, keepdims=True))
+    return dh @ Wr, dh.T @ X, dh.sum(axis=0), dh
+
+
+def layer_backward(x, w_r, b_r, w1, w2, capacity_factor, dout, dloss=1.0,
+                   alpha=0.01, residual=True, idx=None):
+    """Gradients of J = sum(dout * out) + dloss * loss for the top-1 layer.
+
+    ``idx`` (optional) imposes the top-1 choices (e.g. those of another
+    implementation, to compare on identical routing); by default the
+    router's own.  Returns a dict with ``dx [T, d]``, ``dw_r [N, d]``,
+    ``db_r [N]``, ``dw1 [N, F, d]``, ``dw2 [N, d, F]`` (float64) and the
+    intermediates ``dgate [T]``, ``dh [T, N]``, ``idx``, ``gate``, ``drop``,
+    ``counts``, ``slot_token``, ``C``.
+    """
+    T, d = x.shape
+    N = w_r.shape[0]
+    C = capacity(T, N, capacity_factor)
+    r = router(x, w_r, b_r)
+    idx = r["idx"] if idx is None else np.asarray(idx, dtype=np.int64)
+    gate = r["probs"][np.arange(T), idx]
+    dsp = dispatch(idx, N, C)
+    G = as_f64(dout)
+    dx = G.copy() if residual else np.zeros((T, d))
+    dgate = np.zeros(T)
+    dw1 = np.zeros(np.shape(w1))
+    dw2 = np.zeros(np.shape(w2))
+    for e in range(N):
+        n = min(int(dsp["counts"][e]), C)
+        if n == 0:
+            continue
+        rows = dsp["slot_token"][e * C: e * C + n]
+        dg, dxe, dw1[e], dw2[e] = expert_backward(x[rows], w1[e], w2[e], gate[rows], dout[rows])
+        dgate[rows] = dg
+        dx[rows] += dxe
+    dxr, dw_r, db_r, dh = router_backward(x, w_r, r["probs"], idx, dsp["drop"], dgate,
+                                          dsp["counts"], alpha, dloss)
+    dx += dxr
+    return {"dx": dx, "dw_r": dw_r, "db_r": db_r, "dw1": dw1, "dw2": dw2,
+            "dgate": dgate, "dh": dh, "idx": idx, "gate": gate, "drop": dsp["drop"],
+            "counts": dsp["counts"], "slot_token": dsp["slot_token"], "C": C,
+            "probs": r["probs"]}

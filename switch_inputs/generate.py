@@ -19,6 +19,8 @@ Recipe (stated once, used everywhere):
   output-major like a linear layer's ``[out, in]`` weight, so that
   ``E_e(x) = relu(x @ w1[e].T) @ w2[e].T``.  bf16 workloads store ``w1``/``w2``
   as bf16 bit patterns (uint16); the router stays fp32.
+* The backward pass's upstream gradient ``dout ~ N(0, 1)``, shape
+  ``[T, d_model]``, encoded like x (``make_dout``).
 * Workloads with ``zipf_s`` add a router bias ``b_e = beta * ln z_e`` where
   ``z_e`` is the Zipf(s) law over experts (expert 0 heaviest).  ``beta`` is
   fitted so that, with the router's logits modelled as independent Gaussians
@@ -37,7 +39,7 @@ import numpy as np
 
 from .configs import Workload
 
-_TENSOR_IDS = {"x": 1, "w_r": 2, "w1": 3, "w2": 4}
+_TENSOR_IDS = {"x": 1, "w_r": 2, "w1": 3, "w2": 4, "dout": 5}
 INIT_SCALE = 0.1
 
 
@@ -77,6 +79,14 @@ def make_x(wl: Workload) -> np.ndarray:
     rng = _rng(wl, "x")
     x = rng.standard_normal(size=(wl.T, wl.d_model), dtype=np.float32)
     return x if wl.dtype == "f32" else f32_to_bf16_bits(x)
+
+
+def make_dout(wl: Workload) -> np.ndarray:
+    """Upstream gradient of the block output for the backward pass: ``N(0, 1)``
+    of shape ``[T, d_model]``, encoded like x (bf16 bits or fp32)."""
+    rng = _rng(wl, "dout")
+    g = rng.standard_normal(size=(wl.T, wl.d_model), dtype=np.float32)
+    return g if wl.dtype == "f32" else f32_to_bf16_bits(g)
 
 
 def make_router(wl: Workload):
