@@ -1,6 +1,6 @@
 /*
- * switch_moe.h -- C ABI of the Switch-FFN layer forward pass on one NVIDIA
- * B200 (sm_100a).
+ * switch_moe.h -- C ABI of the Switch-FFN layer (forward pass and its
+ * backward) on one NVIDIA B200 (sm_100a).
  *
  * The layer is the one of "Switch Transformers: scaling to trillion-parameter
  * models" (cited below as [P1 section]):
@@ -242,6 +242,48 @@ switch_status_t switch_layer_forward(const switch_config_t* cfg, const void* x,
                                      int32_t* idx, float* gate, int32_t* counts,
                                      float* loss, void* ws, size_t ws_bytes,
                                      void* stream);
+
+/* Backward pass of switch_layer_forward (top-1, bf16): the gradient of
+ *   J = sum(dout * out) + dloss * loss
+ * with respect to x, w_r, b_r, w1 and w2, routing decisions held fixed (the
+ * argmax and the capacity cut are piecewise constant; f_i likewise).  The
+ * gradient reaches the router through the gate value p_idx(x) that scales
+ * the expert output [P1 "Switch Routing: From Top-k to k = 1": the gate
+ * value is what makes the router trainable] and through P_i of the
+ * load-balancing loss [P1 "The Load-Balancing Loss"]:
+ *   dgate[t] = dout[t] . E_idx(x_t)           (kept tokens; 0 if dropped)
+ *   dW2_e = sum_t (gate dout)[t]^T H_t,  dA = (gate dout W2_e) where H > 0,
+ *   dW1_e = sum_t dA_t^T x_t,  dx_t += dA_t W1_e,
+ *   dp[t, i] = [i = idx_t] dgate[t] + dloss alpha N f_i / T,
+ *   dh = p (dp - sum_j p_j dp_j),  dx += dh W_r,  dW_r = dh^T x,
+ *   db_r = sum_t dh,  dx += dout (the residual branch, unless
+ *   SWITCH_FLAG_NO_RESIDUAL).
+ * The call recomputes the forward's routing, dispatch and hidden
+ * activations from its inputs (as activation checkpointing does); it reads
+ * nothing a previous call left in the workspace.
+ *   x [T, d_model] bf16, w_r [N, d_model] fp32, b_r [N] fp32 or NULL,
+ *   w1 [N, d_ff, d_model] bf16, w2 [N, d_model, d_ff] bf16 (as the forward);
+ *   dout [T, d_model] bf16: gradient of J with respect to out;
+ *   dloss: host float, the weight of the loss in J;
+ *   outputs: dx [T, d_model] bf16, dw_r [N, d_model] fp32, db_r [N] fp32 or
+ *   NULL, dw1 [N, d_ff, d_model] bf16, dw2 [N, d_model, d_ff] bf16,
+ *   dgate [T] fp32 or NULL (the gate gradient above).
+ * Arithmetic: expert GEMMs on the tensor cores (bf16 operands, fp32
+ * accumulation; gate * dout, dA and the weight gradients rounded once to
+ * bf16); router backward in fp32 FMA with fixed-order reductions (dW_r and
+ * db_r bit-reproducible).  Workspace: switch_backward_workspace_size()
+ * bytes.  dtype SWITCH_F32 or SWITCH_FLAG_TOP2 return SWITCH_ERR_UNSUPPORTED.
+ * T = 0 writes nothing. */
+switch_status_t switch_layer_backward(const switch_config_t* cfg, const void* x,
+                                      const float* w_r, const float* b_r,
+                                      const void* w1, const void* w2, const void* dout,
+                                      float dloss, void* dx, float* dw_r, float* db_r,
+                                      void* dw1, void* dw2, float* dgate, void* ws,
+                                      size_t ws_bytes, void* stream);
+
+/* Bytes of device workspace switch_layer_backward needs for `cfg` (more
+ * than switch_workspace_size(); every other entry point accepts it too). */
+switch_status_t switch_backward_workspace_size(const switch_config_t* cfg, size_t* bytes);
 
 /* Synchronises `stream`, reads the workspace's device error word, clears
  * it, and returns the recorded status (SWITCH_OK if none).  *where_out and

@@ -34,12 +34,6 @@ namespace smoe {
 
 // ----------------------------------------------------------- tensor maps
 
-typedef CUresult (*PFN_encodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                    const cuuint32_t*, CUtensorMapInterleave,
-                                    CUtensorMapSwizzle, CUtensorMapL2promotion,
-                                    CUtensorMapFloatOOBfill);
-
 PFN_encodeTiled get_encode_fn() {
   static PFN_encodeTiled fn = nullptr;
   if (fn == nullptr) {
@@ -389,7 +383,7 @@ cudaError_t launch_expert_ffn_bf16(const FfnArgs& a, cudaStream_t st) {
   else
     e = gather ? run_gemm<true>(ta1, tb1, to1, g1, a.num_sms, st)
                : run_gemm<false>(ta1, tb1, to1, g1, a.num_sms, st);
-  if (e != cudaSuccess) return e;
+  if (e != cudaSuccess || a.gemm1_only) return e;
 
   GemmParams g2 = g1;
   g2.n_out = a.d;

@@ -80,6 +80,14 @@ bool router_pair_supported(int N, int terms);
 // Bytes of the bf16 split-weight scratch launch_router_tc needs (3 terms).
 size_t router_wsplit_bytes(int N, int d);
 
+// cuTensorMapEncodeTiled, looked up once through the runtime (expert_ffn.cu).
+typedef CUresult (*PFN_encodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                    const cuuint32_t*, CUtensorMapInterleave,
+                                    CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                    CUtensorMapFloatOOBfill);
+PFN_encodeTiled get_encode_fn();
+
 // 2-D bf16 TMA descriptor (expert_ffn.cu): [outer, inner], box
 // box_outer x box_inner, 128-byte swizzle (64-byte when swizzle64).
 bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
@@ -108,6 +116,7 @@ struct FfnArgs {
   int mode2;                // kModeY or kModeCombine for the second GEMM
   bool pair1;               // GEMM1 on CTA pairs (2-SM), else one CTA per tile
   bool pair2;               // GEMM2 on CTA pairs
+  bool gemm1_only;          // stop after GEMM1 (the backward pass recomputes H)
   DevErr* err;
   long long spin;
   int num_sms;

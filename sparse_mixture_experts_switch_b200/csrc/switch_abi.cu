@@ -5,7 +5,7 @@
 #include <cmath>
 #include <cstring>
 
-#include "kernels.cuh"
+#include "backward.cuh"
 
 using namespace smoe;
 
@@ -40,6 +40,9 @@ int64_t capacity_exact(int64_t T, int32_t N, double cf) {
 struct Layout {
   size_t err, hist, base, psum, fpsc, local_rank, idx, gate, rank, drop, counts, counts1,
       slot_token, mtile_start, wsplit, logits, xdisp, hbuf, ybuf, total;
+  // backward pass only (after the forward regions): dA, partial gate
+  // gradients, dh, gate gradient, router part of dx, split-K partials
+  size_t da, dgp, dh, dgate, dxr, rpart, bwd_total;
 };
 
 // Bytes 16..19 of the workspace: the loss kernel's completion ticket (kept
@@ -87,6 +90,14 @@ Layout layout_for(const switch_config_t& c, int64_t C) {
   L.hbuf = take(es * slots * static_cast<size_t>(c.d_ff));
   L.ybuf = take(es * slots * static_cast<size_t>(c.d_model));
   L.total = o;
+  const int64_t ntn = (c.d_ff + 255) / 256;
+  L.da = take(es * slots * static_cast<size_t>(c.d_ff));
+  L.dgp = take(sizeof(float) * slots * ntn);
+  L.dh = take(sizeof(float) * N * T);
+  L.dgate = take(sizeof(float) * T);
+  L.dxr = take(sizeof(float) * T * static_cast<size_t>(c.d_model));
+  L.rpart = take(sizeof(float) * router_bwd_part_floats(T, c.n_experts, c.d_model));
+  L.bwd_total = o;
   return L;
 }
 
@@ -195,6 +206,15 @@ switch_status_t switch_workspace_size(const switch_config_t* cfg, size_t* bytes)
   if (s != SWITCH_OK) return s;
   if (bytes == nullptr) return SWITCH_ERR_INVALID_ARG;
   *bytes = layout_for(*cfg, C).total;
+  return SWITCH_OK;
+}
+
+switch_status_t switch_backward_workspace_size(const switch_config_t* cfg, size_t* bytes) {
+  int64_t C = 0;
+  switch_status_t s = validate(cfg, &C);
+  if (s != SWITCH_OK) return s;
+  if (bytes == nullptr) return SWITCH_ERR_INVALID_ARG;
+  *bytes = layout_for(*cfg, C).bwd_total;
   return SWITCH_OK;
 }
 
@@ -424,6 +444,129 @@ switch_status_t switch_layer_forward(const switch_config_t* cfg, const void* x,
     SMOE_TRY(launch_aux_loss(T, N, nparts, cfg->alpha, counts_loss, psum, loss, nullptr,
                              nullptr, c.at<double>(c.L.fpsc), c.at<unsigned>(kTicketOffset),
                              c.st));
+  return SWITCH_OK;
+}
+
+switch_status_t switch_layer_backward(const switch_config_t* cfg, const void* x,
+                                      const float* w_r, const float* b_r, const void* w1,
+                                      const void* w2, const void* dout, float dloss, void* dx,
+                                      float* dw_r, float* db_r, void* dw1, void* dw2,
+                                      float* dgate, void* ws, size_t ws_bytes, void* stream) {
+  Ctx c{};
+  switch_status_t s = prepare(cfg, ws, ws_bytes, stream, &c);
+  if (s != SWITCH_OK) return s;
+  if (cfg->dtype != SWITCH_BF16 || (cfg->flags & SWITCH_FLAG_TOP2)) return SWITCH_ERR_UNSUPPORTED;
+  if (cfg->T == 0) return SWITCH_OK;
+  if (!x || !w_r || !w1 || !w2 || !dout || !dx || !dw_r || !dw1 || !dw2 || !aligned16(x) ||
+      !aligned16(w1) || !aligned16(w2) || !aligned16(dout) || !aligned16(dx) ||
+      !aligned16(dw1) || !aligned16(dw2))
+    return SWITCH_ERR_INVALID_ARG;
+  if (ws_bytes < c.L.bwd_total) return SWITCH_ERR_WORKSPACE_TOO_SMALL;
+  const int64_t T = cfg->T;
+  const int N = cfg->n_experts;
+  const int d = cfg->d_model, F = cfg->d_ff;
+  const int nt = ntiles_of(T);
+  const int64_t S = static_cast<int64_t>(N) * c.C;
+  int* idx = c.at<int>(c.L.idx);
+  float* gate = c.at<float>(c.L.gate);
+  float* probs = c.at<float>(c.L.dh);          // dh overwrites it in place
+  int* counts = c.at<int>(c.L.counts);
+  int* local_rank = c.at<int>(c.L.local_rank);
+  int* hist = c.at<int>(c.L.hist);
+  int* rank = c.at<int>(c.L.rank);
+  uint8_t* drop = c.at<uint8_t>(c.L.drop);
+  int* slot_token = c.at<int>(c.L.slot_token);
+  int* mtile_start = c.at<int>(c.L.mtile_start);
+  const bool residual = !(cfg->flags & SWITCH_FLAG_NO_RESIDUAL);
+
+  // 1. the forward's routing, dispatch and hidden activations, recomputed
+  // (same kernels, same results): probabilities, slots, x_disp, H
+  RouterOut o{idx, gate, probs, c.at<float>(c.L.psum), nullptr, nullptr, nullptr, nullptr};
+  if (use_tc_router(cfg)) {
+    o.hist = hist;
+    o.local_rank = local_rank;
+    SMOE_TRY(launch_router_tc(T, d, N, router_terms(cfg), x, w_r, b_r, c.ws + c.L.wsplit, o, nt,
+                              c.err, c.spin, c.num_sms, c.st));
+  } else {
+    int nparts = 0;
+    SMOE_TRY(launch_router_simt(T, d, N, true, x, w_r, b_r, c.at<float>(c.L.logits), o, &nparts,
+                                c.st));
+    SMOE_TRY(launch_tile_rank(T, N, idx, nullptr, nullptr, local_rank, hist, nt, c.err, c.st));
+  }
+  SMOE_TRY(launch_scan(N, nt, hist, c.at<int>(c.L.base), counts, c.st));
+  SMOE_TRY(launch_finalize(T, N, c.C, nt, idx, local_rank, c.at<int>(c.L.base), counts, rank,
+                           drop, slot_token, mtile_start, 0, c.st));
+  void* x_disp = c.ws + c.L.xdisp;
+  void* hbuf = c.ws + c.L.hbuf;
+  SMOE_TRY(launch_gather_rows(S, static_cast<int64_t>(d) * 2, slot_token, x, x_disp, c.st));
+  FfnArgs a{};
+  a.T = T;
+  a.d = d;
+  a.F = F;
+  a.N = N;
+  a.C = c.C;
+  a.x = x;
+  a.x_disp = x_disp;
+  a.slot_token = slot_token;
+  a.counts = counts;
+  a.mtile_start = mtile_start;
+  a.w1 = w1;
+  a.w2 = w2;
+  a.hbuf = hbuf;
+  a.mode2 = kModeY;
+  a.pair1 = (cfg->flags & SWITCH_FLAG_GEMM_PAIRS) != 0;
+  a.gemm1_only = true;
+  a.err = c.err;
+  a.spin = c.spin;
+  a.num_sms = c.num_sms;
+  SMOE_TRY(launch_expert_ffn_bf16(a, c.st));
+
+  // 2. dY = gate * dout per kept slot; dA and the gate-gradient partials;
+  // the expert weight gradients
+  void* dys = c.ws + c.L.ybuf;
+  SMOE_TRY(launch_bwd_gather(c.C, N, d, F, counts, slot_token, gate, dout, dys, hbuf, c.st));
+  BwdFfnArgs b{};
+  b.T = T;
+  b.d = d;
+  b.F = F;
+  b.N = N;
+  b.C = c.C;
+  b.counts = counts;
+  b.mtile_start = mtile_start;
+  b.slot_token = slot_token;
+  b.w1 = w1;
+  b.w2 = w2;
+  b.x_disp = x_disp;
+  b.hbuf = hbuf;
+  b.dys = dys;
+  b.da = c.ws + c.L.da;
+  b.dgp = c.at<float>(c.L.dgp);
+  b.dw1 = dw1;
+  b.dw2 = dw2;
+  b.dout = dout;
+  b.dxr = c.at<float>(c.L.dxr);
+  b.dx = dx;
+  b.residual = residual;
+  b.err = c.err;
+  b.spin = c.spin;
+  b.num_sms = c.num_sms;
+  SMOE_TRY(launch_bwd_dh(b, c.st));
+  SMOE_TRY(launch_bwd_dw(b, c.st));
+
+  // 3. router: dh (in place of the probabilities), its input and weight
+  // gradients
+  float* dh = probs;
+  const double ls = static_cast<double>(dloss) * cfg->alpha * N / (static_cast<double>(T) * T);
+  SMOE_TRY(launch_router_bwd_dh(T, N, c.C, (F + 255) / 256, probs, idx, rank, drop, gate,
+                                b.dgp, counts, static_cast<float>(ls), dh,
+                                dgate ? dgate : c.at<float>(c.L.dgate), c.st));
+  SMOE_TRY(launch_router_bwd_dx(T, N, d, dh, w_r, c.at<float>(c.L.dxr), c.st));
+  SMOE_TRY(launch_router_bwd_dw(T, N, d, dh, x, c.at<float>(c.L.rpart), dw_r, db_r, c.st));
+
+  // 4. input gradient: kept tokens in the dX GEMM's epilogue, dropped ones
+  // here
+  SMOE_TRY(launch_bwd_dx(b, c.st));
+  SMOE_TRY(launch_bwd_dropped(T, d, drop, dout, c.at<float>(c.L.dxr), dx, residual, c.st));
   return SWITCH_OK;
 }
 

@@ -71,6 +71,11 @@ def _load():
         "switch_layer_forward": (c_int32, [cfgp, c_void_p, c_void_p, c_void_p, c_void_p,
                                            c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                            c_void_p, c_void_p, c_size_t, c_void_p]),
+        "switch_layer_backward": (c_int32, [cfgp, c_void_p, c_void_p, c_void_p, c_void_p,
+                                            c_void_p, c_void_p, c_float, c_void_p, c_void_p,
+                                            c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                            c_size_t, c_void_p]),
+        "switch_backward_workspace_size": (c_int32, [cfgp, POINTER(c_size_t)]),
         "switch_get_device_error": (c_int32, [c_void_p, c_void_p, POINTER(c_int32),
                                               POINTER(c_int64)]),
         "switch_status_string": (c_char_p, [c_int32]),
@@ -175,6 +180,28 @@ def switch_layer_forward(cfg, x, w_r, b_r, w1, w2, out, idx, gate, counts, loss,
                                      _p(w2), _p(out), _p(idx), _p(gate), _p(counts),
                                      _p(loss), _p(ws), ws.numel(), _stream(stream)),
            "switch_layer_forward")
+
+
+def switch_backward_workspace_size(cfg):
+    n = c_size_t(0)
+    _check(_lib.switch_backward_workspace_size(ctypes.byref(cfg), ctypes.byref(n)),
+           "switch_backward_workspace_size")
+    return n.value
+
+
+def backward_workspace(cfg, device="cuda"):
+    """A zero-filled device workspace of switch_backward_workspace_size(cfg)
+    bytes (every entry point accepts it)."""
+    return torch.zeros(max(switch_backward_workspace_size(cfg), 1), dtype=torch.uint8,
+                       device=device)
+
+
+def switch_layer_backward(cfg, x, w_r, b_r, w1, w2, dout, dloss, dx, dw_r, db_r, dw1, dw2,
+                          dgate, ws, stream=None):
+    _check(_lib.switch_layer_backward(ctypes.byref(cfg), _p(x), _p(w_r), _p(b_r), _p(w1),
+                                      _p(w2), _p(dout), float(dloss), _p(dx), _p(dw_r),
+                                      _p(db_r), _p(dw1), _p(dw2), _p(dgate), _p(ws),
+                                      ws.numel(), _stream(stream)), "switch_layer_backward")
 
 
 def switch_get_device_error(ws, stream=None):

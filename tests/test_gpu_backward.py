@@ -1,0 +1,230 @@
+"""Parity of switch_layer_backward against the oracle's backward pass.
+
+The oracle is re-based on the GPU's top-1 choices (read from a forward call
+on the same inputs; the backward recomputes the same routing), then every
+gradient is compared element by element: bf16 dx, dw1, dw2 and the fp32
+router gradients dw_r, db_r and the gate gradient, each with two bounds
+relative to RMS(oracle):  max |GPU - oracle| <= 4e-2 and RMS(GPU - oracle)
+<= 5e-3.  Derivation: a gradient element passes through up to three bf16
+roundings (gate * dout, dA, and the bf16 output itself; H adds a fourth on
+the dW2 / gate-gradient path), each a relative error of at most 2^-9, while
+the fp32 accumulations add < 1e-5.  A sum of n independently rounded terms
+then has an error of standard deviation about 3 * 2^-9 / sqrt(3) = 3.4e-3 of
+its RMS; over 10^6 elements the largest is about 6 standard deviations
+(0.02), plus the output's own rounding of at most 2^-9 x the largest value
+(about 5 RMS, 0.01): 0.03, bounded by 4e-2.  The RMS bound (1.5 x the
+standard deviation) is what catches a wrong index or a missing term: those
+give errors of the order of the RMS itself.  The router's fp32 gradients
+inherit bf16-level error through the gate gradient.  Routing flips (oracle
+margin < 1e-6) are counted as in the forward tests.
+
+At full size (Base) the oracle computes sampled tokens' dx and gate
+gradients, and sampled experts' weight gradients, one by one; dw_r and db_r
+are checked there through the softmax shift invariance (their sums over
+experts vanish), which holds at any size.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle.switch_oracle as orc
+from switch_inputs import Workload, BASE, make_inputs, make_dout, as_f64
+from gpu_util import dev_float, host_f64, check_routing
+
+pytestmark = pytest.mark.gpu
+
+GRAD_MAX_TOL = 4e-2
+GRAD_RMS_TOL = 5e-3
+
+
+def grad_ok(got, want, name):
+    want = np.asarray(want, np.float64)
+    err = np.asarray(got, np.float64) - want
+    rms = max(float(np.sqrt(np.mean(want * want))), 1e-30)
+    mx = float(np.max(np.abs(err))) / rms
+    rm = float(np.sqrt(np.mean(err * err))) / rms
+    assert mx <= GRAD_MAX_TOL and rm <= GRAD_RMS_TOL, \
+        f"{name}: max err / rms = {mx:.3g}, rms err / rms = {rm:.3g}"
+    return mx, rm
+
+
+@pytest.fixture(scope="module")
+def sm():
+    from sparse_mixture_experts_switch_b200 import switch_moe
+    return switch_moe
+
+
+def _forward_idx(sm, cfg, x, w_r, b_r, w1, w2, ws):
+    out = torch.empty_like(x)
+    idx = torch.empty(cfg.T, dtype=torch.int32, device="cuda")
+    sm.switch_layer_forward(cfg, x, w_r, b_r, w1, w2, out, idx, None, None, None, ws)
+    st, where, info = sm.switch_get_device_error(ws)
+    assert st == 0, f"device error {st} at {where} ({info})"
+    return idx.cpu().numpy().astype(np.int64)
+
+
+def run_backward(sm, wl, inp, dout, dloss=1.0, flags=0, b_r_override=None, reuse_ws=None):
+    cfg = sm.config(wl.T, wl.d_model, wl.d_ff, wl.n_experts, wl.capacity_factor,
+                    dtype=wl.dtype, alpha=wl.alpha, flags=flags)
+    ws = sm.backward_workspace(cfg) if reuse_ws is None else reuse_ws
+    b_np = inp.b_r if b_r_override is None else b_r_override
+    x, w_r, w1, w2 = dev_float(inp.x), dev_float(inp.w_r), dev_float(inp.w1), dev_float(inp.w2)
+    b_r = None if b_np is None else dev_float(b_np)
+    g = dev_float(dout)
+    idx = _forward_idx(sm, cfg, x, w_r, b_r, w1, w2, ws)
+    dx = torch.full_like(x, float("nan"))
+    dw_r = torch.full_like(w_r, float("nan"))
+    db_r = torch.full((wl.n_experts,), float("nan"), device="cuda")
+    dw1 = torch.full_like(w1, float("nan"))
+    dw2 = torch.full_like(w2, float("nan"))
+    dgate = torch.full((wl.T,), float("nan"), device="cuda")
+    sm.switch_layer_backward(cfg, x, w_r, b_r, w1, w2, g, dloss, dx, dw_r, db_r, dw1, dw2,
+                             dgate, ws)
+    st, where, info = sm.switch_get_device_error(ws)
+    assert st == 0, f"device error {st} at {where} ({info})"
+    return idx, {"dx": host_f64(dx), "dw_r": host_f64(dw_r), "db_r": host_f64(db_r),
+                 "dw1": host_f64(dw1), "dw2": host_f64(dw2), "dgate": host_f64(dgate)}
+
+
+def check_backward(sm, wl, dloss=1.0, flags=0, b_r_override=None):
+    inp = make_inputs(wl)
+    dout = make_dout(wl)
+    idx, got = run_backward(sm, wl, inp, dout, dloss, flags, b_r_override)
+    b_np = inp.b_r if b_r_override is None else b_r_override
+    r = orc.router(inp.x, inp.w_r, b_np)
+    flips = check_routing(idx, r)
+    residual = not (flags & sm.FLAG_NO_RESIDUAL)
+    want = orc.layer_backward(inp.x, inp.w_r, b_np, inp.w1, inp.w2, wl.capacity_factor, dout,
+                              dloss=dloss, alpha=wl.alpha, residual=residual, idx=idx)
+    for name in ("dx", "dw1", "dw2", "dw_r", "dgate"):
+        assert np.isfinite(got[name]).all(), name
+        print(wl.name, name, "max/rms err ratios %.3g %.3g" % grad_ok(got[name], want[name], name))
+    if b_np is not None:
+        grad_ok(got["db_r"], want["db_r"], "db_r")
+    return got, want, flips
+
+
+SMALL = Workload("bwd_small", T=3000, d_model=320, d_ff=576, n_experts=8, capacity_factor=1.0,
+                 dtype="bf16", seed=91)
+
+
+def test_backward_small(sm):
+    got, want, _ = check_backward(sm, SMALL)
+    d = want["drop"]
+    assert d.any() and (~d).any()
+    assert np.all(got["dgate"][d] == 0)
+
+
+@pytest.mark.parametrize("flags", [0, 1, 16, 64], ids=["default", "simt_router", "no_residual",
+                                                      "gemm1_pairs"])
+def test_backward_flags(sm, flags):
+    check_backward(sm, SMALL, dloss=0.5, flags=flags)
+
+
+def test_backward_bias_and_loss_only(sm):
+    """Router bias present; dloss = 3 weights the loss's gradient up."""
+    rng = np.random.default_rng(5)
+    bias = (0.05 * rng.standard_normal(SMALL.n_experts)).astype(np.float32)
+    check_backward(sm, SMALL, dloss=3.0, b_r_override=bias)
+
+
+def test_backward_empty_expert_and_heavy_drop(sm):
+    """An expert no token picks has exactly zero weight gradients; with a
+    capacity factor of 0.25 most tokens are dropped."""
+    wl = Workload("bwd_drop", T=2048, d_model=256, d_ff=512, n_experts=8,
+                  capacity_factor=0.25, dtype="bf16", seed=17)
+    bias = np.zeros(wl.n_experts, dtype=np.float32)
+    bias[3] = -60.0
+    got, want, _ = check_backward(sm, wl, b_r_override=bias)
+    assert np.all(got["dw1"][3] == 0) and np.all(got["dw2"][3] == 0)
+    assert want["drop"].mean() > 0.5
+
+
+def test_backward_no_drops_ragged(sm):
+    """Every token kept (capacity factor N); sizes whose tiles are ragged in
+    every dimension (C, d_model and d_ff not multiples of the tile)."""
+    wl = Workload("bwd_ragged", T=1000, d_model=192, d_ff=320, n_experts=6,
+                  capacity_factor=6.0, dtype="bf16", seed=23)
+    got, want, _ = check_backward(sm, wl)
+    assert not want["drop"].any()
+
+
+def test_backward_deterministic(sm):
+    inp = make_inputs(SMALL)
+    dout = make_dout(SMALL)
+    _, a = run_backward(sm, SMALL, inp, dout)
+    _, b = run_backward(sm, SMALL, inp, dout)
+    for k in a:
+        assert np.array_equal(a[k], b[k], equal_nan=True), k
+
+
+def test_backward_rejects_unsupported(sm):
+    wl = SMALL
+    for flags, dtype in ((sm.FLAG_TOP2, "bf16"), (0, "f32")):
+        cfg = sm.config(wl.T, wl.d_model, wl.d_ff, wl.n_experts, wl.capacity_factor,
+                        dtype=dtype, alpha=wl.alpha, flags=flags)
+        ws = sm.backward_workspace(cfg)
+        t = torch.zeros(8, device="cuda")
+        with pytest.raises(sm.SwitchError) as ei:
+            sm.switch_layer_backward(cfg, t, t, None, t, t, t, 1.0, t, t, None, t, t, None, ws)
+        assert ei.value.status == 2
+
+
+def test_backward_workspace_too_small(sm):
+    wl = SMALL
+    cfg = sm.config(wl.T, wl.d_model, wl.d_ff, wl.n_experts, wl.capacity_factor, alpha=wl.alpha)
+    ws = sm.workspace(cfg)                      # the forward's size only
+    assert sm.switch_backward_workspace_size(cfg) > ws.numel()
+    x = torch.zeros(wl.T, wl.d_model, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(sm.SwitchError) as ei:
+        sm.switch_layer_backward(cfg, x, x, None, x, x, x, 1.0, x, x, None, x, x, None, ws)
+    assert ei.value.status == 3
+
+
+# ----------------------------------------------------------- full size
+
+def test_backward_fullsize_base_sampled(sm):
+    wl = BASE
+    inp = make_inputs(wl)
+    dout = make_dout(wl)
+    idx, got = run_backward(sm, wl, inp, dout)
+    T, N = wl.T, wl.n_experts
+    r = orc.router(inp.x, inp.w_r, inp.b_r)
+    check_routing(idx, r)
+    C = orc.capacity(T, N, wl.capacity_factor)
+    dsp = orc.dispatch(idx, N, C)
+    gate = r["probs"][np.arange(T), idx]
+    f_scale = wl.alpha * N * dsp["counts"] / T / T
+    rng = np.random.default_rng(3)
+    toks = np.unique(np.concatenate([[0, T - 1], rng.choice(T, 48, replace=False),
+                                     rng.choice(np.nonzero(dsp["drop"])[0], 8, replace=False)]))
+    want_dx = np.zeros((toks.size, wl.d_model))
+    want_dg = np.zeros(toks.size)
+    for j, t in enumerate(toks):
+        e = int(idx[t])
+        dg, dxe = 0.0, 0.0
+        if not dsp["drop"][t]:
+            dg_a, dxe_a, _, _ = orc.expert_backward(inp.x[t:t + 1], inp.w1[e], inp.w2[e],
+                                                    gate[t:t + 1], dout[t:t + 1])
+            dg, dxe = dg_a[0], dxe_a[0]
+        p = r["probs"][t]
+        dp = f_scale.copy()
+        if not dsp["drop"][t]:
+            dp[e] += dg
+        dh = p * (dp - np.sum(p * dp))
+        want_dx[j] = as_f64(dout[t]) + dxe + dh @ inp.w_r.astype(np.float64)
+        want_dg[j] = dg
+    grad_ok(got["dx"][toks], want_dx, "dx (sampled)")
+    grad_ok(got["dgate"][toks], want_dg, "dgate (sampled)")
+    for e in (0, N // 2, N - 1):
+        n = min(int(dsp["counts"][e]), C)
+        rows = dsp["slot_token"][e * C: e * C + n]
+        _, _, dw1_e, dw2_e = orc.expert_backward(inp.x[rows], inp.w1[e], inp.w2[e], gate[rows],
+                                                 dout[rows])
+        grad_ok(got["dw1"][e], dw1_e, f"dw1[{e}]")
+        grad_ok(got["dw2"][e], dw2_e, f"dw2[{e}]")
+    # softmax shift invariance: sum over experts of dW_r rows and of db_r vanish
+    scale = np.abs(got["dw_r"]).max()
+    assert np.abs(got["dw_r"].sum(axis=0)).max() <= 1e-3 * scale
+    assert np.isfinite(got["dx"]).all() and np.isfinite(got["dw1"]).all()
+    assert np.isfinite(got["dw2"]).all()
