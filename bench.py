@@ -507,6 +507,22 @@ def kernel_rooflines(sm, cfg, wl, C, x, w_r, b_r, w1, w2, ws, flush, stream, dev
         if st2 != 0:
             raise RuntimeError(f"device error {st2} at {where2} ({info2}) in the top-2 layer")
         del ws2
+    # the backward pass of the whole layer (recomputes routing, dispatch and H)
+    t_bwd = None
+    if wl.dtype == "bf16":
+        wsb = sm.backward_workspace(cfg, device=dev)
+        dout = torch.empty_like(x).normal_()
+        dx = torch.empty_like(x)
+        dw_r = torch.empty_like(w_r)
+        db_r = torch.empty(N, dtype=torch.float32, device=dev)
+        dw1 = torch.empty_like(w1)
+        dw2 = torch.empty_like(w2)
+        t_bwd = timed(lambda: sm.switch_layer_backward(cfg, x, w_r, b_r, w1, w2, dout, 1.0, dx,
+                                                       dw_r, db_r, dw1, dw2, None, wsb))
+        stb, whereb, infob = sm.switch_get_device_error(wsb)
+        if stb != 0:
+            raise RuntimeError(f"device error {stb} at {whereb} ({infob}) in the backward pass")
+        del wsb, dout, dx, dw1, dw2
     t_aux = timed(lambda: sm.switch_aux_loss(cfg, counts, probs, loss, None, None, ws))
     st, where, info = sm.switch_get_device_error(ws)
     if st != 0:
@@ -535,6 +551,15 @@ def kernel_rooflines(sm, cfg, wl, C, x, w_r, b_r, w1, w2, ws, flush, stream, dev
         "layer_top2": None if t_top2 is None else {
             "us": t_top2 * 1e6, "tokens_per_s": T / t_top2,
             "capacity": sm.switch_capacity(2 * T, N, wl.capacity_factor)},
+        "layer_backward": None if t_bwd is None else {
+            "us": t_bwd * 1e6, "tokens_per_s": T / t_bwd,
+            # algorithmic: dH, dW2, dW1, dX (2 T_kept d F each) + dW_r and dh W_r
+            "useful_flops": 8.0 * T_kept * d * F + 4.0 * T * N * d,
+            "recompute_flops": 2.0 * T_kept * d * F + 2.0 * T * N * d,
+            "tflops": (8.0 * T_kept * d * F + 4.0 * T * N * d) / t_bwd / 1e12,
+            "tflops_with_recompute": (10.0 * T_kept * d * F + 6.0 * T * N * d) / t_bwd / 1e12,
+            "frac_burst_with_recompute": (10.0 * T_kept * d * F + 6.0 * T * N * d) / t_bwd / 1e12
+                                         / pk["bf16_tflops"]},
         "peaks": {"hbm_gbs": hbm, "bf16_tflops": pk["bf16_tflops"], "kind": pk_kind},
         "_T_kept": T_kept,
     }

@@ -8,8 +8,9 @@
 //     the load-balancing loss through P_i (section "The Load-Balancing
 //     Loss"; f_i is piecewise constant);
 //   * the input gradient of dropped tokens (residual and router only).
-// Router arithmetic is fp32 on CUDA cores (no TF32), every reduction in a
-// fixed order.
+// dh is formed in fp32 and split into hi + lo bf16 planes for the tensor
+// cores (the products with bf16 x, or with W_r's own hi + lo split, are then
+// exact to about 2^-17 relative); every reduction runs in a fixed order.
 #include "backward.cuh"
 
 namespace smoe {
@@ -61,23 +62,26 @@ __global__ void __launch_bounds__(256) bwd_gather_kernel(int64_t S, int64_t C, i
 
 // One warp per token.
 __global__ void __launch_bounds__(256) router_bwd_dh_kernel(
-    int64_t T, int N, int64_t C, int ntn, const float* __restrict__ probs,
+    int64_t T, int N, int Np, int64_t C, int64_t S, int ntn, float* __restrict__ probs,
     const int* __restrict__ idx, const int* __restrict__ rank, const uint8_t* __restrict__ drop,
     const float* __restrict__ gate, const float* __restrict__ dgp, const int* __restrict__ counts,
-    float loss_scale, float* __restrict__ dh, float* __restrict__ dgate) {
+    float loss_scale, __nv_bfloat16* __restrict__ dhp, __nv_bfloat16* __restrict__ dhs,
+    float* __restrict__ dgate, int* __restrict__ drop_list, int* __restrict__ n_drop) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t t = static_cast<int64_t>(blockIdx.x) * kWarpsPerBlock + warp;
   if (t >= T) return;
   const bool kept = drop[t] == 0;
   const int e = idx[t];
+  const int64_t s = static_cast<int64_t>(e) * C + rank[t];     // the token's slot if kept
   float dg = 0.f;
   if (kept) {
-    const int64_t s = static_cast<int64_t>(e) * C + rank[t];
     float sum = 0.f;
     for (int j = 0; j < ntn; ++j) sum += dgp[s * ntn + j];     // fixed order
     dg = sum / gate[t];
+  } else if (lane == 0) {
+    drop_list[atomicAdd(n_drop, 1)] = static_cast<int>(t);
   }
-  const float* prow = probs + t * N;
+  float* prow = probs + t * N;
   float acc = 0.f;
   for (int i = lane; i < N; i += 32) {
     const float dp = loss_scale * static_cast<float>(counts[i]) + ((kept && i == e) ? dg : 0.f);
@@ -85,166 +89,87 @@ __global__ void __launch_bounds__(256) router_bwd_dh_kernel(
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-  float* hrow = dh + t * N;
-  for (int i = lane; i < N; i += 32) {
-    const float dp = loss_scale * static_cast<float>(counts[i]) + ((kept && i == e) ? dg : 0.f);
-    hrow[i] = prow[i] * (dp - acc);
+  __syncwarp();
+  for (int i = lane; i < Np; i += 32) {
+    float v = 0.f;
+    if (i < N) {
+      const float dp = loss_scale * static_cast<float>(counts[i]) + ((kept && i == e) ? dg : 0.f);
+      v = prow[i] * (dp - acc);
+      prow[i] = v;                                   // dh in place of p
+    }
+    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
+    dhp[t * Np + i] = hi;
+    dhp[T * Np + t * Np + i] = lo;
+    if (kept) {
+      dhs[s * Np + i] = hi;
+      dhs[S * Np + s * Np + i] = lo;
+    }
   }
   if (dgate != nullptr && lane == 0) dgate[t] = dg;
 }
 
-constexpr int kSB = 64, kSK = 16;
-
-// dxr [T, d] = dh [T, N] . W_r [N, d]; grid (ceil(T/64), ceil(d/64)),
-// 256 threads, 4 x 4 outputs each.
-__global__ void __launch_bounds__(256) router_bwd_dx_kernel(int64_t T, int N, int d,
-                                                            const float* __restrict__ dh,
-                                                            const float* __restrict__ wr,
-                                                            float* __restrict__ dxr) {
-  __shared__ float As[kSK][kSB + 4];
-  __shared__ float Bs[kSK][kSB + 4];
-  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kSB;
-  const int k0 = blockIdx.y * kSB;
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  float acc[4][4] = {};
-  for (int i0 = 0; i0 < N; i0 += kSK) {
-    for (int q = threadIdx.x; q < kSB * kSK; q += 256) {
-      const int rr = q / kSK, kk = q % kSK;
-      As[kk][rr] = (t0 + rr < T && i0 + kk < N) ? dh[(t0 + rr) * N + i0 + kk] : 0.f;
-      const int kb = q / kSB, cc = q % kSB;
-      Bs[kb][cc] = (i0 + kb < N && k0 + cc < d) ? wr[static_cast<int64_t>(i0 + kb) * d + k0 + cc]
-                                                : 0.f;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int kk = 0; kk < kSK; ++kk) {
-      float av[4], bv[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) av[i] = As[kk][ty * 4 + i];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) bv[j] = Bs[kk][tx * 4 + j];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
-    }
-    __syncthreads();
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int64_t t = t0 + ty * 4 + i;
-    if (t >= T) continue;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int k = k0 + tx * 4 + j;
-      if (k < d) dxr[t * d + k] = acc[i][j];
-    }
-  }
-}
-
-constexpr int64_t kDwChunk = 2048;     // tokens per split-K chunk
-
-int64_t dw_chunks(int64_t T) { return (T + kDwChunk - 1) / kDwChunk; }
-
-// part[c][i][k] = sum over tokens t of chunk c of dh[t, i] x[t, k];
-// partb[c][i] = sum over the chunk of dh[t, i].  grid (ceil(N/64),
-// ceil(d/64), chunks).
-__global__ void __launch_bounds__(256) router_bwd_dw_kernel(int64_t T, int N, int d,
-                                                            const float* __restrict__ dh,
-                                                            const __nv_bfloat16* __restrict__ x,
-                                                            float* __restrict__ part,
-                                                            float* __restrict__ partb) {
-  __shared__ float As[kSK][kSB + 4];
-  __shared__ float Bs[kSK][kSB + 4];
-  const int i0 = blockIdx.x * kSB;
-  const int k0 = blockIdx.y * kSB;
-  const int64_t c = blockIdx.z;
-  const int64_t tb = c * kDwChunk;
-  const int64_t te = tb + kDwChunk < T ? tb + kDwChunk : T;
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  float acc[4][4] = {};
-  float sb = 0.f;
-  for (int64_t u0 = tb; u0 < te; u0 += kSK) {
-    for (int q = threadIdx.x; q < kSB * kSK; q += 256) {
-      const int kk = q / kSB, cc = q % kSB;
-      const int64_t t = u0 + kk;
-      As[kk][cc] = (t < te && i0 + cc < N) ? dh[t * N + i0 + cc] : 0.f;
-      Bs[kk][cc] = (t < te && k0 + cc < d) ? __bfloat162float(x[t * d + k0 + cc]) : 0.f;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int kk = 0; kk < kSK; ++kk) {
-      float av[4], bv[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) av[i] = As[kk][ty * 4 + i];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) bv[j] = Bs[kk][tx * 4 + j];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
-    }
-    if (blockIdx.y == 0 && threadIdx.x < kSB) {
-#pragma unroll
-      for (int kk = 0; kk < kSK; ++kk) sb += As[kk][threadIdx.x];
-    }
-    __syncthreads();
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int ii = i0 + ty * 4 + i;
-    if (ii >= N) continue;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int k = k0 + tx * 4 + j;
-      if (k < d) part[(c * N + ii) * d + k] = acc[i][j];
-    }
-  }
-  if (blockIdx.y == 0 && threadIdx.x < kSB && i0 + static_cast<int>(threadIdx.x) < N)
-    partb[c * N + i0 + threadIdx.x] = sb;
-}
-
-// dw_r[i, k] = sum_c part[c][i][k] in chunk order; db[i] likewise.
-__global__ void router_bwd_reduce_kernel(int64_t nch, int N, int d, const float* __restrict__ part,
-                                         const float* __restrict__ partb, float* __restrict__ dw_r,
-                                         float* __restrict__ db) {
+// wrp[0][i][k] = bf16(W_r[i, k]), wrp[1][i][k] = bf16(W_r[i, k] - hi), zero
+// rows for N <= i < Np.
+__global__ void wr_split_kernel(int N, int Np, int d, const float* __restrict__ w_r,
+                                __nv_bfloat16* __restrict__ wrp) {
   const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t nd = static_cast<int64_t>(N) * d;
-  if (j < nd) {
-    float s = 0.f;
-    for (int64_t c = 0; c < nch; ++c) s += part[c * nd + j];
-    dw_r[j] = s;
-  }
-  if (db != nullptr && j < N) {
-    float s = 0.f;
-    for (int64_t c = 0; c < nch; ++c) s += partb[c * N + j];
-    db[j] = s;
-  }
+  const int64_t n = static_cast<int64_t>(Np) * d;
+  if (j >= n) return;
+  const float w = j < static_cast<int64_t>(N) * d ? w_r[j] : 0.f;
+  const __nv_bfloat16 hi = __float2bfloat16_rn(w);
+  wrp[j] = hi;
+  wrp[n + j] = __float2bfloat16_rn(w - __bfloat162float(hi));
 }
 
-// One warp per token; only dropped tokens are written.
-__global__ void __launch_bounds__(256) bwd_dropped_kernel(int64_t T, int d,
-                                                          const uint8_t* __restrict__ drop,
-                                                          const uint4* __restrict__ dout,
-                                                          const float4* __restrict__ dxr,
-                                                          uint4* __restrict__ dx, int residual) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t t = static_cast<int64_t>(blockIdx.x) * kWarpsPerBlock + warp;
-  if (t >= T || drop[t] == 0) return;
-  const int dv = d / 8;
-  for (int v = lane; v < dv; v += 32) {
-    const float4 a = dxr[(t * dv + v) * 2];
-    const float4 b = dxr[(t * dv + v) * 2 + 1];
-    float o[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-    if (residual) {
-      const uint4 g = dout[t * dv + v];
-      o[0] += bf16_lo(g.x); o[1] += bf16_hi(g.x);
-      o[2] += bf16_lo(g.y); o[3] += bf16_hi(g.y);
-      o[4] += bf16_lo(g.z); o[5] += bf16_hi(g.z);
-      o[6] += bf16_lo(g.w); o[7] += bf16_hi(g.w);
+constexpr int kDropTok = 16;     // dropped tokens per block
+
+// dx[t] = (residual ? dout[t] : 0) + dh[t] . W_r for the listed tokens;
+// block (b, y) takes list entries [16 g, 16 g + 16) for g = b, b + gridDim.x,
+// ... and columns [256 y, 256 y + 256): dh rows staged in shared memory,
+// each W_r element read once per group.
+__global__ void __launch_bounds__(256) bwd_dropped_kernel(
+    int N, int d, const int* __restrict__ drop_list, const int* __restrict__ n_drop,
+    const float* __restrict__ dh, const float* __restrict__ w_r,
+    const __nv_bfloat16* __restrict__ dout, __nv_bfloat16* __restrict__ dx, int residual) {
+  extern __shared__ float sdh[];                       // [kDropTok][N]
+  __shared__ int toks[kDropTok];
+  const int nd = *n_drop;
+  for (int first = blockIdx.x * kDropTok; first < nd; first += gridDim.x * kDropTok) {
+    const int cnt = nd - first < kDropTok ? nd - first : kDropTok;
+    __syncthreads();                                     // previous group done with sdh / toks
+    if (threadIdx.x < kDropTok) toks[threadIdx.x] = threadIdx.x < cnt ? drop_list[first + threadIdx.x] : -1;
+    __syncthreads();
+    for (int q = threadIdx.x; q < kDropTok * N; q += blockDim.x) {
+      const int j = q / N, i = q - j * N;
+      sdh[q] = j < cnt ? dh[static_cast<int64_t>(toks[j]) * N + i] : 0.f;
     }
-    dx[t * dv + v] = make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]),
-                                pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7]));
+    __syncthreads();
+    for (int k = blockIdx.y * blockDim.x + threadIdx.x; k < d; k += gridDim.y * blockDim.x) {
+      float acc[kDropTok];
+#pragma unroll
+      for (int j = 0; j < kDropTok; ++j) acc[j] = 0.f;
+      int i = 0;
+      for (; i + 16 <= N; i += 16) {        // sixteen W_r loads in flight
+        float w[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) w[u] = __ldg(w_r + static_cast<int64_t>(i + u) * d + k);
+#pragma unroll
+        for (int u = 0; u < 16; ++u)
+#pragma unroll
+          for (int j = 0; j < kDropTok; ++j) acc[j] = fmaf(sdh[j * N + i + u], w[u], acc[j]);
+      }
+      for (; i < N; ++i) {
+        const float w = __ldg(w_r + static_cast<int64_t>(i) * d + k);
+#pragma unroll
+        for (int j = 0; j < kDropTok; ++j) acc[j] = fmaf(sdh[j * N + i], w, acc[j]);
+      }
+      for (int j = 0; j < cnt; ++j) {
+        const int64_t o = static_cast<int64_t>(toks[j]) * d + k;
+        const float r = residual ? __bfloat162float(dout[o]) : 0.f;
+        dx[o] = __float2bfloat16_rn(r + acc[j]);
+      }
+    }
   }
 }
 
@@ -265,47 +190,42 @@ cudaError_t launch_bwd_gather(int64_t C, int N, int d, int F, const int* counts,
   return cudaGetLastError();
 }
 
-cudaError_t launch_router_bwd_dh(int64_t T, int N, int64_t C, int ntn, const float* probs,
+cudaError_t launch_router_bwd_dh(int64_t T, int N, int Np, int64_t C, int ntn, float* probs,
                                  const int* idx, const int* rank, const uint8_t* drop,
                                  const float* gate, const float* dgp, const int* counts,
-                                 float loss_scale, float* dh, float* dgate, cudaStream_t st) {
-  router_bwd_dh_kernel<<<warp_blocks(T), 256, 0, st>>>(T, N, C, ntn, probs, idx, rank, drop, gate,
-                                                       dgp, counts, loss_scale, dh, dgate);
+                                 float loss_scale, void* dhp, void* dhs, float* dgate,
+                                 int* drop_list, int* n_drop, cudaStream_t st) {
+  const int64_t S = static_cast<int64_t>(N) * C;
+  router_bwd_dh_kernel<<<warp_blocks(T), 256, 0, st>>>(
+      T, N, Np, C, S, ntn, probs, idx, rank, drop, gate, dgp, counts, loss_scale,
+      static_cast<__nv_bfloat16*>(dhp), static_cast<__nv_bfloat16*>(dhs), dgate, drop_list,
+      n_drop);
   return cudaGetLastError();
 }
 
-cudaError_t launch_router_bwd_dx(int64_t T, int N, int d, const float* dh, const float* w_r,
-                                 float* dxr, cudaStream_t st) {
-  const dim3 grid(static_cast<unsigned>((T + kSB - 1) / kSB), static_cast<unsigned>((d + kSB - 1) / kSB));
-  router_bwd_dx_kernel<<<grid, 256, 0, st>>>(T, N, d, dh, w_r, dxr);
+cudaError_t launch_wr_split(int N, int d, const float* w_r, void* wrp, cudaStream_t st) {
+  const int Np = (N + 63) / 64 * 64;
+  const int64_t n = static_cast<int64_t>(Np) * d;
+  wr_split_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(
+      N, Np, d, w_r, static_cast<__nv_bfloat16*>(wrp));
   return cudaGetLastError();
 }
 
-size_t router_bwd_part_floats(int64_t T, int N, int d) {
-  return static_cast<size_t>(dw_chunks(T)) * static_cast<size_t>(N) * (static_cast<size_t>(d) + 1);
-}
-
-cudaError_t launch_router_bwd_dw(int64_t T, int N, int d, const float* dh, const void* x,
-                                 float* part, float* dw_r, float* db, cudaStream_t st) {
-  const int64_t nch = dw_chunks(T);
-  float* partb = part + nch * N * static_cast<int64_t>(d);
-  const dim3 grid(static_cast<unsigned>((N + kSB - 1) / kSB), static_cast<unsigned>((d + kSB - 1) / kSB),
-                  static_cast<unsigned>(nch));
-  router_bwd_dw_kernel<<<grid, 256, 0, st>>>(T, N, d, dh, static_cast<const __nv_bfloat16*>(x),
-                                             part, partb);
-  cudaError_t e = cudaGetLastError();
+cudaError_t launch_bwd_dropped(int64_t T, int N, int d, const int* drop_list, const int* n_drop,
+                               const float* dh, const float* w_r, const void* dout, void* dx,
+                               bool residual, cudaStream_t st) {
+  const size_t smem = sizeof(float) * kDropTok * static_cast<size_t>(N);
+  static size_t smem_set[64] = {};
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(&bwd_dropped_kernel), smem,
+                                    smem_set);
   if (e != cudaSuccess) return e;
-  const int64_t nd = static_cast<int64_t>(N) * d;
-  router_bwd_reduce_kernel<<<static_cast<unsigned>((nd + 255) / 256), 256, 0, st>>>(
-      nch, N, d, part, partb, dw_r, db);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_bwd_dropped(int64_t T, int d, const uint8_t* drop, const void* dout,
-                               const float* dxr, void* dx, bool residual, cudaStream_t st) {
-  bwd_dropped_kernel<<<warp_blocks(T), 256, 0, st>>>(
-      T, d, drop, static_cast<const uint4*>(dout), reinterpret_cast<const float4*>(dxr),
-      static_cast<uint4*>(dx), residual ? 1 : 0);
+  // a few waves at most: blocks loop over the list in steps of the grid
+  const int64_t groups = (T + kDropTok - 1) / kDropTok;
+  const dim3 blocks(static_cast<unsigned>(groups < 296 ? groups : 296),
+                    static_cast<unsigned>((d + 255) / 256));
+  bwd_dropped_kernel<<<blocks, 256, smem, st>>>(
+      N, d, drop_list, n_drop, dh, w_r, static_cast<const __nv_bfloat16*>(dout),
+      static_cast<__nv_bfloat16*>(dx), residual ? 1 : 0);
   return cudaGetLastError();
 }
 

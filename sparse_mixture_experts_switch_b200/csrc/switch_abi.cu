@@ -41,8 +41,10 @@ struct Layout {
   size_t err, hist, base, psum, fpsc, local_rank, idx, gate, rank, drop, counts, counts1,
       slot_token, mtile_start, wsplit, logits, xdisp, hbuf, ybuf, total;
   // backward pass only (after the forward regions): dA, partial gate
-  // gradients, dh, gate gradient, router part of dx, split-K partials
-  size_t da, dgp, dh, dgate, dxr, rpart, bwd_total;
+  // gradients, dh (fp32, and its bf16 planes per token and per slot), W_r
+  // planes, gate gradient, split-K partials of dW_r, column sums of dh,
+  // dropped-token list and its counter
+  size_t da, dgp, dh, dhp, dhs, wrp, dgate, rpart, colsum, drop_list, n_drop, bwd_total;
 };
 
 // Bytes 16..19 of the workspace: the loss kernel's completion ticket (kept
@@ -93,10 +95,16 @@ Layout layout_for(const switch_config_t& c, int64_t C) {
   const int64_t ntn = (c.d_ff + 255) / 256;
   L.da = take(es * slots * static_cast<size_t>(c.d_ff));
   L.dgp = take(sizeof(float) * slots * ntn);
+  const int64_t Np = (N + 63) / 64 * 64;
   L.dh = take(sizeof(float) * N * T);
+  L.dhp = take(2 * 2 * static_cast<size_t>(T) * Np);
+  L.dhs = take(2 * 2 * static_cast<size_t>(slots) * Np);
+  L.wrp = take(2 * 2 * static_cast<size_t>(Np) * c.d_model);
   L.dgate = take(sizeof(float) * T);
-  L.dxr = take(sizeof(float) * T * static_cast<size_t>(c.d_model));
-  L.rpart = take(sizeof(float) * router_bwd_part_floats(T, c.n_experts, c.d_model));
+  L.rpart = take(sizeof(float) * router_bwd_tc_part_floats(T, c.n_experts, c.d_model, 0));
+  L.colsum = take(sizeof(float) * N * ntiles_of(T));
+  L.drop_list = take(sizeof(int) * T);
+  L.n_drop = take(sizeof(int));
   L.bwd_total = o;
   return L;
 }
@@ -544,29 +552,41 @@ switch_status_t switch_layer_backward(const switch_config_t* cfg, const void* x,
   b.dw1 = dw1;
   b.dw2 = dw2;
   b.dout = dout;
-  b.dxr = c.at<float>(c.L.dxr);
   b.dx = dx;
   b.residual = residual;
+  b.pair_dw = !(cfg->flags & SWITCH_FLAG_GEMM_1SM);
   b.err = c.err;
   b.spin = c.spin;
   b.num_sms = c.num_sms;
   SMOE_TRY(launch_bwd_dh(b, c.st));
   SMOE_TRY(launch_bwd_dw(b, c.st));
 
-  // 3. router: dh (in place of the probabilities), its input and weight
-  // gradients
+  // 3. router: dh (in place of the probabilities) and its bf16 planes, the
+  // weight and bias gradients
   float* dh = probs;
+  const int Np = (N + 63) / 64 * 64;
+  int* n_drop = c.at<int>(c.L.n_drop);
+  int* drop_list = c.at<int>(c.L.drop_list);
   const double ls = static_cast<double>(dloss) * cfg->alpha * N / (static_cast<double>(T) * T);
-  SMOE_TRY(launch_router_bwd_dh(T, N, c.C, (F + 255) / 256, probs, idx, rank, drop, gate,
-                                b.dgp, counts, static_cast<float>(ls), dh,
-                                dgate ? dgate : c.at<float>(c.L.dgate), c.st));
-  SMOE_TRY(launch_router_bwd_dx(T, N, d, dh, w_r, c.at<float>(c.L.dxr), c.st));
-  SMOE_TRY(launch_router_bwd_dw(T, N, d, dh, x, c.at<float>(c.L.rpart), dw_r, db_r, c.st));
+  SMOE_TRY(cudaMemsetAsync(n_drop, 0, sizeof(int), c.st));
+  SMOE_TRY(launch_router_bwd_dh(T, N, Np, c.C, (F + 255) / 256, probs, idx, rank, drop, gate,
+                                b.dgp, counts, static_cast<float>(ls), c.ws + c.L.dhp,
+                                c.ws + c.L.dhs, dgate ? dgate : c.at<float>(c.L.dgate),
+                                drop_list, n_drop, c.st));
+  float* colsum = c.at<float>(c.L.colsum);
+  if (db_r) SMOE_TRY(launch_prob_colsum(T, N, dh, colsum, c.st));
+  SMOE_TRY(launch_router_bwd_dw_tc(T, N, Np, d, c.ws + c.L.dhp, x, c.at<float>(c.L.rpart),
+                                   colsum, dw_r, db_r, c.err, c.spin, c.num_sms, c.st));
 
-  // 4. input gradient: kept tokens in the dX GEMM's epilogue, dropped ones
-  // here
+  // 4. input gradient: kept tokens in the dX GEMM (dA W1_e and dh W_r in one
+  // accumulation), dropped ones from the list
+  SMOE_TRY(launch_wr_split(N, d, w_r, c.ws + c.L.wrp, c.st));
+  b.dhs = c.ws + c.L.dhs;
+  b.wrp = c.ws + c.L.wrp;
+  b.n_router = N;
+  b.n_pad = Np;
   SMOE_TRY(launch_bwd_dx(b, c.st));
-  SMOE_TRY(launch_bwd_dropped(T, d, drop, dout, c.at<float>(c.L.dxr), dx, residual, c.st));
+  SMOE_TRY(launch_bwd_dropped(T, N, d, drop_list, n_drop, dh, w_r, dout, dx, residual, c.st));
   return SWITCH_OK;
 }
 

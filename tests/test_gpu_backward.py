@@ -149,6 +149,13 @@ def test_backward_no_drops_ragged(sm):
     assert not want["drop"].any()
 
 
+def test_backward_many_experts(sm):
+    """N = 100: the router's bf16 planes are padded to 128 columns."""
+    wl = Workload("bwd_n100", T=2500, d_model=128, d_ff=192, n_experts=100,
+                  capacity_factor=1.0, dtype="bf16", seed=29)
+    check_backward(sm, wl, dloss=2.0)
+
+
 def test_backward_deterministic(sm):
     inp = make_inputs(SMALL)
     dout = make_dout(SMALL)
