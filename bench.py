@@ -508,7 +508,7 @@ def kernel_rooflines(sm, cfg, wl, C, x, w_r, b_r, w1, w2, ws, flush, stream, dev
             raise RuntimeError(f"device error {st2} at {where2} ({info2}) in the top-2 layer")
         del ws2
     # the backward pass of the whole layer (recomputes routing, dispatch and H)
-    t_bwd = None
+    t_bwd = t_bwd_saved = t_train = None
     if wl.dtype == "bf16":
         wsb = sm.backward_workspace(cfg, device=dev)
         dout = torch.empty_like(x).normal_()
@@ -522,7 +522,27 @@ def kernel_rooflines(sm, cfg, wl, C, x, w_r, b_r, w1, w2, ws, flush, stream, dev
         stb, whereb, infob = sm.switch_get_device_error(wsb)
         if stb != 0:
             raise RuntimeError(f"device error {stb} at {whereb} ({infob}) in the backward pass")
-        del wsb, dout, dx, dw1, dw2
+        del wsb
+        # training mode: the forward keeps its activations, the backward reads
+        # them (no recompute); and one whole training step of the layer
+        cfg_t = sm.config(T, d, F, N, wl.capacity_factor, dtype=wl.dtype, alpha=wl.alpha,
+                          flags=sm.FLAG_TRAINING)
+        wst = sm.backward_workspace(cfg_t, device=dev)
+
+        def fwd_t():
+            sm.switch_layer_forward(cfg_t, x, w_r, b_r, w1, w2, out, idx, gate, counts, loss, wst)
+
+        def bwd_t():
+            sm.switch_layer_backward(cfg_t, x, w_r, b_r, w1, w2, dout, 1.0, dx, dw_r, db_r, dw1,
+                                     dw2, None, wst)
+
+        fwd_t()
+        t_bwd_saved = timed(bwd_t)
+        t_train = timed(lambda: (fwd_t(), bwd_t()))
+        stb, whereb, infob = sm.switch_get_device_error(wst)
+        if stb != 0:
+            raise RuntimeError(f"device error {stb} at {whereb} ({infob}) in the training step")
+        del wst, dout, dx, dw1, dw2
     t_aux = timed(lambda: sm.switch_aux_loss(cfg, counts, probs, loss, None, None, ws))
     st, where, info = sm.switch_get_device_error(ws)
     if st != 0:
@@ -560,6 +580,16 @@ def kernel_rooflines(sm, cfg, wl, C, x, w_r, b_r, w1, w2, ws, flush, stream, dev
             "tflops_with_recompute": (10.0 * T_kept * d * F + 6.0 * T * N * d) / t_bwd / 1e12,
             "frac_burst_with_recompute": (10.0 * T_kept * d * F + 6.0 * T * N * d) / t_bwd / 1e12
                                          / pk["bf16_tflops"]},
+        "layer_backward_saved": None if t_bwd_saved is None else {
+            "us": t_bwd_saved * 1e6, "tokens_per_s": T / t_bwd_saved,
+            "tflops": (8.0 * T_kept * d * F + 4.0 * T * N * d) / t_bwd_saved / 1e12,
+            "frac_burst": (8.0 * T_kept * d * F + 4.0 * T * N * d) / t_bwd_saved / 1e12
+                          / pk["bf16_tflops"],
+            "note": "SWITCH_FLAG_TRAINING: activations kept by the forward, no recompute"},
+        "training_step": None if t_train is None else {
+            "us": t_train * 1e6, "tokens_per_s": T / t_train,
+            "tflops": (12.0 * T_kept * d * F + 6.0 * T * N * d) / t_train / 1e12,
+            "note": "switch_layer_forward + switch_layer_backward, SWITCH_FLAG_TRAINING"},
         "peaks": {"hbm_gbs": hbm, "bf16_tflops": pk["bf16_tflops"], "kind": pk_kind},
         "_T_kept": T_kept,
     }

@@ -84,7 +84,10 @@ enum {
                                         GEMM2 CTA pairs) */
   SWITCH_FLAG_ROWS_DISPATCHED = 128, /* switch_expert_ffn: x is the dispatched row buffer
                                         x_disp [N*C, d_model] from switch_dispatch */
-  SWITCH_FLAG_TOP2 = 512             /* top-k routing with k = 2 (see "Top-2 routing" below) */
+  SWITCH_FLAG_TOP2 = 512,            /* top-k routing with k = 2 (see "Top-2 routing" below) */
+  SWITCH_FLAG_TRAINING = 1024        /* forward keeps what switch_layer_backward needs in the
+                                        workspace; the backward then reads it instead of
+                                        recomputing (see switch_layer_backward) */
 };
 
 typedef struct {
@@ -258,9 +261,16 @@ switch_status_t switch_layer_forward(const switch_config_t* cfg, const void* x,
  *   dh = p (dp - sum_j p_j dp_j),  dx += dh W_r,  dW_r = dh^T x,
  *   db_r = sum_t dh,  dx += dout (the residual branch, unless
  *   SWITCH_FLAG_NO_RESIDUAL).
- * The call recomputes the forward's routing, dispatch and hidden
- * activations from its inputs (as activation checkpointing does); it reads
- * nothing a previous call left in the workspace.
+ * Saved activations: without SWITCH_FLAG_TRAINING the call recomputes the
+ * forward's routing, dispatch and hidden activations from its inputs (as
+ * activation checkpointing does) and reads nothing a previous call left in
+ * the workspace.  With SWITCH_FLAG_TRAINING, switch_layer_forward (given a
+ * workspace of switch_backward_workspace_size() bytes) keeps the router
+ * probabilities, the routing, the dispatched rows and H there, and this
+ * call reads them instead: it must follow that forward call with the same
+ * config, inputs and workspace, with no other call on the workspace in
+ * between (backward calls may repeat: they leave that state unchanged).
+ * Both ways give bit-identical gradients.
  *   x [T, d_model] bf16, w_r [N, d_model] fp32, b_r [N] fp32 or NULL,
  *   w1 [N, d_ff, d_model] bf16, w2 [N, d_model, d_ff] bf16 (as the forward);
  *   dout [T, d_model] bf16: gradient of J with respect to out;
@@ -272,7 +282,8 @@ switch_status_t switch_layer_forward(const switch_config_t* cfg, const void* x,
  * accumulation; gate * dout, dA and the weight gradients rounded once to
  * bf16); router backward in fp32 FMA with fixed-order reductions (dW_r and
  * db_r bit-reproducible).  Workspace: switch_backward_workspace_size()
- * bytes.  dtype SWITCH_F32 or SWITCH_FLAG_TOP2 return SWITCH_ERR_UNSUPPORTED.
+ * bytes.  dtype SWITCH_F32 or SWITCH_FLAG_TOP2 return SWITCH_ERR_UNSUPPORTED
+ * (so does switch_layer_forward given SWITCH_FLAG_TRAINING with either).
  * T = 0 writes nothing. */
 switch_status_t switch_layer_backward(const switch_config_t* cfg, const void* x,
                                       const float* w_r, const float* b_r,

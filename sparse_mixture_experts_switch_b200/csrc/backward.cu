@@ -62,11 +62,12 @@ __global__ void __launch_bounds__(256) bwd_gather_kernel(int64_t S, int64_t C, i
 
 // One warp per token.
 __global__ void __launch_bounds__(256) router_bwd_dh_kernel(
-    int64_t T, int N, int Np, int64_t C, int64_t S, int ntn, float* __restrict__ probs,
+    int64_t T, int N, int Np, int64_t C, int64_t S, int ntn, const float* __restrict__ probs,
     const int* __restrict__ idx, const int* __restrict__ rank, const uint8_t* __restrict__ drop,
     const float* __restrict__ gate, const float* __restrict__ dgp, const int* __restrict__ counts,
-    float loss_scale, __nv_bfloat16* __restrict__ dhp, __nv_bfloat16* __restrict__ dhs,
-    float* __restrict__ dgate, int* __restrict__ drop_list, int* __restrict__ n_drop) {
+    float loss_scale, float* __restrict__ dh, __nv_bfloat16* __restrict__ dhp,
+    __nv_bfloat16* __restrict__ dhs, float* __restrict__ dgate, int* __restrict__ drop_list,
+    int* __restrict__ n_drop) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t t = static_cast<int64_t>(blockIdx.x) * kWarpsPerBlock + warp;
   if (t >= T) return;
@@ -81,7 +82,7 @@ __global__ void __launch_bounds__(256) router_bwd_dh_kernel(
   } else if (lane == 0) {
     drop_list[atomicAdd(n_drop, 1)] = static_cast<int>(t);
   }
-  float* prow = probs + t * N;
+  const float* prow = probs + t * N;
   float acc = 0.f;
   for (int i = lane; i < N; i += 32) {
     const float dp = loss_scale * static_cast<float>(counts[i]) + ((kept && i == e) ? dg : 0.f);
@@ -95,7 +96,7 @@ __global__ void __launch_bounds__(256) router_bwd_dh_kernel(
     if (i < N) {
       const float dp = loss_scale * static_cast<float>(counts[i]) + ((kept && i == e) ? dg : 0.f);
       v = prow[i] * (dp - acc);
-      prow[i] = v;                                   // dh in place of p
+      dh[t * N + i] = v;
     }
     const __nv_bfloat16 hi = __float2bfloat16_rn(v);
     const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
@@ -190,14 +191,15 @@ cudaError_t launch_bwd_gather(int64_t C, int N, int d, int F, const int* counts,
   return cudaGetLastError();
 }
 
-cudaError_t launch_router_bwd_dh(int64_t T, int N, int Np, int64_t C, int ntn, float* probs,
-                                 const int* idx, const int* rank, const uint8_t* drop,
-                                 const float* gate, const float* dgp, const int* counts,
-                                 float loss_scale, void* dhp, void* dhs, float* dgate,
-                                 int* drop_list, int* n_drop, cudaStream_t st) {
+cudaError_t launch_router_bwd_dh(int64_t T, int N, int Np, int64_t C, int ntn,
+                                 const float* probs, const int* idx, const int* rank,
+                                 const uint8_t* drop, const float* gate, const float* dgp,
+                                 const int* counts, float loss_scale, float* dh, void* dhp,
+                                 void* dhs, float* dgate, int* drop_list, int* n_drop,
+                                 cudaStream_t st) {
   const int64_t S = static_cast<int64_t>(N) * C;
   router_bwd_dh_kernel<<<warp_blocks(T), 256, 0, st>>>(
-      T, N, Np, C, S, ntn, probs, idx, rank, drop, gate, dgp, counts, loss_scale,
+      T, N, Np, C, S, ntn, probs, idx, rank, drop, gate, dgp, counts, loss_scale, dh,
       static_cast<__nv_bfloat16*>(dhp), static_cast<__nv_bfloat16*>(dhs), dgate, drop_list,
       n_drop);
   return cudaGetLastError();

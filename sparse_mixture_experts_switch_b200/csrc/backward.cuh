@@ -95,15 +95,16 @@ cudaError_t launch_bwd_gather(int64_t C, int N, int d, int F, const int* counts,
 //   dh[t, i] = p[t, i] (dp[t, i] - sum_j p[t, j] dp[t, j]).
 // loss_scale = dloss * alpha * N / T^2 (the load-balancing loss's gradient
 // per routed token).
-// Outputs: dh [T, N] fp32 (in place of probs), its hi / lo bf16 planes
+// Outputs: dh [T, N] fp32 (probs is left as it is), its hi / lo bf16 planes
 // dhp [2][T][Np] and, for kept tokens, dhs [2][N*C][Np] at the token's slot
 // (columns N..Np-1 zero), the gate gradient, and the list of dropped tokens
 // (drop_list[0..*n_drop), any order; *n_drop must be zero on entry).
-cudaError_t launch_router_bwd_dh(int64_t T, int N, int Np, int64_t C, int ntn, float* probs,
-                                 const int* idx, const int* rank, const uint8_t* drop,
-                                 const float* gate, const float* dgp, const int* counts,
-                                 float loss_scale, void* dhp, void* dhs, float* dgate,
-                                 int* drop_list, int* n_drop, cudaStream_t st);
+cudaError_t launch_router_bwd_dh(int64_t T, int N, int Np, int64_t C, int ntn,
+                                 const float* probs, const int* idx, const int* rank,
+                                 const uint8_t* drop, const float* gate, const float* dgp,
+                                 const int* counts, float loss_scale, float* dh, void* dhp,
+                                 void* dhs, float* dgate, int* drop_list, int* n_drop,
+                                 cudaStream_t st);
 // wrp [2][N][d] = hi / lo bf16 split of W_r (hi = bf16(W), lo = bf16(W - hi)).
 cudaError_t launch_wr_split(int N, int d, const float* w_r, void* wrp, cudaStream_t st);
 // Dropped tokens (from the list): dx[t] = bf16((residual ? dout[t] : 0) +

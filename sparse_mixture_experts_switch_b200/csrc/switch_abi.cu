@@ -44,7 +44,8 @@ struct Layout {
   // gradients, dh (fp32, and its bf16 planes per token and per slot), W_r
   // planes, gate gradient, split-K partials of dW_r, column sums of dh,
   // dropped-token list and its counter
-  size_t da, dgp, dh, dhp, dhs, wrp, dgate, rpart, colsum, drop_list, n_drop, bwd_total;
+  size_t probs_s, da, dgp, dh, dhp, dhs, wrp, dgate, rpart, colsum, drop_list, n_drop,
+      bwd_total;
 };
 
 // Bytes 16..19 of the workspace: the loss kernel's completion ticket (kept
@@ -93,6 +94,7 @@ Layout layout_for(const switch_config_t& c, int64_t C) {
   L.ybuf = take(es * slots * static_cast<size_t>(c.d_model));
   L.total = o;
   const int64_t ntn = (c.d_ff + 255) / 256;
+  L.probs_s = take(sizeof(float) * N * T);      // router probabilities kept for the backward
   L.da = take(es * slots * static_cast<size_t>(c.d_ff));
   L.dgp = take(sizeof(float) * slots * ntn);
   const int64_t Np = (N + 63) / 64 * 64;
@@ -370,9 +372,17 @@ switch_status_t switch_layer_forward(const switch_config_t* cfg, const void* x,
   const bool top2 = routes_of(*cfg) == 2;
   const int64_t A = routes_of(*cfg) * T;                // assignments, route-major
   const int nta = ntiles_of(A);
-  int* idx_p = idx ? idx : c.at<int>(c.L.idx);
-  float* gate_p = gate ? gate : c.at<float>(c.L.gate);
-  int* counts_p = counts ? counts : c.at<int>(c.L.counts);
+  // SWITCH_FLAG_TRAINING: keep probabilities, routing, x_disp and H in the
+  // workspace for switch_layer_backward (routing arrays always in the
+  // workspace, copied out to the caller's at the end)
+  const bool training = (cfg->flags & SWITCH_FLAG_TRAINING) != 0;
+  if (training) {
+    if (!bf16 || top2) return SWITCH_ERR_UNSUPPORTED;
+    if (ws_bytes < c.L.bwd_total) return SWITCH_ERR_WORKSPACE_TOO_SMALL;
+  }
+  int* idx_p = (idx && !training) ? idx : c.at<int>(c.L.idx);
+  float* gate_p = (gate && !training) ? gate : c.at<float>(c.L.gate);
+  int* counts_p = (counts && !training) ? counts : c.at<int>(c.L.counts);
   int* local_rank = c.at<int>(c.L.local_rank);
   int* hist = c.at<int>(c.L.hist);
   float* psum = c.at<float>(c.L.psum);
@@ -380,8 +390,8 @@ switch_status_t switch_layer_forward(const switch_config_t* cfg, const void* x,
 
   // 1. router (+ per-tile ranks and histograms of the first choices on the
   // tensor-core path)
-  RouterOut o{idx_p, gate_p, nullptr, psum, nullptr, nullptr,
-              top2 ? idx_p + T : nullptr, top2 ? gate_p + T : nullptr};
+  RouterOut o{idx_p, gate_p, training ? c.at<float>(c.L.probs_s) : nullptr, psum, nullptr,
+              nullptr, top2 ? idx_p + T : nullptr, top2 ? gate_p + T : nullptr};
   if (use_tc_router(cfg)) {
     o.hist = hist;
     o.local_rank = local_rank;
@@ -452,6 +462,15 @@ switch_status_t switch_layer_forward(const switch_config_t* cfg, const void* x,
     SMOE_TRY(launch_aux_loss(T, N, nparts, cfg->alpha, counts_loss, psum, loss, nullptr,
                              nullptr, c.at<double>(c.L.fpsc), c.at<unsigned>(kTicketOffset),
                              c.st));
+  if (training) {
+    if (idx)
+      SMOE_TRY(cudaMemcpyAsync(idx, idx_p, sizeof(int) * T, cudaMemcpyDeviceToDevice, c.st));
+    if (gate)
+      SMOE_TRY(cudaMemcpyAsync(gate, gate_p, sizeof(float) * T, cudaMemcpyDeviceToDevice, c.st));
+    if (counts)
+      SMOE_TRY(cudaMemcpyAsync(counts, counts_p, sizeof(int) * N, cudaMemcpyDeviceToDevice,
+                               c.st));
+  }
   return SWITCH_OK;
 }
 
@@ -477,7 +496,7 @@ switch_status_t switch_layer_backward(const switch_config_t* cfg, const void* x,
   const int64_t S = static_cast<int64_t>(N) * c.C;
   int* idx = c.at<int>(c.L.idx);
   float* gate = c.at<float>(c.L.gate);
-  float* probs = c.at<float>(c.L.dh);          // dh overwrites it in place
+  float* probs = c.at<float>(c.L.probs_s);
   int* counts = c.at<int>(c.L.counts);
   int* local_rank = c.at<int>(c.L.local_rank);
   int* hist = c.at<int>(c.L.hist);
@@ -487,47 +506,55 @@ switch_status_t switch_layer_backward(const switch_config_t* cfg, const void* x,
   int* mtile_start = c.at<int>(c.L.mtile_start);
   const bool residual = !(cfg->flags & SWITCH_FLAG_NO_RESIDUAL);
 
-  // 1. the forward's routing, dispatch and hidden activations, recomputed
-  // (same kernels, same results): probabilities, slots, x_disp, H
-  RouterOut o{idx, gate, probs, c.at<float>(c.L.psum), nullptr, nullptr, nullptr, nullptr};
-  if (use_tc_router(cfg)) {
-    o.hist = hist;
-    o.local_rank = local_rank;
-    SMOE_TRY(launch_router_tc(T, d, N, router_terms(cfg), x, w_r, b_r, c.ws + c.L.wsplit, o, nt,
-                              c.err, c.spin, c.num_sms, c.st));
-  } else {
-    int nparts = 0;
-    SMOE_TRY(launch_router_simt(T, d, N, true, x, w_r, b_r, c.at<float>(c.L.logits), o, &nparts,
-                                c.st));
-    SMOE_TRY(launch_tile_rank(T, N, idx, nullptr, nullptr, local_rank, hist, nt, c.err, c.st));
-  }
-  SMOE_TRY(launch_scan(N, nt, hist, c.at<int>(c.L.base), counts, c.st));
-  SMOE_TRY(launch_finalize(T, N, c.C, nt, idx, local_rank, c.at<int>(c.L.base), counts, rank,
-                           drop, slot_token, mtile_start, 0, c.st));
   void* x_disp = c.ws + c.L.xdisp;
   void* hbuf = c.ws + c.L.hbuf;
-  SMOE_TRY(launch_gather_rows(S, static_cast<int64_t>(d) * 2, slot_token, x, x_disp, c.st));
-  FfnArgs a{};
-  a.T = T;
-  a.d = d;
-  a.F = F;
-  a.N = N;
-  a.C = c.C;
-  a.x = x;
-  a.x_disp = x_disp;
-  a.slot_token = slot_token;
-  a.counts = counts;
-  a.mtile_start = mtile_start;
-  a.w1 = w1;
-  a.w2 = w2;
-  a.hbuf = hbuf;
-  a.mode2 = kModeY;
-  a.pair1 = (cfg->flags & SWITCH_FLAG_GEMM_PAIRS) != 0;
-  a.gemm1_only = true;
-  a.err = c.err;
-  a.spin = c.spin;
-  a.num_sms = c.num_sms;
-  SMOE_TRY(launch_expert_ffn_bf16(a, c.st));
+  const bool saved = (cfg->flags & SWITCH_FLAG_TRAINING) != 0;
+  if (saved) {
+    // 1'. the forward (same flag) left probabilities, routing and H here;
+    // only the row copy is missing if it gathered inside GEMM1
+    if (cfg->flags & SWITCH_FLAG_GATHER_IN_GEMM)
+      SMOE_TRY(launch_gather_rows(S, static_cast<int64_t>(d) * 2, slot_token, x, x_disp, c.st));
+  } else {
+    // 1. the forward's routing, dispatch and hidden activations, recomputed
+    // (same kernels, same results): probabilities, slots, x_disp, H
+    RouterOut o{idx, gate, probs, c.at<float>(c.L.psum), nullptr, nullptr, nullptr, nullptr};
+    if (use_tc_router(cfg)) {
+      o.hist = hist;
+      o.local_rank = local_rank;
+      SMOE_TRY(launch_router_tc(T, d, N, router_terms(cfg), x, w_r, b_r, c.ws + c.L.wsplit, o, nt,
+                                c.err, c.spin, c.num_sms, c.st));
+    } else {
+      int nparts = 0;
+      SMOE_TRY(launch_router_simt(T, d, N, true, x, w_r, b_r, c.at<float>(c.L.logits), o, &nparts,
+                                  c.st));
+      SMOE_TRY(launch_tile_rank(T, N, idx, nullptr, nullptr, local_rank, hist, nt, c.err, c.st));
+    }
+    SMOE_TRY(launch_scan(N, nt, hist, c.at<int>(c.L.base), counts, c.st));
+    SMOE_TRY(launch_finalize(T, N, c.C, nt, idx, local_rank, c.at<int>(c.L.base), counts, rank,
+                             drop, slot_token, mtile_start, 0, c.st));
+    SMOE_TRY(launch_gather_rows(S, static_cast<int64_t>(d) * 2, slot_token, x, x_disp, c.st));
+    FfnArgs a{};
+    a.T = T;
+    a.d = d;
+    a.F = F;
+    a.N = N;
+    a.C = c.C;
+    a.x = x;
+    a.x_disp = x_disp;
+    a.slot_token = slot_token;
+    a.counts = counts;
+    a.mtile_start = mtile_start;
+    a.w1 = w1;
+    a.w2 = w2;
+    a.hbuf = hbuf;
+    a.mode2 = kModeY;
+    a.pair1 = (cfg->flags & SWITCH_FLAG_GEMM_PAIRS) != 0;
+    a.gemm1_only = true;
+    a.err = c.err;
+    a.spin = c.spin;
+    a.num_sms = c.num_sms;
+    SMOE_TRY(launch_expert_ffn_bf16(a, c.st));
+  }
 
   // 2. dY = gate * dout per kept slot; dA and the gate-gradient partials;
   // the expert weight gradients
@@ -561,16 +588,15 @@ switch_status_t switch_layer_backward(const switch_config_t* cfg, const void* x,
   SMOE_TRY(launch_bwd_dh(b, c.st));
   SMOE_TRY(launch_bwd_dw(b, c.st));
 
-  // 3. router: dh (in place of the probabilities) and its bf16 planes, the
-  // weight and bias gradients
-  float* dh = probs;
+  // 3. router: dh and its bf16 planes, the weight and bias gradients
+  float* dh = c.at<float>(c.L.dh);
   const int Np = (N + 63) / 64 * 64;
   int* n_drop = c.at<int>(c.L.n_drop);
   int* drop_list = c.at<int>(c.L.drop_list);
   const double ls = static_cast<double>(dloss) * cfg->alpha * N / (static_cast<double>(T) * T);
   SMOE_TRY(cudaMemsetAsync(n_drop, 0, sizeof(int), c.st));
   SMOE_TRY(launch_router_bwd_dh(T, N, Np, c.C, (F + 255) / 256, probs, idx, rank, drop, gate,
-                                b.dgp, counts, static_cast<float>(ls), c.ws + c.L.dhp,
+                                b.dgp, counts, static_cast<float>(ls), dh, c.ws + c.L.dhp,
                                 c.ws + c.L.dhs, dgate ? dgate : c.at<float>(c.L.dgate),
                                 drop_list, n_drop, c.st));
   float* colsum = c.at<float>(c.L.colsum);

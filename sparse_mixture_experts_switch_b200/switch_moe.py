@@ -29,6 +29,7 @@ FLAG_GEMM_1SM = 32
 FLAG_GEMM_PAIRS = 64
 FLAG_ROWS_DISPATCHED = 128
 FLAG_TOP2 = 512
+FLAG_TRAINING = 1024
 
 
 class SwitchConfig(ctypes.Structure):

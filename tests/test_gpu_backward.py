@@ -156,6 +156,64 @@ def test_backward_many_experts(sm):
     check_backward(sm, wl, dloss=2.0)
 
 
+def _forward_all(sm, cfg, dev, ws):
+    x, w_r, b_r, w1, w2 = dev
+    out = torch.empty_like(x)
+    idx = torch.empty(cfg.T, dtype=torch.int32, device="cuda")
+    gate = torch.empty(cfg.T, dtype=torch.float32, device="cuda")
+    counts = torch.empty(cfg.n_experts, dtype=torch.int32, device="cuda")
+    loss = torch.empty(1, dtype=torch.float32, device="cuda")
+    sm.switch_layer_forward(cfg, x, w_r, b_r, w1, w2, out, idx, gate, counts, loss, ws)
+    return [t.cpu() for t in (out, idx, gate, counts, loss)]
+
+
+def _backward_all(sm, cfg, dev, g, ws):
+    x, w_r, b_r, w1, w2 = dev
+    outs = [torch.empty_like(x), torch.empty_like(w_r),
+            torch.empty(cfg.n_experts, device="cuda"), torch.empty_like(w1),
+            torch.empty_like(w2), torch.empty(cfg.T, device="cuda")]
+    dx, dw_r, db_r, dw1, dw2, dgate = outs
+    sm.switch_layer_backward(cfg, x, w_r, b_r, w1, w2, g, 1.0, dx, dw_r, db_r, dw1, dw2, dgate,
+                             ws)
+    st, where, info = sm.switch_get_device_error(ws)
+    assert st == 0, f"device error {st} at {where} ({info})"
+    return [t.cpu() for t in outs]
+
+
+@pytest.mark.parametrize("flags", [0, 8, 1], ids=["default", "gather_in_gemm", "simt_router"])
+def test_backward_saved_forward_state(sm, flags):
+    """SWITCH_FLAG_TRAINING: the forward keeps probabilities, routing, x_disp
+    and H; the backward reads them instead of recomputing.  The forward's
+    outputs and every gradient equal, bit for bit, those of the plain forward
+    and the recomputing backward, and a second backward call repeats them."""
+    wl = SMALL
+    inp = make_inputs(wl)
+    rng = np.random.default_rng(2)
+    bias = (0.05 * rng.standard_normal(wl.n_experts)).astype(np.float32)
+    dev = (dev_float(inp.x), dev_float(inp.w_r), dev_float(bias), dev_float(inp.w1),
+           dev_float(inp.w2))
+    g = dev_float(make_dout(wl))
+    mk = lambda f: sm.config(wl.T, wl.d_model, wl.d_ff, wl.n_experts,  # noqa: E731
+                             wl.capacity_factor, alpha=wl.alpha, flags=f)
+    cfg0, cfg1 = mk(flags), mk(flags | sm.FLAG_TRAINING)
+    ws0 = sm.backward_workspace(cfg0)
+    f0 = _forward_all(sm, cfg0, dev, ws0)
+    b0 = _backward_all(sm, cfg0, dev, g, ws0)
+    ws1 = sm.backward_workspace(cfg1)
+    f1 = _forward_all(sm, cfg1, dev, ws1)
+    b1 = _backward_all(sm, cfg1, dev, g, ws1)
+    b2 = _backward_all(sm, cfg1, dev, g, ws1)
+    for a, b in zip(f0, f1):
+        assert torch.equal(a, b)
+    for a, b, c in zip(b0, b1, b2):
+        assert torch.equal(a, b) and torch.equal(b, c)
+    # the forward's state needs the backward's workspace size
+    small = sm.workspace(cfg1)
+    with pytest.raises(sm.SwitchError) as ei:
+        _forward_all(sm, cfg1, dev, small)
+    assert ei.value.status == 3
+
+
 def test_backward_deterministic(sm):
     inp = make_inputs(SMALL)
     dout = make_dout(SMALL)
