@@ -44,9 +44,9 @@ L2_FLUSH_BYTES = 256 << 20
 GEMM_SOURCES = ("common.cuh", "gemm_common.cuh", "gemm_pair.cuh", "expert_ffn.cu",
                 "expert_ffn_pair.cu")
 GEMM_TRAFFIC = {"workload": "base",
-                "sources_sha256": "0ab85744d10d1b7781851740503a59e5be0ac68493ab955484fd233810972f4a",
-                # GEMM1 715.7 MB read + 373.0 MB written; GEMM2 1239.5 + 93.7 MB
-                "bytes": 715.732480e6 + 372.987392e6 + 1239.501e6 + 93.651456e6}
+                "sources_sha256": "97b31444528b771321d3264df6e72bf3e7d38276351d33b290eca56557619e16",
+                # GEMM1 715.9 MB read + 370.8 MB written; GEMM2 1231.7 + 89.1 MB
+                "bytes": 715.932160e6 + 370.764288e6 + 1231.664896e6 + 89.147392e6}
 
 
 def gemm_sources_sha256():
