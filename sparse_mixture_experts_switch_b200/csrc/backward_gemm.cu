@@ -135,15 +135,7 @@ __device__ __forceinline__ void epi_store(const BwdParams& p, const CUtensorMap*
   const int cols = p.n_out - t.n * kBN < kBN ? p.n_out - t.n * kBN : kBN;
   const int64_t ooff = (static_cast<int64_t>(t.e) * p.M_out + r) * p.n_out + t.n * kBN;
   __nv_bfloat16* orow = p.out + ooff;
-  for (int c = 0; c < cols / 32; ++c) {
-    uint32_t v[32];
-    if (t.kblocks > 0) {
-      tmem_ld32_issue(taddr + static_cast<uint32_t>(c * 32), v);
-      tmem_ld_wait(v);
-    } else {
-#pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = 0u;
-    }
+  auto process = [&](int c, const uint32_t* v) {
     if (bulk) {
       uint32_t pk[16];
 #pragma unroll
@@ -166,6 +158,25 @@ __device__ __forceinline__ void epi_store(const BwdParams& p, const CUtensorMap*
         dst[k] = o;
       }
     }
+  };
+  const int nch = cols / 32;                      // even: n_out is a multiple of 64
+  uint32_t ra[32], rb[32];
+  if (t.kblocks == 0) {                           // no tokens: the accumulator was never written
+#pragma unroll
+    for (int j = 0; j < 32; ++j) ra[j] = 0u;
+    for (int c = 0; c < nch; ++c) process(c, ra);
+    return;
+  }
+  // chunk c + 1's TMEM load is in flight while chunk c is stored
+  tmem_ld32_issue(taddr, ra);
+#pragma unroll 1
+  for (int c = 0; c < nch; c += 2) {
+    tmem_ld_wait(ra);
+    tmem_ld32_issue(taddr + static_cast<uint32_t>((c + 1) * 32), rb);
+    process(c, ra);
+    tmem_ld_wait(rb);
+    if (c + 2 < nch) tmem_ld32_issue(taddr + static_cast<uint32_t>((c + 2) * 32), ra);
+    process(c + 1, rb);
   }
 }
 
@@ -195,14 +206,17 @@ __device__ __forceinline__ void epi_dh(const BwdParams& p, const CUtensorMap* tm
   const int cols = p.n_out - t.n * kBN < kBN ? p.n_out - t.n * kBN : kBN;
   const int64_t off = s * p.n_out + t.n * kBN;
   float dot = 0.f;
-  for (int c = 0; c < cols / 32; ++c) {
-    uint32_t v[32];
-    tmem_ld32_issue(taddr + static_cast<uint32_t>(c * 32), v);
-    tmem_ld_wait(v);
-    if (bulk) {
-      uint4 hv[4];
+  // chunk c + 1's TMEM load and H loads are in flight while chunk c is
+  // processed (nch is even: n_out is a multiple of 64)
+  const int nch = cols / 32;
+  auto load_h = [&](int c, uint4* hv) {
+    if (in_cap) {
 #pragma unroll
       for (int k = 0; k < 4; ++k) hv[k] = ld_u4(p.h + off + c * 32 + 8 * k);
+    }
+  };
+  auto process = [&](int c, const uint32_t* v, const uint4* hv) {
+    if (bulk) {
       uint32_t pk[16];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
@@ -216,9 +230,6 @@ __device__ __forceinline__ void epi_dh(const BwdParams& p, const CUtensorMap* tm
       }
       store_box(tmap_out, stg, nbox, pk, t.n * kBN + c * 32, box_row, lane);
     } else if (in_cap) {
-      uint4 hv[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) hv[k] = ld_u4(p.h + off + c * 32 + 8 * k);
       uint4* dst = reinterpret_cast<uint4*>(p.out + off + c * 32);
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
@@ -238,6 +249,23 @@ __device__ __forceinline__ void epi_dh(const BwdParams& p, const CUtensorMap* tm
         dst[k] = o;
       }
     }
+  };
+  uint32_t ra[32], rb[32];
+  uint4 ha[4], hb[4];
+  tmem_ld32_issue(taddr, ra);
+  load_h(0, ha);
+#pragma unroll 1
+  for (int c = 0; c < nch; c += 2) {
+    tmem_ld_wait(ra);
+    tmem_ld32_issue(taddr + static_cast<uint32_t>((c + 1) * 32), rb);
+    load_h(c + 1, hb);
+    process(c, ra, ha);
+    tmem_ld_wait(rb);
+    if (c + 2 < nch) {
+      tmem_ld32_issue(taddr + static_cast<uint32_t>((c + 2) * 32), ra);
+      load_h(c + 2, ha);
+    }
+    process(c + 1, rb, hb);
   }
   if (kept) p.dgp[s * p.ntiles_n + t.n] = dot;
 }

@@ -18,8 +18,9 @@ give errors of the order of the RMS itself.  The router's fp32 gradients
 inherit bf16-level error through the gate gradient.  Routing flips (oracle
 margin < 1e-6) are counted as in the forward tests.
 
-At full size (Base) the oracle computes sampled tokens' dx and gate
-gradients, and sampled experts' weight gradients, one by one; dw_r and db_r
+At full size (Base, the Zipf-skewed workload with 60% drops, Large and XXL)
+the oracle computes sampled tokens' dx and gate gradients, and sampled
+experts' weight gradients, one by one; dw_r and db_r
 are checked there through the softmax shift invariance (their sums over
 experts vanish), which holds at any size.
 """
@@ -28,7 +29,7 @@ import pytest
 import torch
 
 import oracle.switch_oracle as orc
-from switch_inputs import Workload, BASE, make_inputs, make_dout, as_f64
+from switch_inputs import Workload, WORKLOADS, make_inputs, make_dout, as_f64
 from gpu_util import dev_float, host_f64, check_routing
 
 pytestmark = pytest.mark.gpu
@@ -37,11 +38,32 @@ GRAD_MAX_TOL = 4e-2
 GRAD_RMS_TOL = 5e-3
 
 
-def grad_ok(got, want, name):
+# ReLU decisions near the kink: the GPU takes relu'(A) from its fp32
+# accumulation of A, the oracle from float64; where |A| is below the fp32
+# accumulation error both choices are correct.  A hidden unit counts as
+# ambiguous when |A| < RELU_TAU * sum_k |x_k w_k| (about 17 units in the last
+# place of the sum's L1 mass, an order of magnitude above the expected
+# accumulation error); its whole contribution dH * x (to dW1) or dH * W1 (to
+# dx) is allowed on top of the tolerance.  The RMS bound is not relaxed.
+RELU_TAU = 1e-6
+
+
+def relu_ambiguity(x_rows, w1_e, w2_e, g_rows, dout_rows):
+    """Per-element allowances for dW1_e [F, d] and for the rows' dx [n, d]."""
+    X, W1, W2 = as_f64(x_rows), as_f64(w1_e), as_f64(w2_e)
+    A = X @ W1.T
+    amb = np.abs(A) < RELU_TAU * (np.abs(X) @ np.abs(W1).T)
+    dH = np.asarray(g_rows, np.float64)[:, None] * (as_f64(dout_rows) @ W2)
+    contrib = np.abs(dH) * amb
+    return contrib.T @ np.abs(X), contrib @ np.abs(W1), int(amb.sum())
+
+
+def grad_ok(got, want, name, allow=None):
     want = np.asarray(want, np.float64)
     err = np.asarray(got, np.float64) - want
     rms = max(float(np.sqrt(np.mean(want * want))), 1e-30)
-    mx = float(np.max(np.abs(err))) / rms
+    excess = np.abs(err) if allow is None else np.maximum(np.abs(err) - allow, 0.0)
+    mx = float(np.max(excess)) / rms
     rm = float(np.sqrt(np.mean(err * err))) / rms
     assert mx <= GRAD_MAX_TOL and rm <= GRAD_RMS_TOL, \
         f"{name}: max err / rms = {mx:.3g}, rms err / rms = {rm:.3g}"
@@ -63,7 +85,8 @@ def _forward_idx(sm, cfg, x, w_r, b_r, w1, w2, ws):
     return idx.cpu().numpy().astype(np.int64)
 
 
-def run_backward(sm, wl, inp, dout, dloss=1.0, flags=0, b_r_override=None, reuse_ws=None):
+def run_backward(sm, wl, inp, dout, dloss=1.0, flags=0, b_r_override=None, reuse_ws=None,
+                 to_host=True):
     cfg = sm.config(wl.T, wl.d_model, wl.d_ff, wl.n_experts, wl.capacity_factor,
                     dtype=wl.dtype, alpha=wl.alpha, flags=flags)
     ws = sm.backward_workspace(cfg) if reuse_ws is None else reuse_ws
@@ -82,8 +105,10 @@ def run_backward(sm, wl, inp, dout, dloss=1.0, flags=0, b_r_override=None, reuse
                              dgate, ws)
     st, where, info = sm.switch_get_device_error(ws)
     assert st == 0, f"device error {st} at {where} ({info})"
-    return idx, {"dx": host_f64(dx), "dw_r": host_f64(dw_r), "db_r": host_f64(db_r),
-                 "dw1": host_f64(dw1), "dw2": host_f64(dw2), "dgate": host_f64(dgate)}
+    res = {"dx": dx, "dw_r": dw_r, "db_r": db_r, "dw1": dw1, "dw2": dw2, "dgate": dgate}
+    if to_host:
+        res = {k: host_f64(v) for k, v in res.items()}
+    return idx, res
 
 
 def check_backward(sm, wl, dloss=1.0, flags=0, b_r_override=None):
@@ -248,11 +273,12 @@ def test_backward_workspace_too_small(sm):
 
 # ----------------------------------------------------------- full size
 
-def test_backward_fullsize_base_sampled(sm):
-    wl = BASE
+@pytest.mark.parametrize("name", ["base", "zipf_cf1.0", "large", "xxl"])
+def test_backward_fullsize_sampled(sm, name):
+    wl = WORKLOADS[name]
     inp = make_inputs(wl)
     dout = make_dout(wl)
-    idx, got = run_backward(sm, wl, inp, dout)
+    idx, dev = run_backward(sm, wl, inp, dout, to_host=False)    # weights' gradients stay on the GPU
     T, N = wl.T, wl.n_experts
     r = orc.router(inp.x, inp.w_r, inp.b_r)
     check_routing(idx, r)
@@ -261,35 +287,50 @@ def test_backward_fullsize_base_sampled(sm):
     gate = r["probs"][np.arange(T), idx]
     f_scale = wl.alpha * N * dsp["counts"] / T / T
     rng = np.random.default_rng(3)
+    dropped = np.nonzero(dsp["drop"])[0]
     toks = np.unique(np.concatenate([[0, T - 1], rng.choice(T, 48, replace=False),
-                                     rng.choice(np.nonzero(dsp["drop"])[0], 8, replace=False)]))
+                                     rng.choice(dropped, min(8, dropped.size), replace=False)]))
     want_dx = np.zeros((toks.size, wl.d_model))
     want_dg = np.zeros(toks.size)
+    dxe = np.zeros((toks.size, wl.d_model))
+    allow_dx = np.zeros((toks.size, wl.d_model))
+    kept_j = np.nonzero(~dsp["drop"][toks])[0]
+    for e in np.unique(idx[toks[kept_j]]):          # one oracle call per expert
+        js = kept_j[idx[toks[kept_j]] == e]
+        ts = toks[js]
+        dg_a, dxe_a, _, _ = orc.expert_backward(inp.x[ts], inp.w1[e], inp.w2[e], gate[ts],
+                                                dout[ts])
+        want_dg[js] = dg_a
+        dxe[js] = dxe_a
+        allow_dx[js] = relu_ambiguity(inp.x[ts], inp.w1[e], inp.w2[e], gate[ts], dout[ts])[1]
+    w_r64 = inp.w_r.astype(np.float64)
     for j, t in enumerate(toks):
-        e = int(idx[t])
-        dg, dxe = 0.0, 0.0
-        if not dsp["drop"][t]:
-            dg_a, dxe_a, _, _ = orc.expert_backward(inp.x[t:t + 1], inp.w1[e], inp.w2[e],
-                                                    gate[t:t + 1], dout[t:t + 1])
-            dg, dxe = dg_a[0], dxe_a[0]
         p = r["probs"][t]
         dp = f_scale.copy()
         if not dsp["drop"][t]:
-            dp[e] += dg
+            dp[int(idx[t])] += want_dg[j]
         dh = p * (dp - np.sum(p * dp))
-        want_dx[j] = as_f64(dout[t]) + dxe + dh @ inp.w_r.astype(np.float64)
-        want_dg[j] = dg
-    grad_ok(got["dx"][toks], want_dx, "dx (sampled)")
-    grad_ok(got["dgate"][toks], want_dg, "dgate (sampled)")
+        want_dx[j] = as_f64(dout[t]) + dxe[j] + dh @ w_r64
+    tsel = torch.from_numpy(toks).cuda()
+    grad_ok(host_f64(dev["dx"][tsel]), want_dx, "dx (sampled)", allow_dx)
+    grad_ok(host_f64(dev["dgate"][tsel]), want_dg, "dgate (sampled)")
     for e in (0, N // 2, N - 1):
         n = min(int(dsp["counts"][e]), C)
+        g1, g2 = host_f64(dev["dw1"][e]), host_f64(dev["dw2"][e])
+        if n == 0:
+            assert np.all(g1 == 0) and np.all(g2 == 0)
+            continue
         rows = dsp["slot_token"][e * C: e * C + n]
         _, _, dw1_e, dw2_e = orc.expert_backward(inp.x[rows], inp.w1[e], inp.w2[e], gate[rows],
                                                  dout[rows])
-        grad_ok(got["dw1"][e], dw1_e, f"dw1[{e}]")
-        grad_ok(got["dw2"][e], dw2_e, f"dw2[{e}]")
+        allow_w1, _, n_amb = relu_ambiguity(inp.x[rows], inp.w1[e], inp.w2[e], gate[rows],
+                                            dout[rows])
+        print(name, f"expert {e}: {n_amb} hidden units within the ReLU decision margin")
+        grad_ok(g1, dw1_e, f"dw1[{e}]", allow_w1)
+        grad_ok(g2, dw2_e, f"dw2[{e}]")
     # softmax shift invariance: sum over experts of dW_r rows and of db_r vanish
-    scale = np.abs(got["dw_r"]).max()
-    assert np.abs(got["dw_r"].sum(axis=0)).max() <= 1e-3 * scale
-    assert np.isfinite(got["dx"]).all() and np.isfinite(got["dw1"]).all()
-    assert np.isfinite(got["dw2"]).all()
+    dw_r = host_f64(dev["dw_r"])
+    scale = np.abs(dw_r).max()
+    assert np.abs(dw_r.sum(axis=0)).max() <= 1e-3 * scale
+    for k in ("dx", "dw1", "dw2"):
+        assert bool(torch.isfinite(dev[k]).all()), k
