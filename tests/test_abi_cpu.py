@@ -74,6 +74,26 @@ def test_workspace_validation(sm):
     assert sm.switch_workspace_size(sm.config(512, 64, 256, 4, 1.25, dtype="f32")) > 0
 
 
+def test_backward_workspace_extends_the_forward(sm):
+    """The backward's workspace holds the forward's regions and its own
+    after them: at least the forward size plus dA [N*C, d_ff] bf16, dh [T, N]
+    fp32 and the kept probabilities [T, N] fp32; invalid configs are refused
+    the same way."""
+    for T, d, F, N, cf in ((65536, 768, 3072, 128, 1.25), (1000, 192, 320, 6, 6.0),
+                           (2500, 128, 192, 100, 1.0), (1, 64, 64, 1, 1.0),
+                           (16384, 4096, 10240, 64, 1.25)):
+        cfg = sm.config(T, d, F, N, cf)
+        fwd = sm.switch_workspace_size(cfg)
+        bwd = sm.switch_backward_workspace_size(cfg)
+        C = sm.switch_capacity(T, N, cf)
+        assert bwd >= fwd + N * C * F * 2 + 2 * T * N * 4, (T, d, F, N)
+        top2 = sm.config(T, d, F, max(N, 2), cf, flags=sm.FLAG_TOP2)
+        assert sm.switch_backward_workspace_size(top2) >= sm.switch_workspace_size(top2)
+    with pytest.raises(sm.SwitchError) as ei:
+        sm.switch_backward_workspace_size(sm.config(1024, 100, 3072, 128, 1.25))
+    assert ei.value.status == 2
+
+
 def test_status_strings(sm):
     for s in range(7):
         assert sm.switch_status_string(s)

@@ -174,6 +174,18 @@ def test_backward_no_drops_ragged(sm):
     assert not want["drop"].any()
 
 
+def test_backward_single_expert_and_tiny_batch(sm):
+    """N = 1 (p = 1: the router's gradients vanish, the layer is a dense
+    residual FFN) and a batch smaller than one tile."""
+    for wl in (Workload("bwd_dense", T=700, d_model=192, d_ff=320, n_experts=1,
+                        capacity_factor=1.0, dtype="bf16", seed=31),
+               Workload("bwd_tiny", T=37, d_model=64, d_ff=128, n_experts=4,
+                        capacity_factor=1.0, dtype="bf16", seed=37)):
+        got, want, _ = check_backward(sm, wl)
+        if wl.n_experts == 1:
+            assert np.all(got["dw_r"] == 0) and not want["drop"].any()
+
+
 def test_backward_many_experts(sm):
     """N = 100: the router's bf16 planes are padded to 128 columns."""
     wl = Workload("bwd_n100", T=2500, d_model=128, d_ff=192, n_experts=100,
