@@ -43,9 +43,9 @@ softmax over all experts, not renormalised; the 2T assignments take slots
 first choices first, each route in batch order; ``f_i`` still counts first
 choices.
 
-The backward pass (``layer_backward``) is the chain rule through those
-stages for J = sum(dout * out) + dloss * loss, routing decisions held fixed
-(they are piecewise constant).
+The backward pass (``layer_backward``, ``layer_backward_top2``) is the chain
+rule through those stages for J = sum(dout * out) + dloss * loss, routing
+decisions held fixed (they are piecewise constant).
 
 Arithmetic is float64 throughout (expert matmuls included); floating-point
 inputs are the exact values of the bf16 / fp32 bit patterns the GPU reads.
@@ -436,3 +436,68 @@ def layer_backward(x, w_r, b_r, w1, w2, capacity_factor, dout, dloss=1.0,
             "dgate": dgate, "dh": dh, "idx": idx, "gate": gate, "drop": dsp["drop"],
             "counts": dsp["counts"], "slot_token": dsp["slot_token"], "C": C,
             "probs": r["probs"]}
+
+
+def layer_backward_top2(x, w_r, b_r, w1, w2, capacity_factor, dout, dloss=1.0,
+                        alpha=0.01, residual=True, idx2=None):
+    """Gradients of J = sum(dout * out) + dloss * loss for the top-2 layer.
+
+    Same chain rule as ``layer_backward``, with both kept routes of a token:
+    out = x + sum_r p_{idx_r} E_{idx_r}(x) [P1 §"Switch Routing": the gates
+    are the full-softmax probabilities, not renormalised], so each kept route
+    contributes its own expert gradients and a gate gradient
+    dgate_r = dout . E_{idx_r}(x) at p_{idx_r}; the loss's f_i counts first
+    choices and is held fixed, P_i is differentiated through every p_i.
+    ``idx2`` ([2, T], optional) imposes the choices.  Returns the dict of
+    ``layer_backward`` with ``dgate`` of shape [2, T] and ``drop2``.
+    """
+    T, d = x.shape
+    N = w_r.shape[0]
+    C = capacity(2 * T, N, capacity_factor)
+    r = router_top2(x, w_r, b_r)
+    idx2 = r["idx2"] if idx2 is None else np.asarray(idx2, dtype=np.int64)
+    p = r["probs"]
+    gate2 = np.stack([p[np.arange(T), idx2[0]], p[np.arange(T), idx2[1]]])
+    dsp = dispatch_top2(idx2, N, C)
+    G = as_f64(dout)
+    dx = G.copy() if residual else np.zeros((T, d))
+    dgate = np.zeros((2, T))
+    dw1 = np.zeros(np.shape(w1))
+    dw2 = np.zeros(np.shape(w2))
+    for e in range(N):
+        n = min(int(dsp["counts"][e]), C)
+        if n == 0:
+            continue
+        tok = dsp["slot_token"][e * C: e * C + n]
+        # the route of each slot: the token's first choice if it is e, else its second
+        route = np.where(idx2[0, tok] == e, 0, 1)
+        g = gate2[route, tok]
+        dg, dxe, dw1[e], dw2[e] = expert_backward(x[tok], w1[e], w2[e], g, dout[tok])
+        dgate[route, tok] = dg
+        np.add.at(dx, tok, dxe)
+    counts1 = np.bincount(idx2[0], minlength=N)
+    dxr, dw_r, db_r, dh = router_backward_top2(x, w_r, p, idx2, dsp["drop"], dgate, counts1,
+                                               alpha, dloss)
+    dx += dxr
+    return {"dx": dx, "dw_r": dw_r, "db_r": db_r, "dw1": dw1, "dw2": dw2, "dgate": dgate,
+            "dh": dh, "idx2": idx2, "gate2": gate2, "drop2": dsp["drop"],
+            "counts": dsp["counts"], "C": C}
+
+
+def router_backward_top2(x, w_r, probs, idx2, drop2, dgate2, counts1, alpha, dloss):
+    """Router backward for top-2 routing: as ``router_backward`` with
+    dJ/dp_{t,i} = sum over the token's kept routes r with idx_r = i of
+    dgate_r[t], plus dloss . alpha . N . f_i / T where f_i counts first
+    choices (``counts1``) [P1 §"The Load-Balancing Loss", f through the
+    argmax].  Returns ``(dx_router, dW_r, db, dh)``."""
+    X = as_f64(x)
+    p = np.asarray(probs, dtype=np.float64)
+    T, N = p.shape
+    f = np.asarray(counts1, dtype=np.float64) / T
+    dp = np.tile(dloss * alpha * N * f / T, (T, 1))
+    for rr in range(2):
+        rows = np.nonzero(~np.asarray(drop2[rr], dtype=bool))[0]
+        dp[rows, np.asarray(idx2)[rr, rows]] += np.asarray(dgate2)[rr, rows]
+    dh = p * (dp - np.sum(p * dp, axis=1, keepdims=True))
+    Wr = np.asarray(w_r, dtype=np.float64)
+    return dh @ Wr, dh.T @ X, dh.sum(axis=0), dh

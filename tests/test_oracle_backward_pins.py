@@ -13,7 +13,11 @@ Each check ties the gradient to something other than its own formulas:
 * a dropped token with no loss gradient: its block output is x alone
   (section "Expert Capacity and the Capacity Factor"), so dx = dout exactly;
 * one expert with room for every token: p = 1, the layer is x + FFN(x), and
-  the weight gradients equal torch autograd's for a dense ReLU MLP.
+  the weight gradients equal torch autograd's for a dense ReLU MLP;
+* top-2 (section "Switch Routing: From Top-k to k = 1", the top-k set and its
+  gates): finite differences of the top-2 forward oracle, and with two
+  experts and no drops the gates sum to 1, so the logits' gradients are
+  opposite for every token.
 
 The last test plants plausible mistakes in the backward (on the CPU) and
 checks that some pin catches each one.
@@ -136,9 +140,59 @@ def pin_bwd_single_expert_dense(O):
     np.testing.assert_allclose(got["dx"], X.grad.numpy(), rtol=1e-12, atol=1e-12)
 
 
+def _case_top2(seed, T=12, d=4, F=6, N=4, cf=0.5):
+    """Like _case for top-2: first/second and second/third logit margins and
+    ReLU pre-activations away from their switching points, drops present."""
+    for s_ in range(seed, seed + 2000):
+        rng = np.random.default_rng(s_)
+        x = rng.standard_normal((T, d))
+        w_r = rng.standard_normal((N, d))
+        b_r = 0.3 * rng.standard_normal(N)
+        w1 = rng.standard_normal((N, F, d)) / np.sqrt(d)
+        w2 = rng.standard_normal((N, d, F)) / np.sqrt(F)
+        dout = rng.standard_normal((T, d))
+        hs = np.sort(x @ w_r.T + b_r, axis=1)
+        if np.min(hs[:, -1] - hs[:, -2]) < 1e-2 or np.min(hs[:, -2] - hs[:, -3]) < 1e-2:
+            continue
+        if np.min(np.abs(np.einsum("td,nfd->tnf", x, w1))) < 1e-3:
+            continue
+        r = orc.router_top2(x, w_r, b_r)
+        dsp = orc.dispatch_top2(r["idx2"], N, orc.capacity(2 * T, N, cf))
+        if not dsp["drop"][0].any() and not dsp["drop"][1].any():
+            continue
+        return x, w_r, b_r, w1, w2, dout
+    raise RuntimeError("no smooth top-2 case found")
+
+
+def pin_bwd_top2_finite_differences(O):
+    x, w_r, b_r, w1, w2, dout = _case_top2(7)
+    cf = 0.5
+    got = O.layer_backward_top2(x, w_r, b_r, w1, w2, cf, dout, dloss=2.0, alpha=ALPHA)
+
+    def fun():
+        f = O.layer_forward_top2(x, w_r, b_r, w1, w2, cf, alpha=ALPHA)
+        return float(np.sum(dout * f["out"]) + 2.0 * f["loss"])
+
+    for name, arr in (("dx", x), ("dw_r", w_r), ("db_r", b_r), ("dw1", w1), ("dw2", w2)):
+        np.testing.assert_allclose(got[name], _fd_grad(fun, arr), rtol=1e-6, atol=1e-8,
+                                   err_msg=name)
+    assert got["drop2"][1].any()           # some second routes dropped
+
+
+def pin_bwd_top2_two_experts_gates_sum(O):
+    """N = 2, room for every assignment: both experts take every token and the
+    two gates sum to 1, so the gate gradients enter only through their
+    difference (dh_0 = -dh_1 for every token)."""
+    x, w_r, b_r, w1, w2, dout = _case(61, T=8, N=2)
+    got = O.layer_backward_top2(x, w_r, b_r, w1, w2, 4.0, dout, dloss=0.0, alpha=ALPHA)
+    assert not got["drop2"].any()
+    np.testing.assert_allclose(got["dh"][:, 0], -got["dh"][:, 1], rtol=0, atol=1e-14)
+
+
 PINS = [pin_bwd_finite_differences, pin_bwd_finite_differences_no_residual,
         pin_bwd_loss_only, pin_bwd_softmax_shift, pin_bwd_dropped_passthrough,
-        pin_bwd_single_expert_dense]
+        pin_bwd_single_expert_dense, pin_bwd_top2_finite_differences,
+        pin_bwd_top2_two_experts_gates_sum]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda p: p.__name__)
@@ -209,7 +263,25 @@ def _mut_dropped_get_gate_grad(real):
     return f
 
 
+def _mut_top2_first_route_only(real):
+    def f(x, w_r, probs, idx2, drop2, dgate2, counts1, alpha, dloss):
+        d2 = np.asarray(dgate2, np.float64).copy()
+        d2[1] = 0.0                                    # second gate's gradient lost
+        return real(x, w_r, probs, idx2, drop2, d2, counts1, alpha, dloss)
+    return f
+
+
+def _mut_top2_f_over_both_routes(real):
+    def f(x, w_r, probs, idx2, drop2, dgate2, counts1, alpha, dloss):
+        N = np.shape(probs)[1]
+        both = np.bincount(np.asarray(idx2).reshape(-1), minlength=N)
+        return real(x, w_r, probs, idx2, drop2, dgate2, both, alpha, dloss)
+    return f
+
+
 MUTANTS = {
+    "top2_second_gate_gradient_lost": ("router_backward_top2", _mut_top2_first_route_only),
+    "top2_loss_f_over_both_routes": ("router_backward_top2", _mut_top2_f_over_both_routes),
     "relu_mask_forgotten": ("expert_backward", _mut_no_relu_mask),
     "gate_not_scaling_dY": ("expert_backward", _mut_no_gate_scale),
     "dgate_halved": ("expert_backward", _mut_dgate_of_hidden),
