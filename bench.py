@@ -74,6 +74,9 @@ def parse_args():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="base", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workloads", default=None,
+                    help="comma-separated extra workloads timed after the headline one "
+                         "('all' = every bf16 workload; default: all at N=1, none at N>1)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="budget of the oracle sample timed for cpu_baseline")
     return ap.parse_args()
@@ -179,53 +182,98 @@ def run_reference(args):
 # -------------------------------------------------------------- clocks
 
 class ClockSampler:
+    """SM clock, power and clock-event reasons sampled while the GPU works.
+
+    Reads NVML directly every few milliseconds (read-only queries), so that a
+    timed region of a few tens of milliseconds still gets several samples;
+    falls back to `nvidia-smi -lms 100` when NVML is not importable."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
-    def __init__(self, gpu_id):
+    def __init__(self, gpu_id, uuid=None, period_s=0.002):
         self.gpu_id = gpu_id
-        self.rows = []
+        self.uuid = uuid
+        self.period_s = period_s
+        self.rows = []            # (time, sm_mhz, max_mhz, power_w, reasons)
         self.proc = None
+        self.stop_evt = threading.Event()
+        self.thread = None
+        self.source = None
 
     def start(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = (pynvml.nvmlDeviceGetHandleByUUID(self.uuid) if self.uuid
+                 else pynvml.nvmlDeviceGetHandleByIndex(int(self.gpu_id)))
+            self.source = "nvml"
+            self.thread = threading.Thread(target=self._nvml, args=(pynvml, h), daemon=True)
+            self.thread.start()
+            return
+        except Exception:
+            pass
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
                  "-lms", "100", "-i", str(self.gpu_id)],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.source = "nvidia-smi"
+            self.thread = threading.Thread(target=self._smi, daemon=True)
             self.thread.start()
         except Exception:
             self.proc = None
 
-    def _read(self):
+    def _nvml(self, pynvml, h):
+        bits = (pynvml.nvmlClocksEventReasonHwSlowdown,
+                pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+                pynvml.nvmlClocksEventReasonSwThermalSlowdown,
+                pynvml.nvmlClocksEventReasonSwPowerCap)
+        mx = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+        while not self.stop_evt.is_set():
+            try:
+                sm = float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM))
+                pw = pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0
+                rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                names = [n for n, bit in zip(self.REASONS, bits) if rs & bit]
+                self.rows.append((time.time(), sm, mx, pw, names))
+            except Exception:
+                pass
+            time.sleep(self.period_s)
+
+    def _smi(self):
+        names = self.REASONS
         for ln in self.proc.stdout:
-            self.rows.append((time.time(), [c.strip() for c in ln.split(",")]))
+            r = [c.strip() for c in ln.split(",")]
+            try:
+                self.rows.append((time.time(), float(r[1]), float(r[2]), float(r[3]),
+                                  [n for n, v in zip(names, r[5:9]) if v == "Active"]))
+            except (ValueError, IndexError):
+                pass
 
     def stop(self):
+        self.stop_evt.set()
         if self.proc is not None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
 
     def summary(self, t0, t1):
-        rows = [r for (t, r) in self.rows if t0 - 0.25 <= t <= t1 + 0.25]
-        if not rows:   # timed region shorter than the sampling period: nearest samples
-            rows = [r for (t, r) in sorted(self.rows, key=lambda tr: abs(tr[0] - (t0 + t1) / 2))[:3]]
+        rows = [r for r in self.rows if t0 <= r[0] <= t1]
+        if not rows:   # region shorter than the sampling period: nearest samples
+            rows = sorted(self.rows, key=lambda r: abs(r[0] - (t0 + t1) / 2))[:3]
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v == "Active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
-                "samples": len(rows),
-                "power_w_max": max((float(r[3]) for r in rows if r[3].replace(".", "").isdigit()),
-                                   default=None)}
+        return {"sm_mhz": statistics.median(r[1] for r in rows),
+                "sm_max_mhz": max(r[2] for r in rows),
+                "reasons": sorted({n for r in rows for n in r[4]}),
+                "samples": len(rows), "source": self.source,
+                "power_w_max": max(r[3] for r in rows)}
 
 
 # ------------------------------------------------------------- GPU arm
@@ -287,8 +335,12 @@ def main():
         if world > 1:
             dist.barrier()
 
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        uuid = None
     clocks = ClockSampler(local if not os.environ.get("CUDA_VISIBLE_DEVICES")
-                          else os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local])
+                          else os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local], uuid)
     clocks.start()
     for _ in range(max(3, args.warmup)):
         step()
@@ -345,7 +397,10 @@ def main():
     barrier()
     e2e_value = job_throughput(T, args.steps, world,
                                max_over_ranks(e0.elapsed_time(e1), dev, world))
+    e2e_bytes = (x_host.numel() * x_host.element_size(),
+                 out_host.numel() * out_host.element_size() + loss_host.numel() * 4)
     clocks.stop()
+    del x_host, out_host, step_graph
 
     # --------------------------------------- per-kernel roofline (rank 0)
     line = None
@@ -363,10 +418,15 @@ def main():
                               f"{wl.n_experts}, their time scaled by {wl.n_experts}/{n_exp}"),
                    "host_cpus": os.cpu_count()}
         ffn = kern["expert_ffn"]
-        flops_layer = 2.0 * T * d * N + 4.0 * T_kept * d * F
-        bytes_layer = 3 * T * d * 2 + 2 * N * d * F * 2 + T * d * 2
-        t_layer_min = max(flops_layer / (pk["bf16_tflops"] * 1e12),
-                          bytes_layer / (pk["hbm_gbs"] * 1e9))
+        bounds = layer_bounds(wl, T_kept, pk)
+        t_layer_min = bounds["t_min_us"] * 1e-6
+        extra = extra_workloads(args, world, wl.name)
+        table = {wl.name: workload_row(wl, C, ms_per_step, ffn["us"] * 1e-6, T_kept, pk)}
+        del x, w1, w2, ws, out
+        torch.cuda.empty_cache()
+        for name in extra:
+            table[name] = time_workload(sm, WORKLOADS[name], dev, stream, flush, pk,
+                                        max(5, min(args.steps, 20)))
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
@@ -385,15 +445,15 @@ def main():
                          "peak_kind": f"{pk_kind} bf16 burst",
                          "traffic": gemm_traffic(args.workload),
                          "useful_flops": 4.0 * T_kept * d * F},
-            "layer_roofline": {"t_min_us": t_layer_min * 1e6,
-                               "tokens_per_s": T / t_layer_min,
-                               "frac": (T / t_layer_min and value / world / (T / t_layer_min))},
+            "layer_roofline": {**bounds, "tokens_per_s": T / t_layer_min,
+                               "frac": value / world / (T / t_layer_min)},
             "kernels": kern,
+            "workloads": table,
             "routing": {"T_kept": T_kept, "drop_rate": 1.0 - T_kept / T,
                         "padding": 1.0 - T_kept / (N * C)},
             "cpu_baseline": cpu,
-            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": x.numel() * x.element_size(),
-                    "d2h_bytes_per_step": out.numel() * out.element_size() + 4},
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": e2e_bytes[0],
+                    "d2h_bytes_per_step": e2e_bytes[1]},
             "clocks": clocks.summary(t_wall0, t_wall1),
             "gpu_launches": launches_per_step(cfg, wl) * args.steps,
         }
@@ -402,6 +462,119 @@ def main():
         dist.destroy_process_group()
     if line is not None:
         print(json.dumps(line), flush=True)
+
+
+def layer_bounds(wl, T_kept, pk):
+    """Roofline of the whole layer: useful FLOPs (router + kept tokens' expert
+    GEMMs) at the bf16 burst peak against the layer's minimum bytes (x read
+    three times -- router, row copy, residual -- every expert weight once, out
+    written once) at the HBM peak."""
+    T, d, F, N = wl.T, wl.d_model, wl.d_ff, wl.n_experts
+    es = 2 if wl.dtype == "bf16" else 4
+    flops = 2.0 * T * d * N + 4.0 * T_kept * d * F
+    nbytes = 3 * T * d * es + 2 * N * d * F * es + T * d * es
+    t_c = flops / (pk["bf16_tflops"] * 1e12)
+    t_m = nbytes / (pk["hbm_gbs"] * 1e9)
+    return {"useful_flops": flops, "min_bytes": nbytes, "t_compute_us": t_c * 1e6,
+            "t_mem_us": t_m * 1e6, "bound": "tensor" if t_c >= t_m else "hbm",
+            "t_min_us": max(t_c, t_m) * 1e6}
+
+
+def workload_row(wl, C, t_step_ms, t_ffn_s, T_kept, pk):
+    """One row of the per-workload table: layer tokens/s and the expert GEMMs'
+    throughput against the bf16 peak, with the routing statistics."""
+    T, d, F, N = wl.T, wl.d_model, wl.d_ff, wl.n_experts
+    b = layer_bounds(wl, T_kept, pk)
+    ffn_flops = 4.0 * T_kept * d * F
+    tfl = ffn_flops / t_ffn_s / 1e12
+    return {"T": T, "d_model": d, "d_ff": F, "n_experts": N,
+            "capacity_factor": wl.capacity_factor, "capacity": C,
+            "ms_per_step": t_step_ms, "tokens_per_s": T / (t_step_ms * 1e-3),
+            "layer_tflops": b["useful_flops"] / (t_step_ms * 1e-3) / 1e12,
+            "layer_roofline_frac": b["t_min_us"] / (t_step_ms * 1e3),
+            "t_compute_us": b["t_compute_us"], "t_mem_us": b["t_mem_us"], "bound": b["bound"],
+            "expert_ffn_us": t_ffn_s * 1e6, "expert_ffn_tflops": tfl,
+            "expert_ffn_frac_burst": tfl / pk["bf16_tflops"],
+            "expert_ffn_frac_sustained": tfl / pk["bf16_tflops_sustained"],
+            "T_kept": T_kept, "drop_rate": 1.0 - T_kept / T,
+            "padding": 1.0 - T_kept / (N * C)}
+
+
+def extra_workloads(args, world, headline):
+    if args.workloads is None:
+        names = "all" if world == 1 else ""
+    else:
+        names = args.workloads
+    if names == "all":
+        names = ",".join(n for n, w in WORKLOADS.items() if w.dtype == "bf16")
+    return [n for n in names.split(",") if n and n != headline]
+
+
+def time_replays(fn, flush, stream, dev, reps):
+    """Mean device time of `reps` replays of a CUDA graph of fn, each after an
+    L2 flush, each bracketed by CUDA events on the launching stream."""
+    import torch
+    g = make_graph(fn)
+    g()
+    ts = []
+    for _ in range(reps):
+        flush.zero_()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        g()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ts.append(e0.elapsed_time(e1) * 1e-3)
+    return statistics.mean(ts)
+
+
+def time_workload(sm, wl, dev, stream, flush, pk, steps):
+    """The layer forward and the staged expert FFN of one more workload, timed
+    like the headline (graph replay, L2 flushed before each step)."""
+    import torch
+    inp = host_inputs(wl)
+
+    def to_dev(a):
+        if a is None:
+            return None
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+    T, d, F, N = wl.T, wl.d_model, wl.d_ff, wl.n_experts
+    x, w_r, b_r, w1, w2 = (to_dev(a) for a in (inp.x, inp.w_r, inp.b_r, inp.w1, inp.w2))
+    del inp
+    C = sm.switch_capacity(T, N, wl.capacity_factor)
+    cfg = sm.config(T, d, F, N, wl.capacity_factor, dtype=wl.dtype, alpha=wl.alpha)
+    ws = sm.workspace(cfg, device=dev)
+    out = torch.empty_like(x)
+    i32 = dict(dtype=torch.int32, device=dev)
+    idx, counts = torch.empty(T, **i32), torch.empty(N, **i32)
+    gate = torch.empty(T, dtype=torch.float32, device=dev)
+    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    t_step = time_replays(lambda: sm.switch_layer_forward(cfg, x, w_r, b_r, w1, w2, out, idx,
+                                                          gate, counts, loss, ws),
+                          flush, stream, dev, steps)
+    rank, slot = torch.empty(T, **i32), torch.empty(N * C, **i32)
+    drop = torch.empty(T, dtype=torch.uint8, device=dev)
+    x_disp = torch.empty(N * C, d, dtype=x.dtype, device=dev)
+    y = torch.empty(N * C, d, dtype=x.dtype, device=dev)
+    sm.switch_dispatch(cfg, idx, None, rank, drop, counts, slot, x, x_disp, ws)
+    cfg_rows = sm.config(T, d, F, N, wl.capacity_factor, dtype=wl.dtype, alpha=wl.alpha,
+                         flags=sm.FLAG_ROWS_DISPATCHED)
+    t_ffn = time_replays(lambda: sm.switch_expert_ffn(cfg_rows, x_disp, None, counts, w1, w2,
+                                                      y, ws), flush, stream, dev, 10)
+    st, where, info = sm.switch_get_device_error(ws)
+    if st != 0:
+        raise RuntimeError(f"device error {st} at {where} ({info}) timing {wl.name}")
+    cnt = counts.cpu().numpy().astype(np.int64)
+    T_kept = int(np.minimum(cnt, C).sum())
+    row = workload_row(wl, C, t_step * 1e3, t_ffn, T_kept, pk)
+    row["steps"] = steps
+    del x, w_r, b_r, w1, w2, ws, out, x_disp, y
+    torch.cuda.empty_cache()
+    return row
 
 
 def make_graph(fn, warm=3):

@@ -184,6 +184,9 @@ switch_status_t switch_dispatch(const switch_config_t* cfg, const int32_t* idx,
  *     and launch nothing.
  *   - The first call on a device looks up the array's device address (with
  *     that device current); make that first call before any stream capture.
+ *     The address is kept for the life of the process: after a
+ *     cudaDeviceReset() the library must be unloaded and loaded again before
+ *     this entry point is called on that device.
  *   - All calls share the array: calls that overlap on the GPU (different
  *     streams with no ordering between them) race and give wrong results.
  *   - No device error word: expert ids outside [0, N) make the token dropped

@@ -328,7 +328,14 @@ def layer_forward_top2(x, w_r, b_r, w1, w2, capacity_factor, alpha=0.01,
 
 
 def token_outputs(x, tokens, idx, drop, gate, w1, w2, residual=True):
-    """Block output rows for selected tokens only (for full-size sampling)."""
+    """Block output rows for selected tokens only (for full-size sampling).
+
+    Row j is x[t] + gate[t] . E_idx[t](x[t]) for t = tokens[j] when the token
+    is kept, x[t] when it is dropped (without the x term when ``residual`` is
+    False) [P1 §"Switch Routing", combine equation with one selected expert;
+    §"Expert Capacity and the Capacity Factor", dropped tokens pass through
+    the residual]: the same rows as ``layer_forward``'s output, one token at
+    a time."""
     tokens = np.asarray(tokens)
     rows = as_f64(x[tokens]) if residual else np.zeros((len(tokens), x.shape[1]))
     for j, t in enumerate(tokens):

@@ -10,6 +10,8 @@ import os
 import shutil
 import subprocess
 import sys
+import tempfile
+import zlib
 from concurrent.futures import ThreadPoolExecutor
 
 PKG = os.path.dirname(os.path.abspath(__file__))
@@ -17,7 +19,9 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libswitchmoe.so")
-BUILD_DIR = os.path.join(ROOT, "_build")
+# object files go outside the source tree; only the linked library sits in it
+BUILD_DIR = os.path.join(tempfile.gettempdir(),
+                         "switchmoe_build_%08x" % zlib.crc32(ROOT.encode()))
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",

@@ -1,13 +1,29 @@
 """Full-size parity: every named workload, in the launch configuration the
-benchmark times (switch_layer_forward with default flags).
+benchmark times (switch_layer_forward with default flags), plus the
+no-residual layer and the staged calls on the same inputs.
 
-Checked in full: the top-1 choice (equal to the oracle's except on tokens
-whose oracle top-1/top-2 probability margin is below 1e-6, counted), the
-per-expert counts (bit-exact once the oracle is re-based on the GPU's
-choices), every gate (1e-5 relative) and the load-balancing loss (1e-5
-relative).  Checked on sampled tokens the oracle computes one by one: the
-block output rows (bf16: max |err| <= 2e-2 x RMS of the sampled oracle
-rows; fp32: 1e-5), including dropped tokens, which must equal x bit for bit.
+Checked in full:
+* the top-1 choice (equal to the oracle's except on tokens whose oracle
+  top-1/top-2 probability margin is below 1e-6, counted), every gate (1e-5
+  relative) and the load-balancing loss (1e-5 relative);
+* the dispatch, bit for bit: rank, drop, counts and slot_token of
+  switch_dispatch fed the GPU's choices against the oracle's dispatch of
+  the same choices (and switch_dispatch_noalloc's where its fixed scratch
+  holds the workload).
+
+Checked against the oracle's expert FFNs, each bound relative to the RMS of
+the quantity compared (bf16: max |err| <= 2e-2 x RMS; fp32: 1e-5):
+* the expert term y = gate . E(x) alone (SWITCH_FLAG_NO_RESIDUAL), on every
+  kept token of a few experts (the first, middle and last expert with kept
+  tokens, and the fullest one -- so every M tile and token-tile position of
+  those experts is covered) and on sampled tokens of the others; dropped
+  tokens give exactly 0;
+* Y of the staged switch_expert_ffn on the dispatched rows, on every kept
+  slot of the same experts;
+* the block output with the residual on sampled tokens (dropped tokens equal
+  x bit for bit).  With the 0.1x initialisation the expert term is about
+  1e-3 of x's RMS, below one bf16 ulp of most outputs, so this check alone
+  could not see the experts: the two checks above are the ones that can.
 """
 import numpy as np
 import pytest
@@ -21,6 +37,11 @@ from gpu_util import (dev_float, host_f64, check_routing, rel_err, rms_ratio, PR
 pytestmark = pytest.mark.gpu
 
 NAMES = ["tiny", "base", "zipf_cf1.0", "zipf_cf1.25", "zipf_cf2.0", "large", "xxl"]
+I32 = dict(dtype=torch.int32, device="cuda")
+
+# Largest sizes switch_dispatch_noalloc's fixed scratch holds.
+NOALLOC_MAX_T = 131072
+NOALLOC_MAX_TILES = 131072
 
 
 @pytest.fixture(scope="module")
@@ -39,47 +60,131 @@ def _sample_tokens(T, drop, rng, n=40):
     return np.array(sorted(picks))
 
 
+def _checked_experts(kept):
+    """First, middle and last expert with kept tokens, and the fullest one."""
+    live = np.nonzero(kept > 0)[0]
+    picks = {int(live[0]), int(live[len(live) // 2]), int(live[-1]), int(np.argmax(kept))}
+    return sorted(picks)
+
+
+def _layer(sm, cfg, dev, inp, T, N):
+    out = torch.empty_like(dev["x"])
+    idx = torch.empty(T, **I32)
+    gate = torch.empty(T, dtype=torch.float32, device="cuda")
+    counts = torch.empty(N, **I32)
+    loss = torch.empty(1, dtype=torch.float32, device="cuda")
+    ws = sm.workspace(cfg)
+    sm.switch_layer_forward(cfg, dev["x"], dev["w_r"], dev["b_r"], dev["w1"], dev["w2"], out,
+                            idx, gate, counts, loss, ws)
+    st, where, info = sm.switch_get_device_error(ws)
+    assert st == 0, f"device error {st} at {where} ({info})"
+    return out, idx, gate, counts, loss
+
+
+def _dispatch_outputs(T, N, C):
+    return (torch.full((T,), -7, **I32), torch.full((T,), 9, dtype=torch.uint8, device="cuda"),
+            torch.full((N,), -7, **I32), torch.full((max(N * C, 1),), -7, **I32))
+
+
+def _assert_dispatch(got, want, what):
+    rank, drop, counts, slot = (g.cpu().numpy() for g in got)
+    np.testing.assert_array_equal(rank, want["rank"], err_msg=f"{what}: rank")
+    np.testing.assert_array_equal(drop.astype(bool), want["drop"], err_msg=f"{what}: drop")
+    np.testing.assert_array_equal(counts, want["counts"], err_msg=f"{what}: counts")
+    np.testing.assert_array_equal(slot[:len(want["slot_token"])], want["slot_token"],
+                                  err_msg=f"{what}: slot_token")
+
+
 @pytest.mark.parametrize("name", NAMES)
 def test_fullsize_layer(sm, name):
     wl = WORKLOADS[name]
     inp = make_inputs(wl)
-    cfg = sm.config(wl.T, wl.d_model, wl.d_ff, wl.n_experts, wl.capacity_factor,
-                    dtype=wl.dtype, alpha=wl.alpha)
-    ws = sm.workspace(cfg)
-    x = dev_float(inp.x)
-    w1 = dev_float(inp.w1)
-    w2 = dev_float(inp.w2)
-    out = torch.empty_like(x)
-    idx = torch.empty(wl.T, dtype=torch.int32, device="cuda")
-    gate = torch.empty(wl.T, dtype=torch.float32, device="cuda")
-    counts = torch.empty(wl.n_experts, dtype=torch.int32, device="cuda")
-    loss = torch.empty(1, dtype=torch.float32, device="cuda")
-    sm.switch_layer_forward(cfg, x, dev_float(inp.w_r),
-                            None if inp.b_r is None else dev_float(inp.b_r), w1, w2, out, idx,
-                            gate, counts, loss, ws)
-    st, where, info = sm.switch_get_device_error(ws)
-    assert st == 0, f"device error {st} at {where} ({info})"
-    del w1, w2
+    T, d, N = wl.T, wl.d_model, wl.n_experts
+    tol = BF16_RMS_TOL if wl.dtype == "bf16" else F32_RMS_TOL
+    dev = {"x": dev_float(inp.x), "w_r": dev_float(inp.w_r),
+           "b_r": None if inp.b_r is None else dev_float(inp.b_r),
+           "w1": dev_float(inp.w1), "w2": dev_float(inp.w2)}
+    cfg = sm.config(T, d, wl.d_ff, N, wl.capacity_factor, dtype=wl.dtype, alpha=wl.alpha)
+    out, idx, gate, counts, loss = _layer(sm, cfg, dev, inp, T, N)
     ig = idx.cpu().numpy().astype(np.int64)
 
+    # routing, gates, loss
     r = orc.router(inp.x, inp.w_r, inp.b_r)
     flips = check_routing(ig, r)
-    C = orc.capacity(wl.T, wl.n_experts, wl.capacity_factor)
-    dsp = orc.dispatch(ig, wl.n_experts, C)
+    C = orc.capacity(T, N, wl.capacity_factor)
+    dsp = orc.dispatch(ig, N, C)
     np.testing.assert_array_equal(counts.cpu().numpy(), dsp["counts"])
-    g64 = r["probs"][np.arange(wl.T), ig]
+    g64 = r["probs"][np.arange(T), ig]
     assert rel_err(gate.cpu().numpy(), g64).max() <= PROB_RTOL
     loss_w, _, _ = orc.aux_loss(dsp["counts"], r["probs"], wl.alpha)
     assert abs(loss.item() - loss_w) <= LOSS_RTOL * loss_w
 
+    # dispatch of the GPU's choices, bit for bit, at full size; the row copy
+    # that the staged expert FFN below reads comes with it
+    ws = sm.workspace(cfg)
+    got = _dispatch_outputs(T, N, C)
+    x_disp = torch.empty(N * C, d, dtype=dev["x"].dtype, device="cuda")
+    sm.switch_dispatch(cfg, idx, None, *got, dev["x"], x_disp, ws)
+    st, where, info = sm.switch_get_device_error(ws)
+    assert st == 0, f"device error {st} at {where} ({info})"
+    _assert_dispatch(got, dsp, "switch_dispatch")
+    if T <= NOALLOC_MAX_T and N * ((T + 127) // 128) <= NOALLOC_MAX_TILES:
+        got_na = _dispatch_outputs(T, N, C)
+        sm.switch_dispatch_noalloc(cfg, idx, None, *got_na)
+        torch.cuda.synchronize()
+        _assert_dispatch(got_na, dsp, "switch_dispatch_noalloc")
+
+    # block output with the residual, sampled tokens
     rng = np.random.default_rng(1234)
-    toks = _sample_tokens(wl.T, dsp["drop"], rng)
+    toks = _sample_tokens(T, dsp["drop"], rng)
     want = orc.token_outputs(inp.x, toks, ig, dsp["drop"], g64, inp.w1, inp.w2)
-    got = host_f64(out[torch.from_numpy(toks).cuda()])
-    tol = BF16_RMS_TOL if wl.dtype == "bf16" else F32_RMS_TOL
-    assert rms_ratio(got, want) <= tol
-    d = dsp["drop"][toks]
-    assert (got[d] == as_f64(inp.x[toks])[d]).all()
-    kept = int(np.minimum(dsp["counts"], C).sum())
-    print(f"{name}: flips {flips}, drop rate {1 - kept / wl.T:.4f}, "
-          f"padding {1 - kept / (wl.n_experts * C):.4f}, loss {loss.item():.6f}")
+    got_rows = host_f64(out[torch.from_numpy(toks).cuda()])
+    assert rms_ratio(got_rows, want) <= tol
+    dmask = dsp["drop"][toks]
+    assert (got_rows[dmask] == as_f64(inp.x[toks])[dmask]).all()
+
+    # the oracle's expert outputs on every kept slot of the checked experts
+    kept = np.minimum(dsp["counts"], C)
+    experts = _checked_experts(kept)
+    Y_want = {e: orc.expert(inp.x[dsp["slot_token"][e * C: e * C + kept[e]]], inp.w1[e],
+                            inp.w2[e]) for e in experts}
+
+    # staged expert FFN on the dispatched rows: Y of every kept slot
+    cfg_rows = sm.config(T, d, wl.d_ff, N, wl.capacity_factor, dtype=wl.dtype, alpha=wl.alpha,
+                         flags=sm.FLAG_ROWS_DISPATCHED)
+    y = torch.empty(N * C, d, dtype=dev["x"].dtype, device="cuda")
+    sm.switch_expert_ffn(cfg_rows, x_disp, None, got[2], dev["w1"], dev["w2"], y, ws)
+    st, where, info = sm.switch_get_device_error(ws)
+    assert st == 0, f"device error {st} at {where} ({info})"
+    worst_y = 0.0
+    for e in experts:
+        rows = host_f64(y[e * C: e * C + kept[e]])
+        ratio = rms_ratio(rows, Y_want[e])
+        assert ratio <= tol, f"staged Y of expert {e} ({kept[e]} rows): {ratio:.3e} x RMS"
+        worst_y = max(worst_y, ratio)
+    del y, x_disp
+
+    # the expert term alone: the layer without the residual
+    cfg_nr = sm.config(T, d, wl.d_ff, N, wl.capacity_factor, dtype=wl.dtype, alpha=wl.alpha,
+                       flags=sm.FLAG_NO_RESIDUAL)
+    out_nr, idx_nr, _, _, _ = _layer(sm, cfg_nr, dev, inp, T, N)
+    assert torch.equal(idx_nr, idx)
+    worst_term = 0.0
+    for e in experts:
+        tok_e = dsp["slot_token"][e * C: e * C + kept[e]]
+        want_e = g64[tok_e, None] * Y_want[e]
+        rows = host_f64(out_nr[torch.from_numpy(tok_e).cuda()])
+        ratio = rms_ratio(rows, want_e)
+        assert ratio <= tol, f"expert term of expert {e} ({kept[e]} tokens): {ratio:.3e} x RMS"
+        worst_term = max(worst_term, ratio)
+    others = np.array([t for t in toks if not dsp["drop"][t]])
+    want_o = orc.token_outputs(inp.x, others, ig, dsp["drop"], g64, inp.w1, inp.w2,
+                               residual=False)
+    got_o = host_f64(out_nr[torch.from_numpy(others).cuda()])
+    assert rms_ratio(got_o, want_o) <= tol
+    dropped = np.nonzero(dsp["drop"])[0]
+    if dropped.size:
+        assert (out_nr[torch.from_numpy(dropped).cuda()] == 0).all()
+    print(f"{name}: flips {flips}, drop rate {1 - kept.sum() / T:.4f}, "
+          f"padding {1 - kept.sum() / (N * C):.4f}, loss {loss.item():.6f}, experts "
+          f"{experts}: staged Y {worst_y:.2e}, expert term {worst_term:.2e} x RMS")

@@ -264,7 +264,34 @@ def test_fullsize_base_top2(sm):
                 want[j] += g64[k, t] * orc.expert(inp.x[t:t + 1], inp.w1[e], inp.w2[e])[0]
     got = host_f64(out_d[torch.from_numpy(toks).cuda()])
     assert rms_ratio(got, want) <= BF16_RMS_TOL
-    print(f"base top-2: flips {flips}, C {C}, dropped assignments {dsp['drop'].mean():.4f}")
+
+    # The expert terms alone (no residual; with the 0.1x initialisation they
+    # are below one bf16 ulp of x, so the check above cannot see them): every
+    # token holding a kept slot of the first, middle and last expert, both of
+    # its routes summed, against the oracle, relative to their own RMS.
+    w1, w2 = dev_float(inp.w1), dev_float(inp.w2)
+    out_nr = torch.empty_like(x)
+    cfg_nr = _cfg(sm, wl, sm.FLAG_NO_RESIDUAL)
+    sm.switch_layer_forward(cfg_nr, x, dev_float(inp.w_r), None, w1, w2, out_nr, idx, gate,
+                            counts, loss, ws)
+    _ok(sm, ws)
+    del w1, w2
+    N = wl.n_experts
+    kept = np.minimum(dsp["counts"], C)
+    live = np.nonzero(kept > 0)[0]
+    sel = sorted({int(live[0]), int(live[len(live) // 2]), int(live[-1])})
+    toks = np.unique(np.concatenate([dsp["slot_token"][e * C: e * C + kept[e]] for e in sel]))
+    want = np.zeros((len(toks), wl.d_model))
+    for k in range(2):
+        on = ~dsp["drop"][k, toks]
+        for e in np.unique(ig[k, toks[on]]):
+            j = np.nonzero(on & (ig[k, toks] == e))[0]
+            want[j] += g64[k, toks[j], None] * orc.expert(inp.x[toks[j]], inp.w1[e], inp.w2[e])
+    got = host_f64(out_nr[torch.from_numpy(toks).cuda()])
+    ratio = rms_ratio(got, want)
+    assert ratio <= BF16_RMS_TOL, f"top-2 expert terms: {ratio:.3e} x RMS"
+    print(f"base top-2: flips {flips}, C {C}, dropped assignments {dsp['drop'].mean():.4f}, "
+          f"expert terms of {len(toks)} tokens (experts {sel}) {ratio:.2e} x RMS")
 
 
 def test_top2_expert_ffn_rows_dispatched(sm):

@@ -379,12 +379,64 @@ def pin_top2_signature(O):
         ALPHA * N * np.sum(np.bincount(res["idx2"][0], minlength=N) / T * res["probs"].mean(0)))
 
 
+def pin_token_outputs_signature(O):
+    """The per-token checker used at full size: token t's block row is
+    x_t + p_idx E_idx(x_t) when kept and x_t when dropped (and the same
+    without x when the residual is off), with experts that each write the
+    signature 100 (e + 1) unit(e) through a hidden unit that equals one, so
+    the expected rows are closed forms.  Capacity 0.5 drops tokens."""
+    rng = np.random.default_rng(17)
+    N, dm, T = 3, 4, 30
+    x = rng.standard_normal((T, dm)).astype(np.float32)
+    x[:, 3] = 1.0
+    w_r = rng.standard_normal((N, dm)).astype(np.float32)
+    w1 = np.zeros((N, N, dm), np.float32)
+    w2 = np.zeros((N, dm, N), np.float32)
+    for e in range(N):
+        w1[e, e, 3] = 1.0
+        w2[e, e, e] = 100.0 * (e + 1)
+    r = O.router(x, w_r)
+    C = O.capacity(T, N, 0.5)
+    dsp = O.dispatch(r["idx"], N, C)
+    assert dsp["drop"].any() and not dsp["drop"].all()
+    toks = np.arange(T)[::-1]               # any order of the requested tokens
+    for residual in (True, False):
+        rows = O.token_outputs(x, toks, r["idx"], dsp["drop"], r["gate"], w1, w2,
+                               residual=residual)
+        for j, t in enumerate(toks):
+            want = x[t].astype(np.float64).copy() if residual else np.zeros(dm)
+            if not dsp["drop"][t]:
+                e = r["idx"][t]
+                want[e] += r["gate"][t] * 100.0 * (e + 1)
+            np.testing.assert_allclose(rows[j], want, rtol=1e-12, atol=1e-12)
+
+
+def pin_token_outputs_match_layer(O):
+    """token_outputs on every token equals the whole layer's output (the fp32
+    Tiny workload and a small bf16 one with a Zipf bias and drops), with and
+    without the residual."""
+    from switch_inputs import Workload, make_inputs
+    for wl in (Workload("t32", T=96, d_model=16, d_ff=32, n_experts=4, capacity_factor=0.75,
+                        dtype="f32", seed=21),
+               Workload("tbf", T=80, d_model=64, d_ff=64, n_experts=5, capacity_factor=1.0,
+                        dtype="bf16", zipf_s=1.1, seed=22)):
+        inp = make_inputs(wl)
+        for residual in (True, False):
+            res = O.layer_forward(inp.x, inp.w_r, inp.b_r, inp.w1, inp.w2,
+                                  wl.capacity_factor, ALPHA, residual=residual)
+            assert res["drop"].any()
+            rows = O.token_outputs(inp.x, np.arange(wl.T), res["idx"], res["drop"],
+                                   res["gate"], inp.w1, inp.w2, residual=residual)
+            np.testing.assert_allclose(rows, res["out"], rtol=1e-12, atol=1e-15)
+
+
 PINS = [pin_capacity, pin_softmax_hand, pin_router_invariants, pin_dispatch_hand,
         pin_dispatch_bruteforce, pin_dispatch_via_router, pin_aux_hand,
         pin_aux_uniform, pin_dense_reduction, pin_single_expert_signature,
         pin_dropped_residual, pin_relu_active, pin_top2_router_hand,
         pin_top2_router_invariants, pin_top2_dispatch_hand, pin_top2_dispatch_bruteforce,
-        pin_top2_dense_reduction, pin_top2_signature]
+        pin_top2_dense_reduction, pin_top2_signature, pin_token_outputs_signature,
+        pin_token_outputs_match_layer]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda p: p.__name__)
@@ -506,6 +558,32 @@ def _mut_top2_token_major(real):
     return f
 
 
+def _mut_token_outputs_next_expert(real):
+    def f(x, tokens, idx, drop, gate, w1, w2, residual=True):
+        N = np.shape(w1)[0]
+        return real(x, tokens, (np.asarray(idx) + 1) % N, drop, gate, w1, w2, residual)
+    return f
+
+
+def _mut_token_outputs_first_gate(real):
+    def f(x, tokens, idx, drop, gate, w1, w2, residual=True):
+        g = np.full(len(gate), np.asarray(gate)[0])     # one token's gate for all
+        return real(x, tokens, idx, drop, g, w1, w2, residual)
+    return f
+
+
+def _mut_token_outputs_keeps_dropped(real):
+    def f(x, tokens, idx, drop, gate, w1, w2, residual=True):
+        return real(x, tokens, idx, np.zeros(len(drop), bool), gate, w1, w2, residual)
+    return f
+
+
+def _mut_token_outputs_always_residual(real):
+    def f(x, tokens, idx, drop, gate, w1, w2, residual=True):
+        return real(x, tokens, idx, drop, gate, w1, w2, True)
+    return f
+
+
 MUTANTS = {
     "top2_second_on_last_tie": ("router_top2", _mut_top2_second_highest_index),
     "top2_gates_renormalised": ("router_top2", _mut_top2_renormalised),
@@ -521,6 +599,10 @@ MUTANTS = {
     "dropped_not_residual": ("combine", _mut_combine_drop_zero),
     "P_from_hard_counts": ("aux_loss", _mut_aux_P_from_f),
     "loss_without_N": ("aux_loss", _mut_aux_no_N),
+    "token_outputs_next_expert": ("token_outputs", _mut_token_outputs_next_expert),
+    "token_outputs_first_gate": ("token_outputs", _mut_token_outputs_first_gate),
+    "token_outputs_keeps_dropped": ("token_outputs", _mut_token_outputs_keeps_dropped),
+    "token_outputs_always_residual": ("token_outputs", _mut_token_outputs_always_residual),
 }
 
 

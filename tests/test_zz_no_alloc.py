@@ -11,6 +11,8 @@ import numpy as np
 import pytest
 import torch
 
+import oracle.switch_oracle as orc
+
 pytestmark = pytest.mark.gpu
 
 
@@ -49,6 +51,12 @@ def test_noalloc_dispatch_matches_workspace_dispatch(sm, source):
         for w, g in zip(want, got):
             assert torch.equal(w, g)
         assert int(got[2].sum()) == T
+        # and the oracle's dispatch of the same choices, bit for bit
+        ref = orc.dispatch(idx, N, C)
+        np.testing.assert_array_equal(got[0].cpu().numpy(), ref["rank"])
+        np.testing.assert_array_equal(got[1].cpu().numpy().astype(bool), ref["drop"])
+        np.testing.assert_array_equal(got[2].cpu().numpy(), ref["counts"])
+        np.testing.assert_array_equal(got[3].cpu().numpy(), ref["slot_token"])
 
 
 def test_noalloc_rejects_sizes_beyond_its_array(sm):
