@@ -299,6 +299,85 @@ switch_status_t switch_layer_backward(const switch_config_t* cfg, const void* x,
  * than switch_workspace_size(); every other entry point accepts it too). */
 switch_status_t switch_backward_workspace_size(const switch_config_t* cfg, size_t* bytes);
 
+/* ------------------------------------------------------------------------
+ * Expert parallelism [P1 "Distributed Implementation and the Three
+ * Parallelisms", expert-parallelism row: each device holds some of the
+ * experts and tokens travel to their expert's device and back].
+ *
+ * G ranks (one GPU each) hold N / G experts each -- rank h owns experts
+ * h*N/G .. (h+1)*N/G - 1 -- and cfg->T tokens each (the same T on every
+ * rank).  The global batch is the ranks' batches end to end in rank order
+ * and is ONE routing group: capacity C = switch_capacity(G*T, N, cf), slot
+ * order is global batch order, f_i and P_i are over all G*T tokens.  So the
+ * outputs, counts and loss equal switch_layer_forward's on the
+ * concatenated batch on one GPU (bit for bit when T is a multiple of 128;
+ * otherwise the loss differs by fp32 summation order only).
+ *
+ * One forward step, on every rank, in this order:
+ *   1. switch_ep_route      router + this rank's per-expert counts; writes
+ *                           this rank's exchange record (record_bytes);
+ *   2. [caller] all-gather the records of all ranks, in rank order, into
+ *      `records` [G][record_bytes] (e.g. an NCCL all-gather on the stream);
+ *   3. switch_ep_dispatch   global ranks and drops; stores every kept
+ *                           token's row, source and gate straight into its
+ *                           owner's receive buffer (peer pointers); writes
+ *                           dropped tokens' outputs; the loss;
+ *   4. [caller] barrier: every rank's step 3 has completed;
+ *   5. switch_ep_experts    this rank's experts' GEMMs; the second GEMM's
+ *                           epilogue stores x + gate * E(x) into each
+ *                           token's output row on its home rank (peer
+ *                           pointers);
+ *   6. [caller] barrier before any rank reads its output.
+ * Peer buffers: every rank's receive buffer (recv_bytes, 256-byte aligned)
+ * and output [T, d_model] must be reachable from every rank's GPU (CUDA IPC
+ * or symmetric memory over NVLink); the calls take host arrays of the G
+ * device pointers, entry h being rank h's.  No copy reads another GPU's
+ * memory: the exchange is made of plain stores, none of them multicast.
+ * bf16 only, top-1 only, CTA-pair second GEMM (SWITCH_FLAG_GEMM_1SM and
+ * SWITCH_FLAG_TOP2 return SWITCH_ERR_UNSUPPORTED), N % G == 0, G <= 16,
+ * T < 2^26.  SWITCH_FLAG_NO_RESIDUAL and SWITCH_FLAG_GEMM_PAIRS apply.
+ * T = 0 makes every call a no-op. */
+typedef struct {
+  int32_t world_size;       /* G: ranks of the expert-parallel group */
+  int32_t rank;             /* this rank, 0 <= rank < G */
+} switch_ep_t;
+
+/* Bytes of this rank's workspace (ws_bytes; the same conventions as
+ * switch_workspace_size's), of one exchange record (record_bytes) and of a
+ * receive buffer (recv_bytes).  Any output pointer may be NULL. */
+switch_status_t switch_ep_sizes(const switch_config_t* cfg, const switch_ep_t* ep,
+                                size_t* ws_bytes, size_t* record_bytes, size_t* recv_bytes);
+
+/* Step 1.  x [T, d_model] bf16, w_r [N, d_model] fp32, b_r [N] or NULL as
+ * for switch_router; idx [T] int32 and gate [T] fp32: optional copies of
+ * the top-1 choices and gates.  record: record_bytes of device memory
+ * (16-byte aligned) receiving this rank's per-expert counts and
+ * per-128-token sums of the router probabilities. */
+switch_status_t switch_ep_route(const switch_config_t* cfg, const switch_ep_t* ep,
+                                const void* x, const float* w_r, const float* b_r,
+                                int32_t* idx, float* gate, void* record, void* ws,
+                                size_t ws_bytes, void* stream);
+
+/* Step 3 (after step 2).  records: [G][record_bytes], rank order.
+ * recv_peers: host array of the G ranks' receive buffers.  out: this rank's
+ * output [T, d_model] bf16; this call writes its dropped tokens' rows (x,
+ * or 0 without the residual).  counts [N] int32 (routed tokens of the whole
+ * batch, before the cut) and loss (device fp32 scalar): optional. */
+switch_status_t switch_ep_dispatch(const switch_config_t* cfg, const switch_ep_t* ep,
+                                   const void* x, const void* records, void* const* recv_peers,
+                                   void* out, int32_t* counts, float* loss, void* ws,
+                                   size_t ws_bytes, void* stream);
+
+/* Step 5 (after step 4).  w1_local [N/G, d_ff, d_model] and w2_local
+ * [N/G, d_model, d_ff] bf16: this rank's experts' weights (rows
+ * rank*N/G .. of the full w1 / w2).  recv: this rank's receive buffer.
+ * out_peers: host array of the G ranks' outputs [T, d_model].  Kept
+ * tokens' output rows are written on their home ranks. */
+switch_status_t switch_ep_experts(const switch_config_t* cfg, const switch_ep_t* ep,
+                                  const void* w1_local, const void* w2_local, const void* recv,
+                                  void* const* out_peers, void* ws, size_t ws_bytes,
+                                  void* stream);
+
 /* Synchronises `stream`, reads the workspace's device error word, clears
  * it, and returns the recorded status (SWITCH_OK if none).  *where_out and
  * *info_out (either may be NULL) receive the reporting kernel role and a

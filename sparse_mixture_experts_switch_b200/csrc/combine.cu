@@ -92,25 +92,65 @@ cudaError_t launch_combine(int64_t T, int d, int64_t C, bool bf16, const void* x
 
 // --------------------------------------------------------------- aux loss
 
-// psum[blk][e] = sum over rows blk*128 .. blk*128+127 of probs[row][e],
-// added in row order.
-__global__ void __launch_bounds__(128) prob_colsum_kernel(int64_t T, int N,
+// psum[blk][e] = sum over rows blk*128 .. blk*128+127 of probs[row][e], in a
+// fixed order.  One block per 128-row part; a thread owns one column unit (4
+// experts as a float4 when N % 4 == 0, else one expert) and one of G row
+// groups (rows g, g + G, ...), so a warp reads whole row segments and every
+// thread keeps several independent loads in flight; the G partial sums of a
+// unit are then added in group order.
+template <bool kVec4>
+__global__ void __launch_bounds__(256) prob_colsum_kernel(int64_t T, int N,
                                                           const float* __restrict__ probs,
                                                           float* __restrict__ psum) {
-  const int e = blockIdx.y * 128 + threadIdx.x;
-  if (e >= N) return;
+  __shared__ float4 red[256];
+  const int units = kVec4 ? N / 4 : N;
   const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kTileTok;
-  const int64_t r1 = r0 + kTileTok < T ? r0 + kTileTok : T;
-  float s = 0.f;
-  for (int64_t r = r0; r < r1; ++r) s += probs[r * N + e];
-  psum[static_cast<int64_t>(blockIdx.x) * N + e] = s;
+  const int rows = static_cast<int>(T - r0 < kTileTok ? T - r0 : kTileTok);
+  for (int u0 = 0; u0 < units; u0 += 256) {
+    const int span = units - u0 < 256 ? units - u0 : 256;   // units in this pass
+    const int G = 256 / span;                                // row groups
+    const int u = u0 + static_cast<int>(threadIdx.x) % span;
+    const int g = static_cast<int>(threadIdx.x) / span;
+    float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (g < G) {
+      if (kVec4) {
+        const float4* col = reinterpret_cast<const float4*>(probs + r0 * N) + u;
+#pragma unroll 4
+        for (int r = g; r < rows; r += G) {
+          const float4 v = __ldg(col + static_cast<int64_t>(r) * (N / 4));
+          s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+        }
+      } else {
+        const float* col = probs + r0 * N + u;
+#pragma unroll 4
+        for (int r = g; r < rows; r += G) s.x += __ldg(col + static_cast<int64_t>(r) * N);
+      }
+    }
+    red[threadIdx.x] = s;
+    __syncthreads();
+    if (static_cast<int>(threadIdx.x) < span) {
+      float4 t = red[threadIdx.x];
+      for (int q = 1; q < G; ++q) {
+        const float4 v = red[q * span + threadIdx.x];
+        t.x += v.x; t.y += v.y; t.z += v.z; t.w += v.w;
+      }
+      float* dst = psum + static_cast<int64_t>(blockIdx.x) * N;
+      if (kVec4) reinterpret_cast<float4*>(dst)[u] = t;
+      else dst[u] = t.x;
+    }
+    __syncthreads();
+  }
 }
 
 cudaError_t launch_prob_colsum(int64_t T, int N, const float* probs, float* psum,
                                cudaStream_t st) {
-  const dim3 grid(static_cast<unsigned>((T + kTileTok - 1) / kTileTok),
-                  static_cast<unsigned>((N + 127) / 128));
-  prob_colsum_kernel<<<grid, 128, 0, st>>>(T, N, probs, psum);
+  const unsigned grid = static_cast<unsigned>((T + kTileTok - 1) / kTileTok);
+  const bool vec4 = (N % 4) == 0 && (reinterpret_cast<uintptr_t>(probs) & 15u) == 0 &&
+                    (reinterpret_cast<uintptr_t>(psum) & 15u) == 0;
+  if (vec4)
+    prob_colsum_kernel<true><<<grid, 256, 0, st>>>(T, N, probs, psum);
+  else
+    prob_colsum_kernel<false><<<grid, 256, 0, st>>>(T, N, probs, psum);
   return cudaGetLastError();
 }
 

@@ -204,6 +204,78 @@ cudaError_t launch_finalize(int64_t T, int N, int64_t C, int ntiles, const int* 
   return cudaGetLastError();
 }
 
+// finalize_kernel and the row copy in one pass, one warp per item: items
+// 0 .. T-1 are assignments (lane 0 decides rank / drop / slot, the warp
+// copies the row into its slot), items T .. T + N*C - 1 are slots (a
+// padding slot gets -1 and a zero row).  Slot order, and so every output,
+// is the same as finalize_kernel's followed by gather_rows_kernel's.
+__global__ void __launch_bounds__(256) finalize_gather_kernel(
+    int64_t T, int N, int64_t C, int ntiles, const int* __restrict__ idx,
+    const int* __restrict__ local_rank, const int* __restrict__ base,
+    const int* __restrict__ counts, int* __restrict__ rank, uint8_t* __restrict__ drop,
+    int* __restrict__ slot_token, int* __restrict__ mtile_start, int64_t tok_mod,
+    const uint4* __restrict__ x, uint4* __restrict__ x_disp, int64_t vec_per_row) {
+  if (blockIdx.x == 0 && threadIdx.x < 32 && mtile_start != nullptr)
+    mtile_prefix_warp(N, C, counts, mtile_start);
+  const int lane = threadIdx.x & 31;
+  const int64_t nslots = static_cast<int64_t>(N) * C;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       i < T + nslots; i += warps) {
+    if (i < T) {
+      int64_t slot = -1;
+      const int64_t tok = tok_mod > 0 && i >= tok_mod ? i - tok_mod : i;
+      if (lane == 0) {
+        const int e = idx[i];
+        const int lr = local_rank[i];
+        int r = -1;
+        bool dropped = true;
+        if (e >= 0 && e < N && lr >= 0) {
+          r = base[static_cast<int64_t>(e) * ntiles + (i / kTileTok)] + lr;
+          dropped = r >= C;
+          if (!dropped) {
+            slot = static_cast<int64_t>(e) * C + r;
+            slot_token[slot] = static_cast<int>(tok);
+          }
+        }
+        rank[i] = r;
+        drop[i] = dropped ? 1 : 0;
+      }
+      slot = __shfl_sync(0xffffffffu, slot, 0);
+      if (slot >= 0) {
+        const uint4* src = x + tok * vec_per_row;
+        uint4* dst = x_disp + slot * vec_per_row;
+        for (int64_t v = lane; v < vec_per_row; v += 32) dst[v] = __ldg(src + v);
+      }
+    } else {
+      const int64_t s = i - T;
+      const int e = static_cast<int>(s / C);
+      const int64_t r = s - static_cast<int64_t>(e) * C;
+      const int64_t kept = counts[e] < C ? counts[e] : C;
+      if (r >= kept) {
+        if (lane == 0) slot_token[s] = -1;
+        uint4* dst = x_disp + s * vec_per_row;
+        for (int64_t v = lane; v < vec_per_row; v += 32) dst[v] = make_uint4(0, 0, 0, 0);
+      }
+    }
+  }
+}
+
+cudaError_t launch_finalize_gather(int64_t T, int N, int64_t C, int ntiles, const int* idx,
+                                   const int* local_rank, const int* base, const int* counts,
+                                   int* rank, uint8_t* drop, int* slot_token, int* mtile_start,
+                                   int64_t tok_mod, const void* x, void* x_disp,
+                                   int64_t row_bytes, cudaStream_t st) {
+  const int64_t items = T + static_cast<int64_t>(N) * C;
+  int64_t blocks = (items + 7) / 8;
+  if (blocks > 148 * 8) blocks = 148 * 8;
+  if (blocks < 1) blocks = 1;
+  finalize_gather_kernel<<<static_cast<int>(blocks), 256, 0, st>>>(
+      T, N, C, ntiles, idx, local_rank, base, counts, rank, drop, slot_token, mtile_start,
+      tok_mod, static_cast<const uint4*>(x), static_cast<uint4*>(x_disp), row_bytes / 16);
+  return cudaGetLastError();
+}
+
 __global__ void mtile_table_kernel(int N, int64_t C, const int* counts, int* mtile_start) {
   mtile_prefix_warp(N, C, counts, mtile_start);
 }

@@ -396,6 +396,13 @@ cudaError_t launch_expert_ffn_bf16(const FfnArgs& a, cudaStream_t st) {
   g2.x_res = static_cast<const __nv_bfloat16*>(a.x_res);
   g2.gate = a.gate;
   g2.comb_out = static_cast<__nv_bfloat16*>(a.out);
+  if (a.mode2 == kModeCombineEp) {
+    // expert parallelism: outputs go to each token's home rank (CTA pairs only)
+    if (!a.pair2 || a.peer_out == nullptr || a.n_peers < 1 || a.n_peers > kEpMaxRanks)
+      return cudaErrorInvalidValue;
+    for (int i = 0; i < a.n_peers; ++i)
+      g2.peer_out[i] = static_cast<__nv_bfloat16*>(a.peer_out[i]);
+  }
   return a.pair2 ? run_gemm_pair<false>(ta2, tb2, to2, g2, a.num_sms, st)
                 : run_gemm<false>(ta2, tb2, to2, g2, a.num_sms, st);
 }

@@ -276,8 +276,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     // segments prefetched) while that tile's main loop runs
     CombineMeta meta;
     const int fq = static_cast<int>(rank) * 128 + q * 32;    // warp's feature offset in a tile
-    if (lane == 0 && p.mode != kModeCombine) tma_prefetch_desc(&tmap_out);
-    if (p.mode == kModeCombine) {
+    const bool combine = p.mode == kModeCombine || p.mode == kModeCombineEp;
+    if (lane == 0 && !combine) tma_prefetch_desc(&tmap_out);
+    if (combine) {
       const PairTile t = pair_tile(p, pts, cid);
       combine_meta(p, t, t.f0 + fq, meta, lane);
     }
@@ -303,7 +304,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         if (leader) mbar_arrive(&tempty[acc]);
         else mbar_arrive_remote(tempty_lead + 8u * acc);
       }
-      if (p.mode == kModeCombine && tile + ncl < total) {
+      if (combine && tile + ncl < total) {
         const PairTile tn = pair_tile(p, pts, tile + ncl);
         combine_meta(p, tn, tn.f0 + fq, meta, lane);
       }

@@ -51,6 +51,7 @@ struct GemmParams {
   const __nv_bfloat16* x_res;   // kModeCombine
   const float* gate;
   __nv_bfloat16* comb_out;      // [T, n_out]
+  __nv_bfloat16* peer_out[kEpMaxRanks];   // kModeCombineEp: each rank's output rows
   DevErr* err;
   long long spin;
 };

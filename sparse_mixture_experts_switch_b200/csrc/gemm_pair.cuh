@@ -79,9 +79,13 @@ struct CombineMeta {
   float g[8];
 };
 
+// Expert parallelism (kModeCombineEp): `tok` holds the slot's packed source
+// (home rank, token), the gate is the slot's, and the residual is the slot's
+// own row of the dispatched buffer (a copy of x[token] on this GPU).
 __device__ __forceinline__ void combine_meta(const GemmParams& p, const PairTile& t, int fb,
                                              CombineMeta& m, int lane) {
   const int64_t row0 = static_cast<int64_t>(t.e) * p.C + t.t0;
+  const bool ep = p.mode == kModeCombineEp;
 #pragma unroll
   for (int c = 0; c < 8; ++c) {
     const int col = c * 32 + lane;
@@ -91,9 +95,10 @@ __device__ __forceinline__ void combine_meta(const GemmParams& p, const PairTile
   for (int c = 0; c < 8; ++c) {
     m.g[c] = 0.f;
     if (m.tok[c] >= 0) {
-      m.g[c] = p.gate[m.tok[c]];
+      const int64_t res_row = ep ? row0 + c * 32 + lane : static_cast<int64_t>(m.tok[c]);
+      m.g[c] = p.gate[ep ? res_row : m.tok[c]];
       if (p.x_res != nullptr && fb < p.n_out)
-        prefetch_l2(p.x_res + static_cast<int64_t>(m.tok[c]) * p.n_out + fb);
+        prefetch_l2(p.x_res + res_row * p.n_out + fb);
     }
   }
 }
@@ -132,7 +137,8 @@ __device__ __forceinline__ void epilogue_tile_t(const GemmParams& p, const CUten
   auto chunk_store = [&](int c, const uint32_t* u) {
     const int j0 = c * 32;
     const int jn = t.nv - j0 < 32 ? t.nv - j0 : 32;     // kept tokens in this chunk
-    if (p.mode == kModeCombine) {
+    if (p.mode == kModeCombine || p.mode == kModeCombineEp) {
+      const bool ep = p.mode == kModeCombineEp;
       // transpose: element (token j, feature lane) at row j, 16-byte chunk
       // (lane / 4) ^ (j % 8) of a 128-byte row
 #pragma unroll
@@ -151,9 +157,10 @@ __device__ __forceinline__ void epilogue_tile_t(const GemmParams& p, const CUten
         tk[pass] = __shfl_sync(0xffffffffu, tkc, rr);
         g[pass] = __shfl_sync(0xffffffffu, gcl, rr);
         xr[pass] = make_uint4(0, 0, 0, 0);
+        const int64_t res_row = ep ? row0 + j0 + rr : static_cast<int64_t>(tk[pass]);
         if (tk[pass] >= 0 && p.x_res != nullptr)
-          xr[pass] = __ldg(reinterpret_cast<const uint4*>(
-              p.x_res + static_cast<int64_t>(tk[pass]) * p.n_out + fb + qq * 8));
+          xr[pass] = __ldg(reinterpret_cast<const uint4*>(p.x_res + res_row * p.n_out + fb +
+                                                          qq * 8));
       }
 #pragma unroll
       for (int pass = 0; pass < 4; ++pass) {
@@ -167,8 +174,11 @@ __device__ __forceinline__ void epilogue_tile_t(const GemmParams& p, const CUten
         o.y = pack_bf16x2(fmaf(gg, a.z, bf16_lo(xr[pass].y)), fmaf(gg, a.w, bf16_hi(xr[pass].y)));
         o.z = pack_bf16x2(fmaf(gg, b.x, bf16_lo(xr[pass].z)), fmaf(gg, b.y, bf16_hi(xr[pass].z)));
         o.w = pack_bf16x2(fmaf(gg, b.z, bf16_lo(xr[pass].w)), fmaf(gg, b.w, bf16_hi(xr[pass].w)));
-        *reinterpret_cast<uint4*>(p.comb_out + static_cast<int64_t>(tk[pass]) * p.n_out + fb +
-                                  qq * 8) = o;
+        __nv_bfloat16* orow =
+            ep ? p.peer_out[tk[pass] >> kEpRankShift] +
+                     static_cast<int64_t>(tk[pass] & ((1 << kEpRankShift) - 1)) * p.n_out
+               : p.comb_out + static_cast<int64_t>(tk[pass]) * p.n_out;
+        *reinterpret_cast<uint4*>(orow + fb + qq * 8) = o;
       }
       __syncwarp();                    // the buffer is rewritten by the next chunk
       return;

@@ -26,6 +26,13 @@ cudaError_t launch_finalize(int64_t T, int N, int64_t C, int ntiles, const int* 
                             const int* local_rank, const int* base, const int* counts,
                             int* rank, uint8_t* drop, int* slot_token, int* mtile_start,
                             int64_t tok_mod, cudaStream_t st);
+// launch_finalize and the row copy x_disp[slot] = x[token] (zeros in padding
+// slots) in one kernel; row_bytes % 16 == 0.
+cudaError_t launch_finalize_gather(int64_t T, int N, int64_t C, int ntiles, const int* idx,
+                                   const int* local_rank, const int* base, const int* counts,
+                                   int* rank, uint8_t* drop, int* slot_token, int* mtile_start,
+                                   int64_t tok_mod, const void* x, void* x_disp,
+                                   int64_t row_bytes, cudaStream_t st);
 // Only mtile_start from counts (for a standalone expert-FFN call).
 cudaError_t launch_mtile_table(int N, int64_t C, const int* counts, int* mtile_start,
                                cudaStream_t st);
@@ -94,7 +101,14 @@ bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint6
                        uint32_t box_inner, uint32_t box_outer, bool swizzle64 = false);
 
 // ------------------------------------------------------------ expert FFN
-enum GemmMode : int { kModeHidden = 0, kModeY = 1, kModeCombine = 2 };
+// kModeCombineEp: the combine of expert parallelism.  A slot's row of the
+// dispatched buffer is its residual, `slot_token` holds the slot's source
+// (home rank << kEpRankShift | token on that rank), `gate` is indexed by
+// slot, and the output row goes to the home rank's buffer peer_out[rank].
+enum GemmMode : int { kModeHidden = 0, kModeY = 1, kModeCombine = 2, kModeCombineEp = 3 };
+
+constexpr int kEpMaxRanks = 16;
+constexpr int kEpRankShift = 26;                 // tokens per rank < 2^26
 
 struct FfnArgs {
   int64_t T;
@@ -117,11 +131,45 @@ struct FfnArgs {
   bool pair1;               // GEMM1 on CTA pairs (2-SM), else one CTA per tile
   bool pair2;               // GEMM2 on CTA pairs
   bool gemm1_only;          // stop after GEMM1 (the backward pass recomputes H)
+  void* const* peer_out;    // kModeCombineEp: every rank's output [T_rank, d] (host array)
+  int n_peers;
   DevErr* err;
   long long spin;
   int num_sms;
 };
 cudaError_t launch_expert_ffn_bf16(const FfnArgs& a, cudaStream_t st);
+
+// ------------------------------------------------------ expert parallelism
+// Per-rank exchange record that every rank all-gathers ([G][stride] bytes):
+// the per-part router probability sums [nparts][N] fp32 at offset 0 and the
+// per-expert token counts [N] int32 at `counts_off`.
+struct EpGathered {
+  const uint8_t* base;
+  size_t stride;
+  size_t counts_off;
+};
+struct EpPeers {
+  void* p[kEpMaxRanks];
+};
+// Receiving rank's buffer: dispatched rows [E_loc*C, d] bf16 at offset 0,
+// slot sources [E_loc*C] int32 at src_off, slot gates [E_loc*C] fp32 at
+// gate_off.
+struct EpRecvLayout {
+  size_t src_off;
+  size_t gate_off;
+};
+// Global counts, this rank's experts' counts, and the ranks' probability
+// sums laid end to end [G * nparts][N] for the loss.
+cudaError_t launch_ep_prepare(int N, int G, int me, int e_loc, int nparts, EpGathered g,
+                              int* counts_glob, int* counts_loc, float* psum_cat,
+                              cudaStream_t st);
+// Global batch-order rank of every token of rank r, drop mask, and the kept
+// tokens' rows, sources and gates stored into their owners' buffers.
+cudaError_t launch_ep_dispatch(int64_t T, int N, int64_t C, int G, int r, int e_loc, int ntiles,
+                               const int* idx, const int* local_rank, const int* base,
+                               const float* gate, EpGathered g, const void* x, int64_t row_bytes,
+                               const EpPeers& recv, EpRecvLayout rl, int* rank, uint8_t* drop,
+                               cudaStream_t st);
 cudaError_t launch_expert_ffn_f32(const FfnArgs& a, cudaStream_t st);
 
 }  // namespace smoe

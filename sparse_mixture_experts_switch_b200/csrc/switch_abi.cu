@@ -202,6 +202,96 @@ bool use_tc_router(const switch_config_t* c) {
          (!(c->flags & SWITCH_FLAG_TOP2) || router_pair_supported(c->n_experts, router_terms(c)));
 }
 
+// ------------------------------------------------------ expert parallelism
+
+// Regions of one rank's expert-parallel workspace, of the record every rank
+// all-gathers, and of the receive buffer peers store into.
+struct EpLayout {
+  int G, r, e_loc, nt, nparts, nparts_max;
+  int64_t T, C;
+  bool tc_router;
+  size_t err, hist, base, local_rank, idx, gate, rank, drop, wsplit, logits, psum_cat,
+      counts_glob, counts_loc, mtile_start, fpsc, hbuf, total;
+  size_t payload_counts, payload_total;       // record: psum parts, then counts
+  size_t recv_src, recv_gate, recv_total;     // receive: rows, sources, gates
+};
+
+switch_status_t ep_layout(const switch_config_t* c, const switch_ep_t* ep, EpLayout* L) {
+  if (c == nullptr || ep == nullptr) return SWITCH_ERR_INVALID_ARG;
+  const int G = ep->world_size;
+  if (G < 1 || G > kEpMaxRanks || ep->rank < 0 || ep->rank >= G) return SWITCH_ERR_INVALID_ARG;
+  if (c->T < 0 || c->T >= (int64_t{1} << kEpRankShift) || c->T * G > INT_MAX)
+    return SWITCH_ERR_UNSUPPORTED;
+  switch_config_t whole = *c;                 // the global batch: G ranks' tokens
+  whole.T = c->T * G;
+  int64_t C = 0;
+  switch_status_t s = validate(&whole, &C);
+  if (s != SWITCH_OK) return s;
+  if (c->dtype != SWITCH_BF16 || (c->flags & (SWITCH_FLAG_TOP2 | SWITCH_FLAG_GEMM_1SM)) ||
+      c->n_experts % G != 0)
+    return SWITCH_ERR_UNSUPPORTED;
+  *L = EpLayout{};
+  L->G = G;
+  L->r = ep->rank;
+  L->e_loc = c->n_experts / G;
+  L->T = c->T;
+  L->C = C;
+  L->nt = ntiles_of(c->T);
+  L->tc_router = use_tc_router(c);
+  L->nparts_max = static_cast<int>((c->T + 63) / 64);
+  L->nparts = L->tc_router ? L->nt : L->nparts_max;
+  const int64_t N = c->n_experts, T = c->T;
+  const int64_t S = static_cast<int64_t>(L->e_loc) * C;    // this rank's slots
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = align_up(o + (bytes ? bytes : 1), kAlign);
+    return at;
+  };
+  L->err = take(256);
+  L->hist = take(sizeof(int) * N * L->nt);
+  L->base = take(sizeof(int) * N * L->nt);
+  L->local_rank = take(sizeof(int) * T);
+  L->idx = take(sizeof(int) * T);
+  L->gate = take(sizeof(float) * T);
+  L->rank = take(sizeof(int) * T);
+  L->drop = take(T);
+  L->wsplit = take(router_wsplit_bytes(c->n_experts, c->d_model));
+  L->logits = take(L->tc_router ? 0 : sizeof(float) * N * T);
+  L->psum_cat = take(sizeof(float) * N * L->nparts * G);
+  L->counts_glob = take(sizeof(int) * N);
+  L->counts_loc = take(sizeof(int) * L->e_loc);
+  L->mtile_start = take(sizeof(int) * (L->e_loc + 1));
+  L->fpsc = take(sizeof(double) * N * kAuxChunks);
+  L->hbuf = take(2 * static_cast<size_t>(S) * c->d_ff);
+  L->total = o;
+  L->payload_counts = align_up(sizeof(float) * N * L->nparts_max, 16);
+  L->payload_total = align_up(L->payload_counts + sizeof(int) * N, 16);
+  L->recv_src = align_up(2 * static_cast<size_t>(S) * c->d_model, 256);
+  L->recv_gate = align_up(L->recv_src + sizeof(int) * S, 256);
+  L->recv_total = align_up(L->recv_gate + sizeof(float) * S, 256);
+  return SWITCH_OK;
+}
+
+// Workspace checks shared by the expert-parallel calls.
+switch_status_t ep_prepare_call(const switch_config_t* cfg, const switch_ep_t* ep, void* ws,
+                                size_t ws_bytes, void* stream, EpLayout* L, Ctx* ctx) {
+  switch_status_t s = ep_layout(cfg, ep, L);
+  if (s != SWITCH_OK || cfg->T == 0) return s;
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+    return SWITCH_ERR_INVALID_ARG;
+  if (ws_bytes < L->total) return SWITCH_ERR_WORKSPACE_TOO_SMALL;
+  ctx->C = L->C;
+  ctx->ws = static_cast<uint8_t*>(ws);
+  ctx->err = reinterpret_cast<DevErr*>(ws);
+  ctx->st = static_cast<cudaStream_t>(stream);
+  ctx->spin = cfg->spin_limit > 0 ? cfg->spin_limit : kDefaultSpinCycles;
+  ctx->num_sms = device_sms();
+  if (ctx->num_sms == 0) return SWITCH_ERR_CUDA;
+  if (ctx->num_sms < 0) return SWITCH_ERR_UNSUPPORTED;
+  return SWITCH_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -268,14 +358,18 @@ switch_status_t switch_dispatch(const switch_config_t* cfg, const int32_t* idx,
   SMOE_TRY(launch_tile_rank(A, N, idx, probs, idx ? nullptr : idx_src,
                             c.at<int>(c.L.local_rank), c.at<int>(c.L.hist), nt, c.err, c.st));
   SMOE_TRY(launch_scan(N, nt, c.at<int>(c.L.hist), c.at<int>(c.L.base), counts, c.st));
-  SMOE_TRY(launch_finalize(A, N, c.C, nt, idx_src, c.at<int>(c.L.local_rank),
-                           c.at<int>(c.L.base), counts, rank, drop, slot_token,
-                           c.at<int>(c.L.mtile_start), top2 ? cfg->T : 0, c.st));
   if (x_disp) {
+    // slots and the row copy in one pass
     const int64_t row_bytes =
         static_cast<int64_t>(cfg->d_model) * (cfg->dtype == SWITCH_BF16 ? 2 : 4);
-    SMOE_TRY(launch_gather_rows(static_cast<int64_t>(N) * c.C, row_bytes, slot_token, x,
-                                x_disp, c.st));
+    SMOE_TRY(launch_finalize_gather(A, N, c.C, nt, idx_src, c.at<int>(c.L.local_rank),
+                                    c.at<int>(c.L.base), counts, rank, drop, slot_token,
+                                    c.at<int>(c.L.mtile_start), top2 ? cfg->T : 0, x, x_disp,
+                                    row_bytes, c.st));
+  } else {
+    SMOE_TRY(launch_finalize(A, N, c.C, nt, idx_src, c.at<int>(c.L.local_rank),
+                             c.at<int>(c.L.base), counts, rank, drop, slot_token,
+                             c.at<int>(c.L.mtile_start), top2 ? cfg->T : 0, c.st));
   }
   return SWITCH_OK;
 }
@@ -417,9 +511,18 @@ switch_status_t switch_layer_forward(const switch_config_t* cfg, const void* x,
   int* slot_token = c.at<int>(c.L.slot_token);
   int* rank = c.at<int>(c.L.rank);
   uint8_t* drop = c.at<uint8_t>(c.L.drop);
-  SMOE_TRY(launch_finalize(A, N, c.C, nta, idx_p, local_rank, c.at<int>(c.L.base), counts_p,
-                           rank, drop, slot_token, c.at<int>(c.L.mtile_start),
-                           top2 ? T : 0, c.st));
+  // (bf16, default) the routed rows copied expert by expert in the same pass
+  const bool row_copy = bf16 && !(cfg->flags & SWITCH_FLAG_GATHER_IN_GEMM);
+  if (row_copy)
+    SMOE_TRY(launch_finalize_gather(A, N, c.C, nta, idx_p, local_rank, c.at<int>(c.L.base),
+                                    counts_p, rank, drop, slot_token,
+                                    c.at<int>(c.L.mtile_start), top2 ? T : 0, x,
+                                    c.ws + c.L.xdisp, static_cast<int64_t>(cfg->d_model) * 2,
+                                    c.st));
+  else
+    SMOE_TRY(launch_finalize(A, N, c.C, nta, idx_p, local_rank, c.at<int>(c.L.base), counts_p,
+                             rank, drop, slot_token, c.at<int>(c.L.mtile_start),
+                             top2 ? T : 0, c.st));
   // 4. experts, with the combine fused into the second GEMM unless asked not
   // to (or top-2: two experts write each token, so Y, then one combine)
   const bool fused = !(cfg->flags & SWITCH_FLAG_UNFUSED_COMBINE) && !top2;
@@ -447,12 +550,7 @@ switch_status_t switch_layer_forward(const switch_config_t* cfg, const void* x,
   a.num_sms = c.num_sms;
   a.pair1 = (cfg->flags & SWITCH_FLAG_GEMM_PAIRS) != 0;
   a.pair2 = !(cfg->flags & SWITCH_FLAG_GEMM_1SM);
-  if (bf16 && !(cfg->flags & SWITCH_FLAG_GATHER_IN_GEMM)) {
-    SMOE_TRY(launch_gather_rows(static_cast<int64_t>(N) * c.C,
-                                static_cast<int64_t>(a.d) * 2, slot_token, x, c.ws + c.L.xdisp,
-                                c.st));
-    a.x_disp = c.ws + c.L.xdisp;
-  }
+  if (row_copy) a.x_disp = c.ws + c.L.xdisp;
   SMOE_TRY(bf16 ? launch_expert_ffn_bf16(a, c.st) : launch_expert_ffn_f32(a, c.st));
   // 5. dropped tokens (fused) or every token (unfused)
   SMOE_TRY(launch_combine(T, cfg->d_model, c.C, bf16, x_res, idx_p, rank, drop, gate_p,
@@ -530,9 +628,9 @@ switch_status_t switch_layer_backward(const switch_config_t* cfg, const void* x,
       SMOE_TRY(launch_tile_rank(T, N, idx, nullptr, nullptr, local_rank, hist, nt, c.err, c.st));
     }
     SMOE_TRY(launch_scan(N, nt, hist, c.at<int>(c.L.base), counts, c.st));
-    SMOE_TRY(launch_finalize(T, N, c.C, nt, idx, local_rank, c.at<int>(c.L.base), counts, rank,
-                             drop, slot_token, mtile_start, 0, c.st));
-    SMOE_TRY(launch_gather_rows(S, static_cast<int64_t>(d) * 2, slot_token, x, x_disp, c.st));
+    SMOE_TRY(launch_finalize_gather(T, N, c.C, nt, idx, local_rank, c.at<int>(c.L.base), counts,
+                                    rank, drop, slot_token, mtile_start, 0, x, x_disp,
+                                    static_cast<int64_t>(d) * 2, c.st));
     FfnArgs a{};
     a.T = T;
     a.d = d;
@@ -614,6 +712,146 @@ switch_status_t switch_layer_backward(const switch_config_t* cfg, const void* x,
   SMOE_TRY(launch_bwd_dx(b, c.st));
   SMOE_TRY(launch_bwd_dropped(T, N, d, drop_list, n_drop, dh, w_r, dout, dx, residual, c.st));
   return SWITCH_OK;
+}
+
+switch_status_t switch_ep_sizes(const switch_config_t* cfg, const switch_ep_t* ep,
+                                size_t* ws_bytes, size_t* record_bytes, size_t* recv_bytes) {
+  EpLayout L{};
+  switch_status_t s = ep_layout(cfg, ep, &L);
+  if (s != SWITCH_OK) return s;
+  if (ws_bytes) *ws_bytes = L.total;
+  if (record_bytes) *record_bytes = L.payload_total;
+  if (recv_bytes) *recv_bytes = L.recv_total;
+  return SWITCH_OK;
+}
+
+switch_status_t switch_ep_route(const switch_config_t* cfg, const switch_ep_t* ep, const void* x,
+                                const float* w_r, const float* b_r, int32_t* idx, float* gate,
+                                void* record, void* ws, size_t ws_bytes, void* stream) {
+  EpLayout L{};
+  Ctx c{};
+  switch_status_t s = ep_prepare_call(cfg, ep, ws, ws_bytes, stream, &L, &c);
+  if (s != SWITCH_OK) return s;
+  if (cfg->T == 0) return SWITCH_OK;
+  if (!record || (reinterpret_cast<uintptr_t>(record) & 15u) != 0 || !x || !w_r ||
+      !aligned16(x))
+    return SWITCH_ERR_INVALID_ARG;
+  const int64_t T = cfg->T;
+  const int N = cfg->n_experts;
+  uint8_t* rec = static_cast<uint8_t*>(record);
+  int* idx_w = c.at<int>(L.idx);
+  float* gate_w = c.at<float>(L.gate);
+  int* hist = c.at<int>(L.hist);
+  int* local_rank = c.at<int>(L.local_rank);
+  float* psum = reinterpret_cast<float*>(rec);
+  SMOE_TRY(cudaMemsetAsync(rec, 0, L.payload_counts, c.st));    // unused parts stay zero
+  RouterOut o{idx_w, gate_w, nullptr, psum, nullptr, nullptr, nullptr, nullptr};
+  if (L.tc_router) {
+    o.hist = hist;
+    o.local_rank = local_rank;
+    SMOE_TRY(launch_router_tc(T, cfg->d_model, N, router_terms(cfg), x, w_r, b_r,
+                              c.ws + L.wsplit, o, L.nt, c.err, c.spin, c.num_sms, c.st));
+  } else {
+    int nparts = 0;
+    SMOE_TRY(launch_router_simt(T, cfg->d_model, N, true, x, w_r, b_r, c.at<float>(L.logits),
+                                o, &nparts, c.st));
+    SMOE_TRY(launch_tile_rank(T, N, idx_w, nullptr, nullptr, local_rank, hist, L.nt, c.err,
+                              c.st));
+  }
+  SMOE_TRY(launch_scan(N, L.nt, hist, c.at<int>(L.base),
+                       reinterpret_cast<int*>(rec + L.payload_counts), c.st));
+  if (idx) SMOE_TRY(cudaMemcpyAsync(idx, idx_w, sizeof(int) * T, cudaMemcpyDeviceToDevice, c.st));
+  if (gate)
+    SMOE_TRY(cudaMemcpyAsync(gate, gate_w, sizeof(float) * T, cudaMemcpyDeviceToDevice, c.st));
+  return SWITCH_OK;
+}
+
+switch_status_t switch_ep_dispatch(const switch_config_t* cfg, const switch_ep_t* ep,
+                                   const void* x, const void* records, void* const* recv_peers,
+                                   void* out, int32_t* counts, float* loss, void* ws,
+                                   size_t ws_bytes, void* stream) {
+  EpLayout L{};
+  Ctx c{};
+  switch_status_t s = ep_prepare_call(cfg, ep, ws, ws_bytes, stream, &L, &c);
+  if (s != SWITCH_OK || cfg->T == 0) return s;
+  if (!records || !recv_peers || (reinterpret_cast<uintptr_t>(records) & 15u) != 0)
+    return SWITCH_ERR_INVALID_ARG;
+  EpPeers peers{};
+  for (int i = 0; i < L.G; ++i) {
+    if (recv_peers[i] == nullptr || (reinterpret_cast<uintptr_t>(recv_peers[i]) & 255u) != 0)
+      return SWITCH_ERR_INVALID_ARG;
+    peers.p[i] = recv_peers[i];
+  }
+  if (!x || !out || !aligned16(x) || !aligned16(out)) return SWITCH_ERR_INVALID_ARG;
+  const int N = cfg->n_experts;
+  const int64_t T = cfg->T;
+  const EpGathered g{static_cast<const uint8_t*>(records), L.payload_total, L.payload_counts};
+  int* counts_glob = c.at<int>(L.counts_glob);
+  int* counts_loc = c.at<int>(L.counts_loc);
+  float* psum_cat = c.at<float>(L.psum_cat);
+  SMOE_TRY(launch_ep_prepare(N, L.G, L.r, L.e_loc, L.nparts, g, counts_glob, counts_loc,
+                             psum_cat, c.st));
+  SMOE_TRY(launch_mtile_table(L.e_loc, L.C, counts_loc, c.at<int>(L.mtile_start), c.st));
+  const EpRecvLayout rl{L.recv_src, L.recv_gate};
+  int* rank = c.at<int>(L.rank);
+  uint8_t* drop = c.at<uint8_t>(L.drop);
+  SMOE_TRY(launch_ep_dispatch(T, N, L.C, L.G, L.r, L.e_loc, L.nt, c.at<int>(L.idx),
+                              c.at<int>(L.local_rank), c.at<int>(L.base), c.at<float>(L.gate), g,
+                              x, static_cast<int64_t>(cfg->d_model) * 2, peers, rl, rank, drop,
+                              c.st));
+  // dropped tokens: the residual alone, on this rank
+  const void* x_res = (cfg->flags & SWITCH_FLAG_NO_RESIDUAL) ? nullptr : x;
+  SMOE_TRY(launch_combine(T, cfg->d_model, L.C, true, x_res, c.at<int>(L.idx), rank, drop,
+                          c.at<float>(L.gate), nullptr, out, true, 1, c.st));
+  if (loss)
+    SMOE_TRY(launch_aux_loss(T * L.G, N, L.nparts * L.G, cfg->alpha, counts_glob, psum_cat, loss,
+                             nullptr, nullptr, c.at<double>(L.fpsc),
+                             c.at<unsigned>(kTicketOffset), c.st));
+  if (counts)
+    SMOE_TRY(cudaMemcpyAsync(counts, counts_glob, sizeof(int) * N, cudaMemcpyDeviceToDevice,
+                             c.st));
+  return SWITCH_OK;
+}
+
+switch_status_t switch_ep_experts(const switch_config_t* cfg, const switch_ep_t* ep,
+                                  const void* w1_local, const void* w2_local, const void* recv,
+                                  void* const* out_peers, void* ws, size_t ws_bytes,
+                                  void* stream) {
+  EpLayout L{};
+  Ctx c{};
+  switch_status_t s = ep_prepare_call(cfg, ep, ws, ws_bytes, stream, &L, &c);
+  if (s != SWITCH_OK || cfg->T == 0) return s;
+  if (!w1_local || !w2_local || !recv || !out_peers || !aligned16(w1_local) ||
+      !aligned16(w2_local) || (reinterpret_cast<uintptr_t>(recv) & 255u) != 0)
+    return SWITCH_ERR_INVALID_ARG;
+  for (int i = 0; i < L.G; ++i)
+    if (out_peers[i] == nullptr || !aligned16(out_peers[i])) return SWITCH_ERR_INVALID_ARG;
+  const uint8_t* rb = static_cast<const uint8_t*>(recv);
+  FfnArgs a{};
+  a.T = static_cast<int64_t>(L.e_loc) * L.C;
+  a.d = cfg->d_model;
+  a.F = cfg->d_ff;
+  a.N = L.e_loc;
+  a.C = L.C;
+  a.x = nullptr;
+  a.x_disp = rb;
+  a.slot_token = reinterpret_cast<const int*>(rb + L.recv_src);
+  a.counts = c.at<int>(L.counts_loc);
+  a.mtile_start = c.at<int>(L.mtile_start);
+  a.w1 = w1_local;
+  a.w2 = w2_local;
+  a.hbuf = c.ws + L.hbuf;
+  a.x_res = (cfg->flags & SWITCH_FLAG_NO_RESIDUAL) ? nullptr : rb;
+  a.gate = reinterpret_cast<const float*>(rb + L.recv_gate);
+  a.mode2 = kModeCombineEp;
+  a.pair1 = (cfg->flags & SWITCH_FLAG_GEMM_PAIRS) != 0;
+  a.pair2 = true;
+  a.peer_out = out_peers;
+  a.n_peers = L.G;
+  a.err = c.err;
+  a.spin = c.spin;
+  a.num_sms = c.num_sms;
+  return cuda_status(launch_expert_ffn_bf16(a, c.st));
 }
 
 switch_status_t switch_get_device_error(void* ws, void* stream, int32_t* where_out,

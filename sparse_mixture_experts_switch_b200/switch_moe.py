@@ -39,6 +39,11 @@ class SwitchConfig(ctypes.Structure):
                 ("spin_limit", c_int64)]
 
 
+class SwitchEp(ctypes.Structure):
+    """Expert-parallel group: world_size ranks, this one `rank`."""
+    _fields_ = [("world_size", c_int32), ("rank", c_int32)]
+
+
 class SwitchError(RuntimeError):
     def __init__(self, status, where=None):
         self.status = status
@@ -80,6 +85,16 @@ def _load():
         "switch_get_device_error": (c_int32, [c_void_p, c_void_p, POINTER(c_int32),
                                               POINTER(c_int64)]),
         "switch_status_string": (c_char_p, [c_int32]),
+        "switch_ep_sizes": (c_int32, [cfgp, POINTER(SwitchEp), POINTER(c_size_t),
+                                      POINTER(c_size_t), POINTER(c_size_t)]),
+        "switch_ep_route": (c_int32, [cfgp, POINTER(SwitchEp), c_void_p, c_void_p, c_void_p,
+                                      c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
+                                      c_void_p]),
+        "switch_ep_dispatch": (c_int32, [cfgp, POINTER(SwitchEp), c_void_p, c_void_p,
+                                         POINTER(c_void_p), c_void_p, c_void_p, c_void_p,
+                                         c_void_p, c_size_t, c_void_p]),
+        "switch_ep_experts": (c_int32, [cfgp, POINTER(SwitchEp), c_void_p, c_void_p, c_void_p,
+                                        POINTER(c_void_p), c_void_p, c_size_t, c_void_p]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -203,6 +218,48 @@ def switch_layer_backward(cfg, x, w_r, b_r, w1, w2, dout, dloss, dx, dw_r, db_r,
                                       _p(w2), _p(dout), float(dloss), _p(dx), _p(dw_r),
                                       _p(db_r), _p(dw1), _p(dw2), _p(dgate), _p(ws),
                                       ws.numel(), _stream(stream)), "switch_layer_backward")
+
+
+# ----------------------------------------------------- expert parallelism
+
+def ep(world_size, rank):
+    return SwitchEp(world_size, rank)
+
+
+def switch_ep_sizes(cfg, ep_):
+    """(workspace bytes, exchange-record bytes, receive-buffer bytes)."""
+    a, b, c = c_size_t(0), c_size_t(0), c_size_t(0)
+    _check(_lib.switch_ep_sizes(ctypes.byref(cfg), ctypes.byref(ep_), ctypes.byref(a),
+                                ctypes.byref(b), ctypes.byref(c)), "switch_ep_sizes")
+    return a.value, b.value, c.value
+
+
+def _ptr_array(ptrs):
+    arr = (c_void_p * len(ptrs))()
+    for i, v in enumerate(ptrs):
+        arr[i] = v if isinstance(v, int) else _p(v)
+    return arr
+
+
+def switch_ep_route(cfg, ep_, x, w_r, b_r, idx, gate, record, ws, stream=None):
+    _check(_lib.switch_ep_route(ctypes.byref(cfg), ctypes.byref(ep_), _p(x), _p(w_r), _p(b_r),
+                                _p(idx), _p(gate), _p(record), _p(ws), ws.numel(),
+                                _stream(stream)), "switch_ep_route")
+
+
+def switch_ep_dispatch(cfg, ep_, x, records, recv_peers, out, counts, loss, ws, stream=None):
+    """recv_peers: the G ranks' receive buffers (tensors, or device addresses
+    as ints for buffers mapped from other processes)."""
+    _check(_lib.switch_ep_dispatch(ctypes.byref(cfg), ctypes.byref(ep_), _p(x), _p(records),
+                                   _ptr_array(recv_peers), _p(out), _p(counts), _p(loss),
+                                   _p(ws), ws.numel(), _stream(stream)), "switch_ep_dispatch")
+
+
+def switch_ep_experts(cfg, ep_, w1_local, w2_local, recv, out_peers, ws, stream=None):
+    """out_peers: the G ranks' outputs (tensors or device addresses)."""
+    _check(_lib.switch_ep_experts(ctypes.byref(cfg), ctypes.byref(ep_), _p(w1_local),
+                                  _p(w2_local), _p(recv), _ptr_array(out_peers), _p(ws),
+                                  ws.numel(), _stream(stream)), "switch_ep_experts")
 
 
 def switch_get_device_error(ws, stream=None):

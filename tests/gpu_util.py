@@ -8,6 +8,11 @@ Tolerances (stated once):
   flip is counted;
 * fp32 router probabilities and gates: max relative error 1e-5;
 * bf16 expert / combined outputs: max |GPU - oracle| / RMS(oracle) <= 2e-2;
+  where the output compared is the expert term alone (no residual, whose
+  values spread far beyond their RMS because the gates vary from token to
+  token), each element is first allowed the half ulp of bf16 that rounding
+  the exact value to the output dtype costs (`bf16_rms_excess`): a
+  correctly rounded element 8 RMS from zero is already up to 0.03 RMS off;
 * fp32 expert / combined outputs (fp32 FMA, no TF32): the same ratio <= 1e-5;
 * load-balancing loss: relative error 1e-5.
 """
@@ -40,6 +45,23 @@ def rms_ratio(got, want):
     want = np.asarray(want, dtype=np.float64)
     rms = np.sqrt(np.mean(want * want))
     return float(np.max(np.abs(np.asarray(got, np.float64) - want)) / max(rms, 1e-30))
+
+
+def bf16_half_ulp(want):
+    """Half a unit in the last place of bf16 (8 significant bits) at each
+    value: the most that rounding the exact value to bf16 moves it."""
+    want = np.abs(np.asarray(want, dtype=np.float64))
+    _, ex = np.frexp(want)                 # want = m 2^ex, 0.5 <= m < 1
+    return np.where(want > 0, np.ldexp(1.0, ex - 9), 0.0)
+
+
+def bf16_rms_excess(got, want):
+    """max over elements of (|got - want| - half bf16 ulp of want), over the
+    RMS of want: the error beyond the output's own rounding to bf16."""
+    want = np.asarray(want, dtype=np.float64)
+    rms = np.sqrt(np.mean(want * want))
+    err = np.abs(np.asarray(got, np.float64) - want) - bf16_half_ulp(want)
+    return float(max(np.max(err), 0.0) / max(rms, 1e-30))
 
 
 def check_routing(idx_gpu, r_oracle):

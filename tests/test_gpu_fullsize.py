@@ -12,7 +12,8 @@ Checked in full:
   holds the workload).
 
 Checked against the oracle's expert FFNs, each bound relative to the RMS of
-the quantity compared (bf16: max |err| <= 2e-2 x RMS; fp32: 1e-5):
+the quantity compared (bf16: max |err| <= 2e-2 x RMS beyond each element's
+own rounding to bf16, half an ulp; fp32: 1e-5 x RMS):
 * the expert term y = gate . E(x) alone (SWITCH_FLAG_NO_RESIDUAL), on every
   kept token of a few experts (the first, middle and last expert with kept
   tokens, and the fullest one -- so every M tile and token-tile position of
@@ -31,8 +32,8 @@ import torch
 
 import oracle.switch_oracle as orc
 from switch_inputs import WORKLOADS, make_inputs, as_f64
-from gpu_util import (dev_float, host_f64, check_routing, rel_err, rms_ratio, PROB_RTOL,
-                      BF16_RMS_TOL, F32_RMS_TOL, LOSS_RTOL)
+from gpu_util import (dev_float, host_f64, check_routing, rel_err, rms_ratio, bf16_rms_excess,
+                      PROB_RTOL, BF16_RMS_TOL, F32_RMS_TOL, LOSS_RTOL)
 
 pytestmark = pytest.mark.gpu
 
@@ -101,6 +102,8 @@ def test_fullsize_layer(sm, name):
     inp = make_inputs(wl)
     T, d, N = wl.T, wl.d_model, wl.n_experts
     tol = BF16_RMS_TOL if wl.dtype == "bf16" else F32_RMS_TOL
+    # the expert outputs alone: beyond their own rounding to bf16 (fp32: plain)
+    term_err = bf16_rms_excess if wl.dtype == "bf16" else rms_ratio
     dev = {"x": dev_float(inp.x), "w_r": dev_float(inp.w_r),
            "b_r": None if inp.b_r is None else dev_float(inp.b_r),
            "w1": dev_float(inp.w1), "w2": dev_float(inp.w2)}
@@ -159,7 +162,7 @@ def test_fullsize_layer(sm, name):
     worst_y = 0.0
     for e in experts:
         rows = host_f64(y[e * C: e * C + kept[e]])
-        ratio = rms_ratio(rows, Y_want[e])
+        ratio = term_err(rows, Y_want[e])
         assert ratio <= tol, f"staged Y of expert {e} ({kept[e]} rows): {ratio:.3e} x RMS"
         worst_y = max(worst_y, ratio)
     del y, x_disp
@@ -174,14 +177,14 @@ def test_fullsize_layer(sm, name):
         tok_e = dsp["slot_token"][e * C: e * C + kept[e]]
         want_e = g64[tok_e, None] * Y_want[e]
         rows = host_f64(out_nr[torch.from_numpy(tok_e).cuda()])
-        ratio = rms_ratio(rows, want_e)
+        ratio = term_err(rows, want_e)
         assert ratio <= tol, f"expert term of expert {e} ({kept[e]} tokens): {ratio:.3e} x RMS"
         worst_term = max(worst_term, ratio)
     others = np.array([t for t in toks if not dsp["drop"][t]])
     want_o = orc.token_outputs(inp.x, others, ig, dsp["drop"], g64, inp.w1, inp.w2,
                                residual=False)
     got_o = host_f64(out_nr[torch.from_numpy(others).cuda()])
-    assert rms_ratio(got_o, want_o) <= tol
+    assert term_err(got_o, want_o) <= tol
     dropped = np.nonzero(dsp["drop"])[0]
     if dropped.size:
         assert (out_nr[torch.from_numpy(dropped).cuda()] == 0).all()
