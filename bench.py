@@ -73,6 +73,9 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="base", choices=sorted(WORKLOADS))
+    ap.add_argument("--parallel", default="replicas", choices=["replicas", "ep"],
+                    help="N > 1: independent replicas (default), or expert parallelism "
+                         "(each rank N/G experts and its own T tokens, one routing group)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workloads", default=None,
                     help="comma-separated extra workloads timed after the headline one "
@@ -192,7 +195,7 @@ class ClockSampler:
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
     REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
-    def __init__(self, gpu_id, uuid=None, period_s=0.002):
+    def __init__(self, gpu_id, uuid=None, period_s=0.0005):
         self.gpu_id = gpu_id
         self.uuid = uuid
         self.period_s = period_s
@@ -231,12 +234,16 @@ class ClockSampler:
                 pynvml.nvmlClocksEventReasonSwThermalSlowdown,
                 pynvml.nvmlClocksEventReasonSwPowerCap)
         mx = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+        pw = 0.0
+        n = 0
         while not self.stop_evt.is_set():
             try:
                 sm = float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM))
-                pw = pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0
                 rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
-                names = [n for n, bit in zip(self.REASONS, bits) if rs & bit]
+                if n % 8 == 0:                      # power changes slowly: read it less often
+                    pw = pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0
+                n += 1
+                names = [n_ for n_, bit in zip(self.REASONS, bits) if rs & bit]
                 self.rows.append((time.time(), sm, mx, pw, names))
             except Exception:
                 pass
@@ -278,10 +285,85 @@ class ClockSampler:
 
 # ------------------------------------------------------------- GPU arm
 
+def run_expert_parallel(args):
+    """--parallel ep: the layer expert-parallel over the torchrun ranks.  Each
+    rank holds N / G experts and its own batch of the workload's T tokens
+    (weak scaling: G * T tokens in one routing group); a step is one
+    ExpertParallelSwitch.forward (route, record all-gather, dispatch with peer
+    stores, barrier, experts with the combine stored on the home ranks,
+    barrier), launched eagerly; device time by CUDA events, max over ranks."""
+    import torch
+    import torch.distributed as dist
+    from sparse_mixture_experts_switch_b200.expert_parallel import ExpertParallelSwitch
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    wl = WORKLOADS[args.workload]
+    inp = host_inputs(wl, rank)
+    T, d, F, N = wl.T, wl.d_model, wl.d_ff, wl.n_experts
+    E = N // world
+
+    def to_dev(a):
+        if a is None:
+            return None
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+    x, w_r, b_r = to_dev(inp.x), to_dev(inp.w_r), to_dev(inp.b_r)
+    w1 = to_dev(inp.w1[rank * E:(rank + 1) * E])
+    w2 = to_dev(inp.w2[rank * E:(rank + 1) * E])
+    layer = ExpertParallelSwitch(T, d, F, N, wl.capacity_factor, alpha=wl.alpha, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(max(3, args.warmup)):
+        layer.forward(x, w_r, b_r, w1, w2)
+    torch.cuda.synchronize(dev)
+    st, where, info = layer.lib.switch_get_device_error(layer.ws)
+    if st != 0:
+        raise RuntimeError(f"device error {st} at {where} ({info}) during warm-up")
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    for e0, e1 in evs:
+        flush.zero_()
+        e0.record(stream)
+        layer.forward(x, w_r, b_r, w1, w2)
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    total_ms = max_over_ranks(sum(e0.elapsed_time(e1) for e0, e1 in evs), dev, world)
+    st, where, info = layer.lib.switch_get_device_error(layer.ws)
+    if st != 0:
+        raise RuntimeError(f"device error {st} at {where} ({info}) in the timed region")
+    value = job_throughput(T, args.steps, world, total_ms)
+    if rank == 0:
+        C = layer.lib.switch_capacity(world * T, N, wl.capacity_factor)
+        print(json.dumps({
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": workload_desc(wl), "T_per_rank": T, "d_model": d,
+                       "d_ff": F, "n_experts": N, "capacity_factor": wl.capacity_factor,
+                       "capacity": C, "parallelism": f"expert parallel x{world}",
+                       "l2": "flushed (256 MiB write) before every timed step, outside the events",
+                       "launch": "eager launches of ExpertParallelSwitch.forward"},
+            "gpu_launches": 10 * args.steps}), flush=True)
+    dist.barrier()
+    dist.destroy_process_group()
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.parallel == "ep" and int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        return run_expert_parallel(args)
 
     import torch
     import torch.distributed as dist

@@ -99,10 +99,8 @@ cudaError_t launch_combine(int64_t T, int d, int64_t C, bool bf16, const void* x
 // thread keeps several independent loads in flight; the G partial sums of a
 // unit are then added in group order.
 template <bool kVec4>
-__global__ void __launch_bounds__(256) prob_colsum_kernel(int64_t T, int N,
-                                                          const float* __restrict__ probs,
-                                                          float* __restrict__ psum) {
-  __shared__ float4 red[256];
+__device__ __forceinline__ void colsum_part(int64_t T, int N, const float* __restrict__ probs,
+                                            float* __restrict__ psum, float4* red) {
   const int units = kVec4 ? N / 4 : N;
   const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kTileTok;
   const int rows = static_cast<int>(T - r0 < kTileTok ? T - r0 : kTileTok);
@@ -115,15 +113,32 @@ __global__ void __launch_bounds__(256) prob_colsum_kernel(int64_t T, int N,
     if (g < G) {
       if (kVec4) {
         const float4* col = reinterpret_cast<const float4*>(probs + r0 * N) + u;
-#pragma unroll 4
-        for (int r = g; r < rows; r += G) {
-          const float4 v = __ldg(col + static_cast<int64_t>(r) * (N / 4));
-          s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+        // up to 16 rows' loads in flight per thread, then added in row order
+        for (int r0 = g; r0 < rows; r0 += 16 * G) {
+          float4 v[16];
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            const int r = r0 + k * G;
+            v[k] = r < rows ? __ldg(col + static_cast<int64_t>(r) * (N / 4))
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            s.x += v[k].x; s.y += v[k].y; s.z += v[k].z; s.w += v[k].w;
+          }
         }
       } else {
         const float* col = probs + r0 * N + u;
-#pragma unroll 4
-        for (int r = g; r < rows; r += G) s.x += __ldg(col + static_cast<int64_t>(r) * N);
+        for (int r0 = g; r0 < rows; r0 += 16 * G) {
+          float v[16];
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            const int r = r0 + k * G;
+            v[k] = r < rows ? __ldg(col + static_cast<int64_t>(r) * N) : 0.f;
+          }
+#pragma unroll
+          for (int k = 0; k < 16; ++k) s.x += v[k];
+        }
       }
     }
     red[threadIdx.x] = s;
@@ -140,6 +155,14 @@ __global__ void __launch_bounds__(256) prob_colsum_kernel(int64_t T, int N,
     }
     __syncthreads();
   }
+}
+
+template <bool kVec4>
+__global__ void __launch_bounds__(256) prob_colsum_kernel(int64_t T, int N,
+                                                          const float* __restrict__ probs,
+                                                          float* __restrict__ psum) {
+  __shared__ float4 red[256];
+  colsum_part<kVec4>(T, N, probs, psum, red);
 }
 
 cudaError_t launch_prob_colsum(int64_t T, int N, const float* probs, float* psum,
@@ -225,6 +248,85 @@ cudaError_t launch_aux_loss(int64_t T, int N, int nparts, float alpha, const int
   const dim3 grid(static_cast<unsigned>((N + 31) / 32), static_cast<unsigned>(chunks));
   aux_loss_kernel<<<grid, 256, 0, st>>>(T, N, nparts, alpha, counts, psum, loss, f, P,
                                         part_sum, ticket);
+  return cudaGetLastError();
+}
+
+// The staged loss from full probabilities in one launch: block b sums part b
+// (128 rows, fixed order) into psum[b]; the last block of each of the
+// kAuxChunks runs of parts (a per-run ticket picks which block, not any
+// order of additions) adds the run's parts in order in double into
+// part_sum[run]; the last run to finish forms f_e P_e and the loss in a
+// fixed tree.  Tickets are left at zero for the next call.
+template <bool kVec4>
+__global__ void __launch_bounds__(256) aux_loss_probs_kernel(
+    int64_t T, int N, float alpha, const int* __restrict__ counts,
+    const float* __restrict__ probs, float* __restrict__ psum, float* __restrict__ loss,
+    float* __restrict__ f_out, float* __restrict__ P_out, double* __restrict__ part_sum,
+    unsigned* __restrict__ run_ticket, unsigned* __restrict__ ticket) {
+  __shared__ float4 red4[256];
+  __shared__ double red[256];
+  __shared__ bool last;
+  colsum_part<kVec4>(T, N, probs, psum, red4);
+  const int nparts = static_cast<int>(gridDim.x);
+  const int per = (nparts + kAuxChunks - 1) / kAuxChunks;   // parts per run
+  const int nruns = (nparts + per - 1) / per;                // runs that hold parts
+  const int run = static_cast<int>(blockIdx.x) / per;
+  const int p0 = run * per;
+  const int p1 = p0 + per < nparts ? p0 + per : nparts;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) last = atomicAdd(&run_ticket[run], 1u) == static_cast<unsigned>(p1 - p0 - 1);
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  for (int e = threadIdx.x; e < N; e += 256) {
+    double tot = 0.0;
+    for (int pp = p0; pp < p1; ++pp)
+      tot += static_cast<double>(__ldcg(psum + static_cast<int64_t>(pp) * N + e));
+    part_sum[static_cast<int64_t>(run) * N + e] = tot;
+  }
+  if (threadIdx.x == 0) run_ticket[run] = 0;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) last = atomicAdd(ticket, 1u) == static_cast<unsigned>(nruns - 1);
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  double acc = 0.0;
+  for (int i = threadIdx.x; i < N; i += 256) {
+    double tot = 0.0;
+    for (int c = 0; c < nruns; ++c) tot += __ldcg(part_sum + static_cast<int64_t>(c) * N + i);
+    const double P = tot / static_cast<double>(T);
+    const double f = static_cast<double>(counts[i]) / static_cast<double>(T);
+    if (f_out) f_out[i] = static_cast<float>(f);
+    if (P_out) P_out[i] = static_cast<float>(P);
+    acc += f * P;
+  }
+  red[threadIdx.x] = acc;
+  __syncthreads();
+  for (int st = 128; st > 0; st >>= 1) {
+    if (threadIdx.x < st) red[threadIdx.x] += red[threadIdx.x + st];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    if (loss) *loss = static_cast<float>(static_cast<double>(alpha) * N * red[0]);
+    *ticket = 0;
+  }
+}
+
+cudaError_t launch_aux_loss_probs(int64_t T, int N, float alpha, const int* counts,
+                                  const float* probs, float* psum, float* loss, float* f,
+                                  float* P, double* part_sum, unsigned* run_ticket,
+                                  unsigned* ticket, cudaStream_t st) {
+  const unsigned grid = static_cast<unsigned>((T + kTileTok - 1) / kTileTok);
+  const bool vec4 = (N % 4) == 0 && (reinterpret_cast<uintptr_t>(probs) & 15u) == 0 &&
+                    (reinterpret_cast<uintptr_t>(psum) & 15u) == 0;
+  if (vec4)
+    aux_loss_probs_kernel<true><<<grid, 256, 0, st>>>(T, N, alpha, counts, probs, psum, loss, f,
+                                                       P, part_sum, run_ticket, ticket);
+  else
+    aux_loss_probs_kernel<false><<<grid, 256, 0, st>>>(T, N, alpha, counts, probs, psum, loss, f,
+                                                        P, part_sum, run_ticket, ticket);
   return cudaGetLastError();
 }
 

@@ -535,6 +535,18 @@ __device__ __forceinline__ void prefetch_l2(const void* p) {
 // Raise a kernel's dynamic shared-memory limit to `bytes`, once per kernel
 // and device (steady-state calls then launch with no extra driver call).
 // `cache` is a per-kernel array of 64 entries, one per device.
+// Programmatic dependent launch: a kernel launched with the programmatic
+// stream-serialization attribute may start while the previous kernel on the
+// stream still runs, once that kernel has signalled launch_dependents; a
+// thread that reads the previous kernel's results first waits for it to
+// complete (both are no-ops for kernels launched the ordinary way).
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait_prerequisites() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 inline cudaError_t ensure_smem_limit(const void* func, size_t bytes, size_t* cache) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);

@@ -204,12 +204,17 @@ cudaError_t launch_finalize(int64_t T, int N, int64_t C, int ntiles, const int* 
   return cudaGetLastError();
 }
 
-// finalize_kernel and the row copy in one pass, one warp per item: items
-// 0 .. T-1 are assignments (lane 0 decides rank / drop / slot, the warp
-// copies the row into its slot), items T .. T + N*C - 1 are slots (a
-// padding slot gets -1 and a zero row).  Slot order, and so every output,
-// is the same as finalize_kernel's followed by gather_rows_kernel's.
-__global__ void __launch_bounds__(256) finalize_gather_kernel(
+// finalize_kernel and the row copy in one pass.  Items 0 .. T-1 are
+// assignments, items T .. T + N*C - 1 are slots.  A warp takes kGatherGroup
+// consecutive items: lane j < kGatherGroup decides item j as finalize_kernel
+// does (an assignment's rank, drop and slot; a padding slot's -1), so those
+// metadata loads are in flight together; then the warp copies the items'
+// rows one after another (16 bytes per lane per access): a kept token's row
+// into its slot, zeros into a padding slot.  Groups are small so that many
+// warps per SM each have a row in flight.
+constexpr int kGatherGroup = 8;
+
+__global__ void __launch_bounds__(256, 4) finalize_gather_kernel(
     int64_t T, int N, int64_t C, int ntiles, const int* __restrict__ idx,
     const int* __restrict__ local_rank, const int* __restrict__ base,
     const int* __restrict__ counts, int* __restrict__ rank, uint8_t* __restrict__ drop,
@@ -219,44 +224,58 @@ __global__ void __launch_bounds__(256) finalize_gather_kernel(
     mtile_prefix_warp(N, C, counts, mtile_start);
   const int lane = threadIdx.x & 31;
   const int64_t nslots = static_cast<int64_t>(N) * C;
+  const int64_t items = T + nslots;
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
-       i < T + nslots; i += warps) {
+  for (int64_t g0 = (static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5)) *
+                    kGatherGroup;
+       g0 < items; g0 += warps * kGatherGroup) {
+    const int64_t i = lane < kGatherGroup ? g0 + lane : items;   // other lanes: no item
+    int64_t dst = -1;        // x_disp row this lane's item writes
+    int64_t src = -1;        // x row copied into it (-1: zeros)
     if (i < T) {
-      int64_t slot = -1;
-      const int64_t tok = tok_mod > 0 && i >= tok_mod ? i - tok_mod : i;
-      if (lane == 0) {
-        const int e = idx[i];
-        const int lr = local_rank[i];
-        int r = -1;
-        bool dropped = true;
-        if (e >= 0 && e < N && lr >= 0) {
-          r = base[static_cast<int64_t>(e) * ntiles + (i / kTileTok)] + lr;
-          dropped = r >= C;
-          if (!dropped) {
-            slot = static_cast<int64_t>(e) * C + r;
-            slot_token[slot] = static_cast<int>(tok);
-          }
+      const int e = idx[i];
+      const int lr = local_rank[i];
+      int r = -1;
+      bool dropped = true;
+      if (e >= 0 && e < N && lr >= 0) {
+        r = base[static_cast<int64_t>(e) * ntiles + (i / kTileTok)] + lr;
+        dropped = r >= C;
+        if (!dropped) {
+          const int64_t tok = tok_mod > 0 && i >= tok_mod ? i - tok_mod : i;
+          dst = static_cast<int64_t>(e) * C + r;
+          src = tok;
+          slot_token[dst] = static_cast<int>(tok);
         }
-        rank[i] = r;
-        drop[i] = dropped ? 1 : 0;
       }
-      slot = __shfl_sync(0xffffffffu, slot, 0);
-      if (slot >= 0) {
-        const uint4* src = x + tok * vec_per_row;
-        uint4* dst = x_disp + slot * vec_per_row;
-        for (int64_t v = lane; v < vec_per_row; v += 32) dst[v] = __ldg(src + v);
-      }
-    } else {
+      rank[i] = r;
+      drop[i] = dropped ? 1 : 0;
+    } else if (i < items) {
       const int64_t s = i - T;
       const int e = static_cast<int>(s / C);
       const int64_t r = s - static_cast<int64_t>(e) * C;
       const int64_t kept = counts[e] < C ? counts[e] : C;
       if (r >= kept) {
-        if (lane == 0) slot_token[s] = -1;
-        uint4* dst = x_disp + s * vec_per_row;
-        for (int64_t v = lane; v < vec_per_row; v += 32) dst[v] = make_uint4(0, 0, 0, 0);
+        slot_token[s] = -1;
+        dst = s;
       }
+    }
+    // the group's rows side by side: every lane has one 16-byte load of each
+    // row in flight before it stores any of them
+    int d_j[kGatherGroup], s_j[kGatherGroup];          // row ids fit int32 (validated)
+#pragma unroll
+    for (int j = 0; j < kGatherGroup; ++j) {
+      d_j[j] = __shfl_sync(0xffffffffu, static_cast<int>(dst), j);
+      s_j[j] = __shfl_sync(0xffffffffu, static_cast<int>(src), j);
+    }
+    for (int64_t v = lane; v < vec_per_row; v += 32) {
+      uint4 val[kGatherGroup];
+#pragma unroll
+      for (int j = 0; j < kGatherGroup; ++j)
+        val[j] = (d_j[j] >= 0 && s_j[j] >= 0) ? __ldg(x + static_cast<int64_t>(s_j[j]) * vec_per_row + v)
+                                              : make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int j = 0; j < kGatherGroup; ++j)
+        if (d_j[j] >= 0) x_disp[static_cast<int64_t>(d_j[j]) * vec_per_row + v] = val[j];
     }
   }
 }
@@ -267,7 +286,7 @@ cudaError_t launch_finalize_gather(int64_t T, int N, int64_t C, int ntiles, cons
                                    int64_t tok_mod, const void* x, void* x_disp,
                                    int64_t row_bytes, cudaStream_t st) {
   const int64_t items = T + static_cast<int64_t>(N) * C;
-  int64_t blocks = (items + 7) / 8;
+  int64_t blocks = (items + 8 * kGatherGroup - 1) / (8 * kGatherGroup);   // 8 warps a block
   if (blocks > 148 * 8) blocks = 148 * 8;
   if (blocks < 1) blocks = 1;
   finalize_gather_kernel<<<static_cast<int>(blocks), 256, 0, st>>>(

@@ -59,6 +59,14 @@ cudaError_t launch_aux_loss(int64_t T, int N, int nparts, float alpha, const int
                             const float* psum, float* loss, float* f, float* P,
                             double* part_sum, unsigned* ticket, cudaStream_t st);
 
+// The loss from full probabilities [T, N] in one launch (column sums per
+// 128-row part into psum, then as launch_aux_loss).  run_ticket:
+// kAuxChunks zero-initialised counters, ticket: one (all left zero).
+cudaError_t launch_aux_loss_probs(int64_t T, int N, float alpha, const int* counts,
+                                  const float* probs, float* psum, float* loss, float* f,
+                                  float* P, double* part_sum, unsigned* run_ticket,
+                                  unsigned* ticket, cudaStream_t st);
+
 // ---------------------------------------------------------------- router
 struct RouterOut {
   int* idx;          // [T]

@@ -190,6 +190,9 @@ cudaError_t launch_router_simt(int64_t T, int d, int N, bool bf16, const void* x
 // so one accumulator chunk of 32 x terms columns holds all of them).
 __global__ void wsplit_kernel(int N, int N_pad, int d, int terms, bool interleave,
                               const float* __restrict__ w_r, __nv_bfloat16* __restrict__ out) {
+  // the router that follows may start its prologue and its x loads now; it
+  // waits for this kernel before it reads the split
+  pdl_launch_dependents();
   const int64_t n = static_cast<int64_t>(N_pad) * d;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -577,13 +580,15 @@ __global__ void __launch_bounds__(kRouterThreads, 1) router_tc_kernel(
 // B operand, Nt = terms x N_pad; with two terms, one term per CTA).  The
 // leader issues tcgen05.mma.cta_group::2 (M = 256, N = Nt, K = 16); each
 // CTA's TMEM receives its 128 tokens x all Nt columns.  Every SM streams 16 KB
-// of x and Nt/2 x 128 B of weights per 64-deep K step through a six-stage
-// ring.  Two TMEM accumulators alternate between tiles, each drained by its
-// own group of four epilogue warps, so the softmax of one tile overlaps the
-// main loop of the next.
+// of x and Nt/2 x 128 B of weights per 64-deep K step.  x comes from DRAM
+// and the weights from L2, so they have rings of their own: a deep one for x
+// (the bytes in flight that DRAM's latency needs) and a shallow one for the
+// weights, each filled by its own producer thread.  Two TMEM accumulators
+// alternate between tiles; all eight epilogue warps drain every tile, so the
+// softmax of one tile overlaps the main loop of the next.
 struct RouterPairParams {
   int64_t T;
-  int d, N, N_pad, ntiles, npairs, stages;
+  int d, N, N_pad, ntiles, npairs, xstages, wstages;
   uint32_t x_bytes, w_bytes;       // per stage and CTA
   int w_half_rows;
   const float* b_r;
@@ -592,23 +597,28 @@ struct RouterPairParams {
   long long spin;
 };
 
-constexpr int kRouterPairMaxStages = 8;
+constexpr int kRouterPairMaxXStages = 12;
+constexpr int kRouterPairMaxWStages = 10;
+// warp 0 x producer, warp 1 MMA, warp 2 weight producer, warps 3-10 epilogue
+constexpr int kRouterPairThreads = 96 + 256;
 
 template <int NCH, int TERMS>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kRouterThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kRouterPairThreads, 1)
     router_pair_kernel(const __grid_constant__ CUtensorMap tmap_x,
                        const __grid_constant__ CUtensorMap tmap_w, RouterPairParams prm) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-  const int STAGES = prm.stages;
-  const uint32_t stage_bytes = prm.x_bytes + prm.w_bytes;
+  const int XST = prm.xstages, WST = prm.wstages;
   const int N = prm.N, N_pad = prm.N_pad;
   constexpr int NT = NCH * 32 * TERMS;                   // accumulator columns per tile
-  uint8_t* tail = smem + static_cast<size_t>(STAGES) * stage_bytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(tail);    // leader: bytes of both CTAs
-  uint64_t* empty = full + kRouterPairMaxStages;         // local: stage consumed
-  uint64_t* tfull = empty + kRouterPairMaxStages;        // local: accumulator g ready
+  uint8_t* wring = smem + static_cast<size_t>(XST) * prm.x_bytes;
+  uint8_t* tail = wring + static_cast<size_t>(WST) * prm.w_bytes;
+  uint64_t* xfull = reinterpret_cast<uint64_t*>(tail);   // leader: x bytes of both CTAs
+  uint64_t* xempty = xfull + kRouterPairMaxXStages;      // local: x stage consumed
+  uint64_t* wfull = xempty + kRouterPairMaxXStages;      // leader: weight bytes of both CTAs
+  uint64_t* wempty = wfull + kRouterPairMaxWStages;      // local: weight stage consumed
+  uint64_t* tfull = wempty + kRouterPairMaxWStages;      // local: accumulator g ready
   uint64_t* tempty = tfull + 2;                          // leader: accumulator g drained
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
@@ -632,9 +642,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kRouterThreads, 1)
   const long long lim = prm.spin;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+    for (int s = 0; s < XST; ++s) {
+      mbar_init(&xfull[s], 1);
+      mbar_init(&xempty[s], 1);
+    }
+    for (int s = 0; s < WST; ++s) {
+      mbar_init(&wfull[s], 1);
+      mbar_init(&wempty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
@@ -658,30 +672,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kRouterThreads, 1)
   cluster_sync();                          // the peer's barriers exist before any remote use
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
-  const uint32_t full_lead = map_to_rank(smem_u32(full), 0);
+  const uint32_t xfull_lead = map_to_rank(smem_u32(xfull), 0);
+  const uint32_t wfull_lead = map_to_rank(smem_u32(wfull), 0);
   const uint32_t tempty_lead = map_to_rank(smem_u32(tempty), 0);
 
-  if (warp == 0) {
-    // ------------------------------------------------------- TMA producer
+  if (warp == 0 || warp == 2) {
+    // ------------------------------------------- TMA producers (x; weights)
     if (lane == 0) {
-      tma_prefetch_desc(&tmap_x);
-      tma_prefetch_desc(&tmap_w);
+      const bool is_x = warp == 0;
+      const int nst = is_x ? XST : WST;
+      uint64_t* fullb = is_x ? xfull : wfull;
+      uint64_t* emptyb = is_x ? xempty : wempty;
+      const uint32_t full_lead = is_x ? xfull_lead : wfull_lead;
+      const uint32_t bytes = is_x ? prm.x_bytes : prm.w_bytes;
+      uint8_t* ring = is_x ? smem : wring;
+      tma_prefetch_desc(is_x ? &tmap_x : &tmap_w);
+      // the weight split is the previous kernel's output (launched as a
+      // programmatic dependent of it, this kernel may be running already)
+      if (!is_x) pdl_wait_prerequisites();
       int stage = 0;
       uint32_t phase = 0, issued_mask = 0, issued_phase = 0;
       bool ok = true;
       for (int pt = cid; pt < prm.npairs && ok && !*abort_flag; pt += ncl) {
-        const int xrow = pt * 256 + static_cast<int>(rank) * 128;
+        const int row = is_x ? pt * 256 + static_cast<int>(rank) * 128
+                             : static_cast<int>(rank) * prm.w_half_rows;
         for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, lim)) { ok = false; break; }
-          uint8_t* sx = smem + static_cast<size_t>(stage) * stage_bytes;
-          const uint32_t bar = full_lead + 8u * stage;
-          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * stage_bytes);
-          tma_load_2d_pair(sx, &tmap_x, bar, kb * 64, xrow);
-          tma_load_2d_pair(sx + prm.x_bytes, &tmap_w, bar, kb * 64,
-                           static_cast<int>(rank) * prm.w_half_rows);
+          if (!mbar_wait(&emptyb[stage], phase ^ 1u, lim)) { ok = false; break; }
+          if (leader) mbar_arrive_expect_tx(&fullb[stage], 2 * bytes);
+          tma_load_2d_pair(ring + static_cast<size_t>(stage) * bytes, is_x ? &tmap_x : &tmap_w,
+                           full_lead + 8u * stage, kb * 64, row);
           issued_mask |= 1u << stage;
           issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          if (++stage == nst) { stage = 0; phase ^= 1u; }
         }
       }
       if (!ok) {
@@ -691,17 +713,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kRouterThreads, 1)
       // Both CTAs' bytes land on the leader's barriers: the leader waits for
       // every issued stage before the final cluster barrier.
       if (leader)
-        for (int s = 0; s < STAGES; ++s)
+        for (int s = 0; s < nst; ++s)
           if (((issued_mask >> s) & 1u) &&
-              !mbar_wait_cluster(&full[s], (issued_phase >> s) & 1u, kDefaultSpinCycles))
+              !mbar_wait_cluster(&fullb[s], (issued_phase >> s) & 1u, kDefaultSpinCycles))
             report_error(prm.err, SWITCH_ERR_TIMEOUT, kWhereDrain, s);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer
     if (leader && lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(256, NT);
-      int stage = 0;
-      uint32_t phase = 0;
+      int xs = 0, ws = 0;
+      uint32_t xph = 0, wph = 0;
       bool ok = true, any = false;
       int li = 0;                                        // local tile count
       for (int pt = cid; pt < prm.npairs && ok && !*abort_flag; pt += ncl, ++li) {
@@ -711,17 +733,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kRouterThreads, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * 256);
         for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait_cluster(&full[stage], phase, lim)) { ok = false; break; }
+          if (!mbar_wait_cluster(&xfull[xs], xph, lim) ||
+              !mbar_wait_cluster(&wfull[ws], wph, lim)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t sx = smem_u32(smem + static_cast<size_t>(stage) * stage_bytes);
-          const uint64_t xd = sw128_kmajor_desc(sx);
-          const uint64_t wd = sw128_kmajor_desc(sx + prm.x_bytes);
+          const uint64_t xd = sw128_kmajor_desc(smem_u32(smem + static_cast<size_t>(xs) * prm.x_bytes));
+          const uint64_t wd = sw128_kmajor_desc(smem_u32(wring + static_cast<size_t>(ws) * prm.w_bytes));
 #pragma unroll
           for (int k = 0; k < 4; ++k)
             umma_bf16_pair(d_tmem, xd + 2 * k, wd + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
           any = true;
-          umma_commit_pair(&empty[stage], 0x3);
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          umma_commit_pair(&xempty[xs], 0x3);
+          umma_commit_pair(&wempty[ws], 0x3);
+          if (++xs == XST) { xs = 0; xph ^= 1u; }
+          if (++ws == WST) { ws = 0; wph ^= 1u; }
         }
         if (!ok) break;
         umma_commit_pair(&tfull[acc], 0x3);
@@ -747,9 +771,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kRouterThreads, 1)
     // with the tile's parity.
     constexpr int NH = (NCH + 1) / 2;                  // chunks per half
     const int q = warp & 3;
-    const int h = (warp - 2) >> 2;
+    const int h = (warp - 3) >> 2;
     const int row = q * 32 + lane;
-    const int et = threadIdx.x - 64;                   // 0 .. 255
+    const int et = threadIdx.x - 96;                   // 0 .. 255
     const int N_h = N - h * NH * 32;                   // experts of this half (may be <= 0)
     int li = 0;
     for (int pt = cid; pt < prm.npairs; pt += ncl, ++li) {
@@ -781,19 +805,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kRouterThreads, 1)
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(acc * 256);
       if (here) {
+        // every TMEM load of this thread's logits in flight at once, one wait
+        uint32_t r[NH][TERMS][32];
 #pragma unroll
         for (int cc = 0; cc < NH; ++cc) {
           const int c = h * NH + cc;
 #pragma unroll
-          for (int p = 0; p < TERMS; ++p) {
-            uint32_t r[32];
-            if (c < NCH) {                                // warp-uniform
-              tmem_ld32_issue(taddr + static_cast<uint32_t>((c * TERMS + p) * 32), r);
-              tmem_ld_wait(r);
-            }
+          for (int p = 0; p < TERMS; ++p)
+            if (c < NCH)                                  // warp-uniform
+              tmem_ld32_issue(taddr + static_cast<uint32_t>((c * TERMS + p) * 32), r[cc][p]);
+        }
+        // (the first wait covers every load; each call also orders its array's
+        // register uses after the wait)
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              v[cc * 32 + j] = p == 0 ? __uint_as_float(r[j]) : v[cc * 32 + j] + __uint_as_float(r[j]);
+        for (int cc = 0; cc < NH; ++cc)
+#pragma unroll
+          for (int p = 0; p < TERMS; ++p)
+            if (h * NH + cc < NCH) tmem_ld_wait(r[cc][p]);
+#pragma unroll
+        for (int cc = 0; cc < NH; ++cc) {
+          const int c = h * NH + cc;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            float a = __uint_as_float(r[cc][0][j]);
+#pragma unroll
+            for (int p = 1; p < TERMS; ++p) a += __uint_as_float(r[cc][p][j]);
+            v[cc * 32 + j] = a;
           }
           if (prm.b_r != nullptr)
 #pragma unroll
@@ -995,8 +1032,19 @@ static cudaError_t run_router_pair_t(const CUtensorMap& tx, const CUtensorMap& t
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(&router_pair_kernel<NCH, TERMS>),
                                     smem, smem_set);
   if (e != cudaSuccess) return e;
-  router_pair_kernel<NCH, TERMS><<<grid, kRouterThreads, smem, st>>>(tx, tw, p);
-  return cudaGetLastError();
+  // launched as a programmatic dependent of the weight split: its prologue,
+  // TMEM allocation and first x loads overlap that kernel
+  cudaLaunchConfig_t lc{};
+  lc.gridDim = dim3(grid);
+  lc.blockDim = dim3(kRouterPairThreads);
+  lc.dynamicSmemBytes = smem;
+  lc.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  return cudaLaunchKernelEx(&lc, router_pair_kernel<NCH, TERMS>, tx, tw, p);
 }
 
 // CTA-pair router: terms x N_pad <= 256.
@@ -1022,18 +1070,23 @@ static cudaError_t launch_router_pair(int64_t T, int d, int N, int N_pad, int te
   const size_t tail_bytes =
       512 + sizeof(float) * N_pad * 9 + sizeof(int) * N_pad * 8 + 5 * sizeof(float) * 512;
   const size_t budget = 227 * 1024 - 1024 - tail_bytes;
-  int stages = static_cast<int>(budget / (p.x_bytes + p.w_bytes));
-  if (stages > kRouterPairMaxStages) stages = kRouterPairMaxStages;
-  if (stages < 2) return cudaErrorInvalidConfiguration;
-  p.stages = stages;
+  // x comes from DRAM: eight 16 KB stages (128 KB in flight per SM); the
+  // weights from L2, whose latency under this load is still microseconds:
+  // the rest of shared memory (the same bytes per K step as x)
+  int xst = 8;
+  int wst = static_cast<int>((budget - static_cast<size_t>(xst) * p.x_bytes) / p.w_bytes);
+  if (wst > kRouterPairMaxWStages) wst = kRouterPairMaxWStages;
+  if (wst < 2) return cudaErrorInvalidConfiguration;
+  p.xstages = xst;
+  p.wstages = wst;
   CUtensorMap tx, tw;
   if (!make_tmap_bf16_2d(&tx, x, static_cast<uint64_t>(d), static_cast<uint64_t>(T), 64, 128))
     return cudaErrorInvalidValue;
   if (!make_tmap_bf16_2d(&tw, wsplit, static_cast<uint64_t>(d), static_cast<uint64_t>(nt), 64,
                          static_cast<uint32_t>(nt / 2)))
     return cudaErrorInvalidValue;
-  const size_t smem =
-      1024 + static_cast<size_t>(stages) * (p.x_bytes + p.w_bytes) + tail_bytes;
+  const size_t smem = 1024 + static_cast<size_t>(xst) * p.x_bytes +
+                      static_cast<size_t>(wst) * p.w_bytes + tail_bytes;
   int clusters = num_sms / 2;
   if (clusters > p.npairs) clusters = p.npairs;
   if (clusters < 1) clusters = 1;

@@ -51,6 +51,10 @@ struct Layout {
 // Bytes 16..19 of the workspace: the loss kernel's completion ticket (kept
 // at zero between calls, like the error word in bytes 0..15).
 constexpr size_t kTicketOffset = 16;
+// Bytes 32 .. 32 + 4 kAuxChunks: the staged loss's per-run tickets (also
+// left at zero).
+constexpr size_t kRunTicketOffset = 32;
+static_assert(kRunTicketOffset + 4 * kAuxChunks <= 256, "tickets live in the first 256 bytes");
 
 int ntiles_of(int64_t T) { return static_cast<int>((T + kTileTok - 1) / kTileTok); }
 
@@ -442,10 +446,10 @@ switch_status_t switch_aux_loss(const switch_config_t* cfg, const int32_t* count
   if (s != SWITCH_OK || cfg->T == 0) return s;
   if (!counts || !probs || !loss) return SWITCH_ERR_INVALID_ARG;
   float* psum = c.at<float>(c.L.psum);
-  SMOE_TRY(launch_prob_colsum(cfg->T, cfg->n_experts, probs, psum, c.st));
-  return cuda_status(launch_aux_loss(cfg->T, cfg->n_experts, ntiles_of(cfg->T), cfg->alpha,
-                                     counts, psum, loss, f, P, c.at<double>(c.L.fpsc),
-                                     c.at<unsigned>(kTicketOffset), c.st));
+  return cuda_status(launch_aux_loss_probs(cfg->T, cfg->n_experts, cfg->alpha, counts, probs,
+                                           psum, loss, f, P, c.at<double>(c.L.fpsc),
+                                           c.at<unsigned>(kRunTicketOffset),
+                                           c.at<unsigned>(kTicketOffset), c.st));
 }
 
 switch_status_t switch_layer_forward(const switch_config_t* cfg, const void* x,
