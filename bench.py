@@ -42,11 +42,11 @@ L2_FLUSH_BYTES = 256 << 20
 # taken on: the bench reports them as `traffic` while the sources hash the
 # same, and null once a kernel has changed.
 GEMM_SOURCES = ("common.cuh", "gemm_common.cuh", "gemm_pair.cuh", "expert_ffn.cu",
-                "expert_ffn_pair.cu")
+                "expert_ffn_pair.cu", "expert_ffn_pair_rows.cu")
 GEMM_TRAFFIC = {"workload": "base",
-                "sources_sha256": "97b31444528b771321d3264df6e72bf3e7d38276351d33b290eca56557619e16",
-                # GEMM1 715.9 MB read + 370.8 MB written; GEMM2 1231.7 + 89.1 MB
-                "bytes": 715.932160e6 + 370.764288e6 + 1231.664896e6 + 89.147392e6}
+                "sources_sha256": "f115382257c4210eec65746c4eb1247239b854e35d34c5d5ea0879661d8ffed6",
+                # GEMM1 715.8 MB read + 367.7 MB written; GEMM2 1231.6 + 89.2 MB
+                "bytes": 715.76e6 + 367.73e6 + 1231.59e6 + 89.25e6}
 
 
 def gemm_sources_sha256():
@@ -79,7 +79,7 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workloads", default=None,
                     help="comma-separated extra workloads timed after the headline one "
-                         "('all' = every bf16 workload; default: all at N=1, none at N>1)")
+                         "('all' = every bf16 workload, 'none'; default: all at N=1, none at N>1)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="budget of the oracle sample timed for cpu_baseline")
     return ap.parse_args()
@@ -589,6 +589,11 @@ def extra_workloads(args, world, headline):
         names = args.workloads
     if names == "all":
         names = ",".join(n for n, w in WORKLOADS.items() if w.dtype == "bf16")
+    if names == "none":
+        return []
+    unknown = [n for n in names.split(",") if n and n not in WORKLOADS]
+    if unknown:
+        raise SystemExit(f"unknown workloads: {unknown}")
     return [n for n in names.split(",") if n and n != headline]
 
 

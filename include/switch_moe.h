@@ -85,9 +85,12 @@ enum {
   SWITCH_FLAG_ROWS_DISPATCHED = 128, /* switch_expert_ffn: x is the dispatched row buffer
                                         x_disp [N*C, d_model] from switch_dispatch */
   SWITCH_FLAG_TOP2 = 512,            /* top-k routing with k = 2 (see "Top-2 routing" below) */
-  SWITCH_FLAG_TRAINING = 1024        /* forward keeps what switch_layer_backward needs in the
+  SWITCH_FLAG_TRAINING = 1024,       /* forward keeps what switch_layer_backward needs in the
                                         workspace; the backward then reads it instead of
                                         recomputing (see switch_layer_backward) */
+  SWITCH_FLAG_GEMM1_ROWS_PAIRS = 2048 /* bf16 GEMM1 on CTA pairs with 256 dispatched rows x 256
+                                        columns per tile (needs the row copy: not with
+                                        SWITCH_FLAG_GATHER_IN_GEMM) */
 };
 
 typedef struct {

@@ -342,8 +342,9 @@ cudaError_t launch_expert_ffn_bf16(const FfnArgs& a, cudaStream_t st) {
   const uint64_t slots = static_cast<uint64_t>(a.N) * static_cast<uint64_t>(a.C);
   CUtensorMap ta1, tb1, ta2, tb2, to1, to2;
   const bool gather = a.x_disp == nullptr;
+  const bool rows1 = a.pair1_rows && !gather;   // row-major pairs read rows by TMA only
   // CTA pairs load half a weight tile each (128 rows); single CTAs all 256.
-  const uint32_t b_rows1 = a.pair1 ? 128u : static_cast<uint32_t>(kBN);
+  const uint32_t b_rows1 = (a.pair1 || rows1) ? 128u : static_cast<uint32_t>(kBN);
   const uint32_t b_rows2 = a.pair2 ? 128u : static_cast<uint32_t>(kBN);
   bool ok = true;
   if (gather)
@@ -377,7 +378,9 @@ cudaError_t launch_expert_ffn_bf16(const FfnArgs& a, cudaStream_t st) {
   g1.err = a.err;
   g1.spin = a.spin;
   cudaError_t e;
-  if (a.pair1)
+  if (rows1)
+    e = run_gemm_pair_rows(ta1, tb1, to1, g1, a.num_sms, st);
+  else if (a.pair1)
     e = gather ? run_gemm_pair<true>(ta1, tb1, to1, g1, a.num_sms, st)
                : run_gemm_pair<false>(ta1, tb1, to1, g1, a.num_sms, st);
   else

@@ -198,6 +198,13 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, const CUtenso
   }
 }
 
+// Row-major CTA-pair kernel launcher (expert_ffn_pair_rows.cu): 256-row x
+// 256-column tiles of row-contiguous operands (no gather).
+cudaError_t run_gemm_pair_rows(const CUtensorMap& ta, const CUtensorMap& tw, const CUtensorMap& to,
+                               const GemmParams& gp, int num_sms, cudaStream_t st);
+// Dynamic shared memory of the CTA-pair kernels for N experts.
+size_t gemm_pair_smem_bytes(int N);
+
 // CTA-pair kernel launcher (expert_ffn_pair.cu).
 template <bool kGather>
 cudaError_t run_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to,

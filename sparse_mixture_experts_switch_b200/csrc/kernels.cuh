@@ -138,6 +138,7 @@ struct FfnArgs {
   int mode2;                // kModeY or kModeCombine for the second GEMM
   bool pair1;               // GEMM1 on CTA pairs (2-SM), else one CTA per tile
   bool pair2;               // GEMM2 on CTA pairs
+  bool pair1_rows;          // GEMM1 on CTA pairs with the rows as M (256-row tiles)
   bool gemm1_only;          // stop after GEMM1 (the backward pass recomputes H)
   void* const* peer_out;    // kModeCombineEp: every rank's output [T_rank, d] (host array)
   int n_peers;

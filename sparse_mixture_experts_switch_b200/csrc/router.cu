@@ -188,28 +188,47 @@ cudaError_t launch_router_simt(int64_t T, int d, int N, bool bf16, const void* x
 // stacked, p * N_pad + e (each term's experts together); interleaved,
 // (e / 32 * terms + p) * 32 + e % 32 (the terms of 32 experts side by side,
 // so one accumulator chunk of 32 x terms columns holds all of them).
+// Eight consecutive elements of one row per thread: two 16-byte loads of
+// W_r, one 16-byte store per term.
 __global__ void wsplit_kernel(int N, int N_pad, int d, int terms, bool interleave,
                               const float* __restrict__ w_r, __nv_bfloat16* __restrict__ out) {
   // the router that follows may start its prologue and its x loads now; it
   // waits for this kernel before it reads the split
   pdl_launch_dependents();
-  const int64_t n = static_cast<int64_t>(N_pad) * d;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+  const int d8 = d / 8;
+  const int64_t n8 = static_cast<int64_t>(N_pad) * d8;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int e = static_cast<int>(i / d);
-    const int64_t k = i - static_cast<int64_t>(e) * d;
-    const float w = e < N ? w_r[i] : 0.f;
-    const __nv_bfloat16 hi = __float2bfloat16_rn(w);
-    const float r1 = w - __bfloat162float(hi);           // exact
-    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
-    const float r2 = r1 - __bfloat162float(mid);          // exact
+    const int e = static_cast<int>(i / d8);
+    const int64_t k0 = (i - static_cast<int64_t>(e) * d8) * 8;
+    float w[8];
+    if (e < N) {
+      const float4* src = reinterpret_cast<const float4*>(w_r + static_cast<int64_t>(e) * d + k0);
+      const float4 a = __ldg(src), b = __ldg(src + 1);
+      w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w; w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) w[j] = 0.f;
+    }
+    uint32_t hi[4], mid[4], lo[4];
+#pragma unroll
+    for (int j = 0; j < 8; j += 2) {
+      const __nv_bfloat16 h0 = __float2bfloat16_rn(w[j]), h1 = __float2bfloat16_rn(w[j + 1]);
+      const float r0 = w[j] - __bfloat162float(h0), r1 = w[j + 1] - __bfloat162float(h1);   // exact
+      const __nv_bfloat16 m0 = __float2bfloat16_rn(r0), m1 = __float2bfloat16_rn(r1);
+      const float s0 = r0 - __bfloat162float(m0), s1 = r1 - __bfloat162float(m1);           // exact
+      hi[j / 2] = pack_bf16x2(__bfloat162float(h0), __bfloat162float(h1));
+      mid[j / 2] = pack_bf16x2(__bfloat162float(m0), __bfloat162float(m1));
+      lo[j / 2] = pack_bf16x2(s0, s1);                    // exact: <= 8 bits each
+    }
     auto row = [&](int p) -> int64_t {
       return interleave ? static_cast<int64_t>((e >> 5) * terms + p) * 32 + (e & 31)
                         : static_cast<int64_t>(p) * N_pad + e;
     };
-    out[row(0) * d + k] = hi;
-    out[row(1) * d + k] = mid;
-    if (terms == 3) out[row(2) * d + k] = __float2bfloat16_rn(r2);   // exact: <= 8 bits
+    *reinterpret_cast<uint4*>(out + row(0) * d + k0) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    *reinterpret_cast<uint4*>(out + row(1) * d + k0) = make_uint4(mid[0], mid[1], mid[2], mid[3]);
+    if (terms == 3)
+      *reinterpret_cast<uint4*>(out + row(2) * d + k0) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
   }
 }
 
@@ -1113,10 +1132,10 @@ cudaError_t launch_router_tc(int64_t T, int d, int N, int terms, const void* x,
   const int N_pad = router_n_pad(N);
   const bool pair = terms * N_pad <= 256 && num_sms >= 2;
   {
-    const int64_t n = static_cast<int64_t>(N_pad) * d;
-    int blocks = static_cast<int>((n + 255) / 256);
+    const int64_t n8 = static_cast<int64_t>(N_pad) * (d / 8);     // d % 64 == 0
+    int blocks = static_cast<int>((n8 + 127) / 128);
     if (blocks > 1024) blocks = 1024;
-    wsplit_kernel<<<blocks, 256, 0, st>>>(N, N_pad, d, terms, pair, w_r,
+    wsplit_kernel<<<blocks, 128, 0, st>>>(N, N_pad, d, terms, pair, w_r,
                                           static_cast<__nv_bfloat16*>(wsplit));
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;

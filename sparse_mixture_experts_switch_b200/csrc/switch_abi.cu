@@ -195,6 +195,17 @@ switch_status_t cuda_status(cudaError_t e) {
     if (_e != cudaSuccess) return SWITCH_ERR_CUDA; \
   } while (0)
 
+// GEMM1 on row-major CTA pairs: asked for, or by default when every
+// expert's kept rows fit one 256-row pair tile but not one 128-row tile
+// (128 < C <= 256): then the pair tile has no more padding rows than two
+// single-CTA tiles, and each SM streams a third fewer operand bytes.
+bool gemm1_rows_pairs(const switch_config_t* c, int64_t C) {
+  if (c->flags & SWITCH_FLAG_GEMM1_ROWS_PAIRS) return true;
+  if (c->flags & (SWITCH_FLAG_GEMM_1SM | SWITCH_FLAG_GEMM_PAIRS | SWITCH_FLAG_GATHER_IN_GEMM))
+    return false;
+  return C > 128 && C <= 256;
+}
+
 int router_terms(const switch_config_t* c) {
   return (c->flags & SWITCH_FLAG_ROUTER_3TERM) ? 3 : 2;
 }
@@ -328,7 +339,8 @@ switch_status_t switch_router(const switch_config_t* cfg, const void* x, const f
   Ctx c{};
   switch_status_t s = prepare(cfg, ws, ws_bytes, stream, &c);
   if (s != SWITCH_OK || cfg->T == 0) return s;
-  if (!x || !w_r || !idx || !gate || !aligned16(x) || (probs && !aligned16(probs)))
+  if (!x || !w_r || !idx || !gate || !aligned16(x) || !aligned16(w_r) ||
+      (probs && !aligned16(probs)))
     return SWITCH_ERR_INVALID_ARG;
   const bool top2 = routes_of(*cfg) == 2;
   RouterOut o{idx, gate, probs, c.at<float>(c.L.psum), nullptr, nullptr,
@@ -409,6 +421,7 @@ switch_status_t switch_expert_ffn(const switch_config_t* cfg, const void* x,
   a.num_sms = c.num_sms;
   a.pair1 = (cfg->flags & SWITCH_FLAG_GEMM_PAIRS) != 0;
   a.pair2 = !(cfg->flags & SWITCH_FLAG_GEMM_1SM);
+  a.pair1_rows = gemm1_rows_pairs(cfg, c.C);
   if (dispatched) {
     a.x = nullptr;
     a.x_disp = x;
@@ -460,8 +473,8 @@ switch_status_t switch_layer_forward(const switch_config_t* cfg, const void* x,
   Ctx c{};
   switch_status_t s = prepare(cfg, ws, ws_bytes, stream, &c);
   if (s != SWITCH_OK || cfg->T == 0) return s;
-  if (!x || !w_r || !w1 || !w2 || !out || !aligned16(x) || !aligned16(w1) || !aligned16(w2) ||
-      !aligned16(out))
+  if (!x || !w_r || !w1 || !w2 || !out || !aligned16(x) || !aligned16(w_r) || !aligned16(w1) ||
+      !aligned16(w2) || !aligned16(out))
     return SWITCH_ERR_INVALID_ARG;
   const int64_t T = cfg->T;
   const int N = cfg->n_experts;
@@ -554,6 +567,7 @@ switch_status_t switch_layer_forward(const switch_config_t* cfg, const void* x,
   a.num_sms = c.num_sms;
   a.pair1 = (cfg->flags & SWITCH_FLAG_GEMM_PAIRS) != 0;
   a.pair2 = !(cfg->flags & SWITCH_FLAG_GEMM_1SM);
+  a.pair1_rows = gemm1_rows_pairs(cfg, c.C);
   if (row_copy) a.x_disp = c.ws + c.L.xdisp;
   SMOE_TRY(bf16 ? launch_expert_ffn_bf16(a, c.st) : launch_expert_ffn_f32(a, c.st));
   // 5. dropped tokens (fused) or every token (unfused)
@@ -587,6 +601,7 @@ switch_status_t switch_layer_backward(const switch_config_t* cfg, const void* x,
   if (cfg->dtype != SWITCH_BF16 || (cfg->flags & SWITCH_FLAG_TOP2)) return SWITCH_ERR_UNSUPPORTED;
   if (cfg->T == 0) return SWITCH_OK;
   if (!x || !w_r || !w1 || !w2 || !dout || !dx || !dw_r || !dw1 || !dw2 || !aligned16(x) ||
+      !aligned16(w_r) ||
       !aligned16(w1) || !aligned16(w2) || !aligned16(dout) || !aligned16(dx) ||
       !aligned16(dw1) || !aligned16(dw2))
     return SWITCH_ERR_INVALID_ARG;
@@ -651,6 +666,7 @@ switch_status_t switch_layer_backward(const switch_config_t* cfg, const void* x,
     a.hbuf = hbuf;
     a.mode2 = kModeY;
     a.pair1 = (cfg->flags & SWITCH_FLAG_GEMM_PAIRS) != 0;
+    a.pair1_rows = gemm1_rows_pairs(cfg, c.C);
     a.gemm1_only = true;
     a.err = c.err;
     a.spin = c.spin;
@@ -738,7 +754,7 @@ switch_status_t switch_ep_route(const switch_config_t* cfg, const switch_ep_t* e
   if (s != SWITCH_OK) return s;
   if (cfg->T == 0) return SWITCH_OK;
   if (!record || (reinterpret_cast<uintptr_t>(record) & 15u) != 0 || !x || !w_r ||
-      !aligned16(x))
+      !aligned16(x) || !aligned16(w_r))
     return SWITCH_ERR_INVALID_ARG;
   const int64_t T = cfg->T;
   const int N = cfg->n_experts;
@@ -849,6 +865,7 @@ switch_status_t switch_ep_experts(const switch_config_t* cfg, const switch_ep_t*
   a.gate = reinterpret_cast<const float*>(rb + L.recv_gate);
   a.mode2 = kModeCombineEp;
   a.pair1 = (cfg->flags & SWITCH_FLAG_GEMM_PAIRS) != 0;
+  a.pair1_rows = gemm1_rows_pairs(cfg, c.C);
   a.pair2 = true;
   a.peer_out = out_peers;
   a.n_peers = L.G;

@@ -30,6 +30,7 @@ FLAG_GEMM_PAIRS = 64
 FLAG_ROWS_DISPATCHED = 128
 FLAG_TOP2 = 512
 FLAG_TRAINING = 1024
+FLAG_GEMM1_ROWS_PAIRS = 2048
 
 
 class SwitchConfig(ctypes.Structure):

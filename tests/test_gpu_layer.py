@@ -71,13 +71,24 @@ E2E = Workload("e2e", T=3000, d_model=320, d_ff=576, n_experts=8, capacity_facto
                dtype="bf16", seed=71)
 
 
-@pytest.mark.parametrize("flags", [0, 1, 2, 4, 8, 1 | 4 | 8, 32, 32 | 8, 64, 64 | 8],
+@pytest.mark.parametrize("flags", [0, 1, 2, 4, 8, 1 | 4 | 8, 32, 32 | 8, 64, 64 | 8, 2048,
+                                   2048 | 4, 2048 | 32],
                          ids=["fused", "simt_router", "three_term", "unfused", "gather_in_gemm",
                               "simt_unfused_gather", "gemm_1sm", "gemm_1sm_gather", "gemm_pairs",
-                              "gemm_pairs_gather"])
+                              "gemm_pairs_gather", "gemm1_rows_pairs", "gemm1_rows_pairs_unfused",
+                              "gemm1_rows_pairs_1sm"])
 def test_layer_bf16(sm, flags):
     flips, drop_rate = check_layer(sm, E2E, flags)
     assert drop_rate > 0     # cf = 1.0 with random routing overflows some experts
+
+
+def test_layer_capacity_within_one_pair_tile(sm):
+    """128 < C <= 256: the default GEMM1 runs on row-major CTA pairs."""
+    wl = Workload("c160", T=2048, d_model=256, d_ff=512, n_experts=16, capacity_factor=1.25,
+                  dtype="bf16", seed=74)
+    assert 128 < sm.switch_capacity(wl.T, wl.n_experts, wl.capacity_factor) <= 256
+    check_layer(sm, wl)
+    check_layer(sm, wl, sm.FLAG_NO_RESIDUAL, residual=False)
 
 
 def test_layer_no_residual(sm):

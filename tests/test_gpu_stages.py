@@ -207,9 +207,9 @@ FFN_CASES = [
 ]
 
 
-@pytest.mark.parametrize("flags", [0, 8, 32, 40, 64, 72],
+@pytest.mark.parametrize("flags", [0, 8, 32, 40, 64, 72, 2048, 2048 | 8],
                          ids=["default", "gather_in_gemm", "one_sm", "one_sm_gather", "pairs",
-                              "pairs_gather"])
+                              "pairs_gather", "rows_pairs", "rows_pairs_gather"])
 @pytest.mark.parametrize("wl", FFN_CASES, ids=lambda w: w.name)
 def test_expert_ffn(sm, wl, flags):
     inp = make_inputs(wl)
@@ -235,7 +235,8 @@ def test_expert_ffn(sm, wl, flags):
     assert np.isnan(yg[~kept]).all()     # padding rows untouched
 
 
-@pytest.mark.parametrize("flags", [128, 128 | 32, 128 | 64], ids=["default", "one_sm", "pairs"])
+@pytest.mark.parametrize("flags", [128, 128 | 32, 128 | 64, 128 | 2048],
+                         ids=["default", "one_sm", "pairs", "rows_pairs"])
 @pytest.mark.parametrize("wl", FFN_CASES, ids=lambda w: w.name)
 def test_expert_ffn_rows_dispatched(sm, wl, flags):
     """x_disp from switch_dispatch fed to switch_expert_ffn (ROWS_DISPATCHED):
