@@ -860,8 +860,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kRouterPairThreads, 
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {                                    // TMEM of this tile no longer read
-        if (leader) mbar_arrive(&tempty[acc]);
-        else mbar_arrive_remote(tempty_lead + 8u * acc);
+        if (leader) mbar_arrive_relaxed(&tempty[acc]);
+        else mbar_arrive_remote_relaxed(tempty_lead + 8u * acc);
       }
       if (!here) continue;
       const int par = li & 1;
