@@ -280,9 +280,17 @@ __global__ void __launch_bounds__(256) aux_loss_probs_kernel(
   if (!last) return;
   __threadfence();
   for (int e = threadIdx.x; e < N; e += 256) {
+    // 16 parts' loads in flight at a time, added in part order
     double tot = 0.0;
-    for (int pp = p0; pp < p1; ++pp)
-      tot += static_cast<double>(__ldcg(psum + static_cast<int64_t>(pp) * N + e));
+    for (int pb = p0; pb < p1; pb += 16) {
+      float v[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        v[j] = pb + j < p1 ? __ldcg(psum + static_cast<int64_t>(pb + j) * N + e) : 0.f;
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        if (pb + j < p1) tot += static_cast<double>(v[j]);
+    }
     part_sum[static_cast<int64_t>(run) * N + e] = tot;
   }
   if (threadIdx.x == 0) run_ticket[run] = 0;
@@ -294,8 +302,14 @@ __global__ void __launch_bounds__(256) aux_loss_probs_kernel(
   __threadfence();
   double acc = 0.0;
   for (int i = threadIdx.x; i < N; i += 256) {
+    double v[kAuxChunks];                 // every run's sum in flight, added in run order
+#pragma unroll
+    for (int c = 0; c < kAuxChunks; ++c)
+      v[c] = c < nruns ? __ldcg(part_sum + static_cast<int64_t>(c) * N + i) : 0.0;
     double tot = 0.0;
-    for (int c = 0; c < nruns; ++c) tot += __ldcg(part_sum + static_cast<int64_t>(c) * N + i);
+#pragma unroll
+    for (int c = 0; c < kAuxChunks; ++c)
+      if (c < nruns) tot += v[c];
     const double P = tot / static_cast<double>(T);
     const double f = static_cast<double>(counts[i]) / static_cast<double>(T);
     if (f_out) f_out[i] = static_cast<float>(f);
