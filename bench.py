@@ -755,20 +755,24 @@ def kernel_rooflines(sm, cfg, wl, C, x, w_r, b_r, w1, w2, ws, flush, stream, dev
     t_comb = timed(lambda: sm.switch_combine(cfg, x, idx, rank, drop, gate, y, out))
     # the top-2 routing variant of the whole layer (capacity over 2T)
     t_top2 = None
+    T_kept2 = 0
     if N >= 2:
         cfg2 = sm.config(T, d, F, N, wl.capacity_factor, dtype=wl.dtype, alpha=wl.alpha,
                          flags=sm.FLAG_TOP2)
         ws2 = sm.workspace(cfg2, device=dev)
         idx2 = torch.empty(2 * T, **i32)
         gate2 = torch.empty(2 * T, dtype=torch.float32, device=dev)
+        counts2 = torch.empty(N, **i32)
         t_top2 = timed(lambda: sm.switch_layer_forward(cfg2, x, w_r, b_r, w1, w2, out, idx2,
-                                                       gate2, counts, loss, ws2))
+                                                       gate2, counts2, loss, ws2))
         st2, where2, info2 = sm.switch_get_device_error(ws2)
         if st2 != 0:
             raise RuntimeError(f"device error {st2} at {where2} ({info2}) in the top-2 layer")
+        C2 = sm.switch_capacity(2 * T, N, wl.capacity_factor)
+        T_kept2 = int(np.minimum(counts2.cpu().numpy().astype(np.int64), C2).sum())
         del ws2
     # the backward pass of the whole layer (recomputes routing, dispatch and H)
-    t_bwd = t_bwd_saved = t_train = None
+    t_bwd = t_bwd_saved = t_train = t_bwd2 = None
     if wl.dtype == "bf16":
         wsb = sm.backward_workspace(cfg, device=dev)
         dout = torch.empty_like(x).normal_()
@@ -802,7 +806,19 @@ def kernel_rooflines(sm, cfg, wl, C, x, w_r, b_r, w1, w2, ws, flush, stream, dev
         stb, whereb, infob = sm.switch_get_device_error(wst)
         if stb != 0:
             raise RuntimeError(f"device error {stb} at {whereb} ({infob}) in the training step")
-        del wst, dout, dx, dw1, dw2
+        del wst
+        # the top-2 backward (recomputes the top-2 routing, dispatch and H)
+        if N >= 2:
+            wsb2 = sm.backward_workspace(cfg2, device=dev)
+            t_bwd2 = timed(lambda: sm.switch_layer_backward(cfg2, x, w_r, b_r, w1, w2, dout, 1.0,
+                                                            dx, dw_r, db_r, dw1, dw2, None,
+                                                            wsb2))
+            stb, whereb, infob = sm.switch_get_device_error(wsb2)
+            if stb != 0:
+                raise RuntimeError(f"device error {stb} at {whereb} ({infob}) in the top-2 "
+                                   "backward pass")
+            del wsb2
+        del dout, dx, dw1, dw2
     t_aux = timed(lambda: sm.switch_aux_loss(cfg, counts, probs, loss, None, None, ws))
     st, where, info = sm.switch_get_device_error(ws)
     if st != 0:
@@ -846,6 +862,11 @@ def kernel_rooflines(sm, cfg, wl, C, x, w_r, b_r, w1, w2, ws, flush, stream, dev
             "frac_burst": (8.0 * T_kept * d * F + 4.0 * T * N * d) / t_bwd_saved / 1e12
                           / pk["bf16_tflops"],
             "note": "SWITCH_FLAG_TRAINING: activations kept by the forward, no recompute"},
+        "layer_backward_top2": None if t_bwd2 is None else {
+            "us": t_bwd2 * 1e6, "tokens_per_s": T / t_bwd2, "kept_assignments": T_kept2,
+            "useful_flops": 8.0 * T_kept2 * d * F + 4.0 * T * N * d,
+            "tflops_with_recompute": (10.0 * T_kept2 * d * F + 6.0 * T * N * d) / t_bwd2 / 1e12,
+            "note": "SWITCH_FLAG_TOP2, routing, dispatch and H recomputed"},
         "training_step": None if t_train is None else {
             "us": t_train * 1e6, "tokens_per_s": T / t_train,
             "tflops": (12.0 * T_kept * d * F + 6.0 * T * N * d) / t_train / 1e12,

@@ -252,7 +252,7 @@ switch_status_t switch_layer_forward(const switch_config_t* cfg, const void* x,
                                      float* loss, void* ws, size_t ws_bytes,
                                      void* stream);
 
-/* Backward pass of switch_layer_forward (top-1, bf16): the gradient of
+/* Backward pass of switch_layer_forward (bf16; top-1, or top-2 below): the gradient of
  *   J = sum(dout * out) + dloss * loss
  * with respect to x, w_r, b_r, w1 and w2, routing decisions held fixed (the
  * argmax and the capacity cut are piecewise constant; f_i likewise).  The
@@ -284,12 +284,24 @@ switch_status_t switch_layer_forward(const switch_config_t* cfg, const void* x,
  *   outputs: dx [T, d_model] bf16, dw_r [N, d_model] fp32, db_r [N] fp32 or
  *   NULL, dw1 [N, d_ff, d_model] bf16, dw2 [N, d_model, d_ff] bf16,
  *   dgate [T] fp32 or NULL (the gate gradient above).
+ * Top-2 (SWITCH_FLAG_TOP2) [P1 "Switch Routing": out = x + sum over the
+ * top-k set of p_i E_i(x), p the full softmax, not renormalised]: every kept
+ * route r of token t (expert idx_r, gate p_{idx_r}) contributes its own
+ * expert gradients and its own gate gradient
+ *   dgate[r T + t] = dout[t] . E_{idx_r}(x_t)  (0 for a dropped route),
+ *   dp[t, i] = sum over kept r with idx_r = i of dgate[r T + t]
+ *              + dloss alpha N f_i / T,
+ * f_i over the first choices (as the forward's loss); dx adds both kept
+ * routes' dA W1_e rows (kept in fp32 per slot, then summed per token in
+ * route order with the residual and dh W_r).  dgate is then [2 T] fp32,
+ * route-major.  A route whose gate underflowed to 0 reports dgate 0 (its
+ * dY is 0; p = 0 removes it from dh in any case).
  * Arithmetic: expert GEMMs on the tensor cores (bf16 operands, fp32
  * accumulation; gate * dout, dA and the weight gradients rounded once to
  * bf16); router backward in fp32 FMA with fixed-order reductions (dW_r and
  * db_r bit-reproducible).  Workspace: switch_backward_workspace_size()
- * bytes.  dtype SWITCH_F32 or SWITCH_FLAG_TOP2 return SWITCH_ERR_UNSUPPORTED
- * (so does switch_layer_forward given SWITCH_FLAG_TRAINING with either).
+ * bytes.  dtype SWITCH_F32 returns SWITCH_ERR_UNSUPPORTED (so does
+ * switch_layer_forward given SWITCH_FLAG_TRAINING with it).
  * T = 0 writes nothing. */
 switch_status_t switch_layer_backward(const switch_config_t* cfg, const void* x,
                                       const float* w_r, const float* b_r,

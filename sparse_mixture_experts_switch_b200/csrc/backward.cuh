@@ -1,4 +1,4 @@
-// Backward pass of the top-1 Switch-FFN layer: parameters of the backward
+// Backward pass of the Switch-FFN layer (top-1 and top-2): parameters of the backward
 // GEMM kernel and the launch wrappers the C-ABI layer calls.
 #pragma once
 
@@ -7,7 +7,7 @@
 namespace smoe {
 
 enum BwdSched : int { kSchedRows = 0, kSchedWeight = 1, kSchedSplit = 2 };
-enum BwdEpi : int { kEpiDH = 0, kEpiStore = 1, kEpiDX = 2, kEpiStoreF32 = 3 };
+enum BwdEpi : int { kEpiDH = 0, kEpiStore = 1, kEpiDX = 2, kEpiStoreF32 = 3, kEpiDXSlot = 4 };
 
 struct BwdParams {
   int N;                 // experts
@@ -28,7 +28,7 @@ struct BwdParams {
   const int* slot_token;
   const __nv_bfloat16* h;      // dH epilogue: H [N*C, n_out]
   __nv_bfloat16* out;          // dH: dA [N*C, n_out]; store: [N * M_out, n_out]
-  float* out_f32;              // store-f32: [batches * M_out, n_out]
+  float* out_f32;              // store-f32: [batches * M_out, n_out]; dX per slot: [N*C, n_out]
   float* dgp;                  // dH: [N*C, ntiles_n] partial gate gradients
   const __nv_bfloat16* dout;   // dX: [T, n_out]
   __nv_bfloat16* dx;           // dX: [T, n_out]
@@ -58,6 +58,8 @@ struct BwdFfnArgs {
   const void* wrp;          // [2][N][d] bf16: hi / lo planes of W_r
   int n_router, n_pad;      // router experts N and the planes' row length Np
   void* dx;                 // [T, d] bf16 out (kept tokens)
+  float* dxs;               // top-2: [N*C, d] fp32 out, the dX GEMM's rows per kept slot
+                            // (then added per token by launch_bwd_combine_top2); null: top-1
   bool residual;
   bool pair_dw;             // weight gradients on CTA pairs (256 x 256 tiles)
   DevErr* err;
@@ -70,7 +72,9 @@ cudaError_t launch_bwd_dh(const BwdFfnArgs& a, cudaStream_t st);
 // dW2_e = dY_e^T H_e, dW1_e = dA_e^T X_e for every expert (zeros when empty).
 cudaError_t launch_bwd_dw(const BwdFfnArgs& a, cudaStream_t st);
 // dx of kept tokens: residual + dA W1_e + dh W_r (the router term as three
-// extra bf16 split terms of the same accumulation).
+// extra bf16 split terms of the same accumulation).  With a.dxs (top-2: two
+// slots may hold one token) each kept slot's fp32 row dA W1_e + dh_s W_r is
+// stored at its slot instead, without the residual.
 cudaError_t launch_bwd_dx(const BwdFfnArgs& a, cudaStream_t st);
 // dW_r [N, d] = dh^T x on the tensor cores: dh as hi + lo bf16 planes
 // dhp [2][T][Np] (x is exact in bf16), split-K over token chunks into fp32
@@ -82,12 +86,15 @@ cudaError_t launch_router_bwd_dw_tc(int64_t T, int N, int Np, int d, const void*
                                     float* dw_r, float* db, DevErr* err, long long spin,
                                     int num_sms, cudaStream_t st);
 
-// dys[s] = bf16(gate[t] * dout[t]) for kept slot s of token t, zero for
-// padding; H rows in [kept, min(C, kept rounded up to 64)) of each expert
-// are zeroed (the weight-gradient GEMMs read whole 64-row K blocks).
+// dys[s] = bf16(g * dout[t]) for kept slot s of token t, zero for padding;
+// g = gate[t] (top-1), or with top-2 (T2 = T > 0) the gate of the route that
+// put t in expert e = s / C: gate[t] if idx[t] == e (its first choice), else
+// gate[T2 + t].  H rows in [kept, min(C, kept rounded up to 64)) of each
+// expert are zeroed (the weight-gradient GEMMs read whole 64-row K blocks).
 cudaError_t launch_bwd_gather(int64_t C, int N, int d, int F, const int* counts,
-                              const int* slot_token, const float* gate, const void* dout,
-                              void* dys, void* hbuf, cudaStream_t st);
+                              const int* slot_token, const float* gate, const int* idx,
+                              int64_t T2, const void* dout, void* dys, void* hbuf,
+                              cudaStream_t st);
 
 // Router backward for top-1 routing:
 //   dgate[t] = sum_j dgp[idx*C + rank][j] / gate[t] (kept tokens, else 0),
@@ -105,6 +112,30 @@ cudaError_t launch_router_bwd_dh(int64_t T, int N, int Np, int64_t C, int ntn,
                                  const int* counts, float loss_scale, float* dh, void* dhp,
                                  void* dhs, float* dgate, int* drop_list, int* n_drop,
                                  cudaStream_t st);
+// Router backward for top-2 routing: per token t and route r (entry
+// a = r T + t of the route-major arrays idx, rank, drop, gate, dgate),
+//   dgate[a] = sum_j dgp[idx_a*C + rank_a][j] / gate[a] (kept route, gate > 0;
+//              else 0),
+//   dp[t, i] = loss_scale * counts1[i] + sum over kept r with idx_a = i of dgate[a],
+//   dh[t, i] = p[t, i] (dp[t, i] - sum_j p[t, j] dp[t, j]);
+// counts1 are the first choices' totals (the loss's f_i).  dh's hi / lo
+// planes go to dhp [2][T][Np], and to dhs [2][N*C][Np] at the token's first
+// kept slot (route 0 if kept, else route 1); a second kept slot gets zero
+// planes, so the router term dh W_r enters the token's dx once.  Tokens with
+// both routes dropped are listed in drop_list (any order).
+cudaError_t launch_router_bwd_dh_top2(int64_t T, int N, int Np, int64_t C, int ntn,
+                                      const float* probs, const int* idx, const int* rank,
+                                      const uint8_t* drop, const float* gate, const float* dgp,
+                                      const int* counts1, float loss_scale, float* dh,
+                                      void* dhp, void* dhs, float* dgate, int* drop_list,
+                                      int* n_drop, cudaStream_t st);
+// Top-2 input gradient of tokens with at least one kept route:
+//   dx[t] = bf16((residual ? dout[t] : 0) + dxs[s_0] + dxs[s_1])  (kept routes'
+// slots s_r = idx_a*C + rank_a, added in route order in fp32).  Tokens with
+// both routes dropped are left to launch_bwd_dropped.
+cudaError_t launch_bwd_combine_top2(int64_t T, int d, int64_t C, const int* idx, const int* rank,
+                                    const uint8_t* drop, const float* dxs, const void* dout,
+                                    void* dx, bool residual, cudaStream_t st);
 // wrp [2][N][d] = hi / lo bf16 split of W_r (hi = bf16(W), lo = bf16(W - hi)).
 cudaError_t launch_wr_split(int N, int d, const float* w_r, void* wrp, cudaStream_t st);
 // Dropped tokens (from the list): dx[t] = bf16((residual ? dout[t] : 0) +

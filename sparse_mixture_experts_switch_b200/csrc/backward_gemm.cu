@@ -20,7 +20,9 @@
 //     product with H for the gate gradient (sum over the tile's columns);
 //   * store: bf16 rows of a weight gradient (zeros for an expert with no
 //     tokens);
-//   * dX: dx[token] = dout[token] (residual) + router term + dX row.
+//   * dX: dx[token] = dout[token] (residual) + router term + dX row;
+//   * dX per slot (top-2, where two slots can hold one token): the fp32 row
+//     (router term + dX row) stored at the slot, added per token afterwards.
 #include <cstring>
 
 #include "gemm_common.cuh"
@@ -310,6 +312,29 @@ __device__ __forceinline__ void epi_dx(const BwdParams& p, const BTile& t, uint3
   }
 }
 
+// dX tile for top-2: kept slot rows store their fp32 accumulator (dA W1_e
+// plus the router term where the slot carries it) at the slot; the token's
+// sum over its slots and the residual are added by a later kernel.
+__device__ __forceinline__ void epi_dx_slot(const BwdParams& p, const BTile& t, uint32_t taddr,
+                                            int q, int lane) {
+  const int64_t r_in = static_cast<int64_t>(t.m) * kBM + q * 32 + lane;
+  const int64_t cnt = p.counts[t.e];
+  const int64_t ne = cnt < p.C ? cnt : p.C;
+  const bool kept = r_in < ne;
+  const int cols = p.n_out - t.n * kBN < kBN ? p.n_out - t.n * kBN : kBN;
+  const int64_t off = (static_cast<int64_t>(t.e) * p.C + r_in) * p.n_out + t.n * kBN;
+  for (int c = 0; c < cols / 32; ++c) {
+    uint32_t v[32];
+    tmem_ld32_issue(taddr + static_cast<uint32_t>(c * 32), v);
+    tmem_ld_wait(v);
+    if (kept) {
+      uint4* dst = reinterpret_cast<uint4*>(p.out_f32 + off + c * 32);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) dst[k] = make_uint4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+    }
+  }
+}
+
 }  // namespace
 
 template <int kSched, int kEpi>
@@ -516,6 +541,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_gemm_kernel(
       if (kEpi == kEpiStore) epi_store<false>(p, &tmap_a2, t, taddr, q, lane, stg, nbox);
       else if (kEpi == kEpiStoreF32) epi_store<true>(p, &tmap_a2, t, taddr, q, lane, stg, nbox);
       else if (kEpi == kEpiDH) epi_dh(p, &tmap_a2, t, taddr, q, lane, stg, nbox);
+      else if (kEpi == kEpiDXSlot) epi_dx_slot(p, t, taddr, q, lane);
       else epi_dx(p, t, taddr, q, lane);
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
@@ -889,6 +915,10 @@ cudaError_t launch_bwd_dx(const BwdFfnArgs& a, cudaStream_t st) {
   p.dout = static_cast<const __nv_bfloat16*>(a.dout);
   p.dx = static_cast<__nv_bfloat16*>(a.dx);
   p.residual = a.residual ? 1 : 0;
+  if (a.dxs) {
+    p.out_f32 = a.dxs;
+    return run_bwd<kSchedRows, kEpiDXSlot>(ta, tb, ta2, tb2, p, a.num_sms, st);
+  }
   return run_bwd<kSchedRows, kEpiDX>(ta, tb, ta2, tb2, p, a.num_sms, st);
 }
 

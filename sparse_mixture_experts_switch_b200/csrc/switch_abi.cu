@@ -42,9 +42,10 @@ struct Layout {
       slot_token, mtile_start, wsplit, logits, xdisp, hbuf, ybuf, total;
   // backward pass only (after the forward regions): dA, partial gate
   // gradients, dh (fp32, and its bf16 planes per token and per slot), W_r
-  // planes, gate gradient, split-K partials of dW_r, column sums of dh,
-  // dropped-token list and its counter
-  size_t probs_s, da, dgp, dh, dhp, dhs, wrp, dgate, rpart, colsum, drop_list, n_drop,
+  // planes, gate gradient (per route), split-K partials of dW_r, column
+  // sums of dh, dropped-token list and its counter; top-2 only: the dX
+  // GEMM's fp32 rows per slot
+  size_t probs_s, da, dgp, dh, dhp, dhs, wrp, dgate, rpart, colsum, drop_list, n_drop, dxs,
       bwd_total;
 };
 
@@ -106,11 +107,12 @@ Layout layout_for(const switch_config_t& c, int64_t C) {
   L.dhp = take(2 * 2 * static_cast<size_t>(T) * Np);
   L.dhs = take(2 * 2 * static_cast<size_t>(slots) * Np);
   L.wrp = take(2 * 2 * static_cast<size_t>(Np) * c.d_model);
-  L.dgate = take(sizeof(float) * T);
+  L.dgate = take(sizeof(float) * A);
   L.rpart = take(sizeof(float) * router_bwd_tc_part_floats(T, c.n_experts, c.d_model, 0));
   L.colsum = take(sizeof(float) * N * ntiles_of(T));
   L.drop_list = take(sizeof(int) * T);
   L.n_drop = take(sizeof(int));
+  L.dxs = take(routes_of(c) == 2 ? sizeof(float) * slots * static_cast<size_t>(c.d_model) : 0);
   L.bwd_total = o;
   return L;
 }
@@ -488,7 +490,7 @@ switch_status_t switch_layer_forward(const switch_config_t* cfg, const void* x,
   // workspace, copied out to the caller's at the end)
   const bool training = (cfg->flags & SWITCH_FLAG_TRAINING) != 0;
   if (training) {
-    if (!bf16 || top2) return SWITCH_ERR_UNSUPPORTED;
+    if (!bf16) return SWITCH_ERR_UNSUPPORTED;
     if (ws_bytes < c.L.bwd_total) return SWITCH_ERR_WORKSPACE_TOO_SMALL;
   }
   int* idx_p = (idx && !training) ? idx : c.at<int>(c.L.idx);
@@ -580,9 +582,9 @@ switch_status_t switch_layer_forward(const switch_config_t* cfg, const void* x,
                              c.st));
   if (training) {
     if (idx)
-      SMOE_TRY(cudaMemcpyAsync(idx, idx_p, sizeof(int) * T, cudaMemcpyDeviceToDevice, c.st));
+      SMOE_TRY(cudaMemcpyAsync(idx, idx_p, sizeof(int) * A, cudaMemcpyDeviceToDevice, c.st));
     if (gate)
-      SMOE_TRY(cudaMemcpyAsync(gate, gate_p, sizeof(float) * T, cudaMemcpyDeviceToDevice, c.st));
+      SMOE_TRY(cudaMemcpyAsync(gate, gate_p, sizeof(float) * A, cudaMemcpyDeviceToDevice, c.st));
     if (counts)
       SMOE_TRY(cudaMemcpyAsync(counts, counts_p, sizeof(int) * N, cudaMemcpyDeviceToDevice,
                                c.st));
@@ -598,7 +600,7 @@ switch_status_t switch_layer_backward(const switch_config_t* cfg, const void* x,
   Ctx c{};
   switch_status_t s = prepare(cfg, ws, ws_bytes, stream, &c);
   if (s != SWITCH_OK) return s;
-  if (cfg->dtype != SWITCH_BF16 || (cfg->flags & SWITCH_FLAG_TOP2)) return SWITCH_ERR_UNSUPPORTED;
+  if (cfg->dtype != SWITCH_BF16) return SWITCH_ERR_UNSUPPORTED;
   if (cfg->T == 0) return SWITCH_OK;
   if (!x || !w_r || !w1 || !w2 || !dout || !dx || !dw_r || !dw1 || !dw2 || !aligned16(x) ||
       !aligned16(w_r) ||
@@ -611,10 +613,16 @@ switch_status_t switch_layer_backward(const switch_config_t* cfg, const void* x,
   const int d = cfg->d_model, F = cfg->d_ff;
   const int nt = ntiles_of(T);
   const int64_t S = static_cast<int64_t>(N) * c.C;
+  // top-2: route-major arrays of A = 2T assignments (entry T + t is token
+  // t's second choice); counts1 = the first choices' totals (the loss's f_i)
+  const bool top2 = routes_of(*cfg) == 2;
+  const int64_t A = routes_of(*cfg) * T;
+  const int nta = ntiles_of(A);
   int* idx = c.at<int>(c.L.idx);
   float* gate = c.at<float>(c.L.gate);
   float* probs = c.at<float>(c.L.probs_s);
   int* counts = c.at<int>(c.L.counts);
+  int* counts1 = top2 ? c.at<int>(c.L.counts1) : counts;
   int* local_rank = c.at<int>(c.L.local_rank);
   int* hist = c.at<int>(c.L.hist);
   int* rank = c.at<int>(c.L.rank);
@@ -634,7 +642,8 @@ switch_status_t switch_layer_backward(const switch_config_t* cfg, const void* x,
   } else {
     // 1. the forward's routing, dispatch and hidden activations, recomputed
     // (same kernels, same results): probabilities, slots, x_disp, H
-    RouterOut o{idx, gate, probs, c.at<float>(c.L.psum), nullptr, nullptr, nullptr, nullptr};
+    RouterOut o{idx, gate, probs, c.at<float>(c.L.psum), nullptr, nullptr,
+                top2 ? idx + T : nullptr, top2 ? gate + T : nullptr};
     if (use_tc_router(cfg)) {
       o.hist = hist;
       o.local_rank = local_rank;
@@ -646,9 +655,15 @@ switch_status_t switch_layer_backward(const switch_config_t* cfg, const void* x,
                                   c.st));
       SMOE_TRY(launch_tile_rank(T, N, idx, nullptr, nullptr, local_rank, hist, nt, c.err, c.st));
     }
-    SMOE_TRY(launch_scan(N, nt, hist, c.at<int>(c.L.base), counts, c.st));
-    SMOE_TRY(launch_finalize_gather(T, N, c.C, nt, idx, local_rank, c.at<int>(c.L.base), counts,
-                                    rank, drop, slot_token, mtile_start, 0, x, x_disp,
+    if (top2) {
+      // as the forward: first choices' totals, then the 2T assignments ranked
+      SMOE_TRY(launch_scan(N, nt, hist, c.at<int>(c.L.base), counts1, c.st));
+      SMOE_TRY(launch_tile_rank(A, N, idx, nullptr, nullptr, local_rank, hist, nta, c.err,
+                                c.st));
+    }
+    SMOE_TRY(launch_scan(N, nta, hist, c.at<int>(c.L.base), counts, c.st));
+    SMOE_TRY(launch_finalize_gather(A, N, c.C, nta, idx, local_rank, c.at<int>(c.L.base), counts,
+                                    rank, drop, slot_token, mtile_start, top2 ? T : 0, x, x_disp,
                                     static_cast<int64_t>(d) * 2, c.st));
     FfnArgs a{};
     a.T = T;
@@ -677,7 +692,8 @@ switch_status_t switch_layer_backward(const switch_config_t* cfg, const void* x,
   // 2. dY = gate * dout per kept slot; dA and the gate-gradient partials;
   // the expert weight gradients
   void* dys = c.ws + c.L.ybuf;
-  SMOE_TRY(launch_bwd_gather(c.C, N, d, F, counts, slot_token, gate, dout, dys, hbuf, c.st));
+  SMOE_TRY(launch_bwd_gather(c.C, N, d, F, counts, slot_token, gate, idx, top2 ? T : 0, dout,
+                             dys, hbuf, c.st));
   BwdFfnArgs b{};
   b.T = T;
   b.d = d;
@@ -713,10 +729,16 @@ switch_status_t switch_layer_backward(const switch_config_t* cfg, const void* x,
   int* drop_list = c.at<int>(c.L.drop_list);
   const double ls = static_cast<double>(dloss) * cfg->alpha * N / (static_cast<double>(T) * T);
   SMOE_TRY(cudaMemsetAsync(n_drop, 0, sizeof(int), c.st));
-  SMOE_TRY(launch_router_bwd_dh(T, N, Np, c.C, (F + 255) / 256, probs, idx, rank, drop, gate,
-                                b.dgp, counts, static_cast<float>(ls), dh, c.ws + c.L.dhp,
-                                c.ws + c.L.dhs, dgate ? dgate : c.at<float>(c.L.dgate),
-                                drop_list, n_drop, c.st));
+  float* dgate_p = dgate ? dgate : c.at<float>(c.L.dgate);
+  if (top2)
+    SMOE_TRY(launch_router_bwd_dh_top2(T, N, Np, c.C, (F + 255) / 256, probs, idx, rank, drop,
+                                       gate, b.dgp, counts1, static_cast<float>(ls), dh,
+                                       c.ws + c.L.dhp, c.ws + c.L.dhs, dgate_p, drop_list, n_drop,
+                                       c.st));
+  else
+    SMOE_TRY(launch_router_bwd_dh(T, N, Np, c.C, (F + 255) / 256, probs, idx, rank, drop, gate,
+                                  b.dgp, counts, static_cast<float>(ls), dh, c.ws + c.L.dhp,
+                                  c.ws + c.L.dhs, dgate_p, drop_list, n_drop, c.st));
   float* colsum = c.at<float>(c.L.colsum);
   if (db_r) SMOE_TRY(launch_prob_colsum(T, N, dh, colsum, c.st));
   SMOE_TRY(launch_router_bwd_dw_tc(T, N, Np, d, c.ws + c.L.dhp, x, c.at<float>(c.L.rpart),
@@ -729,7 +751,13 @@ switch_status_t switch_layer_backward(const switch_config_t* cfg, const void* x,
   b.wrp = c.ws + c.L.wrp;
   b.n_router = N;
   b.n_pad = Np;
+  // top-2: the dX GEMM's rows stay per slot (two slots can hold one token)
+  // and are added per token, with the residual, afterwards
+  if (top2) b.dxs = c.at<float>(c.L.dxs);
   SMOE_TRY(launch_bwd_dx(b, c.st));
+  if (top2)
+    SMOE_TRY(launch_bwd_combine_top2(T, d, c.C, idx, rank, drop, b.dxs, dout, dx, residual,
+                                     c.st));
   SMOE_TRY(launch_bwd_dropped(T, N, d, drop_list, n_drop, dh, w_r, dout, dx, residual, c.st));
   return SWITCH_OK;
 }
