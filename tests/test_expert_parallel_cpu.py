@@ -172,3 +172,52 @@ def test_ep_protocol_two_gloo_ranks():
         assert out[q]["C"] == C
         assert out[q]["counts"] == want["counts"].tolist()
         assert out[q]["loss"] == pytest.approx(loss_want, rel=1e-6)
+
+
+def _rank_leaves_main(rank, world, port, out):
+    """Both ranks run one step; rank 1 then leaves (between steps, nothing in
+    flight); rank 0's next step must end with an error from its first
+    collective (the peer's connection closes, or the short process-group
+    timeout runs out) instead of waiting for ever."""
+    import datetime
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=5))
+    from sparse_mixture_experts_switch_b200 import switch_moe
+    from sparse_mixture_experts_switch_b200.expert_parallel import ExpertParallelSwitch
+    inp = make_inputs(WL)
+    Tr = WL.T // world
+    lib = OracleEpLib(switch_moe, WL, inp.x[rank * Tr:(rank + 1) * Tr], rank)
+
+    def peer_alloc(shape, dtype, device):
+        return torch.zeros(shape, dtype=dtype), [0] * world
+
+    layer = ExpertParallelSwitch(Tr, WL.d_model, WL.d_ff, WL.n_experts, WL.capacity_factor,
+                                 alpha=WL.alpha, device="cpu", peer_alloc=peer_alloc, lib=lib)
+    w_r, b_r = torch.from_numpy(inp.w_r), torch.from_numpy(inp.b_r)
+    layer.forward(None, w_r, b_r, None, None)
+    if rank == 1:
+        out[1] = "left"
+        os._exit(0)                      # gone without a goodbye
+    import time
+    t0 = time.monotonic()
+    try:
+        layer.forward(None, w_r, b_r, None, None)
+        out[0] = "completed"
+    except Exception as e:               # noqa: BLE001 -- any collective error counts
+        out[0] = f"error after {time.monotonic() - t0:.1f} s: {type(e).__name__}"
+    os._exit(0)
+
+
+def test_ep_rank_leaving_ends_the_next_step_with_an_error():
+    world = 2
+    port = _free_port()
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    ctx = mp.start_processes(_rank_leaves_main, args=(world, port, out), nprocs=world,
+                             join=False, start_method="spawn")
+    assert ctx.join(timeout=120) or ctx.join(timeout=60), "ranks did not finish"
+    assert out[1] == "left"
+    assert out[0].startswith("error after"), out[0]
+    assert float(out[0].split()[2]) < 60.0
+    print(out[0])

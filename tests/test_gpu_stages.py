@@ -332,31 +332,43 @@ def test_combine(sm, residual, dtype):
 
 # --------------------------------------------------------------- aux loss
 
-def test_aux_loss(sm):
-    wl = Workload("a", T=3333, d_model=128, d_ff=64, n_experts=24, capacity_factor=1.0,
+# (T, N): float4 columns; one column per thread (N % 4 != 0); blocks left
+# with no rows (T = 9473 over 148 blocks of 65 rows); N >= 512 (several
+# passes over the experts in the final sum), also with scalar columns
+AUX_CASES = [(3333, 24), (10000, 37), (9473, 128), (2000, 600), (777, 1001)]
+
+
+@pytest.mark.parametrize("T,N", AUX_CASES, ids=lambda v: str(v))
+def test_aux_loss(sm, T, N):
+    wl = Workload("a", T=T, d_model=128, d_ff=64, n_experts=N, capacity_factor=1.0,
                   dtype="bf16", seed=61)
     x = make_x(wl)
     w_r, _ = make_router(wl)
     r = orc.router(x, w_r)
-    C = orc.capacity(wl.T, 24, 1.0)
-    counts = orc.dispatch(r["idx"], 24, C)["counts"]
+    C = orc.capacity(wl.T, N, 1.0)
+    counts = orc.dispatch(r["idx"], N, C)["counts"]
     p32 = r["probs"].astype(np.float32)
     loss_w, f_w, P_w = orc.aux_loss(counts, p32.astype(np.float64), wl.alpha)
     cfg = _cfg(sm, wl)
     ws = sm.workspace(cfg)
     loss = torch.empty(1, **F32)
-    f = torch.empty(24, **F32)
-    P = torch.empty(24, **F32)
-    sm.switch_aux_loss(cfg, torch.from_numpy(counts.astype(np.int32)).cuda(),
-                       torch.from_numpy(p32).cuda(), loss, f, P, ws)
+    f = torch.empty(N, **F32)
+    P = torch.empty(N, **F32)
+    cnt = torch.from_numpy(counts.astype(np.int32)).cuda()
+    pd = torch.from_numpy(p32).cuda()
+    sm.switch_aux_loss(cfg, cnt, pd, loss, f, P, ws)
     _ok(sm, ws)
     assert abs(loss.item() - loss_w) <= LOSS_RTOL * loss_w
     assert rel_err(P.cpu().numpy(), P_w).max() <= LOSS_RTOL
     np.testing.assert_allclose(f.cpu().numpy(), f_w, rtol=1e-7)
+    # the same call again: bit for bit (fixed order of additions)
+    loss2, P2 = torch.empty_like(loss), torch.empty_like(P)
+    sm.switch_aux_loss(cfg, cnt, pd, loss2, None, P2, ws)
+    _ok(sm, ws)
+    assert torch.equal(loss, loss2) and torch.equal(P, P2)
     # uniform router: loss = alpha exactly in exact arithmetic
-    pu = np.full((wl.T, 24), 1.0 / 24, np.float32)
-    sm.switch_aux_loss(cfg, torch.from_numpy(counts.astype(np.int32)).cuda(),
-                       torch.from_numpy(pu).cuda(), loss, None, None, ws)
+    pu = np.full((wl.T, N), 1.0 / N, np.float32)
+    sm.switch_aux_loss(cfg, cnt, torch.from_numpy(pu).cuda(), loss, None, None, ws)
     _ok(sm, ws)
     assert abs(loss.item() - wl.alpha) <= LOSS_RTOL * wl.alpha
 
