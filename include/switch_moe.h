@@ -252,7 +252,7 @@ switch_status_t switch_layer_forward(const switch_config_t* cfg, const void* x,
                                      float* loss, void* ws, size_t ws_bytes,
                                      void* stream);
 
-/* Backward pass of switch_layer_forward (bf16; top-1, or top-2 below): the gradient of
+/* Backward pass of switch_layer_forward (bf16 or fp32; top-1, or top-2 below): the gradient of
  *   J = sum(dout * out) + dloss * loss
  * with respect to x, w_r, b_r, w1 and w2, routing decisions held fixed (the
  * argmax and the capacity cut are piecewise constant; f_i likewise).  The
@@ -277,13 +277,14 @@ switch_status_t switch_layer_forward(const switch_config_t* cfg, const void* x,
  * config, inputs and workspace, with no other call on the workspace in
  * between (backward calls may repeat: they leave that state unchanged).
  * Both ways give bit-identical gradients.
- *   x [T, d_model] bf16, w_r [N, d_model] fp32, b_r [N] fp32 or NULL,
- *   w1 [N, d_ff, d_model] bf16, w2 [N, d_model, d_ff] bf16 (as the forward);
- *   dout [T, d_model] bf16: gradient of J with respect to out;
+ *   x [T, d_model], w_r [N, d_model] fp32, b_r [N] fp32 or NULL,
+ *   w1 [N, d_ff, d_model], w2 [N, d_model, d_ff] (as the forward);
+ *   dout [T, d_model]: gradient of J with respect to out;
  *   dloss: host float, the weight of the loss in J;
- *   outputs: dx [T, d_model] bf16, dw_r [N, d_model] fp32, db_r [N] fp32 or
- *   NULL, dw1 [N, d_ff, d_model] bf16, dw2 [N, d_model, d_ff] bf16,
- *   dgate [T] fp32 or NULL (the gate gradient above).
+ *   outputs: dx [T, d_model], dw_r [N, d_model] fp32, db_r [N] fp32 or
+ *   NULL, dw1 [N, d_ff, d_model], dw2 [N, d_model, d_ff], dgate [T] fp32
+ *   or NULL (the gate gradient above); x, w1, w2, dout, dx, dw1 and dw2 in
+ *   cfg->dtype (bf16 or fp32).
  * Top-2 (SWITCH_FLAG_TOP2) [P1 "Switch Routing": out = x + sum over the
  * top-k set of p_i E_i(x), p the full softmax, not renormalised]: every kept
  * route r of token t (expert idx_r, gate p_{idx_r}) contributes its own
@@ -296,12 +297,13 @@ switch_status_t switch_layer_forward(const switch_config_t* cfg, const void* x,
  * route order with the residual and dh W_r).  dgate is then [2 T] fp32,
  * route-major.  A route whose gate underflowed to 0 reports dgate 0 (its
  * dY is 0; p = 0 removes it from dh in any case).
- * Arithmetic: expert GEMMs on the tensor cores (bf16 operands, fp32
- * accumulation; gate * dout, dA and the weight gradients rounded once to
- * bf16); router backward in fp32 FMA with fixed-order reductions (dW_r and
- * db_r bit-reproducible).  Workspace: switch_backward_workspace_size()
- * bytes.  dtype SWITCH_F32 returns SWITCH_ERR_UNSUPPORTED (so does
- * switch_layer_forward given SWITCH_FLAG_TRAINING with it).
+ * Arithmetic: bf16 -- expert GEMMs on the tensor cores (bf16 operands,
+ * fp32 accumulation; gate * dout, dA and the weight gradients rounded once
+ * to bf16); router backward in fp32 FMA with fixed-order reductions (dW_r
+ * and db_r bit-reproducible).  fp32 -- every product and sum in fp32 on
+ * CUDA-core FMA tiles (the path of small full-precision configurations),
+ * each output element one fixed-order loop, so all gradients are
+ * bit-reproducible.  Workspace: switch_backward_workspace_size() bytes.
  * T = 0 writes nothing. */
 switch_status_t switch_layer_backward(const switch_config_t* cfg, const void* x,
                                       const float* w_r, const float* b_r,

@@ -136,6 +136,40 @@ cudaError_t launch_router_bwd_dh_top2(int64_t T, int N, int Np, int64_t C, int n
 cudaError_t launch_bwd_combine_top2(int64_t T, int d, int64_t C, const int* idx, const int* rank,
                                     const uint8_t* drop, const float* dxs, const void* dout,
                                     void* dx, bool residual, cudaStream_t st);
+// ------------------------------------------------------------ fp32 path
+// The backward in fp32 on CUDA-core FMA tiles (backward_f32.cu).
+struct BwdF32Args {
+  int64_t T;
+  int d, F, N;
+  int64_t C;
+  const int* counts;        // [N]
+  const int* slot_token;    // [N*C]
+  const float* gate;        // [routes * T]
+  const int* idx;           // [routes * T]
+  int64_t T2;               // top-2: T (a slot's route from idx), else 0
+  const float* dout;        // [T, d]
+  const float* x;           // [T, d]
+  const float* w1;          // [N, F, d]
+  const float* w2;          // [N, d, F]
+  const float* h;           // [N*C, F] hidden activations of the forward
+  float* dys;               // [N*C, d] out: gate * dout per kept slot
+  float* da;                // [N*C, F] out
+  float* dgp;               // [N*C, bwd_f32_dgp_parts(F)] out
+  float* dw1;               // [N, F, d] out
+  float* dw2;               // [N, d, F] out
+  float* dxs;               // [N*C, d] out: dA W1_e per kept slot
+};
+// Gate-gradient partials per slot of the fp32 dH (one per 64 columns).
+int bwd_f32_dgp_parts(int F);
+// dY, dA and its gate-gradient partials, dW2, dW1 and the dX rows per slot.
+cudaError_t launch_bwd_f32_experts(const BwdF32Args& a, cudaStream_t st);
+// dW_r = dh^T x, db_r = column sums of dh (if db_r), and
+// dx[t] = residual + the token's kept slots' dX rows + dh[t] W_r.
+cudaError_t launch_bwd_f32_router(const BwdF32Args& a, int routes, const int* rank,
+                                  const uint8_t* drop, const float* dh, const float* w_r,
+                                  float* dw_r, float* db_r, float* dx, bool residual,
+                                  cudaStream_t st);
+
 // wrp [2][N][d] = hi / lo bf16 split of W_r (hi = bf16(W), lo = bf16(W - hi)).
 cudaError_t launch_wr_split(int N, int d, const float* w_r, void* wrp, cudaStream_t st);
 // Dropped tokens (from the list): dx[t] = bf16((residual ? dout[t] : 0) +

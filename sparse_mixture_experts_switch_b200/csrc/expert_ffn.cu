@@ -493,7 +493,7 @@ cudaError_t launch_expert_ffn_f32(const FfnArgs& a, cudaStream_t st) {
                                       static_cast<const float*>(a.w1),
                                       static_cast<float*>(a.hbuf), nullptr, nullptr);
   cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  if (e != cudaSuccess || a.gemm1_only) return e;
   const dim3 g2(static_cast<unsigned>((a.C + kSB - 1) / kSB),
                 static_cast<unsigned>((a.d + kSB - 1) / kSB), static_cast<unsigned>(a.N));
   float* out2 = a.mode2 == kModeCombine ? static_cast<float*>(a.out) : static_cast<float*>(a.y);

@@ -1,6 +1,7 @@
 // C ABI of the Switch-FFN layer (declared in include/switch_moe.h):
 // argument validation, exact capacity, workspace carving and the launch
 // sequence of each entry point.  No device memory is allocated here.
+#include <algorithm>
 #include <climits>
 #include <cmath>
 #include <cstring>
@@ -43,8 +44,8 @@ struct Layout {
   // backward pass only (after the forward regions): dA, partial gate
   // gradients, dh (fp32, and its bf16 planes per token and per slot), W_r
   // planes, gate gradient (per route), split-K partials of dW_r, column
-  // sums of dh, dropped-token list and its counter; top-2 only: the dX
-  // GEMM's fp32 rows per slot
+  // sums of dh, dropped-token list and its counter; top-2 and fp32 only:
+  // the dX GEMM's fp32 rows per slot
   size_t probs_s, da, dgp, dh, dhp, dhs, wrp, dgate, rpart, colsum, drop_list, n_drop, dxs,
       bwd_total;
 };
@@ -101,7 +102,8 @@ Layout layout_for(const switch_config_t& c, int64_t C) {
   const int64_t ntn = (c.d_ff + 255) / 256;
   L.probs_s = take(sizeof(float) * N * T);      // router probabilities kept for the backward
   L.da = take(es * slots * static_cast<size_t>(c.d_ff));
-  L.dgp = take(sizeof(float) * slots * ntn);
+  // gate-gradient partials: one per 256 columns (bf16 tiles) or 64 (fp32)
+  L.dgp = take(sizeof(float) * slots * std::max<int64_t>(ntn, (c.d_ff + 63) / 64));
   const int64_t Np = (N + 63) / 64 * 64;
   L.dh = take(sizeof(float) * N * T);
   L.dhp = take(2 * 2 * static_cast<size_t>(T) * Np);
@@ -112,7 +114,9 @@ Layout layout_for(const switch_config_t& c, int64_t C) {
   L.colsum = take(sizeof(float) * N * ntiles_of(T));
   L.drop_list = take(sizeof(int) * T);
   L.n_drop = take(sizeof(int));
-  L.dxs = take(routes_of(c) == 2 ? sizeof(float) * slots * static_cast<size_t>(c.d_model) : 0);
+  L.dxs = take(routes_of(c) == 2 || c.dtype != SWITCH_BF16
+                   ? sizeof(float) * slots * static_cast<size_t>(c.d_model)
+                   : 0);
   L.bwd_total = o;
   return L;
 }
@@ -489,10 +493,7 @@ switch_status_t switch_layer_forward(const switch_config_t* cfg, const void* x,
   // workspace for switch_layer_backward (routing arrays always in the
   // workspace, copied out to the caller's at the end)
   const bool training = (cfg->flags & SWITCH_FLAG_TRAINING) != 0;
-  if (training) {
-    if (!bf16) return SWITCH_ERR_UNSUPPORTED;
-    if (ws_bytes < c.L.bwd_total) return SWITCH_ERR_WORKSPACE_TOO_SMALL;
-  }
+  if (training && ws_bytes < c.L.bwd_total) return SWITCH_ERR_WORKSPACE_TOO_SMALL;
   int* idx_p = (idx && !training) ? idx : c.at<int>(c.L.idx);
   float* gate_p = (gate && !training) ? gate : c.at<float>(c.L.gate);
   int* counts_p = (counts && !training) ? counts : c.at<int>(c.L.counts);
@@ -600,8 +601,8 @@ switch_status_t switch_layer_backward(const switch_config_t* cfg, const void* x,
   Ctx c{};
   switch_status_t s = prepare(cfg, ws, ws_bytes, stream, &c);
   if (s != SWITCH_OK) return s;
-  if (cfg->dtype != SWITCH_BF16) return SWITCH_ERR_UNSUPPORTED;
   if (cfg->T == 0) return SWITCH_OK;
+  const bool bf16 = cfg->dtype == SWITCH_BF16;
   if (!x || !w_r || !w1 || !w2 || !dout || !dx || !dw_r || !dw1 || !dw2 || !aligned16(x) ||
       !aligned16(w_r) ||
       !aligned16(w1) || !aligned16(w2) || !aligned16(dout) || !aligned16(dx) ||
@@ -636,8 +637,8 @@ switch_status_t switch_layer_backward(const switch_config_t* cfg, const void* x,
   const bool saved = (cfg->flags & SWITCH_FLAG_TRAINING) != 0;
   if (saved) {
     // 1'. the forward (same flag) left probabilities, routing and H here;
-    // only the row copy is missing if it gathered inside GEMM1
-    if (cfg->flags & SWITCH_FLAG_GATHER_IN_GEMM)
+    // only the row copy is missing if it gathered inside GEMM1 (bf16)
+    if (bf16 && (cfg->flags & SWITCH_FLAG_GATHER_IN_GEMM))
       SMOE_TRY(launch_gather_rows(S, static_cast<int64_t>(d) * 2, slot_token, x, x_disp, c.st));
   } else {
     // 1. the forward's routing, dispatch and hidden activations, recomputed
@@ -651,8 +652,8 @@ switch_status_t switch_layer_backward(const switch_config_t* cfg, const void* x,
                                 c.err, c.spin, c.num_sms, c.st));
     } else {
       int nparts = 0;
-      SMOE_TRY(launch_router_simt(T, d, N, true, x, w_r, b_r, c.at<float>(c.L.logits), o, &nparts,
-                                  c.st));
+      SMOE_TRY(launch_router_simt(T, d, N, bf16, x, w_r, b_r, c.at<float>(c.L.logits), o,
+                                  &nparts, c.st));
       SMOE_TRY(launch_tile_rank(T, N, idx, nullptr, nullptr, local_rank, hist, nt, c.err, c.st));
     }
     if (top2) {
@@ -662,9 +663,13 @@ switch_status_t switch_layer_backward(const switch_config_t* cfg, const void* x,
                                 c.st));
     }
     SMOE_TRY(launch_scan(N, nta, hist, c.at<int>(c.L.base), counts, c.st));
-    SMOE_TRY(launch_finalize_gather(A, N, c.C, nta, idx, local_rank, c.at<int>(c.L.base), counts,
-                                    rank, drop, slot_token, mtile_start, top2 ? T : 0, x, x_disp,
-                                    static_cast<int64_t>(d) * 2, c.st));
+    if (bf16)
+      SMOE_TRY(launch_finalize_gather(A, N, c.C, nta, idx, local_rank, c.at<int>(c.L.base),
+                                      counts, rank, drop, slot_token, mtile_start, top2 ? T : 0,
+                                      x, x_disp, static_cast<int64_t>(d) * 2, c.st));
+    else      // fp32: GEMM1 gathers its rows from x
+      SMOE_TRY(launch_finalize(A, N, c.C, nta, idx, local_rank, c.at<int>(c.L.base), counts, rank,
+                               drop, slot_token, mtile_start, top2 ? T : 0, c.st));
     FfnArgs a{};
     a.T = T;
     a.d = d;
@@ -672,7 +677,7 @@ switch_status_t switch_layer_backward(const switch_config_t* cfg, const void* x,
     a.N = N;
     a.C = c.C;
     a.x = x;
-    a.x_disp = x_disp;
+    a.x_disp = bf16 ? x_disp : nullptr;
     a.slot_token = slot_token;
     a.counts = counts;
     a.mtile_start = mtile_start;
@@ -686,7 +691,54 @@ switch_status_t switch_layer_backward(const switch_config_t* cfg, const void* x,
     a.err = c.err;
     a.spin = c.spin;
     a.num_sms = c.num_sms;
-    SMOE_TRY(launch_expert_ffn_bf16(a, c.st));
+    SMOE_TRY(bf16 ? launch_expert_ffn_bf16(a, c.st) : launch_expert_ffn_f32(a, c.st));
+  }
+
+  const int Np = (N + 63) / 64 * 64;
+  float* dh = c.at<float>(c.L.dh);
+  int* n_drop = c.at<int>(c.L.n_drop);
+  int* drop_list = c.at<int>(c.L.drop_list);
+  const double ls = static_cast<double>(dloss) * cfg->alpha * N / (static_cast<double>(T) * T);
+  float* dgate_p = dgate ? dgate : c.at<float>(c.L.dgate);
+  if (!bf16) {
+    // fp32: the expert gradients on CUDA-core tiles, then the router's; dx
+    // per token from its slots' rows, the router term and the residual
+    BwdF32Args f{};
+    f.T = T;
+    f.d = d;
+    f.F = F;
+    f.N = N;
+    f.C = c.C;
+    f.counts = counts;
+    f.slot_token = slot_token;
+    f.gate = gate;
+    f.idx = idx;
+    f.T2 = top2 ? T : 0;
+    f.dout = static_cast<const float*>(dout);
+    f.x = static_cast<const float*>(x);
+    f.w1 = static_cast<const float*>(w1);
+    f.w2 = static_cast<const float*>(w2);
+    f.h = static_cast<const float*>(hbuf);
+    f.dys = c.at<float>(c.L.ybuf);
+    f.da = c.at<float>(c.L.da);
+    f.dgp = c.at<float>(c.L.dgp);
+    f.dw1 = static_cast<float*>(dw1);
+    f.dw2 = static_cast<float*>(dw2);
+    f.dxs = c.at<float>(c.L.dxs);
+    SMOE_TRY(launch_bwd_f32_experts(f, c.st));
+    SMOE_TRY(cudaMemsetAsync(n_drop, 0, sizeof(int), c.st));
+    const int ntn = bwd_f32_dgp_parts(F);
+    if (top2)
+      SMOE_TRY(launch_router_bwd_dh_top2(T, N, Np, c.C, ntn, probs, idx, rank, drop, gate, f.dgp,
+                                         counts1, static_cast<float>(ls), dh, c.ws + c.L.dhp,
+                                         c.ws + c.L.dhs, dgate_p, drop_list, n_drop, c.st));
+    else
+      SMOE_TRY(launch_router_bwd_dh(T, N, Np, c.C, ntn, probs, idx, rank, drop, gate, f.dgp,
+                                    counts, static_cast<float>(ls), dh, c.ws + c.L.dhp,
+                                    c.ws + c.L.dhs, dgate_p, drop_list, n_drop, c.st));
+    SMOE_TRY(launch_bwd_f32_router(f, routes_of(*cfg), rank, drop, dh, w_r, dw_r, db_r,
+                                   static_cast<float*>(dx), residual, c.st));
+    return SWITCH_OK;
   }
 
   // 2. dY = gate * dout per kept slot; dA and the gate-gradient partials;
@@ -723,13 +775,7 @@ switch_status_t switch_layer_backward(const switch_config_t* cfg, const void* x,
   SMOE_TRY(launch_bwd_dw(b, c.st));
 
   // 3. router: dh and its bf16 planes, the weight and bias gradients
-  float* dh = c.at<float>(c.L.dh);
-  const int Np = (N + 63) / 64 * 64;
-  int* n_drop = c.at<int>(c.L.n_drop);
-  int* drop_list = c.at<int>(c.L.drop_list);
-  const double ls = static_cast<double>(dloss) * cfg->alpha * N / (static_cast<double>(T) * T);
   SMOE_TRY(cudaMemsetAsync(n_drop, 0, sizeof(int), c.st));
-  float* dgate_p = dgate ? dgate : c.at<float>(c.L.dgate);
   if (top2)
     SMOE_TRY(launch_router_bwd_dh_top2(T, N, Np, c.C, (F + 255) / 256, probs, idx, rank, drop,
                                        gate, b.dgp, counts1, static_cast<float>(ls), dh,

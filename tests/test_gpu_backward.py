@@ -260,16 +260,19 @@ def test_backward_deterministic(sm):
         assert np.array_equal(a[k], b[k], equal_nan=True), k
 
 
-def test_backward_rejects_unsupported(sm):
+def test_backward_rejects_misaligned_arguments(sm):
+    """A pointer that is not 16-byte aligned is refused before any launch
+    (both dtypes); nothing is written."""
     wl = SMALL
-    for flags, dtype in ((0, "f32"),):
+    for dtype in ("bf16", "f32"):
         cfg = sm.config(wl.T, wl.d_model, wl.d_ff, wl.n_experts, wl.capacity_factor,
-                        dtype=dtype, alpha=wl.alpha, flags=flags)
+                        dtype=dtype, alpha=wl.alpha)
         ws = sm.backward_workspace(cfg)
-        t = torch.zeros(8, device="cuda")
+        t = torch.zeros(64, device="cuda")
         with pytest.raises(sm.SwitchError) as ei:
-            sm.switch_layer_backward(cfg, t, t, None, t, t, t, 1.0, t, t, None, t, t, None, ws)
-        assert ei.value.status == 2
+            sm.switch_layer_backward(cfg, t[1:], t, None, t, t, t, 1.0, t, t, None, t, t, None,
+                                     ws)
+        assert ei.value.status == 1
 
 
 def test_backward_workspace_too_small(sm):
