@@ -18,6 +18,7 @@ import argparse
 import datetime
 import json
 import os
+import select
 import statistics
 import subprocess
 import sys
@@ -44,9 +45,10 @@ L2_FLUSH_BYTES = 256 << 20
 GEMM_SOURCES = ("common.cuh", "gemm_common.cuh", "gemm_pair.cuh", "expert_ffn.cu",
                 "expert_ffn_pair.cu", "expert_ffn_pair_rows.cu")
 GEMM_TRAFFIC = {"workload": "base",
-                "sources_sha256": "f115382257c4210eec65746c4eb1247239b854e35d34c5d5ea0879661d8ffed6",
-                # GEMM1 715.8 MB read + 367.7 MB written; GEMM2 1231.6 + 89.2 MB
-                "bytes": 715.76e6 + 367.73e6 + 1231.59e6 + 89.25e6}
+                "sources_sha256": "6aab2fb984fd416352e3c1c71cb906257297a029786ee11003080e3aa3259b90",
+                # GEMM1 715.75 MB read + 368.26 MB written; GEMM2 1233.39 + 89.68 MB
+                # (mean of four forwards; profiles/layer_kernels_dram_base.md)
+                "bytes": 715.75e6 + 368.26e6 + 1233.39e6 + 89.68e6}
 
 
 def gemm_sources_sha256():
@@ -205,18 +207,55 @@ class ClockSampler:
         self.thread = None
         self.source = None
 
+    # The NVML loop runs in a child process of its own, so that the bench
+    # process's interpreter lock (held while it launches and waits) cannot
+    # starve it; each line carries the child's wall-clock time of the sample.
+    NVML_CHILD = r"""
+import sys, time, pynvml
+pynvml.nvmlInit()
+uuid, idx, period = sys.argv[1], int(sys.argv[2]), float(sys.argv[3])
+h = pynvml.nvmlDeviceGetHandleByUUID(uuid) if uuid else pynvml.nvmlDeviceGetHandleByIndex(idx)
+bits = (pynvml.nvmlClocksEventReasonHwSlowdown, pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+        pynvml.nvmlClocksEventReasonSwThermalSlowdown, pynvml.nvmlClocksEventReasonSwPowerCap)
+mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+pw, n = 0.0, 0
+for _ in range(3):          # the first queries are slow: make them before reporting ready
+    pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+    pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+    pynvml.nvmlDeviceGetPowerUsage(h)
+print("ready", flush=True)
+while True:
+    try:
+        sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+        rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+        if n % 8 == 0:
+            pw = pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0
+        n += 1
+        flags = "".join("1" if rs & b else "0" for b in bits)
+        print(f"{time.time():.6f},{sm},{mx},{pw:.1f},{flags}", flush=True)
+    except pynvml.NVMLError:
+        pass
+    time.sleep(period)
+"""
+
     def start(self):
         try:
-            import pynvml
-            pynvml.nvmlInit()
-            h = (pynvml.nvmlDeviceGetHandleByUUID(self.uuid) if self.uuid
-                 else pynvml.nvmlDeviceGetHandleByIndex(int(self.gpu_id)))
+            import pynvml  # noqa: F401 -- the child needs it too
+            self.proc = subprocess.Popen(
+                [sys.executable, "-c", self.NVML_CHILD, self.uuid or "", str(self.gpu_id or 0),
+                 str(self.period_s)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            ready, _, _ = select.select([self.proc.stdout], [], [], 30.0)
+            if not ready or self.proc.stdout.readline().strip() != "ready":
+                raise RuntimeError("NVML sampler did not start")
             self.source = "nvml"
-            self.thread = threading.Thread(target=self._nvml, args=(pynvml, h), daemon=True)
+            self.thread = threading.Thread(target=self._nvml_lines, daemon=True)
             self.thread.start()
             return
         except Exception:
-            pass
+            if self.proc is not None:
+                self.proc.kill()
+                self.proc = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
@@ -228,26 +267,14 @@ class ClockSampler:
         except Exception:
             self.proc = None
 
-    def _nvml(self, pynvml, h):
-        bits = (pynvml.nvmlClocksEventReasonHwSlowdown,
-                pynvml.nvmlClocksEventReasonHwThermalSlowdown,
-                pynvml.nvmlClocksEventReasonSwThermalSlowdown,
-                pynvml.nvmlClocksEventReasonSwPowerCap)
-        mx = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
-        pw = 0.0
-        n = 0
-        while not self.stop_evt.is_set():
+    def _nvml_lines(self):
+        for ln in self.proc.stdout:
+            r = ln.strip().split(",")
             try:
-                sm = float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM))
-                rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
-                if n % 8 == 0:                      # power changes slowly: read it less often
-                    pw = pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0
-                n += 1
-                names = [n_ for n_, bit in zip(self.REASONS, bits) if rs & bit]
-                self.rows.append((time.time(), sm, mx, pw, names))
-            except Exception:
+                self.rows.append((float(r[0]), float(r[1]), float(r[2]), float(r[3]),
+                                  [n for n, f in zip(self.REASONS, r[4]) if f == "1"]))
+            except (ValueError, IndexError):
                 pass
-            time.sleep(self.period_s)
 
     def _smi(self):
         names = self.REASONS
