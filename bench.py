@@ -481,35 +481,67 @@ def main():
     value = job_throughput(T, args.steps, world, total_ms)
 
     # ------------------------------------------- end to end (host buffers)
+    # Each step copies its input from pinned host memory, runs the layer
+    # through the public call, and copies its output and loss back, as a
+    # serving loop would: on three streams, so that step i's input copy and
+    # step i-1's output copy (separate copy engines, both PCIe directions)
+    # run while step i-1 / step i compute; two device input and output
+    # buffers alternate, and events order every reuse.
     x_host = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
     x_host.copy_(x)
-    out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-    loss_host = torch.empty(1, dtype=torch.float32, pin_memory=True)
+    out_host = [torch.empty(out.shape, dtype=out.dtype, pin_memory=True) for _ in range(2)]
+    loss_host = [torch.empty(1, dtype=torch.float32, pin_memory=True) for _ in range(2)]
+    xb = [x, torch.empty_like(x)]
+    ob = [out, torch.empty_like(out)]
+    lb = [loss, torch.empty_like(loss)]
+    s_in = torch.cuda.Stream(dev)
+    s_out = torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()                        # noqa: E731
 
-    def e2e_step():
-        x.copy_(x_host, non_blocking=True)
-        step()
-        out_host.copy_(out, non_blocking=True)
-        loss_host.copy_(loss, non_blocking=True)
+    def e2e_run(n):
+        """n pipelined steps; returns (first event, last event) for timing."""
+        t_first = torch.cuda.Event(enable_timing=True)
+        t_last = torch.cuda.Event(enable_timing=True)
+        in_done, comp_done, out_done = {}, {}, {}
+        t_first.record(s_in)
+        for i in range(n):
+            b = i % 2
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(comp_done[i - 2])      # step i-2 has read xb[b]
+                xb[b].copy_(x_host, non_blocking=True)
+                in_done[i] = ev()
+                in_done[i].record(s_in)
+            stream.wait_event(in_done[i])
+            if i >= 2:
+                stream.wait_event(out_done[i - 2])         # ob[b] copied out
+            sm.switch_layer_forward(cfg, xb[b], w_r, b_r, w1, w2, ob[b], None, None, None,
+                                    lb[b], ws)
+            comp_done[i] = ev()
+            comp_done[i].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(comp_done[i])
+                out_host[b].copy_(ob[b], non_blocking=True)
+                loss_host[b].copy_(lb[b], non_blocking=True)
+                out_done[i] = ev()
+                out_done[i].record(s_out)
+        s_in.wait_stream(s_out)
+        s_in.wait_stream(stream)
+        t_last.record(s_in)
+        return t_first, t_last
 
-    for _ in range(max(3, args.warmup)):
-        e2e_step()
+    e2e_run(max(3, args.warmup))
     barrier()
     torch.cuda.synchronize(dev)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e1.record(stream)
+    e0, e1 = e2e_run(args.steps)
     torch.cuda.synchronize(dev)
     barrier()
     e2e_value = job_throughput(T, args.steps, world,
                                max_over_ranks(e0.elapsed_time(e1), dev, world))
     e2e_bytes = (x_host.numel() * x_host.element_size(),
-                 out_host.numel() * out_host.element_size() + loss_host.numel() * 4)
+                 out_host[0].numel() * out_host[0].element_size() + loss_host[0].numel() * 4)
     clocks.stop()
-    del x_host, out_host, step_graph
+    del x_host, out_host, step_graph, xb, ob
 
     # --------------------------------------- per-kernel roofline (rank 0)
     line = None
