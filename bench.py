@@ -38,16 +38,16 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 L2_FLUSH_BYTES = 256 << 20
 
 # DRAM bytes (read + written) of one GEMM1 + GEMM2 launch pair on the Base
-# workload, from ncu captures of those kernels (profiles/
-# expert_gemm_base_full.md), valid only for the kernel sources they were
-# taken on: the bench reports them as `traffic` while the sources hash the
-# same, and null once a kernel has changed.
+# workload, from a one-pass ncu capture of those kernels (dram__bytes_read.sum
+# + dram__bytes_write.sum, caches flushed before each kernel), valid only for
+# the kernel sources they were taken on: the bench reports them as `traffic`
+# while the sources hash the same, and null once a kernel has changed.
 GEMM_SOURCES = ("common.cuh", "gemm_common.cuh", "gemm_pair.cuh", "expert_ffn.cu",
                 "expert_ffn_pair.cu", "expert_ffn_pair_rows.cu")
 GEMM_TRAFFIC = {"workload": "base",
                 "sources_sha256": "6aab2fb984fd416352e3c1c71cb906257297a029786ee11003080e3aa3259b90",
                 # GEMM1 715.75 MB read + 368.26 MB written; GEMM2 1233.39 + 89.68 MB
-                # (mean of four forwards; profiles/layer_kernels_dram_base.md)
+                # (mean of four forwards of one capture)
                 "bytes": 715.75e6 + 368.26e6 + 1233.39e6 + 89.68e6}
 
 
