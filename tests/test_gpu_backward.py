@@ -193,6 +193,17 @@ def test_backward_many_experts(sm):
     check_backward(sm, wl, dloss=2.0)
 
 
+def test_backward_wide_router(sm):
+    """N = 300: the tensor-core router with several weight tiles, planes padded
+    to 320 columns, five extra K blocks per term in the dX GEMM.  About 40
+    kept tokens per expert, so that a weight gradient is a sum of as many
+    terms as the tolerance's derivation assumes (with ~10 its error tail is
+    heavier)."""
+    wl = Workload("bwd_n300", T=12000, d_model=128, d_ff=128, n_experts=300,
+                  capacity_factor=1.5, dtype="bf16", seed=33)
+    check_backward(sm, wl, dloss=1.5)
+
+
 def _forward_all(sm, cfg, dev, ws):
     x, w_r, b_r, w1, w2 = dev
     out = torch.empty_like(x)

@@ -145,6 +145,15 @@ def test_backward_top2_many_experts_tiny_batch(sm):
         check_backward_top2(sm, wl, dloss=2.0)
 
 
+def test_backward_top2_wide_router(sm):
+    """N = 300 with top-2: the FMA router (the CTA-pair router's top-2 form
+    takes N <= 128), planes padded to 320 columns; about 40 kept assignments
+    per expert."""
+    wl = Workload("bwd2_n300", T=6000, d_model=128, d_ff=128, n_experts=300,
+                  capacity_factor=1.5, dtype="bf16", seed=35)
+    check_backward_top2(sm, wl, dloss=1.5)
+
+
 def _all_grads(sm, cfg, dev, g, ws):
     x, w_r, b_r, w1, w2 = dev
     outs = [torch.empty_like(x), torch.empty_like(w_r),
