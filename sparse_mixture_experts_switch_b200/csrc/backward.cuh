@@ -69,6 +69,10 @@ struct BwdFfnArgs {
 
 // dA = (dY W2_e) masked by H > 0, and the per-slot partial gate gradients.
 cudaError_t launch_bwd_dh(const BwdFfnArgs& a, cudaStream_t st);
+// 3-D bf16 TMA descriptor [outer][mid][inner], box 1 x box_mid x box_inner,
+// 128-byte swizzle (backward_gemm.cu).
+bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t mid,
+                       uint64_t outer, uint32_t box_inner, uint32_t box_mid);
 // dW2_e = dY_e^T H_e, dW1_e = dA_e^T X_e for every expert (zeros when empty).
 cudaError_t launch_bwd_dw(const BwdFfnArgs& a, cudaStream_t st);
 // dx of kept tokens: residual + dA W1_e + dh W_r (the router term as three
@@ -76,6 +80,9 @@ cudaError_t launch_bwd_dw(const BwdFfnArgs& a, cudaStream_t st);
 // slots may hold one token) each kept slot's fp32 row dA W1_e + dh_s W_r is
 // stored at its slot instead, without the residual.
 cudaError_t launch_bwd_dx(const BwdFfnArgs& a, cudaStream_t st);
+// The same on operand-swapped CTA pairs (output features x slots per tile,
+// slots as the MMA's flexible N; backward_pair.cu).
+cudaError_t launch_bwd_dx_pair(const BwdFfnArgs& a, cudaStream_t st);
 // dW_r [N, d] = dh^T x on the tensor cores: dh as hi + lo bf16 planes
 // dhp [2][T][Np] (x is exact in bf16), split-K over token chunks into fp32
 // partials `part`, then summed in a fixed order; db [N] (or null) = sum of

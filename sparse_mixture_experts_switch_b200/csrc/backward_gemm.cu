@@ -778,8 +778,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBwdThreads, 1)
 
 // 3-D bf16 tensor [outer][mid][inner] (inner contiguous), 128-byte swizzle,
 // box box_inner x box_mid x 1; out-of-range elements read as zero.
-static bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t mid,
-                              uint64_t outer, uint32_t box_inner, uint32_t box_mid) {
+bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t mid,
+                       uint64_t outer, uint32_t box_inner, uint32_t box_mid) {
   PFN_encodeTiled enc = get_encode_fn();
   if (enc == nullptr) return false;
   const cuuint64_t dims[3] = {inner, mid, outer};

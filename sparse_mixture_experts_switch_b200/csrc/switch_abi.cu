@@ -800,7 +800,9 @@ switch_status_t switch_layer_backward(const switch_config_t* cfg, const void* x,
   // top-2: the dX GEMM's rows stay per slot (two slots can hold one token)
   // and are added per token, with the residual, afterwards
   if (top2) b.dxs = c.at<float>(c.L.dxs);
-  SMOE_TRY(launch_bwd_dx(b, c.st));
+  // on operand-swapped CTA pairs unless one-CTA GEMMs are asked for
+  SMOE_TRY((cfg->flags & SWITCH_FLAG_GEMM_1SM) ? launch_bwd_dx(b, c.st)
+                                               : launch_bwd_dx_pair(b, c.st));
   if (top2)
     SMOE_TRY(launch_bwd_combine_top2(T, d, c.C, idx, rank, drop, b.dxs, dout, dx, residual,
                                      c.st));
