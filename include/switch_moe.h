@@ -89,8 +89,10 @@ enum {
                                         workspace; the backward then reads it instead of
                                         recomputing (see switch_layer_backward) */
   SWITCH_FLAG_GEMM1_ROWS_PAIRS = 2048 /* bf16 GEMM1 on CTA pairs with 256 dispatched rows x 256
-                                        columns per tile (needs the row copy: not with
-                                        SWITCH_FLAG_GATHER_IN_GEMM) */
+                                        columns per tile, an expert's last 128 rows as a half
+                                        tile (needs the row copy: not with
+                                        SWITCH_FLAG_GATHER_IN_GEMM); the default already when
+                                        128 < C <= 256 or d_model >= 2048 */
 };
 
 typedef struct {

@@ -378,8 +378,13 @@ cudaError_t launch_expert_ffn_bf16(const FfnArgs& a, cudaStream_t st) {
   g1.err = a.err;
   g1.spin = a.spin;
   cudaError_t e;
-  if (rows1)
-    e = run_gemm_pair_rows(ta1, tb1, to1, g1, a.num_sms, st);
+  if (rows1) {
+    // the half tiles' 64-row boxes of the dispatched rows
+    CUtensorMap ta1h;
+    if (!make_tmap_bf16_2d(&ta1h, a.x_disp, a.d, slots, kBK, kBM / 2))
+      return cudaErrorInvalidValue;
+    e = run_gemm_pair_rows(ta1, ta1h, tb1, to1, g1, a.num_sms, st);
+  }
   else if (a.pair1)
     e = gather ? run_gemm_pair<true>(ta1, tb1, to1, g1, a.num_sms, st)
                : run_gemm_pair<false>(ta1, tb1, to1, g1, a.num_sms, st);

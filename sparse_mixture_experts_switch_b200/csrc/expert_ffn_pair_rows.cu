@@ -9,12 +9,22 @@
 // tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 16), and each CTA's TMEM
 // receives its 128 rows x all 256 columns.  So every SM streams 32 KB per
 // 64-deep K step (instead of 48 KB for a one-CTA 128 x 256 tile) for the same
-// tensor work, and the MMA's N is always full.  The price is that an
-// expert's last row tile is padded to 256 rows instead of 128.
+// tensor work, and the MMA's N is always full.
 //
-// The epilogue is the one-CTA kernel's (epilogue_tile: one TMEM lane = one
+// An expert's last pair tile, when it covers only one 128-row M tile (its
+// kept rows end in the first half of the 256), is a half tile: each CTA
+// loads 64 of the rows (a 64-row box) and the leader issues the M = 128 form
+// of tcgen05.mma.cta_group::2, so the tile costs half a pair tile instead of
+// padding the expert to 256 rows.  Its accumulator is laid out across the
+// pair's TMEM in the 2 x 2 datapath form: in each CTA, TMEM lanes 0-63 hold
+// that CTA's 64 rows x output columns 0-127, lanes 64-127 the same rows x
+// columns 128-255, both at accumulator columns 0-127.
+//
+// The epilogue is the one-CTA kernel's (epilogue_rows: one TMEM lane = one
 // output row per thread; ReLU and 32 x 32 TMA box stores for the hidden
-// activations), run by each CTA on its 128 rows.  Two TMEM accumulators
+// activations), run by each CTA on its 128 rows (on a half tile: warps of
+// lane quarters 0-1 on the first 128 columns of its 64 rows, quarters 2-3 on
+// the last 128).  Two TMEM accumulators
 // alternate between tiles; the four epilogue warps of both CTAs hand an
 // accumulator back to the leader.  No copy here is multicast.
 #include <cstring>
@@ -25,6 +35,7 @@ namespace smoe {
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     expert_gemm_pair_rows_kernel(const __grid_constant__ CUtensorMap tmap_a,
+                                 const __grid_constant__ CUtensorMap tmap_a64,
                                  const __grid_constant__ CUtensorMap tmap_w,
                                  const __grid_constant__ CUtensorMap tmap_out, GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -88,6 +99,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     // ------------------------------------------------------- TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&tmap_a);
+      tma_prefetch_desc(&tmap_a64);
       tma_prefetch_desc(&tmap_w);
       int stage = 0;
       uint32_t phase = 0;
@@ -97,9 +109,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         if (*abort_flag) break;
         int e, tt, n;
         decode_tile(tile, pts, p.N, p.ntiles_n, e, tt, n);
+        const bool half = 2 * tt + 1 == mts[e + 1] - mts[e];   // one 128-row M tile
         const int a_row = static_cast<int>(static_cast<int64_t>(e) * p.C + tt * 256 +
-                                           static_cast<int>(rank) * 128);
+                                           static_cast<int>(rank) * (half ? 64 : 128));
         const int w_row = e * p.n_out + n * kBN + static_cast<int>(rank) * 128;
+        const uint32_t tx = 2 * (half ? kPairTokBytes / 2 + kPairWBytes : kPairStageBytes);
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, lim)) {
             report_error(p.err, SWITCH_ERR_TIMEOUT, kWhereGemmProducer, tile);
@@ -109,8 +123,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           }
           uint8_t* sa = smem + stage * kPairStageBytes;
           const uint32_t bar = full_lead + 8u * stage;
-          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * kPairStageBytes);
-          tma_load_2d_pair(sa, &tmap_a, bar, kb * kBK, a_row);
+          if (leader) mbar_arrive_expect_tx(&full[stage], tx);
+          tma_load_2d_pair(sa, half ? &tmap_a64 : &tmap_a, bar, kb * kBK, a_row);
           tma_load_2d_pair(sa + kPairTokBytes, &tmap_w, bar, kb * kBK, w_row);
           issued_mask |= 1u << stage;
           issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
@@ -129,13 +143,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   } else if (warp == 1) {
     // ----------------------------------------------------- MMA issuer
     if (leader && lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(2 * kBM, kBN);
+      constexpr uint32_t idesc_full = idesc_bf16_f32(2 * kBM, kBN);
+      constexpr uint32_t idesc_half = idesc_bf16_f32(kBM, kBN);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool any = false;
       for (int tile = cid; tile < total && !*abort_flag; tile += ncl) {
+        int e, tt, n;
+        decode_tile(tile, pts, p.N, p.ntiles_n, e, tt, n);
+        const uint32_t idesc = 2 * tt + 1 == mts[e + 1] - mts[e] ? idesc_half : idesc_full;
         if (!mbar_wait_cluster(&tempty[acc], acc_phase ^ 1u, lim)) {
           report_error(p.err, SWITCH_ERR_TIMEOUT, kWhereGemmMma, tile);
           *abort_flag = 1;
@@ -194,11 +212,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       int e, tt, n;
       decode_tile(tile, pts, p.N, p.ntiles_n, e, tt, n);
-      // this CTA's rows are the 128-row tile 2 tt + rank of the expert
-      epilogue_tile(p, &tmap_out, e, 2 * tt + static_cast<int>(rank), n,
-                    tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                        static_cast<uint32_t>(acc * kBN),
-                    stg, tokw, q, lane);
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                             static_cast<uint32_t>(acc * kBN);
+      if (2 * tt + 1 != mts[e + 1] - mts[e]) {
+        // this CTA's rows are the 128-row tile 2 tt + rank of the expert
+        epilogue_tile(p, &tmap_out, e, 2 * tt + static_cast<int>(rank), n, taddr, stg, tokw, q,
+                      lane);
+      } else {
+        // half tile: rows tt*256 + 64 rank + 32 (q % 2) .., columns
+        // n*256 + 128 (q / 2) .., at accumulator columns 0-127
+        const int col_base = n * kBN + (q >> 1) * 128;
+        const int ncols = p.n_out - col_base < 128 ? p.n_out - col_base : 128;
+        if (ncols > 0)
+          epilogue_rows(p, &tmap_out, e,
+                        static_cast<int64_t>(tt) * 256 + static_cast<int>(rank) * 64 +
+                            (q & 1) * 32,
+                        col_base, ncols, taddr, stg, tokw, lane);
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
@@ -218,7 +248,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   if (warp == 1) tmem_dealloc_pair(tmem_base, kTmemCols);
 }
 
-cudaError_t run_gemm_pair_rows(const CUtensorMap& ta, const CUtensorMap& tw, const CUtensorMap& to,
+cudaError_t run_gemm_pair_rows(const CUtensorMap& ta, const CUtensorMap& ta64,
+                               const CUtensorMap& tw, const CUtensorMap& to,
                                const GemmParams& gp, int num_sms, cudaStream_t st) {
   const size_t smem = gemm_pair_smem_bytes(gp.N);
   static size_t smem_set[64] = {};
@@ -226,7 +257,7 @@ cudaError_t run_gemm_pair_rows(const CUtensorMap& ta, const CUtensorMap& tw, con
                                     smem, smem_set);
   if (e != cudaSuccess) return e;
   const int grid = (num_sms / 2) * 2;
-  expert_gemm_pair_rows_kernel<<<grid, kGemmThreads, smem, st>>>(ta, tw, to, gp);
+  expert_gemm_pair_rows_kernel<<<grid, kGemmThreads, smem, st>>>(ta, ta64, tw, to, gp);
   return cudaGetLastError();
 }
 

@@ -94,16 +94,19 @@ __device__ __forceinline__ void prefetch_residual(const GemmParams& p, int tok, 
 //     transposed through the buffer so that each global store instruction
 //     writes 8 rows x 64 bytes, rows past the expert's count skipped; the
 //     combine adds the residual row and scales by the token's gate.
-__device__ __forceinline__ void epilogue_tile(const GemmParams& p, const CUtensorMap* tmap_out,
-                                              int e, int m, int n, uint32_t taddr, uint32_t stg,
-                                              int* tokw, int q, int lane) {
+// The general form: the warp's 32 rows start at row `rbase` of expert e,
+// and its accumulator holds `ncols` output columns from `col_base` (a
+// multiple of 64) on, read from TMEM at taddr, taddr + 32, ...
+__device__ __forceinline__ void epilogue_rows(const GemmParams& p, const CUtensorMap* tmap_out,
+                                              int e, int64_t rbase, int col_base, int ncols,
+                                              uint32_t taddr, uint32_t stg, int* tokw,
+                                              int lane) {
   const int qq = lane & 3;          // 8-column group in the transposed pass
   const int rr0 = lane >> 2;        // row within an 8-row pass
   const int64_t n_e = kept_rows(p, e);
-  const int64_t rbase = static_cast<int64_t>(m) * kBM + q * 32;   // first row of this warp
   const bool valid = rbase + lane < n_e;
   const bool bulk = p.mode != kModeCombine && rbase + 32 <= n_e;
-  const int nch = (p.n_out - n * kBN < kBN ? p.n_out - n * kBN : kBN) / 32;   // even: n_out % 64 == 0
+  const int nch = ncols / 32;       // even: n_out % 64 == 0
   float g = 1.f;
   if (p.mode == kModeCombine) {
     const int tk = valid ? p.slot_token[static_cast<int64_t>(e) * p.C + rbase + lane] : 0;
@@ -135,13 +138,13 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, const CUtenso
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
-      tma_store_2d(tmap_out, buf, n * kBN + c * 32, box_row);
+      tma_store_2d(tmap_out, buf, col_base + c * 32, box_row);
       bulk_commit();
     }
   };
 
   auto chunk_lsu = [&](int c, const uint32_t* u) {
-    const int col0 = n * kBN + c * 32;
+    const int col0 = col_base + c * 32;
     float v[32];
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
@@ -198,9 +201,19 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, const CUtenso
   }
 }
 
+// One 128-row x 256-column tile (M tile m, column tile n): warp q drains rows
+// m * 128 + q * 32 .. + 31, all the tile's columns.
+__device__ __forceinline__ void epilogue_tile(const GemmParams& p, const CUtensorMap* tmap_out,
+                                              int e, int m, int n, uint32_t taddr, uint32_t stg,
+                                              int* tokw, int q, int lane) {
+  epilogue_rows(p, tmap_out, e, static_cast<int64_t>(m) * kBM + q * 32, n * kBN,
+                p.n_out - n * kBN < kBN ? p.n_out - n * kBN : kBN, taddr, stg, tokw, lane);
+}
+
 // Row-major CTA-pair kernel launcher (expert_ffn_pair_rows.cu): 256-row x
 // 256-column tiles of row-contiguous operands (no gather).
-cudaError_t run_gemm_pair_rows(const CUtensorMap& ta, const CUtensorMap& tw, const CUtensorMap& to,
+cudaError_t run_gemm_pair_rows(const CUtensorMap& ta, const CUtensorMap& ta64,
+                               const CUtensorMap& tw, const CUtensorMap& to,
                                const GemmParams& gp, int num_sms, cudaStream_t st);
 // Dynamic shared memory of the CTA-pair kernels for N experts.
 size_t gemm_pair_smem_bytes(int N);

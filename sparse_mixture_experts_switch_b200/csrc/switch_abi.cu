@@ -201,15 +201,18 @@ switch_status_t cuda_status(cudaError_t e) {
     if (_e != cudaSuccess) return SWITCH_ERR_CUDA; \
   } while (0)
 
-// GEMM1 on row-major CTA pairs: asked for, or by default when every
-// expert's kept rows fit one 256-row pair tile but not one 128-row tile
-// (128 < C <= 256): then the pair tile has no more padding rows than two
-// single-CTA tiles, and each SM streams a third fewer operand bytes.
+// GEMM1 on row-major CTA pairs (each SM streams a third fewer operand bytes
+// per K step; an expert's last 128 rows take a half tile, not a padded pair
+// tile): asked for, or by default when C > 128 and either every expert's
+// rows fit one pair tile (C <= 256) or d_model >= 2048, where a tile's long
+// K loop amortises its epilogue (measured: XXL 1364-1376 vs 1394-1422 us;
+// with d_model 768 and C 512-1024 the one-CTA kernel is as fast or 1.5%
+// faster).
 bool gemm1_rows_pairs(const switch_config_t* c, int64_t C) {
   if (c->flags & SWITCH_FLAG_GEMM1_ROWS_PAIRS) return true;
   if (c->flags & (SWITCH_FLAG_GEMM_1SM | SWITCH_FLAG_GEMM_PAIRS | SWITCH_FLAG_GATHER_IN_GEMM))
     return false;
-  return C > 128 && C <= 256;
+  return C > 128 && (C <= 256 || c->d_model >= 2048);
 }
 
 int router_terms(const switch_config_t* c) {
