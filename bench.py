@@ -45,10 +45,10 @@ L2_FLUSH_BYTES = 256 << 20
 GEMM_SOURCES = ("common.cuh", "gemm_common.cuh", "gemm_pair.cuh", "expert_ffn.cu",
                 "expert_ffn_pair.cu", "expert_ffn_pair_rows.cu")
 GEMM_TRAFFIC = {"workload": "base",
-                "sources_sha256": "6aab2fb984fd416352e3c1c71cb906257297a029786ee11003080e3aa3259b90",
-                # GEMM1 715.75 MB read + 368.26 MB written; GEMM2 1233.39 + 89.68 MB
+                "sources_sha256": "d2067776da057fb3b27aa075813009009823d377f68b9d645996937a3265cdba",
+                # GEMM1 715.71 MB read + 369.03 MB written; GEMM2 1234.02 + 89.47 MB
                 # (mean of four forwards of one capture)
-                "bytes": 715.75e6 + 368.26e6 + 1233.39e6 + 89.68e6}
+                "bytes": 715.71e6 + 369.03e6 + 1234.02e6 + 89.47e6}
 
 
 def gemm_sources_sha256():
