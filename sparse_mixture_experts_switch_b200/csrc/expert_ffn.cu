@@ -341,18 +341,27 @@ static cudaError_t run_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const 
 cudaError_t launch_expert_ffn_bf16(const FfnArgs& a, cudaStream_t st) {
   const uint64_t slots = static_cast<uint64_t>(a.N) * static_cast<uint64_t>(a.C);
   CUtensorMap ta1, tb1, ta2, tb2, to1, to2;
+  // 64- and 32-row boxes of the token rows (half tiles; ragged pair tiles)
+  CUtensorMap ta1h, ta1q, ta2h, ta2q;
   const bool gather = a.x_disp == nullptr;
   const bool rows1 = a.pair1_rows && !gather;   // row-major pairs read rows by TMA only
   // CTA pairs load half a weight tile each (128 rows); single CTAs all 256.
   const uint32_t b_rows1 = (a.pair1 || rows1) ? 128u : static_cast<uint32_t>(kBN);
   const uint32_t b_rows2 = a.pair2 ? 128u : static_cast<uint32_t>(kBN);
   bool ok = true;
-  if (gather)
+  if (gather) {
     memset(&ta1, 0, sizeof(ta1));          // unused: rows are gathered with cp.async
-  else
+    memset(&ta1h, 0, sizeof(ta1h));
+    memset(&ta1q, 0, sizeof(ta1q));
+  } else {
     ok = make_tmap_bf16_2d(&ta1, a.x_disp, a.d, slots, kBK, kBM);
+    ok = ok && make_tmap_bf16_2d(&ta1h, a.x_disp, a.d, slots, kBK, kBM / 2);
+    ok = ok && make_tmap_bf16_2d(&ta1q, a.x_disp, a.d, slots, kBK, kBM / 4);
+  }
   ok = ok && make_tmap_bf16_2d(&tb1, a.w1, a.d, static_cast<uint64_t>(a.N) * a.F, kBK, b_rows1);
   ok = ok && make_tmap_bf16_2d(&ta2, a.hbuf, a.F, slots, kBK, kBM);
+  ok = ok && make_tmap_bf16_2d(&ta2h, a.hbuf, a.F, slots, kBK, kBM / 2);
+  ok = ok && make_tmap_bf16_2d(&ta2q, a.hbuf, a.F, slots, kBK, kBM / 4);
   ok = ok && make_tmap_bf16_2d(&tb2, a.w2, a.F, static_cast<uint64_t>(a.N) * a.d, kBK, b_rows2);
   // epilogue boxes: 32 rows x 32 columns of H (GEMM1) or Y (GEMM2, unfused)
   ok = ok && make_tmap_bf16_2d(&to1, a.hbuf, a.F, slots, 32, 32, true);
@@ -378,16 +387,11 @@ cudaError_t launch_expert_ffn_bf16(const FfnArgs& a, cudaStream_t st) {
   g1.err = a.err;
   g1.spin = a.spin;
   cudaError_t e;
-  if (rows1) {
-    // the half tiles' 64-row boxes of the dispatched rows
-    CUtensorMap ta1h;
-    if (!make_tmap_bf16_2d(&ta1h, a.x_disp, a.d, slots, kBK, kBM / 2))
-      return cudaErrorInvalidValue;
+  if (rows1)
     e = run_gemm_pair_rows(ta1, ta1h, tb1, to1, g1, a.num_sms, st);
-  }
   else if (a.pair1)
-    e = gather ? run_gemm_pair<true>(ta1, tb1, to1, g1, a.num_sms, st)
-               : run_gemm_pair<false>(ta1, tb1, to1, g1, a.num_sms, st);
+    e = gather ? run_gemm_pair<true>(ta1, ta1, ta1, tb1, to1, g1, a.num_sms, st)
+               : run_gemm_pair<false>(ta1, ta1h, ta1q, tb1, to1, g1, a.num_sms, st);
   else
     e = gather ? run_gemm<true>(ta1, tb1, to1, g1, a.num_sms, st)
                : run_gemm<false>(ta1, tb1, to1, g1, a.num_sms, st);
@@ -411,7 +415,7 @@ cudaError_t launch_expert_ffn_bf16(const FfnArgs& a, cudaStream_t st) {
     for (int i = 0; i < a.n_peers; ++i)
       g2.peer_out[i] = static_cast<__nv_bfloat16*>(a.peer_out[i]);
   }
-  return a.pair2 ? run_gemm_pair<false>(ta2, tb2, to2, g2, a.num_sms, st)
+  return a.pair2 ? run_gemm_pair<false>(ta2, ta2h, ta2q, tb2, to2, g2, a.num_sms, st)
                 : run_gemm<false>(ta2, tb2, to2, g2, a.num_sms, st);
 }
 

@@ -34,9 +34,18 @@
 
 namespace smoe {
 
+// Token rows per CTA of a tile (nmma / 2) decide its token box when the rows
+// come by TMA: 32, 64 or 128 rows, so a ragged tile with few tokens does not
+// stream a full 128-row box (its MMA reads only nmma / 2 rows per CTA).
+__device__ __forceinline__ int tok_box_rows(int nmma) {
+  return nmma <= 64 ? 32 : (nmma <= 128 ? 64 : 128);
+}
+
 template <bool kGather>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     expert_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_tok,
+                            const __grid_constant__ CUtensorMap tmap_tok64,
+                            const __grid_constant__ CUtensorMap tmap_tok32,
                             const __grid_constant__ CUtensorMap tmap_w,
                             const __grid_constant__ CUtensorMap tmap_out, GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -106,7 +115,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     const bool lead_warp = warp == 0;
     if (!kGather && !lead_warp) goto producer_done;
     {
-      if (lead_warp && lane == 0 && !kGather) tma_prefetch_desc(&tmap_tok);
+      if (lead_warp && lane == 0 && !kGather) {
+        tma_prefetch_desc(&tmap_tok);
+        tma_prefetch_desc(&tmap_tok64);
+        tma_prefetch_desc(&tmap_tok32);
+      }
       if (lead_warp && lane == 0) tma_prefetch_desc(&tmap_w);
       const int ch = lane & 7;
       const int gw = lead_warp ? 0 : warp - 5;                // 0..3
@@ -114,7 +127,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       const uint32_t vec_per_row = static_cast<uint32_t>(p.K / 8);
       const uint32_t sw_even = static_cast<uint32_t>((ch ^ (row0 & 7)) << 4);
       const uint32_t sw_odd = static_cast<uint32_t>((ch ^ ((row0 + 4) & 7)) << 4);
-      const uint32_t tx_bytes = kGather ? 2 * kPairWBytes : 2 * kPairStageBytes;
+      // bytes the TMA copies of one stage bring (both CTAs): the weights, plus
+      // the token rows' box when they come by TMA (gathered rows: cp.async)
+      auto tx_bytes_of = [&](const PairTile& t) {
+        return kGather ? 2 * kPairWBytes
+                       : 2 * (kPairWBytes + static_cast<uint32_t>(tok_box_rows(t.nmma)) * kBK * 2);
+      };
       int stage = 0;
       uint32_t phase = 0;
       uint32_t issued_mask = 0, issued_phase = 0;
@@ -140,6 +158,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         const int tok_row = static_cast<int>(static_cast<int64_t>(t.e) * p.C + t.t0 +
                                              static_cast<int>(rank) * (t.nmma >> 1));
         const int w_row = t.e * p.n_out + t.f0 + static_cast<int>(rank) * 128;
+        const uint32_t tx_bytes = tx_bytes_of(t);
+        const int box_rows = tok_box_rows(t.nmma);
+        const CUtensorMap* tmap_t = box_rows == 32 ? &tmap_tok32
+                                   : (box_rows == 64 ? &tmap_tok64 : &tmap_tok);
         uint32_t roff_next[8];
         const int next = tile + ncl;
         if (kGather && next < total) load_rows(next, roff_next);   // in flight meanwhile
@@ -172,7 +194,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             const uint32_t bar = full_lead + 8u * stage;
             if (leader) mbar_arrive_expect_tx(&full[stage], tx_bytes);
             tma_load_2d_pair(sw, &tmap_w, bar, kb * kBK, w_row);
-            if (!kGather) tma_load_2d_pair(stok, &tmap_tok, bar, kb * kBK, tok_row);
+            if (!kGather) tma_load_2d_pair(stok, tmap_t, bar, kb * kBK, tok_row);
           }
           issued_mask |= 1u << stage;
           issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
@@ -326,7 +348,8 @@ size_t gemm_pair_smem_bytes(int N) {
 }
 
 template <bool kGather>
-cudaError_t run_gemm_pair(const CUtensorMap& ttok, const CUtensorMap& tw, const CUtensorMap& to,
+cudaError_t run_gemm_pair(const CUtensorMap& ttok, const CUtensorMap& ttok64,
+                          const CUtensorMap& ttok32, const CUtensorMap& tw, const CUtensorMap& to,
                           const GemmParams& gp, int num_sms, cudaStream_t st) {
   const size_t smem = gemm_pair_smem_bytes(gp.N);
   static size_t smem_set[64] = {};
@@ -334,14 +357,17 @@ cudaError_t run_gemm_pair(const CUtensorMap& ttok, const CUtensorMap& tw, const 
       reinterpret_cast<const void*>(&expert_gemm_pair_kernel<kGather>), smem, smem_set);
   if (e != cudaSuccess) return e;
   const int grid = (num_sms / 2) * 2;
-  expert_gemm_pair_kernel<kGather><<<grid, kGemmThreads, smem, st>>>(ttok, tw, to, gp);
+  expert_gemm_pair_kernel<kGather><<<grid, kGemmThreads, smem, st>>>(ttok, ttok64, ttok32, tw,
+                                                                      to, gp);
   return cudaGetLastError();
 }
 
 template cudaError_t run_gemm_pair<true>(const CUtensorMap&, const CUtensorMap&,
+                                         const CUtensorMap&, const CUtensorMap&,
                                          const CUtensorMap&, const GemmParams&, int,
                                          cudaStream_t);
 template cudaError_t run_gemm_pair<false>(const CUtensorMap&, const CUtensorMap&,
+                                          const CUtensorMap&, const CUtensorMap&,
                                           const CUtensorMap&, const GemmParams&, int,
                                           cudaStream_t);
 

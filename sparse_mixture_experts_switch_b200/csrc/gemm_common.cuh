@@ -218,9 +218,11 @@ cudaError_t run_gemm_pair_rows(const CUtensorMap& ta, const CUtensorMap& ta64,
 // Dynamic shared memory of the CTA-pair kernels for N experts.
 size_t gemm_pair_smem_bytes(int N);
 
-// CTA-pair kernel launcher (expert_ffn_pair.cu).
+// CTA-pair kernel launcher (expert_ffn_pair.cu).  ta, ta64, ta32: the token
+// rows with 128-, 64- and 32-row boxes (unused when gathered).
 template <bool kGather>
-cudaError_t run_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to,
-                          const GemmParams& gp, int num_sms, cudaStream_t st);
+cudaError_t run_gemm_pair(const CUtensorMap& ta, const CUtensorMap& ta64, const CUtensorMap& ta32,
+                          const CUtensorMap& tb, const CUtensorMap& to, const GemmParams& gp,
+                          int num_sms, cudaStream_t st);
 
 }  // namespace smoe
