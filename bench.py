@@ -45,10 +45,10 @@ L2_FLUSH_BYTES = 256 << 20
 GEMM_SOURCES = ("common.cuh", "gemm_common.cuh", "gemm_pair.cuh", "expert_ffn.cu",
                 "expert_ffn_pair.cu", "expert_ffn_pair_rows.cu")
 GEMM_TRAFFIC = {"workload": "base",
-                "sources_sha256": "d2067776da057fb3b27aa075813009009823d377f68b9d645996937a3265cdba",
-                # GEMM1 715.71 MB read + 369.03 MB written; GEMM2 1234.02 + 89.47 MB
+                "sources_sha256": "1c28c5c52cbea4c75ac7c940e1cb64e1f1aaa45af6027d39d79d5e7c275d7071",
+                # GEMM1 715.73 MB read + 367.61 MB written; GEMM2 1205.44 + 89.26 MB
                 # (mean of four forwards of one capture)
-                "bytes": 715.71e6 + 369.03e6 + 1234.02e6 + 89.47e6}
+                "bytes": 715.73e6 + 367.61e6 + 1205.44e6 + 89.26e6}
 
 
 def gemm_sources_sha256():
