@@ -540,7 +540,6 @@ def main():
                                max_over_ranks(e0.elapsed_time(e1), dev, world))
     e2e_bytes = (x_host.numel() * x_host.element_size(),
                  out_host[0].numel() * out_host[0].element_size() + loss_host[0].numel() * 4)
-    clocks.stop()
     del x_host, out_host, step_graph, xb, ob
 
     # --------------------------------------- per-kernel roofline (rank 0)
@@ -566,8 +565,12 @@ def main():
         del x, w1, w2, ws, out
         torch.cuda.empty_cache()
         for name in extra:
+            tw0 = time.time()
             table[name] = time_workload(sm, WORKLOADS[name], dev, stream, flush, pk,
                                         max(5, min(args.steps, 20)))
+            # the SM clock while this workload's layer and expert FFN were timed
+            # (a long tensor-bound workload can reach the power cap)
+            table[name]["clocks"] = clocks.summary(tw0, time.time())
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
@@ -598,6 +601,7 @@ def main():
             "clocks": clocks.summary(t_wall0, t_wall1),
             "gpu_launches": launches_per_step(cfg, wl) * args.steps,
         }
+    clocks.stop()
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
