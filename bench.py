@@ -84,6 +84,9 @@ def parse_args():
                          "('all' = every bf16 workload, 'none'; default: all at N=1, none at N>1)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="budget of the oracle sample timed for cpu_baseline")
+    ap.add_argument("--stage", default=None, choices=sorted(STAGES),
+                    help="time one staged call alone on --workload (--steps replays after "
+                         "--warmup) and print its line instead of the layer's")
     return ap.parse_args()
 
 
@@ -389,6 +392,8 @@ def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.stage is not None:
+        return run_stage(args)
     if args.parallel == "ep" and int(os.environ.get("WORLD_SIZE", "1")) > 1:
         return run_expert_parallel(args)
 
@@ -607,6 +612,80 @@ def main():
         dist.destroy_process_group()
     if line is not None:
         print(json.dumps(line), flush=True)
+
+
+# staged calls that --stage times alone: algorithmic bytes as in the kernel table
+STAGES = ("router", "router_probs", "dispatch", "dispatch_gather", "combine", "aux_loss")
+
+
+def run_stage(args):
+    """One staged call on one GPU, on the workload's synthetic inputs: the
+    router (with probabilities) and the dispatch run once to give it real
+    routing; then `steps` graph replays of the call, each after an L2 flush."""
+    import torch
+    from sparse_mixture_experts_switch_b200 import switch_moe as sm
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    wl = WORKLOADS[args.workload]
+    w_r_h, b_r_h = make_router(wl)          # no expert weights: no stage here reads them
+    T, d, N = wl.T, wl.d_model, wl.n_experts
+    C = sm.switch_capacity(T, N, wl.capacity_factor)
+    tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+
+    def to_dev(a):
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+    x, w_r = to_dev(make_x(wl)), to_dev(w_r_h)
+    b_r = None if b_r_h is None else to_dev(b_r_h)
+    cfg = sm.config(T, d, wl.d_ff, N, wl.capacity_factor, dtype=wl.dtype, alpha=wl.alpha)
+    ws = sm.workspace(cfg, device=dev)
+    i32 = dict(dtype=torch.int32, device=dev)
+    idx, rank, counts = torch.empty(T, **i32), torch.empty(T, **i32), torch.empty(N, **i32)
+    gate = torch.empty(T, dtype=torch.float32, device=dev)
+    probs = torch.empty(T, N, dtype=torch.float32, device=dev)
+    drop = torch.empty(T, dtype=torch.uint8, device=dev)
+    slot = torch.empty(N * C, **i32)
+    x_disp = torch.empty(N * C, d, dtype=tdt, device=dev)
+    y = torch.empty(N * C, d, dtype=tdt, device=dev).normal_()
+    out = torch.empty_like(x)
+    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    sm.switch_router(cfg, x, w_r, b_r, idx, gate, probs, ws)
+    sm.switch_dispatch(cfg, idx, None, rank, drop, counts, slot, None, None, ws)
+    torch.cuda.synchronize(dev)
+    T_kept = int(np.minimum(counts.cpu().numpy().astype(np.int64), C).sum())
+    es = x.element_size()
+    calls = {
+        "router": (lambda: sm.switch_router(cfg, x, w_r, b_r, idx, gate, None, ws),
+                   T * d * es + N * d * 4 + T * 8),
+        "router_probs": (lambda: sm.switch_router(cfg, x, w_r, b_r, idx, gate, probs, ws),
+                         T * d * es + N * d * 4 + T * 8 + T * N * 4),
+        "dispatch": (lambda: sm.switch_dispatch(cfg, idx, None, rank, drop, counts, slot, None,
+                                                None, ws),
+                     T * 4 + T * 5 + N * 4 + N * C * 4),
+        "dispatch_gather": (lambda: sm.switch_dispatch(cfg, idx, None, rank, drop, counts, slot,
+                                                       x, x_disp, ws),
+                            T * 9 + N * 4 + N * C * 4 + T_kept * d * es + N * C * d * es),
+        "combine": (lambda: sm.switch_combine(cfg, x, idx, rank, drop, gate, y, out),
+                    2 * T * d * es + T_kept * d * es + T * 13),
+        "aux_loss": (lambda: sm.switch_aux_loss(cfg, counts, probs, loss, None, None, ws),
+                     T * N * 4 + N * 4),
+    }
+    fn, nbytes = calls[args.stage]
+    for _ in range(max(0, args.warmup - 3)):
+        fn()
+    t = time_replays(fn, flush, torch.cuda.current_stream(dev), dev, args.steps)
+    st, where, info = sm.switch_get_device_error(ws)
+    if st != 0:
+        raise RuntimeError(f"device error {st} at {where} ({info}) in {args.stage}")
+    pk, pk_kind = peaks()
+    print(json.dumps({"stage": args.stage, "workload": workload_desc(wl), "us": t * 1e6,
+                      "bytes": nbytes, "gbs": nbytes / t / 1e9,
+                      "frac_hbm": nbytes / t / 1e9 / pk["hbm_gbs"], "peak_kind": pk_kind,
+                      "steps": args.steps, "warmup": max(3, args.warmup),
+                      "l2": "flushed (256 MiB write) before every replay"}), flush=True)
 
 
 def layer_bounds(wl, T_kept, pk):
