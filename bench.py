@@ -503,8 +503,10 @@ def main():
     s_out = torch.cuda.Stream(dev)
     ev = lambda: torch.cuda.Event()                        # noqa: E731
 
-    def e2e_run(n):
-        """n pipelined steps; returns (first event, last event) for timing."""
+    def e2e_run(n, compute=True):
+        """n pipelined steps; returns (first event, last event) for timing.
+        compute=False runs the same copies and ordering without the layer:
+        the copy-bound ceiling of this loop on this host."""
         t_first = torch.cuda.Event(enable_timing=True)
         t_last = torch.cuda.Event(enable_timing=True)
         in_done, comp_done, out_done = {}, {}, {}
@@ -520,8 +522,9 @@ def main():
             stream.wait_event(in_done[i])
             if i >= 2:
                 stream.wait_event(out_done[i - 2])         # ob[b] copied out
-            sm.switch_layer_forward(cfg, xb[b], w_r, b_r, w1, w2, ob[b], None, None, None,
-                                    lb[b], ws)
+            if compute:
+                sm.switch_layer_forward(cfg, xb[b], w_r, b_r, w1, w2, ob[b], None, None, None,
+                                        lb[b], ws)
             comp_done[i] = ev()
             comp_done[i].record(stream)
             with torch.cuda.stream(s_out):
@@ -545,6 +548,13 @@ def main():
                                max_over_ranks(e0.elapsed_time(e1), dev, world))
     e2e_bytes = (x_host.numel() * x_host.element_size(),
                  out_host[0].numel() * out_host[0].element_size() + loss_host[0].numel() * 4)
+    # the same loop with the copies alone: what the host link allows
+    e2e_run(max(3, args.warmup), compute=False)
+    torch.cuda.synchronize(dev)
+    c0, c1 = e2e_run(args.steps, compute=False)
+    torch.cuda.synchronize(dev)
+    copy_ms = max_over_ranks(c0.elapsed_time(c1), dev, world)
+    copy_bound = job_throughput(T, args.steps, world, copy_ms)
     del x_host, out_host, step_graph, xb, ob
 
     # --------------------------------------- per-kernel roofline (rank 0)
@@ -602,7 +612,11 @@ def main():
                         "padding": 1.0 - T_kept / (N * C)},
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": e2e_bytes[0],
-                    "d2h_bytes_per_step": e2e_bytes[1]},
+                    "d2h_bytes_per_step": e2e_bytes[1],
+                    # the same pipelined loop with its copies only (no layer)
+                    "copy_bound": copy_bound,
+                    "frac_of_copy_bound": e2e_value / copy_bound,
+                    "h2d_gbs_per_gpu": e2e_bytes[0] * args.steps / (copy_ms * 1e-3) / 1e9},
             "clocks": clocks.summary(t_wall0, t_wall1),
             "gpu_launches": launches_per_step(cfg, wl) * args.steps,
         }
