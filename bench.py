@@ -856,9 +856,10 @@ def job_throughput(tokens_per_rank, steps, world, max_total_ms):
 def launches_per_step(cfg, wl):
     """Kernels switch_layer_forward launches with the default flags on this
     workload: router (weight split + tensor-core router, or SIMT router +
-    tile ranks), scan, finalize (with the row copy for bf16), GEMM1, GEMM2,
-    the dropped-token copy and the loss."""
-    return 2 + 1 + 1 + 2 + 1 + 1
+    tile ranks), the scan (which also forms the loss), finalize (for bf16
+    with the row copy, which also writes the dropped tokens' rows), GEMM1,
+    GEMM2 (with the combine); fp32 adds the dropped-token copy."""
+    return 2 + 1 + 1 + 2 + (0 if wl.dtype == "bf16" else 1)
 
 
 def kernel_rooflines(sm, cfg, wl, C, x, w_r, b_r, w1, w2, ws, flush, stream, dev, pk, pk_kind,

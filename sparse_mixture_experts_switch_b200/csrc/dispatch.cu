@@ -72,10 +72,18 @@ cudaError_t launch_tile_rank(int64_t T, int N, const int* idx_in, const float* p
 }
 
 // One block per expert: exclusive scan over its ntiles histogram entries.
+// With a loss (ScanLoss::loss set), each block then also forms its expert's
+// f_e P_e from the router's per-part probability sums, and the last block
+// to finish (a ticket picks which block, not any order of additions) adds
+// them into the loss: the additions are those of aux_loss_kernel, in the
+// same order, so both give the same bits.
 __global__ void __launch_bounds__(256) scan_kernel(int ntiles, const int* __restrict__ hist,
                                                    int* __restrict__ base,
-                                                   int* __restrict__ counts) {
+                                                   int* __restrict__ counts, ScanLoss L) {
   __shared__ int warp_tot[8];
+  __shared__ double cpart[kAuxChunks][8];
+  __shared__ double red[256];
+  __shared__ bool last;
   const int e = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const int* h = hist + static_cast<int64_t>(e) * ntiles;
@@ -115,11 +123,57 @@ __global__ void __launch_bounds__(256) scan_kernel(int ntiles, const int* __rest
     __syncthreads();
   }
   if (tid == 0) counts[e] = carry;
+  if (L.loss == nullptr) return;
+
+  // P_e: chunk `by` of the parts, warp lane w of it (parts p0 + w, + 8, ...)
+  const int N = static_cast<int>(gridDim.x);
+  const int chunks = L.nparts < kAuxChunks ? (L.nparts > 0 ? L.nparts : 1) : kAuxChunks;
+  const int per = (L.nparts + chunks - 1) / chunks;
+  if (tid < chunks * 8) {
+    const int by = tid >> 3, wq = tid & 7;
+    const int p0 = by * per;
+    const int p1 = p0 + per < L.nparts ? p0 + per : L.nparts;
+    double sp = 0.0;
+    for (int pp = p0 + wq; pp < p1; pp += 8)
+      sp += static_cast<double>(L.psum[static_cast<int64_t>(pp) * N + e]);
+    cpart[by][wq] = sp;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    double tot = 0.0;
+    for (int by = 0; by < chunks; ++by) {
+      double part = 0.0;
+      for (int q = 0; q < 8; ++q) part += cpart[by][q];
+      tot += part;
+    }
+    const double P = tot / static_cast<double>(L.T);
+    const double f = static_cast<double>(carry) / static_cast<double>(L.T);
+    L.fp[e] = f * P;
+    __threadfence();
+    last = atomicAdd(L.ticket, 1u) == gridDim.x - 1;
+  }
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  double acc = 0.0;
+  for (int i = tid; i < N; i += 256) acc += __ldcg(L.fp + i);
+  red[tid] = acc;
+  __syncthreads();
+  for (int stp = 128; stp > 0; stp >>= 1) {
+    if (tid < stp) red[tid] += red[tid + stp];
+    __syncthreads();
+  }
+  if (tid == 0) {
+    *L.loss = static_cast<float>(static_cast<double>(L.alpha) * N * red[0]);
+    *L.ticket = 0;               // ready for the next call on this workspace
+  }
 }
 
 cudaError_t launch_scan(int N, int ntiles, const int* hist, int* base, int* counts,
-                        cudaStream_t st) {
-  scan_kernel<<<N, 256, 0, st>>>(ntiles, hist, base, counts);
+                        cudaStream_t st, const ScanLoss* loss) {
+  ScanLoss L{};
+  if (loss != nullptr) L = *loss;
+  scan_kernel<<<N, 256, 0, st>>>(ntiles, hist, base, counts, L);
   return cudaGetLastError();
 }
 
@@ -211,7 +265,10 @@ cudaError_t launch_finalize(int64_t T, int N, int64_t C, int ntiles, const int* 
 // metadata loads are in flight together; then the warp copies the items'
 // rows one after another (16 bytes per lane per access): a kept token's row
 // into its slot, zeros into a padding slot.  Groups are small so that many
-// warps per SM each have a row in flight.
+// warps per SM each have a row in flight.  With `out` (top-1 layer, combine
+// fused into the second GEMM) a dropped token's output row is written here
+// as well: its residual x row (zeros without a residual), which is all the
+// combine gives a token that no expert processed.
 constexpr int kGatherGroup = 8;
 
 __global__ void __launch_bounds__(256, 4) finalize_gather_kernel(
@@ -219,7 +276,8 @@ __global__ void __launch_bounds__(256, 4) finalize_gather_kernel(
     const int* __restrict__ local_rank, const int* __restrict__ base,
     const int* __restrict__ counts, int* __restrict__ rank, uint8_t* __restrict__ drop,
     int* __restrict__ slot_token, int* __restrict__ mtile_start, int64_t tok_mod,
-    const uint4* __restrict__ x, uint4* __restrict__ x_disp, int64_t vec_per_row) {
+    const uint4* __restrict__ x, uint4* __restrict__ x_disp, int64_t vec_per_row,
+    uint4* __restrict__ out, bool out_residual) {
   if (blockIdx.x == 0 && threadIdx.x < 32 && mtile_start != nullptr)
     mtile_prefix_warp(N, C, counts, mtile_start);
   const int lane = threadIdx.x & 31;
@@ -232,6 +290,7 @@ __global__ void __launch_bounds__(256, 4) finalize_gather_kernel(
     const int64_t i = lane < kGatherGroup ? g0 + lane : items;   // other lanes: no item
     int64_t dst = -1;        // x_disp row this lane's item writes
     int64_t src = -1;        // x row copied into it (-1: zeros)
+    int64_t odst = -1;       // out row (a dropped token's) this item writes
     if (i < T) {
       const int e = idx[i];
       const int lr = local_rank[i];
@@ -246,6 +305,10 @@ __global__ void __launch_bounds__(256, 4) finalize_gather_kernel(
           src = tok;
           slot_token[dst] = static_cast<int>(tok);
         }
+      }
+      if (dropped && out != nullptr) {
+        odst = i;
+        src = out_residual ? i : -1;
       }
       rank[i] = r;
       drop[i] = dropped ? 1 : 0;
@@ -262,10 +325,22 @@ __global__ void __launch_bounds__(256, 4) finalize_gather_kernel(
     // the group's rows side by side: every lane has one 16-byte load of each
     // row in flight before it stores any of them
     int d_j[kGatherGroup], s_j[kGatherGroup];          // row ids fit int32 (validated)
+    const bool any_out = __any_sync(0xffffffffu, odst >= 0);
 #pragma unroll
     for (int j = 0; j < kGatherGroup; ++j) {
       d_j[j] = __shfl_sync(0xffffffffu, static_cast<int>(dst), j);
       s_j[j] = __shfl_sync(0xffffffffu, static_cast<int>(src), j);
+    }
+    if (any_out) {
+      // a dropped token among the group's items: one row at a time
+      for (int j = 0; j < kGatherGroup; ++j) {
+        const int o_j = __shfl_sync(0xffffffffu, static_cast<int>(odst), j);
+        if (o_j < 0) continue;
+        for (int64_t v = lane; v < vec_per_row; v += 32)
+          out[static_cast<int64_t>(o_j) * vec_per_row + v] =
+              s_j[j] >= 0 ? __ldg(x + static_cast<int64_t>(s_j[j]) * vec_per_row + v)
+                          : make_uint4(0, 0, 0, 0);
+      }
     }
     for (int64_t v = lane; v < vec_per_row; v += 32) {
       uint4 val[kGatherGroup];
@@ -284,14 +359,17 @@ cudaError_t launch_finalize_gather(int64_t T, int N, int64_t C, int ntiles, cons
                                    const int* local_rank, const int* base, const int* counts,
                                    int* rank, uint8_t* drop, int* slot_token, int* mtile_start,
                                    int64_t tok_mod, const void* x, void* x_disp,
-                                   int64_t row_bytes, cudaStream_t st) {
+                                   int64_t row_bytes, cudaStream_t st, void* out,
+                                   bool out_residual) {
+  if (out != nullptr && tok_mod != 0) return cudaErrorInvalidValue;   // top-1 only
   const int64_t items = T + static_cast<int64_t>(N) * C;
   int64_t blocks = (items + 8 * kGatherGroup - 1) / (8 * kGatherGroup);   // 8 warps a block
   if (blocks > 148 * 8) blocks = 148 * 8;
   if (blocks < 1) blocks = 1;
   finalize_gather_kernel<<<static_cast<int>(blocks), 256, 0, st>>>(
       T, N, C, ntiles, idx, local_rank, base, counts, rank, drop, slot_token, mtile_start,
-      tok_mod, static_cast<const uint4*>(x), static_cast<uint4*>(x_disp), row_bytes / 16);
+      tok_mod, static_cast<const uint4*>(x), static_cast<uint4*>(x_disp), row_bytes / 16,
+      static_cast<uint4*>(out), out_residual);
   return cudaGetLastError();
 }
 

@@ -14,10 +14,23 @@ constexpr int kTileTok = 128;   // tokens per dispatch/router tile
 cudaError_t launch_tile_rank(int64_t T, int N, const int* idx_in, const float* probs,
                              int* idx_out, int* local_rank, int* hist, int ntiles,
                              DevErr* err, cudaStream_t st);
+// The load-balancing loss formed by the scan (as launch_aux_loss would from
+// the same counts and per-part sums psum[nparts][N]): fp[N] doubles of
+// scratch, ticket one zero-initialised counter (left zero).
+struct ScanLoss {
+  int64_t T;
+  int nparts;
+  float alpha;
+  const float* psum;
+  float* loss;
+  double* fp;
+  unsigned* ticket;
+};
 // Exclusive scan of every expert's tile histogram in tile order:
-// base[e * ntiles + tile]; counts[e] = total.
+// base[e * ntiles + tile]; counts[e] = total; with `loss`, also the loss
+// from these counts.
 cudaError_t launch_scan(int N, int ntiles, const int* hist, int* base, int* counts,
-                        cudaStream_t st);
+                        cudaStream_t st, const ScanLoss* loss = nullptr);
 // rank/drop per token, slot_token (kept tokens and -1 padding), and the
 // per-expert prefix of 128-row M tiles mtile_start[N + 1].
 // tok_mod > 0: entries are route-major assignments of tok_mod tokens, and
@@ -27,12 +40,14 @@ cudaError_t launch_finalize(int64_t T, int N, int64_t C, int ntiles, const int* 
                             int* rank, uint8_t* drop, int* slot_token, int* mtile_start,
                             int64_t tok_mod, cudaStream_t st);
 // launch_finalize and the row copy x_disp[slot] = x[token] (zeros in padding
-// slots) in one kernel; row_bytes % 16 == 0.
+// slots) in one kernel; row_bytes % 16 == 0.  out (top-1 only, tok_mod 0):
+// also out[t] = x[t] (out_residual) or zeros for every dropped token t.
 cudaError_t launch_finalize_gather(int64_t T, int N, int64_t C, int ntiles, const int* idx,
                                    const int* local_rank, const int* base, const int* counts,
                                    int* rank, uint8_t* drop, int* slot_token, int* mtile_start,
                                    int64_t tok_mod, const void* x, void* x_disp,
-                                   int64_t row_bytes, cudaStream_t st);
+                                   int64_t row_bytes, cudaStream_t st, void* out = nullptr,
+                                   bool out_residual = true);
 // Only mtile_start from counts (for a standalone expert-FFN call).
 cudaError_t launch_mtile_table(int N, int64_t C, const int* counts, int* mtile_start,
                                cudaStream_t st);

@@ -523,33 +523,40 @@ switch_status_t switch_layer_forward(const switch_config_t* cfg, const void* x,
   // 2-3. dispatch: scan over tiles, then rank / drop / slots / tile table.
   // Top-2: the first choices' totals are the loss's counts; then the 2T
   // assignments are ranked as one sequence, first choices first.
-  int* counts_loss = counts_p;
+  // The load-balancing loss (f_i over the first choices) is formed by the
+  // scan that counts the first choices.
+  const ScanLoss sl{T, nparts, cfg->alpha, psum, loss, c.at<double>(c.L.fpsc),
+                    c.at<unsigned>(kTicketOffset)};
+  const ScanLoss* slp = loss ? &sl : nullptr;
   if (top2) {
-    counts_loss = c.at<int>(c.L.counts1);
-    SMOE_TRY(launch_scan(N, nt, hist, c.at<int>(c.L.base), counts_loss, c.st));
+    SMOE_TRY(launch_scan(N, nt, hist, c.at<int>(c.L.base), c.at<int>(c.L.counts1), c.st, slp));
     SMOE_TRY(launch_tile_rank(A, N, idx_p, nullptr, nullptr, local_rank, hist, nta, c.err,
                               c.st));
   }
-  SMOE_TRY(launch_scan(N, nta, hist, c.at<int>(c.L.base), counts_p, c.st));
+  SMOE_TRY(launch_scan(N, nta, hist, c.at<int>(c.L.base), counts_p, c.st, top2 ? nullptr : slp));
   int* slot_token = c.at<int>(c.L.slot_token);
   int* rank = c.at<int>(c.L.rank);
   uint8_t* drop = c.at<uint8_t>(c.L.drop);
-  // (bf16, default) the routed rows copied expert by expert in the same pass
+  // (bf16, default) the routed rows copied expert by expert in the same pass;
+  // with the combine fused into the second GEMM (top-1), the dropped tokens'
+  // output rows too
   const bool row_copy = bf16 && !(cfg->flags & SWITCH_FLAG_GATHER_IN_GEMM);
+  const bool fused = !(cfg->flags & SWITCH_FLAG_UNFUSED_COMBINE) && !top2;
+  const bool residual = !(cfg->flags & SWITCH_FLAG_NO_RESIDUAL);
+  const bool dropped_in_copy = row_copy && fused;
   if (row_copy)
     SMOE_TRY(launch_finalize_gather(A, N, c.C, nta, idx_p, local_rank, c.at<int>(c.L.base),
                                     counts_p, rank, drop, slot_token,
                                     c.at<int>(c.L.mtile_start), top2 ? T : 0, x,
                                     c.ws + c.L.xdisp, static_cast<int64_t>(cfg->d_model) * 2,
-                                    c.st));
+                                    c.st, dropped_in_copy ? out : nullptr, residual));
   else
     SMOE_TRY(launch_finalize(A, N, c.C, nta, idx_p, local_rank, c.at<int>(c.L.base), counts_p,
                              rank, drop, slot_token, c.at<int>(c.L.mtile_start),
                              top2 ? T : 0, c.st));
   // 4. experts, with the combine fused into the second GEMM unless asked not
   // to (or top-2: two experts write each token, so Y, then one combine)
-  const bool fused = !(cfg->flags & SWITCH_FLAG_UNFUSED_COMBINE) && !top2;
-  const void* x_res = (cfg->flags & SWITCH_FLAG_NO_RESIDUAL) ? nullptr : x;
+  const void* x_res = residual ? x : nullptr;
   FfnArgs a{};
   a.T = T;
   a.d = cfg->d_model;
@@ -576,14 +583,11 @@ switch_status_t switch_layer_forward(const switch_config_t* cfg, const void* x,
   a.pair1_rows = gemm1_rows_pairs(cfg, c.C);
   if (row_copy) a.x_disp = c.ws + c.L.xdisp;
   SMOE_TRY(bf16 ? launch_expert_ffn_bf16(a, c.st) : launch_expert_ffn_f32(a, c.st));
-  // 5. dropped tokens (fused) or every token (unfused)
-  SMOE_TRY(launch_combine(T, cfg->d_model, c.C, bf16, x_res, idx_p, rank, drop, gate_p,
-                          c.ws + c.L.ybuf, out, fused, routes_of(*cfg), c.st));
-  // 6. load-balancing loss (f_i over the first choices)
-  if (loss)
-    SMOE_TRY(launch_aux_loss(T, N, nparts, cfg->alpha, counts_loss, psum, loss, nullptr,
-                             nullptr, c.at<double>(c.L.fpsc), c.at<unsigned>(kTicketOffset),
-                             c.st));
+  // 5. dropped tokens (fused; unless the row copy wrote them) or every token
+  // (unfused)
+  if (!dropped_in_copy)
+    SMOE_TRY(launch_combine(T, cfg->d_model, c.C, bf16, x_res, idx_p, rank, drop, gate_p,
+                            c.ws + c.L.ybuf, out, fused, routes_of(*cfg), c.st));
   if (training) {
     if (idx)
       SMOE_TRY(cudaMemcpyAsync(idx, idx_p, sizeof(int) * A, cudaMemcpyDeviceToDevice, c.st));
