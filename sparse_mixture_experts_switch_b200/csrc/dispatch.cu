@@ -265,7 +265,8 @@ cudaError_t launch_finalize(int64_t T, int N, int64_t C, int ntiles, const int* 
 // metadata loads are in flight together; then the warp copies the items'
 // rows one after another (16 bytes per lane per access): a kept token's row
 // into its slot, zeros into a padding slot.  Groups are small so that many
-// warps per SM each have a row in flight.  With `out` (top-1 layer, combine
+// warps per SM each have a row in flight.  Without zero_pad the padding
+// slots' rows are left as they are (their slot_token is still -1).  With `out` (top-1 layer, combine
 // fused into the second GEMM) a dropped token's output row is written here
 // as well: its residual x row (zeros without a residual), which is all the
 // combine gives a token that no expert processed.
@@ -277,7 +278,7 @@ __global__ void __launch_bounds__(256, 4) finalize_gather_kernel(
     const int* __restrict__ counts, int* __restrict__ rank, uint8_t* __restrict__ drop,
     int* __restrict__ slot_token, int* __restrict__ mtile_start, int64_t tok_mod,
     const uint4* __restrict__ x, uint4* __restrict__ x_disp, int64_t vec_per_row,
-    uint4* __restrict__ out, bool out_residual) {
+    uint4* __restrict__ out, bool out_residual, bool zero_pad) {
   if (blockIdx.x == 0 && threadIdx.x < 32 && mtile_start != nullptr)
     mtile_prefix_warp(N, C, counts, mtile_start);
   const int lane = threadIdx.x & 31;
@@ -319,7 +320,7 @@ __global__ void __launch_bounds__(256, 4) finalize_gather_kernel(
       const int64_t kept = counts[e] < C ? counts[e] : C;
       if (r >= kept) {
         slot_token[s] = -1;
-        dst = s;
+        dst = zero_pad ? s : -1;
       }
     }
     // the group's rows side by side: every lane has one 16-byte load of each
@@ -360,7 +361,7 @@ cudaError_t launch_finalize_gather(int64_t T, int N, int64_t C, int ntiles, cons
                                    int* rank, uint8_t* drop, int* slot_token, int* mtile_start,
                                    int64_t tok_mod, const void* x, void* x_disp,
                                    int64_t row_bytes, cudaStream_t st, void* out,
-                                   bool out_residual) {
+                                   bool out_residual, bool zero_pad) {
   if (out != nullptr && tok_mod != 0) return cudaErrorInvalidValue;   // top-1 only
   const int64_t items = T + static_cast<int64_t>(N) * C;
   int64_t blocks = (items + 8 * kGatherGroup - 1) / (8 * kGatherGroup);   // 8 warps a block
@@ -369,7 +370,7 @@ cudaError_t launch_finalize_gather(int64_t T, int N, int64_t C, int ntiles, cons
   finalize_gather_kernel<<<static_cast<int>(blocks), 256, 0, st>>>(
       T, N, C, ntiles, idx, local_rank, base, counts, rank, drop, slot_token, mtile_start,
       tok_mod, static_cast<const uint4*>(x), static_cast<uint4*>(x_disp), row_bytes / 16,
-      static_cast<uint4*>(out), out_residual);
+      static_cast<uint4*>(out), out_residual, zero_pad);
   return cudaGetLastError();
 }
 

@@ -42,12 +42,14 @@ cudaError_t launch_finalize(int64_t T, int N, int64_t C, int ntiles, const int* 
 // launch_finalize and the row copy x_disp[slot] = x[token] (zeros in padding
 // slots) in one kernel; row_bytes % 16 == 0.  out (top-1 only, tok_mod 0):
 // also out[t] = x[t] (out_residual) or zeros for every dropped token t.
+// zero_pad false: padding rows of x_disp are not written (for a consumer
+// that never uses them: the forward GEMMs store no result of a padding row).
 cudaError_t launch_finalize_gather(int64_t T, int N, int64_t C, int ntiles, const int* idx,
                                    const int* local_rank, const int* base, const int* counts,
                                    int* rank, uint8_t* drop, int* slot_token, int* mtile_start,
                                    int64_t tok_mod, const void* x, void* x_disp,
                                    int64_t row_bytes, cudaStream_t st, void* out = nullptr,
-                                   bool out_residual = true);
+                                   bool out_residual = true, bool zero_pad = true);
 // Only mtile_start from counts (for a standalone expert-FFN call).
 cudaError_t launch_mtile_table(int N, int64_t C, const int* counts, int* mtile_start,
                                cudaStream_t st);

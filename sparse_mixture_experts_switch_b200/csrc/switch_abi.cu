@@ -549,7 +549,8 @@ switch_status_t switch_layer_forward(const switch_config_t* cfg, const void* x,
                                     counts_p, rank, drop, slot_token,
                                     c.at<int>(c.L.mtile_start), top2 ? T : 0, x,
                                     c.ws + c.L.xdisp, static_cast<int64_t>(cfg->d_model) * 2,
-                                    c.st, dropped_in_copy ? out : nullptr, residual));
+                                    c.st, dropped_in_copy ? out : nullptr, residual,
+                                    /*zero_pad=*/training));
   else
     SMOE_TRY(launch_finalize(A, N, c.C, nta, idx_p, local_rank, c.at<int>(c.L.base), counts_p,
                              rank, drop, slot_token, c.at<int>(c.L.mtile_start),
