@@ -440,7 +440,7 @@ def main():
     def step():
         sm.switch_layer_forward(cfg, x, w_r, b_r, w1, w2, out, idx, gate, counts, loss, ws)
 
-    # One forward = 8 kernel launches with no host synchronisation inside, so
+    # One forward = 6 kernel launches with no host synchronisation inside, so
     # it is captured once as a CUDA graph and replayed: the timed region then
     # measures the kernels, not the host's launch latency.
     step_graph = make_graph(step)
