@@ -406,6 +406,12 @@ cudaError_t launch_expert_ffn_bf16(const FfnArgs& a, cudaStream_t st) {
   g2.out = static_cast<__nv_bfloat16*>(a.y);
   g2.ldo = a.d;
   g2.x_res = static_cast<const __nv_bfloat16*>(a.x_res);
+  g2.res_by_slot = false;
+  if (a.res_by_slot && a.x_res != nullptr && a.mode2 == kModeCombine && a.pair2 &&
+      a.x_disp != nullptr) {
+    g2.x_res = static_cast<const __nv_bfloat16*>(a.x_disp);
+    g2.res_by_slot = true;
+  }
   g2.gate = a.gate;
   g2.comb_out = static_cast<__nv_bfloat16*>(a.out);
   if (a.mode2 == kModeCombineEp) {

@@ -54,6 +54,10 @@ struct GemmParams {
   __nv_bfloat16* peer_out[kEpMaxRanks];   // kModeCombineEp: each rank's output rows
   DevErr* err;
   long long spin;
+  // kModeCombine on CTA pairs: x_res is the dispatched buffer and a slot's
+  // residual row is its own row there (a copy of x[token]), so a tile reads
+  // consecutive rows instead of its tokens' scattered rows of x.
+  bool res_by_slot;
 };
 
 // Rows (m*128 + r) of expert e in this tile that hold a token.

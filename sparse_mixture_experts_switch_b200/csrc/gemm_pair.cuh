@@ -95,8 +95,9 @@ __device__ __forceinline__ void combine_meta(const GemmParams& p, const PairTile
   for (int c = 0; c < 8; ++c) {
     m.g[c] = 0.f;
     if (m.tok[c] >= 0) {
-      const int64_t res_row = ep ? row0 + c * 32 + lane : static_cast<int64_t>(m.tok[c]);
-      m.g[c] = p.gate[ep ? res_row : m.tok[c]];
+      const int64_t res_row =
+          (ep || p.res_by_slot) ? row0 + c * 32 + lane : static_cast<int64_t>(m.tok[c]);
+      m.g[c] = p.gate[ep ? row0 + c * 32 + lane : m.tok[c]];
       if (p.x_res != nullptr && fb < p.n_out)
         prefetch_l2(p.x_res + res_row * p.n_out + fb);
     }
@@ -157,7 +158,8 @@ __device__ __forceinline__ void epilogue_tile_t(const GemmParams& p, const CUten
         tk[pass] = __shfl_sync(0xffffffffu, tkc, rr);
         g[pass] = __shfl_sync(0xffffffffu, gcl, rr);
         xr[pass] = make_uint4(0, 0, 0, 0);
-        const int64_t res_row = ep ? row0 + j0 + rr : static_cast<int64_t>(tk[pass]);
+        const int64_t res_row =
+            (ep || p.res_by_slot) ? row0 + j0 + rr : static_cast<int64_t>(tk[pass]);
         if (tk[pass] >= 0 && p.x_res != nullptr)
           xr[pass] = __ldg(reinterpret_cast<const uint4*>(p.x_res + res_row * p.n_out + fb +
                                                           qq * 8));

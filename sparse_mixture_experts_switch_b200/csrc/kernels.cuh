@@ -157,6 +157,9 @@ struct FfnArgs {
   bool pair2;               // GEMM2 on CTA pairs
   bool pair1_rows;          // GEMM1 on CTA pairs with the rows as M (256-row tiles)
   bool gemm1_only;          // stop after GEMM1 (the backward pass recomputes H)
+  // kModeCombine on CTA pairs with x_disp holding every kept row: the
+  // residual is read from x_disp by slot (x_res must then be x)
+  bool res_by_slot;
   void* const* peer_out;    // kModeCombineEp: every rank's output [T_rank, d] (host array)
   int n_peers;
   DevErr* err;

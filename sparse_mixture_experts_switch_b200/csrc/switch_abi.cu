@@ -583,6 +583,7 @@ switch_status_t switch_layer_forward(const switch_config_t* cfg, const void* x,
   a.pair2 = !(cfg->flags & SWITCH_FLAG_GEMM_1SM);
   a.pair1_rows = gemm1_rows_pairs(cfg, c.C);
   if (row_copy) a.x_disp = c.ws + c.L.xdisp;
+  a.res_by_slot = row_copy;            // the residual rows from the dispatched copy
   SMOE_TRY(bf16 ? launch_expert_ffn_bf16(a, c.st) : launch_expert_ffn_f32(a, c.st));
   // 5. dropped tokens (fused; unless the row copy wrote them) or every token
   // (unfused)
