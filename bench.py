@@ -45,10 +45,10 @@ L2_FLUSH_BYTES = 256 << 20
 GEMM_SOURCES = ("common.cuh", "gemm_common.cuh", "gemm_pair.cuh", "expert_ffn.cu",
                 "expert_ffn_pair.cu", "expert_ffn_pair_rows.cu")
 GEMM_TRAFFIC = {"workload": "base",
-                "sources_sha256": "1c28c5c52cbea4c75ac7c940e1cb64e1f1aaa45af6027d39d79d5e7c275d7071",
-                # GEMM1 715.73 MB read + 367.61 MB written; GEMM2 1205.44 + 89.26 MB
+                "sources_sha256": "7d69bded4bbe40d742d5bf14338b0e2e0207cab2b4923298d9e9ec395ba85062",
+                # GEMM1 715.74 MB read + 368.30 MB written; GEMM2 1203.28 + 89.06 MB
                 # (mean of four forwards of one capture)
-                "bytes": 715.73e6 + 367.61e6 + 1205.44e6 + 89.26e6}
+                "bytes": 715.74e6 + 368.30e6 + 1203.28e6 + 89.06e6}
 
 
 def gemm_sources_sha256():
