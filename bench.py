@@ -30,7 +30,9 @@ sys.path.insert(0, ROOT)
 
 import numpy as np  # noqa: E402
 
-from switch_inputs import WORKLOADS, make_x, make_router, make_w1, make_w2, Inputs  # noqa: E402
+from switch_inputs import (WORKLOADS, PROFILE_WORKLOADS, make_x, make_router, make_w1,  # noqa: E402
+                           make_w2, Inputs)
+ALL_WORKLOADS = {**WORKLOADS, **PROFILE_WORKLOADS}
 
 METRIC = "Switch-layer fwd tokens/s"
 UNIT = "tokens/s"
@@ -74,7 +76,10 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="base", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="base",
+                    choices=sorted(WORKLOADS) + sorted(PROFILE_WORKLOADS),
+                    help="the headline workload (default base); base_e64, Base's per-expert "
+                         "shape at half the tokens and experts, is for counter captures")
     ap.add_argument("--parallel", default="replicas", choices=["replicas", "ep"],
                     help="N > 1: independent replicas (default), or expert parallelism "
                          "(each rank N/G experts and its own T tokens, one routing group)")
@@ -162,7 +167,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    wl = WORKLOADS[args.workload]
+    wl = ALL_WORKLOADS[args.workload]
     inp = host_inputs(wl)
     per_step_budget = max(1.0, min(8.0, 150.0 / max(1, args.steps + args.warmup)))
     est, n_exp = oracle_sample(inp, per_step_budget)          # sizes the sample
@@ -332,7 +337,7 @@ def run_expert_parallel(args):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
-    wl = WORKLOADS[args.workload]
+    wl = ALL_WORKLOADS[args.workload]
     inp = host_inputs(wl, rank)
     T, d, F, N = wl.T, wl.d_model, wl.d_ff, wl.n_experts
     E = N // world
@@ -410,7 +415,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=dev)
 
-    wl = WORKLOADS[args.workload]
+    wl = ALL_WORKLOADS[args.workload]
     inp = host_inputs(wl, rank)
     T, d, F, N = wl.T, wl.d_model, wl.d_ff, wl.n_experts
     C = sm.switch_capacity(T, N, wl.capacity_factor)
@@ -629,7 +634,8 @@ def main():
 
 
 # staged calls that --stage times alone: algorithmic bytes as in the kernel table
-STAGES = ("router", "router_probs", "dispatch", "dispatch_gather", "combine", "aux_loss")
+STAGES = ("router", "router_probs", "dispatch", "dispatch_gather", "combine", "aux_loss",
+          "expert_ffn")
 
 
 def run_stage(args):
@@ -640,8 +646,8 @@ def run_stage(args):
     from sparse_mixture_experts_switch_b200 import switch_moe as sm
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    wl = WORKLOADS[args.workload]
-    w_r_h, b_r_h = make_router(wl)          # no expert weights: no stage here reads them
+    wl = ALL_WORKLOADS[args.workload]
+    w_r_h, b_r_h = make_router(wl)          # expert weights only for the expert FFN stage
     T, d, N = wl.T, wl.d_model, wl.n_experts
     C = sm.switch_capacity(T, N, wl.capacity_factor)
     tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
@@ -667,9 +673,15 @@ def run_stage(args):
     loss = torch.empty(1, dtype=torch.float32, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     sm.switch_router(cfg, x, w_r, b_r, idx, gate, probs, ws)
-    sm.switch_dispatch(cfg, idx, None, rank, drop, counts, slot, None, None, ws)
+    sm.switch_dispatch(cfg, idx, None, rank, drop, counts, slot, x, x_disp, ws)
     torch.cuda.synchronize(dev)
     T_kept = int(np.minimum(counts.cpu().numpy().astype(np.int64), C).sum())
+    ffn = None
+    if args.stage == "expert_ffn":
+        w1, w2 = to_dev(make_w1(wl)), to_dev(make_w2(wl))
+        cfg_rows = sm.config(T, d, wl.d_ff, N, wl.capacity_factor, dtype=wl.dtype,
+                             alpha=wl.alpha, flags=sm.FLAG_ROWS_DISPATCHED)
+        ffn = lambda: sm.switch_expert_ffn(cfg_rows, x_disp, None, counts, w1, w2, y, ws)  # noqa: E731
     es = x.element_size()
     calls = {
         "router": (lambda: sm.switch_router(cfg, x, w_r, b_r, idx, gate, None, ws),
@@ -686,6 +698,8 @@ def run_stage(args):
                     2 * T * d * es + T_kept * d * es + T * 13),
         "aux_loss": (lambda: sm.switch_aux_loss(cfg, counts, probs, loss, None, None, ws),
                      T * N * 4 + N * 4),
+        # FLOPs, not bytes: the line's "gbs" is then useful GFLOP/s
+        "expert_ffn": (ffn, 4.0 * T_kept * d * wl.d_ff),
     }
     fn, nbytes = calls[args.stage]
     for _ in range(max(0, args.warmup - 3)):
@@ -695,11 +709,16 @@ def run_stage(args):
     if st != 0:
         raise RuntimeError(f"device error {st} at {where} ({info}) in {args.stage}")
     pk, pk_kind = peaks()
-    print(json.dumps({"stage": args.stage, "workload": workload_desc(wl), "us": t * 1e6,
-                      "bytes": nbytes, "gbs": nbytes / t / 1e9,
-                      "frac_hbm": nbytes / t / 1e9 / pk["hbm_gbs"], "peak_kind": pk_kind,
-                      "steps": args.steps, "warmup": max(3, args.warmup),
-                      "l2": "flushed (256 MiB write) before every replay"}), flush=True)
+    line = {"stage": args.stage, "workload": workload_desc(wl), "us": t * 1e6}
+    if args.stage == "expert_ffn":
+        line.update({"useful_flops": nbytes, "tflops": nbytes / t / 1e12,
+                     "frac_burst": nbytes / t / 1e12 / pk["bf16_tflops"]})
+    else:
+        line.update({"bytes": nbytes, "gbs": nbytes / t / 1e9,
+                     "frac_hbm": nbytes / t / 1e9 / pk["hbm_gbs"]})
+    line.update({"peak_kind": pk_kind, "steps": args.steps, "warmup": max(3, args.warmup),
+                 "l2": "flushed (256 MiB write) before every replay"})
+    print(json.dumps(line), flush=True)
 
 
 def layer_bounds(wl, T_kept, pk):

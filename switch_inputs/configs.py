@@ -42,3 +42,9 @@ XXL = Workload("xxl", T=16384, d_model=4096, d_ff=10240, n_experts=64,
 
 WORKLOADS = {w.name: w for w in
              (TINY, BASE, ZIPF_100, ZIPF_125, ZIPF_200, LARGE, XXL)}
+
+# A smaller case with Base's per-expert shape (half the tokens and half the
+# experts: the same capacity and tile shapes), for counter captures that
+# replay a kernel many times; not one of the benchmark's workloads.
+BASE_E64 = BASE.with_(name="base_e64", T=32768, n_experts=64, seed=1005)
+PROFILE_WORKLOADS = {w.name: w for w in (BASE_E64,)}
