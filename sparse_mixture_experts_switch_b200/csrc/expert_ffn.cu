@@ -407,6 +407,7 @@ cudaError_t launch_expert_ffn_bf16(const FfnArgs& a, cudaStream_t st) {
   g2.ldo = a.d;
   g2.x_res = static_cast<const __nv_bfloat16*>(a.x_res);
   g2.res_by_slot = false;
+  g2.reverse_tiles = a.pair2;          // GEMM1 ran just before: its last rows are in L2
   if (a.res_by_slot && a.x_res != nullptr && a.mode2 == kModeCombine && a.pair2 &&
       a.x_disp != nullptr) {
     g2.x_res = static_cast<const __nv_bfloat16*>(a.x_disp);

@@ -58,6 +58,10 @@ struct GemmParams {
   // residual row is its own row there (a copy of x[token]), so a tile reads
   // consecutive rows instead of its tokens' scattered rows of x.
   bool res_by_slot;
+  // CTA-pair kernel: take the tile list from its end (the last experts
+  // first).  Right after GEMM1 the last experts' hidden rows are the ones
+  // still in L2, so GEMM2 reads them before they are evicted.
+  bool reverse_tiles;
 };
 
 // Rows (m*128 + r) of expert e in this tile that hold a token.

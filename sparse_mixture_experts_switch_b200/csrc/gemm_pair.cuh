@@ -53,6 +53,7 @@ struct PairTile {
 __device__ __forceinline__ PairTile pair_tile(const GemmParams& p, const int* pts, int tile) {
   PairTile t;
   int tt, mf;
+  if (p.reverse_tiles) tile = pts[p.N] * p.ntiles_n - 1 - tile;
   decode_tile(tile, pts, p.N, p.ntiles_n, t.e, tt, mf);
   t.t0 = tt * 256;
   const int64_t rem = kept_rows(p, t.e) - t.t0;
