@@ -47,10 +47,10 @@ L2_FLUSH_BYTES = 256 << 20
 GEMM_SOURCES = ("common.cuh", "gemm_common.cuh", "gemm_pair.cuh", "expert_ffn.cu",
                 "expert_ffn_pair.cu", "expert_ffn_pair_rows.cu")
 GEMM_TRAFFIC = {"workload": "base",
-                "sources_sha256": "7d69bded4bbe40d742d5bf14338b0e2e0207cab2b4923298d9e9ec395ba85062",
-                # GEMM1 715.74 MB read + 368.30 MB written; GEMM2 1203.28 + 89.06 MB
+                "sources_sha256": "c4fce9f41a3dd7e284f8129f86b81096d3c4c9f22e2d073bac49b74f260f4f6a",
+                # GEMM1 715.75 MB read + 368.88 MB written; GEMM2 1197.38 + 89.05 MB
                 # (mean of four forwards of one capture)
-                "bytes": 715.74e6 + 368.30e6 + 1203.28e6 + 89.06e6}
+                "bytes": 715.75e6 + 368.88e6 + 1197.38e6 + 89.05e6}
 
 
 def gemm_sources_sha256():
