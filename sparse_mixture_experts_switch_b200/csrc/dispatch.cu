@@ -283,7 +283,9 @@ __global__ void __launch_bounds__(256, 4) finalize_gather_kernel(
     mtile_prefix_warp(N, C, counts, mtile_start);
   const int lane = threadIdx.x & 31;
   const int64_t nslots = static_cast<int64_t>(N) * C;
-  const int64_t items = T + nslots;
+  // without zero_pad nothing reads the padding slots (their slot_token
+  // entries included), so only the assignments are items
+  const int64_t items = T + (zero_pad ? nslots : 0);
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   for (int64_t g0 = (static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5)) *
                     kGatherGroup;
@@ -363,7 +365,7 @@ cudaError_t launch_finalize_gather(int64_t T, int N, int64_t C, int ntiles, cons
                                    int64_t row_bytes, cudaStream_t st, void* out,
                                    bool out_residual, bool zero_pad) {
   if (out != nullptr && tok_mod != 0) return cudaErrorInvalidValue;   // top-1 only
-  const int64_t items = T + static_cast<int64_t>(N) * C;
+  const int64_t items = T + (zero_pad ? static_cast<int64_t>(N) * C : 0);
   int64_t blocks = (items + 8 * kGatherGroup - 1) / (8 * kGatherGroup);   // 8 warps a block
   if (blocks > 148 * 8) blocks = 148 * 8;
   if (blocks < 1) blocks = 1;

@@ -42,8 +42,9 @@ cudaError_t launch_finalize(int64_t T, int N, int64_t C, int ntiles, const int* 
 // launch_finalize and the row copy x_disp[slot] = x[token] (zeros in padding
 // slots) in one kernel; row_bytes % 16 == 0.  out (top-1 only, tok_mod 0):
 // also out[t] = x[t] (out_residual) or zeros for every dropped token t.
-// zero_pad false: padding rows of x_disp are not written (for a consumer
-// that never uses them: the forward GEMMs store no result of a padding row).
+// zero_pad false: padding slots are not touched at all, neither their rows
+// of x_disp nor their slot_token entries (for a consumer that never reads
+// them: the forward GEMMs use only kept slots).
 cudaError_t launch_finalize_gather(int64_t T, int N, int64_t C, int ntiles, const int* idx,
                                    const int* local_rank, const int* base, const int* counts,
                                    int* rank, uint8_t* drop, int* slot_token, int* mtile_start,
