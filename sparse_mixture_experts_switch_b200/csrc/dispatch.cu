@@ -266,10 +266,11 @@ cudaError_t launch_finalize(int64_t T, int N, int64_t C, int ntiles, const int* 
 // rows one after another (16 bytes per lane per access): a kept token's row
 // into its slot, zeros into a padding slot.  Groups are small so that many
 // warps per SM each have a row in flight.  Without zero_pad the padding
-// slots' rows are left as they are (their slot_token is still -1).  With `out` (top-1 layer, combine
-// fused into the second GEMM) a dropped token's output row is written here
-// as well: its residual x row (zeros without a residual), which is all the
-// combine gives a token that no expert processed.
+// slots are not items at all (neither their rows nor their slot_token
+// entries are written).  With `out` (top-1 layer, combine fused into the
+// second GEMM) a dropped token's output row is written here as well: its
+// residual x row (zeros without a residual), which is all the combine gives
+// a token that no expert processed.
 constexpr int kGatherGroup = 8;
 
 __global__ void __launch_bounds__(256, 4) finalize_gather_kernel(
@@ -320,9 +321,9 @@ __global__ void __launch_bounds__(256, 4) finalize_gather_kernel(
       const int e = static_cast<int>(s / C);
       const int64_t r = s - static_cast<int64_t>(e) * C;
       const int64_t kept = counts[e] < C ? counts[e] : C;
-      if (r >= kept) {
+      if (r >= kept) {             // (only with zero_pad: see `items`)
         slot_token[s] = -1;
-        dst = zero_pad ? s : -1;
+        dst = s;
       }
     }
     // the group's rows side by side: every lane has one 16-byte load of each
