@@ -97,3 +97,16 @@ def test_backward_workspace_extends_the_forward(sm):
 def test_status_strings(sm):
     for s in range(7):
         assert sm.switch_status_string(s)
+
+
+def test_binding_flags_match_the_header(sm):
+    """Every SWITCH_FLAG_* of the header has the same value in the binding,
+    and the binding defines no flag the header does not."""
+    src = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    header = {m.group(1): int(m.group(2))
+              for m in re.finditer(r"\bSWITCH_FLAG_([A-Z0-9_]+)\s*=\s*(\d+)", src)}
+    binding = {k[len("FLAG_"):]: v for k, v in vars(sm).items()
+               if k.startswith("FLAG_") and isinstance(v, int)}
+    assert header and header == binding
+    assert len(set(header.values())) == len(header)          # distinct bits
+    assert all(v & (v - 1) == 0 for v in header.values())    # one bit each
