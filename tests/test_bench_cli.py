@@ -41,3 +41,27 @@ def test_launch_count_matches_the_forward(monkeypatch):
     # bf16: weight split, router, scan (+ loss), slots + row copy, GEMM1, GEMM2
     assert bench.launches_per_step(None, WORKLOADS["base"]) == 6
     assert bench.launches_per_step(None, WORKLOADS["tiny"]) == 7
+
+
+def test_layer_roofline_arithmetic():
+    """The bench's layer roofline for Base, by hand: useful FLOPs
+    2·T·d·N (router) + 4·T_kept·d·F (the two expert GEMMs) at the bf16 peak,
+    against x read three times, every expert weight once and out written
+    once at the HBM peak."""
+    import bench
+    wl = WORKLOADS["base"]
+    pk = {"bf16_tflops": 1646.3, "hbm_gbs": 6433.9, "bf16_tflops_sustained": 1394.0}
+    T_kept = 65484
+    b = bench.layer_bounds(wl, T_kept, pk)
+    flops = 2 * 65536 * 768 * 128 + 4 * T_kept * 768 * 3072
+    nbytes = 4 * 65536 * 768 * 2 + 2 * 128 * 768 * 3072 * 2
+    assert b["useful_flops"] == pytest.approx(flops, rel=1e-12)
+    assert b["min_bytes"] == nbytes
+    assert b["t_compute_us"] == pytest.approx(flops / 1646.3e12 * 1e6, rel=1e-12)
+    assert b["t_mem_us"] == pytest.approx(nbytes / 6433.9e9 * 1e6, rel=1e-12)
+    assert b["bound"] == "tensor" and 380 < b["t_compute_us"] < 386 and 248 < b["t_mem_us"] < 252
+    row = bench.workload_row(wl, 640, 0.661, 571e-6, T_kept, pk)
+    assert row["tokens_per_s"] == pytest.approx(65536 / 0.661e-3)
+    assert row["expert_ffn_frac_burst"] == pytest.approx(4 * T_kept * 768 * 3072 / 571e-6
+                                                         / 1e12 / 1646.3)
+    assert row["padding"] == pytest.approx(1 - T_kept / (128 * 640))
